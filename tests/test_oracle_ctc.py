@@ -1,0 +1,70 @@
+"""Pins of the oracle's CTC head, greedy collapse and INT8 g64 dequantisation."""
+import itertools
+
+import numpy as np
+import pytest
+
+import oracle
+from conformer_speech_recognition_b200 import synth
+from conftest import read_golden_rows
+
+
+def test_collapse_hand_cases():
+    rows = read_golden_rows("collapse.txt")
+    assert len(rows) >= 6
+    for blank, seq, expected in rows:
+        seq = [int(t) for t in seq.split()]
+        exp = [int(t) for t in expected.split()]
+        assert oracle.greedy_collapse(seq, int(blank)) == exp
+
+
+def test_collapse_vs_groupby_bruteforce():
+    rng = np.random.default_rng(0)
+    for _ in range(500):
+        blank = int(rng.integers(1, 5))
+        seq = rng.integers(0, blank + 1, size=int(rng.integers(0, 20))).tolist()
+        ref = [k for k, _ in itertools.groupby(seq) if k != blank]
+        assert oracle.greedy_collapse(seq, blank) == ref
+
+
+def test_ctc_head_logsoftmax_and_first_argmax():
+    rng = np.random.default_rng(1)
+    d, C, T = 6, 5, 4
+    W = {"head.weight": rng.normal(size=(C, d)), "head.bias": np.zeros(C)}
+    enc = rng.normal(size=(T, d))
+    z, logp, a = oracle.ctc_head(enc, W)
+    np.testing.assert_allclose(np.exp(logp).sum(axis=1), 1.0, rtol=1e-12)
+    np.testing.assert_allclose(z - logp, np.broadcast_to(np.log(np.exp(z).sum(axis=1))[:, None], z.shape), rtol=1e-12)
+    np.testing.assert_array_equal(a, [int(np.argmax(r)) for r in z])
+    # ties: lowest index wins
+    W2 = {"head.weight": np.zeros((C, d)), "head.bias": np.array([0.0, 2.0, 2.0, 1.0, 2.0])}
+    _, _, a2 = oracle.ctc_head(enc, W2)
+    assert np.all(a2 == 1)
+
+
+def test_int8_g64_round_trip_bound():
+    rng = np.random.default_rng(2)
+    w = (rng.normal(0, 0.02, size=(16, 256))).astype(np.float16)
+    w[3, 64:128] = 0  # an all-zero group
+    q, s = synth.quantize_g64(w)
+    assert q.dtype == np.int8 and s.dtype == np.float16 and s.shape == (16, 4)
+    assert np.abs(q).max() <= 127
+    back = oracle.dequant_g64(q, s)
+    err = np.abs(back - w.astype(np.float64))
+    bound = np.repeat(s.astype(np.float64), 64, axis=1) / 2
+    assert np.all(err <= bound * (1 + 1e-9) + 1e-12)
+    assert s[3, 1] == 1.0 and np.all(q[3, 64:128] == 0)
+    # the largest magnitude of each group maps to +-127 (up to fp16 rounding of the scale)
+    g = np.abs(q.reshape(16, 4, 64)).max(axis=2)
+    assert np.all((g >= 126) | (s == 1.0))
+
+
+def test_int8_weights_replace_every_linear():
+    cfg = synth.model_config(dict(synth.LARGE, n_layers=1, d_model=128, n_heads=2, ffn_dim=256), 257, "int8_g64")
+    W = synth.random_weights(cfg)
+    names = synth.quantized_linear_names(cfg)
+    assert len(names) == 11
+    for n in names:
+        assert n + ".weight" not in W and W[n + ".weight_q"].dtype == np.int8
+        w, b = oracle.get_linear(W, n)
+        assert w.shape[0] == b.shape[0]
