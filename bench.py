@@ -1,0 +1,393 @@
+#!/usr/bin/env python
+"""Throughput of the GigaAM Conformer encoder + CTC path on B200.
+
+One step = gam_encode + gam_ctc_greedy over one batch of a synthetic workload
+(audio already resident in device memory).  Prints ONE JSON line (rank 0).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+Multi-GPU (launched by torchrun, one process per GPU): every rank runs its own
+copy of the workload batch (independent clips, no data-path collective), the
+elapsed time is the max over ranks, value = total audio seconds / that time
+(weak scaling).
+
+``--impl reference`` times the CPU oracle (the plain NumPy definition of the
+path) on this machine's host cores, one bounded sample per step.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from conformer_speech_recognition_b200 import synth  # noqa: E402
+
+METRIC = "audio-sec/sec (×realtime) encoder+CTC at 1 B200; GEMM TFLOP/s vs fp16 peak"
+UNIT = "audio-sec/sec"
+DEFAULT_WORKLOAD = "c2_varlen_b32_d768"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+# ---------------------------------------------------------------------------
+# helpers
+# ---------------------------------------------------------------------------
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        d["source"] = "measured"
+        return d
+    d = dict(FALLBACK_PEAKS)
+    d["source"] = "fallback"
+    return d
+
+
+def algorithmic_work(cfg, lens):
+    """Per-kernel-family algorithmic FLOPs or bytes for ONE step, and the number of
+    launches of each family per step.  Valid frames only (padding excluded)."""
+    from conformer_speech_recognition_b200 import gam
+    fr, el, fmax, tmax = gam.gam_plan_lengths(cfg, lens)
+    d, f, L, C = cfg["d_model"], cfg["ffn_dim"], cfg["n_layers"], cfg["n_classes"]
+    Kdw = cfg["conv_kernel"]
+    M = float(np.sum(el))
+    L1 = float(np.sum((fr - 1) // 2))
+    att = float(np.sum(el.astype(np.float64) ** 2))
+    wbytes = 1 if cfg["precision"] == "int8_g64" else 2
+    act = 2  # fp16 activations
+    fl = {
+        "gemm_subsampling": 2 * L1 * 5 * cfg["n_mels"] * d + 2 * M * 5 * d * d,
+        "gemm_ffn_up": 2 * L * 2 * M * d * f,
+        "gemm_ffn_down": 2 * L * 2 * M * f * d,
+        "gemm_qkv": L * 2 * M * d * 3 * d,
+        "gemm_attn_out": L * 2 * M * d * d,
+        "gemm_pw1_glu": L * 2 * M * d * 2 * d,
+        "gemm_pw2": L * 2 * M * d * d,
+        "attention": L * 4 * att * d,
+        "ctc_gemm": 2 * M * d * C,
+        "frontend": float(np.sum(fr)) * (2 * 320 * 320 + 2 * 161 * 64),
+    }
+    by = {
+        "layernorm": L * 5 * M * d * (4 + act),
+        "dwconv": L * M * d * 2 * act,
+        "frontend": float(np.sum(lens)) * 4 + float(np.sum(fr)) * 64 * act,
+    }
+    launches = {"gemm_subsampling": 2, "gemm_ffn_up": 2 * L, "gemm_ffn_down": 2 * L, "gemm_qkv": L,
+                "gemm_attn_out": L, "gemm_pw1_glu": L, "gemm_pw2": L, "attention": L, "ctc_gemm": 1,
+                "frontend": 1, "layernorm": 4 * L + 1, "dwconv": L}
+    _ = wbytes
+    return fl, by, launches
+
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        if self.thread:
+            self.thread.join(timeout=2)
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                smax.append(float(parts[1]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[4:8]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def oracle_throughput(name, budget_s, clip_indices=None):
+    """The CPU oracle (fp32, as it stands) on a bounded sample of the workload.
+    Returns (audio seconds per second, description, threads)."""
+    import oracle
+    cfg = synth.workload_config(name)
+    W = synth.random_weights(cfg, seed=0)
+    audio, lens = synth.workload_audio(name)
+    order = clip_indices if clip_indices is not None else list(range(len(lens)))
+    done_audio = 0.0
+    used = []
+    t0 = time.perf_counter()
+    for i in order:
+        oracle.transcribe_clip(audio[i, :lens[i]], W, cfg, np.float32)
+        done_audio += lens[i] / synth.SAMPLE_RATE
+        used.append(int(i))
+        if time.perf_counter() - t0 >= budget_s:
+            break
+    el = time.perf_counter() - t0
+    try:
+        from threadpoolctl import threadpool_info
+        threads = max((p.get("num_threads", 1) for p in threadpool_info()), default=os.cpu_count())
+    except Exception:
+        threads = os.cpu_count()
+    desc = f"{len(used)} clip(s) {used[:8]}{'...' if len(used) > 8 else ''} of {name}, {done_audio:.1f} audio-s, " \
+           f"fp32 NumPy oracle, {el:.1f} s"
+    return done_audio / el, desc, threads
+
+
+# ---------------------------------------------------------------------------
+# reference arm: the oracle on the host cores
+# ---------------------------------------------------------------------------
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return 0
+    name = args.workload
+    cfg = synth.workload_config(name)
+    import oracle
+    W = synth.random_weights(cfg, seed=0)
+    audio, lens = synth.workload_audio(name)
+    order = list(np.argsort(lens))  # shortest clips first keeps every step bounded
+    per_step = []
+    audio_s = []
+
+    def one(i):
+        t0 = time.perf_counter()
+        oracle.transcribe_clip(audio[i, :lens[i]], W, cfg, np.float32)
+        return time.perf_counter() - t0, lens[i] / synth.SAMPLE_RATE
+
+    k = 0
+    for _ in range(args.warmup):
+        one(order[k % len(order)])
+        k += 1
+    for _ in range(args.steps):
+        t, a = one(order[k % len(order)])
+        per_step.append(t)
+        audio_s.append(a)
+        k += 1
+    total_t, total_a = sum(per_step), sum(audio_s)
+    value = total_a / total_t
+    try:
+        from threadpoolctl import threadpool_info
+        threads = max((p.get("num_threads", 1) for p in threadpool_info()), default=os.cpu_count())
+    except Exception:
+        threads = os.cpu_count()
+    sample = f"one clip per step (shortest first) of {name}: {total_a:.1f} audio-s over {args.steps} steps"
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000 * total_t / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": {"workload": name, "batch": 1, "precision": "fp32 oracle (NumPy)"},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------------------
+# our arm
+# ---------------------------------------------------------------------------
+
+def run_ours(args, rank, world, local_rank):
+    import torch
+    from conformer_speech_recognition_b200 import gam
+    dist = world > 1
+    if dist:
+        import torch.distributed as td
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    name = args.workload
+    cfg = synth.workload_config(name)
+    W = synth.random_weights(cfg, seed=0)
+    audio_np, lens = synth.workload_audio(name)
+    B, nmax = audio_np.shape
+    ctx = gam.gam_create(cfg, W, B, nmax, device=local_rank)
+    audio = torch.from_numpy(audio_np).to(dev)
+    fr, el, fmax, tmax = gam.gam_plan_lengths(cfg, lens)
+    enc = torch.empty((B, tmax, cfg["d_model"]), dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    audio_seconds = float(np.sum(lens)) / synth.SAMPLE_RATE
+
+    def step():
+        gam.gam_encode(ctx, audio, lens, out=enc, stream=stream)
+        return gam.gam_ctc_greedy(ctx, enc, el, stream=stream)
+
+    # warm-up with every family timed: picks the dominant kernel family
+    gam.gam_profile_enable(ctx, -1)
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    warm = gam.gam_profile_all(ctx)
+    kinds = {gam.gam_profile_kind_name(k): k for k in range(gam.gam_profile_kinds())}
+    dominant = max(warm, key=lambda n: warm[n][0])
+
+    # timed region: only the dominant family carries event pairs
+    gam.gam_profile_enable(ctx, 1 << kinds[dominant])
+    clocks = ClockSampler(local_rank) if rank == 0 else None
+    if dist:
+        td.barrier()
+    torch.cuda.synchronize(dev)
+    if clocks:
+        clocks.start()
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    t_start.record(stream)
+    for _ in range(args.steps):
+        step()
+    t_end.record(stream)
+    torch.cuda.synchronize(dev)
+    elapsed_ms = t_start.elapsed_time(t_end)
+    clock_info = clocks.stop() if clocks else None
+    prof = gam.gam_profile_all(ctx)
+    launches = sum(v[1] for v in prof.values())
+    dom_ms, dom_n = prof[dominant]
+    gam.gam_device_status(ctx)
+
+    # end to end through the public host-buffer call (copies inside the timed region)
+    pinned = torch.from_numpy(audio_np).pin_memory()
+    tok_h = torch.empty((B, tmax), dtype=torch.int32).pin_memory()
+    cnt_h = torch.empty((B,), dtype=torch.int32).pin_memory()
+    gam.gam_profile_enable(ctx, 0)
+    for _ in range(max(1, args.warmup)):
+        gam.gam_transcribe(ctx, pinned, lens, tok_h, cnt_h, stream=stream)
+    if dist:
+        td.barrier()
+    torch.cuda.synchronize(dev)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        gam.gam_transcribe(ctx, pinned, lens, tok_h, cnt_h, stream=stream)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = e0.elapsed_time(e1)
+
+    if dist:
+        t = torch.tensor([elapsed_ms, e2e_ms], dtype=torch.float64, device=dev)
+        td.all_reduce(t, op=td.ReduceOp.MAX)
+        elapsed_ms, e2e_ms = float(t[0]), float(t[1])
+
+    if rank == 0:
+        peaks = load_peaks()
+        fl, by, _ = algorithmic_work(cfg, lens)
+        value = world * audio_seconds * args.steps / (elapsed_ms / 1e3)
+        e2e_value = world * audio_seconds * args.steps / (e2e_ms / 1e3)
+        avg_launch_ms = dom_ms / max(dom_n, 1)
+        per_step_launches_dom = dom_n / args.steps
+        if dominant in fl and dominant != "frontend":
+            per_launch = fl[dominant] / per_step_launches_dom
+            achieved = per_launch / (avg_launch_ms / 1e3) / 1e12
+            peak = peaks["bf16_tflops_sustained"]
+            roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                    "frac": achieved / peak, "traffic": None, "kernel": dominant,
+                    "peak_source": f"{peaks['source']} bf16 sustained (fp16 dense rate equal to bf16)"}
+        else:
+            per_launch = by.get(dominant, 0.0) / max(per_step_launches_dom, 1)
+            achieved = per_launch / (avg_launch_ms / 1e3) / 1e9
+            peak = peaks["hbm_gbs"]
+            roof = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                    "traffic": None, "kernel": dominant, "peak_source": f"{peaks['source']} HBM copy"}
+        gemm_flops = sum(v for k, v in fl.items() if k.startswith("gemm_"))
+        # GEMM kernel time per step from the warm-up pass (every family timed there)
+        gemm_ms = sum(v[0] for k, v in warm.items() if k.startswith("gemm_")) / max(args.warmup, 1)
+        cpu = None
+        if not args.no_cpu_baseline and world == 1:
+            v, desc, threads = oracle_throughput(name, args.cpu_budget)
+            cpu = {"value": v, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": desc}
+        h2d = int(B * nmax * 4 + 5 * (B + 1) * 4 + B * 4)
+        d2h = int(B * tmax * 4 + B * 4)
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": elapsed_ms / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f16", "data": "synthetic",
+            "config": {"workload": name, "batch": B, "audio_seconds_per_step": audio_seconds,
+                       "valid_encoder_frames": int(np.sum(el)), "precision": cfg["precision"],
+                       "layers": cfg["n_layers"], "d_model": cfg["d_model"],
+                       "l2": "not flushed: the fp16 weights (442 MB) and activations stream through the 126 MB L2 "
+                             "every step",
+                       "parallelism": f"replicas x{world} (independent batches, no collective on the data path)"},
+            "roofline": roof,
+            "gemm_tflops_per_step_algorithmic": gemm_flops / 1e12,
+            "gemm_tflops_per_s_of_gemm_time": gemm_flops / (gemm_ms / 1e3) / 1e12 if gemm_ms > 0 else None,
+            "gemm_frac_of_fp16_peak": (gemm_flops / (gemm_ms / 1e3) / 1e12) / peaks["bf16_tflops_sustained"]
+            if gemm_ms > 0 else None,
+            "cpu_baseline": cpu,
+            "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+            "gpu_launches": int(launches),
+            "clocks": clock_info,
+            "warmup_profile_ms": {k: round(v[0] / max(args.warmup, 1), 4) for k, v in warm.items() if v[1]},
+        }
+        print(json.dumps(line), flush=True)
+    ctx.close()
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(synth.WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle CPU time for cpu_baseline")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        print("warning: at least 3 warm-up steps are required for a valid number", file=sys.stderr)
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        return run_reference(args, rank, world)
+    if world > 1:
+        import datetime
+        import torch.distributed as td
+        td.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    try:
+        return run_ours(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch.distributed as td
+            td.destroy_process_group()
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,28 @@
+// Tensor-core (tcgen05 / TMEM / TMA) kernels: GEMM with fused epilogues and
+// masked flash attention.  Host-side interface used by the runtime.
+#pragma once
+
+#include "common.cuh"
+
+namespace gam {
+
+// Per-context state of the tensor-core kernels (tensor-map cache, status word).
+struct TcGemmCache {
+  int* status = nullptr;  // device word set when a bounded wait gives up
+};
+
+// True when the tensor-core GEMM handles this operand / shape / epilogue combination.
+bool tc_supported(int a_dtype, int b_dtype, int N, int K, int epi);
+
+cudaError_t launch_gemm_tc(TcGemmCache* cache, const void* A, const void* A2, int n_split, int lda, WeightOp B,
+                           int M, int N, int K, int epi, const EpiParams& ep, cudaStream_t s);
+
+// Masked multi-head attention: tensor cores for fp16 activations, CUDA cores for fp32.
+cudaError_t launch_attention(TcGemmCache* cache, const void* qk, const void* vt, Clips clips, void* o, int t_half,
+                             int rows_pad, int n_heads, int d_head, int t_max, cudaStream_t s);
+
+cudaError_t tc_read_status(TcGemmCache* cache, int* status);
+cudaError_t tc_reset_status(TcGemmCache* cache);
+void tc_release(TcGemmCache* cache);
+
+}  // namespace gam

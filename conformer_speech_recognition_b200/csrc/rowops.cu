@@ -1,0 +1,359 @@
+// Memory-bound row kernels of the Conformer block and the CTC decoder.
+//
+//  * LayerNorm over d (one warp per row, float4 loads, two-pass statistics in
+//    registers), in three forms: plain; fused with the rotary embedding of
+//    "GigaAM on MLX: the transcripts matched, but the model was broken",
+//    "Trap 2" (u = LN(x) feeds V, u_rot = u * cos + rotate_half(u) * sin per
+//    head feeds Q and K; tables of base 5000 from "Trap 1"); and chained
+//    (block-final LayerNorm written back to the residual stream, then the next
+//    block's first LayerNorm).
+//  * Depthwise conv over time with BatchNorm folded into its weights and
+//    bias, then Swish (textbook Conformer convolution module), rows outside
+//    the clip read as zero.
+//  * Encoder output scatter to the padded [B, T', d] layout.
+//  * CTC: log-softmax + first-index argmax per frame, then greedy collapse
+//    (runs merged, blanks dropped) with a block-wide scan.
+#include "common.cuh"
+
+namespace gam {
+namespace {
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+template <typename T>
+__device__ __forceinline__ void store4(T* p, float4 v);
+template <>
+__device__ __forceinline__ void store4<float>(float* p, float4 v) { *reinterpret_cast<float4*>(p) = v; }
+template <>
+__device__ __forceinline__ void store4<__half>(__half* p, float4 v) {
+  __half2 a = __floats2half2_rn(v.x, v.y), b = __floats2half2_rn(v.z, v.w);
+  uint2 u;
+  u.x = *reinterpret_cast<uint32_t*>(&a);
+  u.y = *reinterpret_cast<uint32_t*>(&b);
+  *reinterpret_cast<uint2*>(p) = u;
+}
+
+__device__ __forceinline__ float ld1(const float* p) { return *p; }
+__device__ __forceinline__ float ld1(const __half* p) { return __half2float(*p); }
+
+// Normalise the row held in v[0..nv) (float4 chunks, chunk j at column 4(32 j + lane)).
+__device__ __forceinline__ void ln_row(float4 (&v)[8], int nv, int d, float eps, const float* g, const float* b,
+                                       int lane) {
+  float s = 0.f;
+#pragma unroll
+  for (int j = 0; j < 8; ++j)
+    if (j < nv) s += v[j].x + v[j].y + v[j].z + v[j].w;
+  const float mean = warp_sum(s) / d;
+  float q = 0.f;
+#pragma unroll
+  for (int j = 0; j < 8; ++j)
+    if (j < nv) {
+      v[j].x -= mean; v[j].y -= mean; v[j].z -= mean; v[j].w -= mean;
+      q += v[j].x * v[j].x + v[j].y * v[j].y + v[j].z * v[j].z + v[j].w * v[j].w;
+    }
+  const float rstd = rsqrtf(warp_sum(q) / d + eps);
+#pragma unroll
+  for (int j = 0; j < 8; ++j)
+    if (j < nv) {
+      const int c = (j * 32 + lane) * 4;
+      const float4 gg = *reinterpret_cast<const float4*>(g + c);
+      const float4 bb = *reinterpret_cast<const float4*>(b + c);
+      v[j].x = v[j].x * rstd * gg.x + bb.x;
+      v[j].y = v[j].y * rstd * gg.y + bb.y;
+      v[j].z = v[j].z * rstd * gg.z + bb.z;
+      v[j].w = v[j].w * rstd * gg.w + bb.w;
+    }
+}
+
+__device__ __forceinline__ void load_row(const float* x, float4 (&v)[8], int nv, int lane) {
+#pragma unroll
+  for (int j = 0; j < 8; ++j)
+    if (j < nv) v[j] = *reinterpret_cast<const float4*>(x + (j * 32 + lane) * 4);
+}
+
+template <typename T>
+__global__ void __launch_bounds__(256)
+ln_kernel(const float* __restrict__ x, const float* __restrict__ g, const float* __restrict__ b, float eps,
+          T* __restrict__ u, int rows, int d) {
+  const int row = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+  if (row >= rows) return;
+  const int nv = d >> 7;
+  float4 v[8];
+  load_row(x + (size_t)row * d, v, nv, lane);
+  ln_row(v, nv, d, eps, g, b, lane);
+#pragma unroll
+  for (int j = 0; j < 8; ++j)
+    if (j < nv) store4<T>(u + (size_t)row * d + (j * 32 + lane) * 4, v[j]);
+}
+
+template <typename T>
+__global__ void __launch_bounds__(256)
+ln_chain_kernel(float* __restrict__ x, const float* __restrict__ g1, const float* __restrict__ b1,
+                const float* __restrict__ g2, const float* __restrict__ b2, float eps, T* __restrict__ u, int rows,
+                int d) {
+  const int row = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+  if (row >= rows) return;
+  const int nv = d >> 7;
+  float4 v[8];
+  float* xr = x + (size_t)row * d;
+  load_row(xr, v, nv, lane);
+  ln_row(v, nv, d, eps, g1, b1, lane);
+#pragma unroll
+  for (int j = 0; j < 8; ++j)
+    if (j < nv) *reinterpret_cast<float4*>(xr + (j * 32 + lane) * 4) = v[j];
+  ln_row(v, nv, d, eps, g2, b2, lane);
+#pragma unroll
+  for (int j = 0; j < 8; ++j)
+    if (j < nv) store4<T>(u + (size_t)row * d + (j * 32 + lane) * 4, v[j]);
+}
+
+template <typename T>
+__global__ void __launch_bounds__(256)
+ln_rope_kernel(const float* __restrict__ x, const float* __restrict__ g, const float* __restrict__ b, float eps,
+               const float* __restrict__ cos_tab, const float* __restrict__ sin_tab, Clips clips, T* __restrict__ u,
+               T* __restrict__ urot, int rows, int d, int dh) {
+  __shared__ __align__(16) float srow[8][1024];
+  const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int row = blockIdx.x * 8 + w;
+  if (row >= rows) return;
+  const int nv = d >> 7;
+  float4 v[8];
+  load_row(x + (size_t)row * d, v, nv, lane);
+  ln_row(v, nv, d, eps, g, b, lane);
+  float* sr = srow[w];
+#pragma unroll
+  for (int j = 0; j < 8; ++j)
+    if (j < nv) {
+      const int c = (j * 32 + lane) * 4;
+      store4<T>(u + (size_t)row * d + c, v[j]);
+      *reinterpret_cast<float4*>(sr + c) = v[j];
+    }
+  __syncwarp();
+  const int ci = clips.find(row, 1);
+  int t = row - clips.e(ci);
+  if (t < 0 || t >= clips.L2(ci)) t = 0;  // gap row: any finite rotation
+  const int half = dh >> 1;
+  const float* ct = cos_tab + (size_t)t * half;
+  const float* st = sin_tab + (size_t)t * half;
+#pragma unroll
+  for (int j = 0; j < 8; ++j)
+    if (j < nv) {
+      const int c0 = (j * 32 + lane) * 4;
+      float o[4];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const int c = c0 + k;
+        const int cc = c % dh;
+        const int i = cc < half ? cc : cc - half;
+        const float cs = __ldg(ct + i), sn = __ldg(st + i);
+        o[k] = cc < half ? sr[c] * cs - sr[c + half] * sn : sr[c] * cs + sr[c - half] * sn;
+      }
+      store4<T>(urot + (size_t)row * d + c0, make_float4(o[0], o[1], o[2], o[3]));
+    }
+}
+
+// Depthwise conv: CTA = 32 rows x 128 channels; input rows [r0 - pad, r0 + 32 + pad)
+// staged in shared memory; w is tap-major [K][d] with BatchNorm folded in.
+template <typename T>
+__global__ void __launch_bounds__(256)
+dwconv_kernel(const T* __restrict__ g, const float* __restrict__ w, const float* __restrict__ bias, Clips clips,
+              T* __restrict__ out, int rows, int d, int K) {
+  __shared__ float tile[94][128];
+  const int pad = (K - 1) / 2;
+  const int r0 = blockIdx.x * 32, c0 = blockIdx.y * 128;
+  const int nrow = 32 + 2 * pad;
+  for (int idx = threadIdx.x; idx < nrow * 128; idx += 256) {
+    const int rr = idx >> 7, cc = idx & 127;
+    const int src = r0 - pad + rr;
+    tile[rr][cc] = (src >= 0 && src < rows) ? ld1(g + (size_t)src * d + c0 + cc) : 0.f;
+  }
+  __syncthreads();
+  const int cc = threadIdx.x & 127, c = c0 + cc;
+  const float bv = __ldg(bias + c);
+  for (int j = threadIdx.x >> 7; j < 32; j += 2) {
+    const int r = r0 + j;
+    if (r >= rows) break;
+    const int ci = clips.find(r, 1);
+    const int lo = clips.e(ci), hi = lo + clips.L2(ci);
+    float v = 0.f;
+    if (r >= lo && r < hi) {
+      float acc = bv;
+      for (int k = 0; k < K; ++k) {
+        const int src = r + k - pad;
+        if (src >= lo && src < hi) acc = fmaf(__ldg(w + (size_t)k * d + c), tile[j + k][cc], acc);
+      }
+      v = acc / (1.f + __expf(-acc));
+    }
+    if constexpr (sizeof(T) == 2) out[(size_t)r * d + c] = __float2half_rn(v);
+    else out[(size_t)r * d + c] = v;
+  }
+}
+
+__global__ void scatter_kernel(const float* __restrict__ x, Clips clips, float* __restrict__ out, int t_max, int d) {
+  const int row = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+  if (row >= clips.B * t_max) return;
+  const int b = row / t_max, t = row - b * t_max;
+  float* o = out + (size_t)row * d;
+  if (t < clips.L2(b)) {
+    const float* xr = x + (size_t)(clips.e(b) + t) * d;
+    for (int c = lane * 4; c < d; c += 128)
+      *reinterpret_cast<float4*>(o + c) = *reinterpret_cast<const float4*>(xr + c);
+  } else {
+    for (int c = lane * 4; c < d; c += 128) *reinterpret_cast<float4*>(o + c) = make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+}
+
+__global__ void logsoftmax_argmax_kernel(const float* __restrict__ logits, int ld, const int* __restrict__ lens,
+                                         int batch, int t_max, int C, float* __restrict__ logp,
+                                         int* __restrict__ argmax) {
+  const int row = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+  if (row >= batch * t_max) return;
+  const int b = row / t_max, t = row - b * t_max;
+  if (t >= __ldg(lens + b)) {
+    if (logp)
+      for (int c = lane; c < C; c += 32) logp[(size_t)row * C + c] = 0.f;
+    if (lane == 0) argmax[row] = -1;
+    return;
+  }
+  const float* z = logits + (size_t)row * ld;
+  float best = -INFINITY;
+  int bi = 0x7fffffff;
+  for (int c = lane; c < C; c += 32) {
+    const float v = z[c];
+    if (v > best) { best = v; bi = c; }  // lane-local scan is in increasing c: keeps the first maximum
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    const float ob = __shfl_xor_sync(0xffffffffu, best, o);
+    const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+    if (ob > best || (ob == best && oi < bi)) { best = ob; bi = oi; }
+  }
+  float s = 0.f;
+  for (int c = lane; c < C; c += 32) s += expf(z[c] - best);
+  s = warp_sum(s);
+  const float lse = best + logf(s);
+  if (logp)
+    for (int c = lane; c < C; c += 32) logp[(size_t)row * C + c] = z[c] - lse;
+  if (lane == 0) argmax[row] = bi;
+}
+
+// One CTA (256 threads) per clip: keep_t = a_t != blank && (t == 0 || a_t != a_{t-1}),
+// exclusive scan of keep flags over contiguous per-thread chunks, compaction.
+__global__ void __launch_bounds__(256)
+collapse_kernel(const int* __restrict__ argmax, const int* __restrict__ lens, int t_max, int blank,
+                int* __restrict__ tokens, int* __restrict__ counts) {
+  __shared__ int warp_tot[8];
+  __shared__ int s_total;
+  const int b = blockIdx.x, tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
+  const int L = min(__ldg(lens + b), t_max);
+  const int* a = argmax + (size_t)b * t_max;
+  const int chunk = (L + 255) / 256;
+  const int t0 = tid * chunk, t1 = min(t0 + chunk, L);
+  int cnt = 0;
+  for (int t = t0; t < t1; ++t) {
+    const int v = a[t];
+    cnt += (v != blank && (t == 0 || v != a[t - 1])) ? 1 : 0;
+  }
+  // inclusive warp scan
+  int inc = cnt;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, inc, o);
+    if (lane >= o) inc += y;
+  }
+  if (lane == 31) warp_tot[w] = inc;
+  __syncthreads();
+  if (tid == 0) {
+    int run = 0;
+    for (int i = 0; i < 8; ++i) { const int v = warp_tot[i]; warp_tot[i] = run; run += v; }
+    s_total = run;
+  }
+  __syncthreads();
+  int pos = warp_tot[w] + inc - cnt;
+  int* tok = tokens + (size_t)b * t_max;
+  for (int t = t0; t < t1; ++t) {
+    const int v = a[t];
+    if (v != blank && (t == 0 || v != a[t - 1])) tok[pos++] = v;
+  }
+  const int total = s_total;
+  for (int t = total + tid; t < t_max; t += 256) tok[t] = -1;
+  if (tid == 0) counts[b] = total;
+}
+
+__global__ void f32_to_f16_kernel(const float* __restrict__ in, __half* __restrict__ out, int64_t n) {
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x)
+    out[i] = __float2half_rn(in[i]);
+}
+
+}  // namespace
+
+cudaError_t launch_layernorm(const float* x, const float* g, const float* b, float eps, void* u, int u_half, int rows,
+                             int d, cudaStream_t s) {
+  if (d % 128 || d > 1024) return cudaErrorInvalidValue;
+  const int grid = (rows + 7) / 8;
+  if (u_half) ln_kernel<__half><<<grid, 256, 0, s>>>(x, g, b, eps, (__half*)u, rows, d);
+  else ln_kernel<float><<<grid, 256, 0, s>>>(x, g, b, eps, (float*)u, rows, d);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_layernorm_chain(float* x, const float* g1, const float* b1, const float* g2, const float* b2,
+                                   float eps, void* u, int u_half, int rows, int d, cudaStream_t s) {
+  if (d % 128 || d > 1024) return cudaErrorInvalidValue;
+  const int grid = (rows + 7) / 8;
+  if (u_half) ln_chain_kernel<__half><<<grid, 256, 0, s>>>(x, g1, b1, g2, b2, eps, (__half*)u, rows, d);
+  else ln_chain_kernel<float><<<grid, 256, 0, s>>>(x, g1, b1, g2, b2, eps, (float*)u, rows, d);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_layernorm_rope(const float* x, const float* g, const float* b, float eps, const float* cos_tab,
+                                  const float* sin_tab, Clips clips, void* u, void* urot, int u_half, int rows, int d,
+                                  int d_head, cudaStream_t s) {
+  if (d % 128 || d > 1024 || d_head % 4) return cudaErrorInvalidValue;
+  const int grid = (rows + 7) / 8;
+  if (u_half)
+    ln_rope_kernel<__half><<<grid, 256, 0, s>>>(x, g, b, eps, cos_tab, sin_tab, clips, (__half*)u, (__half*)urot,
+                                                rows, d, d_head);
+  else
+    ln_rope_kernel<float><<<grid, 256, 0, s>>>(x, g, b, eps, cos_tab, sin_tab, clips, (float*)u, (float*)urot, rows,
+                                               d, d_head);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_dwconv(const void* g, const float* w, const float* bias, Clips clips, void* out, int t_half,
+                          int rows, int d, int K, cudaStream_t s) {
+  if (d % 128 || K > 63 || (K & 1) == 0) return cudaErrorInvalidValue;
+  dim3 grid((rows + 31) / 32, d / 128);
+  if (t_half) dwconv_kernel<__half><<<grid, 256, 0, s>>>((const __half*)g, w, bias, clips, (__half*)out, rows, d, K);
+  else dwconv_kernel<float><<<grid, 256, 0, s>>>((const float*)g, w, bias, clips, (float*)out, rows, d, K);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_scatter_out(const float* x, Clips clips, float* out, int t_max, int d, cudaStream_t s) {
+  const int rows = clips.B * t_max;
+  scatter_kernel<<<(rows + 7) / 8, 256, 0, s>>>(x, clips, out, t_max, d);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_logsoftmax_argmax(const float* logits, int ld, const int* lens, int batch, int t_max, int C,
+                                     float* logp, int* argmax, cudaStream_t s) {
+  const int rows = batch * t_max;
+  logsoftmax_argmax_kernel<<<(rows + 7) / 8, 256, 0, s>>>(logits, ld, lens, batch, t_max, C, logp, argmax);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_collapse(const int* argmax, const int* lens, int batch, int t_max, int blank, int* tokens,
+                            int* counts, cudaStream_t s) {
+  collapse_kernel<<<batch, 256, 0, s>>>(argmax, lens, t_max, blank, tokens, counts);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_f32_to_f16(const float* in, __half* out, int64_t n, cudaStream_t s) {
+  f32_to_f16_kernel<<<148 * 8, 256, 0, s>>>(in, out, n);
+  return cudaGetLastError();
+}
+
+}  // namespace gam

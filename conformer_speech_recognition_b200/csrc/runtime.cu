@@ -1,0 +1,960 @@
+// Host runtime behind include/gam.h: argument checks, weight validation and
+// repacking, one preallocated workspace per context, per-call length planning
+// (segment layout, see common.cuh), the launch sequence of the encoder and of
+// the CTC decoder, launch counting / CUDA-event profiling and host-side fault
+// injection.
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+#include <map>
+#include <string>
+#include <vector>
+
+#include "../../include/gam.h"
+#include "common.cuh"
+#include "gemm_tc.cuh"
+
+using namespace gam;
+
+namespace {
+
+thread_local std::string g_create_error;
+
+const char* kKindNames[PK_COUNT] = {"frontend",  "gemm_subsampling", "gemm_ffn_up",  "gemm_ffn_down",
+                                    "gemm_qkv",  "gemm_attn_out",    "gemm_pw1_glu", "gemm_pw2",
+                                    "attention", "layernorm",        "dwconv",       "ctc_gemm",
+                                    "ctc_softmax_argmax", "ctc_collapse", "misc"};
+
+inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+inline int64_t round_up(int64_t a, int64_t b) { return ceil_div(a, b) * b; }
+
+// Lengths of one clip (see gam.h).
+struct ClipLen {
+  int F, T1, T2, L1, L2;
+};
+ClipLen clip_len(int64_t n, const gam_config& c) {
+  ClipLen r{0, 0, 0, 0, 0};
+  if (n < c.win) return r;
+  r.F = (int)(1 + (n - c.win) / c.hop);
+  const int k = c.sub_kernel, p = k / 2;
+  r.T1 = (r.F + 2 * p - k) / 2 + 1;
+  r.T2 = (r.T1 + 2 * p - k) / 2 + 1;
+  r.L1 = (r.F - 1) / 2;
+  r.L2 = r.L1 >= 1 ? (r.L1 - 1) / 2 : 0;
+  return r;
+}
+// Encoder rows reserved for a clip of F frames (segment layout).
+int seg_rows(const ClipLen& l) {
+  int64_t a = ceil_div(l.F + 2, 4), b = ceil_div(l.L1 + 2, 2), c = l.L2 + 1;
+  return (int)round_up(std::max(a, std::max(b, c)), 8);
+}
+
+struct DevLinear {
+  void* w = nullptr;        // [N, K] f32 / f16 / int8
+  __half* scale = nullptr;  // int8: [N, K/64]
+  float* b = nullptr;       // [N]
+  int N = 0, K = 0, dtype = 0;
+  WeightOp op() const { return WeightOp{w, scale, dtype}; }
+};
+struct DevLN {
+  float* g = nullptr;
+  float* b = nullptr;
+};
+struct DevLayer {
+  DevLN ln_ffn1, ln_attn, ln_conv, ln_ffn2, ln_out;
+  DevLinear ffn1_up, ffn1_down, qkv, out, pw1, pw2, ffn2_up, ffn2_down;
+  float* dw_w = nullptr;  // [K][d], BatchNorm folded
+  float* dw_b = nullptr;  // [d]
+};
+
+struct Prof {
+  uint32_t mask = 0;  // families whose launches are timed
+  int64_t launches[PK_COUNT] = {};
+  double ms[PK_COUNT] = {};
+  std::vector<cudaEvent_t> ev;  // pairs
+  std::vector<int> kind;        // per recorded pair
+  size_t used = 0;
+};
+
+constexpr int kRing = 8;
+
+}  // namespace
+
+struct gam_ctx {
+  gam_config cfg{};
+  int device = 0;
+  int act_half = 0;  // activations between GEMMs in fp16 (1) or fp32 (0)
+  int wdtype = 0;    // GEMM weight dtype: 0 f32, 1 f16, 2 int8-g64
+  int d_head = 0;
+  std::string err;
+  std::vector<void*> allocs;
+  // weights
+  float* basis = nullptr;  // [320][320]
+  float* fb = nullptr;     // [161][64]
+  DevLinear conv1, conv2, head;
+  std::vector<DevLayer> layers;
+  float* rope_cos = nullptr;  // [T2_cap][d_head/2]
+  float* rope_sin = nullptr;
+  // capacity
+  int F_cap = 0, T2_cap = 0;
+  int64_t E_cap = 0, R1_cap = 0, R0_cap = 0;
+  // workspace
+  void* mel = nullptr;
+  void* c1 = nullptr;
+  float* x = nullptr;
+  void* u = nullptr;
+  void* urot = nullptr;
+  void* g = nullptr;
+  void* h = nullptr;
+  void* qk = nullptr;
+  void* vt = nullptr;
+  float* logits = nullptr;
+  int* argmax = nullptr;
+  float* audio_stage = nullptr;
+  float* enc_stage = nullptr;
+  int* tokens_stage = nullptr;
+  int* counts_stage = nullptr;
+  int* dev_status = nullptr;
+  // per-call table ring (pinned host -> device)
+  int* tab_host[kRing] = {};
+  int* tab_dev[kRing] = {};
+  cudaEvent_t tab_ev[kRing] = {};
+  int ring = 0;
+  cudaStream_t last_stream = nullptr;
+  // tcgen05 GEMM plans
+  TcGemmCache tc;
+  Prof prof;
+  int inject_err = 0, inject_count = 0;
+};
+
+namespace {
+
+gam_status fail(gam_ctx* c, gam_status s, const std::string& msg) {
+  if (c) c->err = msg;
+  else g_create_error = msg;
+  return s;
+}
+
+gam_status cuda_check(gam_ctx* c, cudaError_t e, const char* what) {
+  if (c && c->inject_count > 0) {
+    c->inject_count--;
+    e = (cudaError_t)c->inject_err;
+  }
+  if (e == cudaSuccess) return GAM_OK;
+  return fail(c, GAM_ERR_CUDA, std::string(what) + ": " + cudaGetErrorName(e) + " (" + cudaGetErrorString(e) + ")");
+}
+
+#define GAM_TRY(expr)                  \
+  do {                                 \
+    gam_status _s = (expr);            \
+    if (_s != GAM_OK) return _s;       \
+  } while (0)
+
+template <class F>
+gam_status run_kernel(gam_ctx* c, int kind, cudaStream_t s, F&& launch) {
+  Prof& p = c->prof;
+  p.launches[kind]++;
+  const bool timed = ((p.mask >> kind) & 1u) && p.used + 2 <= p.ev.size();
+  if (timed) cudaEventRecord(p.ev[p.used], s);
+  cudaError_t e = launch();
+  if (timed) {
+    cudaEventRecord(p.ev[p.used + 1], s);
+    p.kind.push_back(kind);
+    p.used += 2;
+  }
+  return cuda_check(c, e, kKindNames[kind]);
+}
+
+gam_status dev_alloc(gam_ctx* c, void** p, size_t bytes) {
+  if (bytes == 0) bytes = 16;
+  cudaError_t e = cudaMalloc(p, bytes);
+  if (e != cudaSuccess) return cuda_check(c, e, "cudaMalloc");
+  c->allocs.push_back(*p);
+  return GAM_OK;
+}
+template <class T>
+gam_status upload(gam_ctx* c, T** dst, const void* src, size_t bytes) {
+  GAM_TRY(dev_alloc(c, (void**)dst, bytes));
+  return cuda_check(c, cudaMemcpy(*dst, src, bytes, cudaMemcpyHostToDevice), "cudaMemcpy weights");
+}
+
+// ---- weight table ----
+struct WeightTable {
+  std::map<std::string, const gam_tensor*> by_name;
+};
+
+gam_status find(gam_ctx* c, const WeightTable& t, const std::string& name, std::vector<int64_t> shape,
+                const gam_tensor** out, bool allow_trailing_one = false) {
+  auto it = t.by_name.find(name);
+  if (it == t.by_name.end()) return fail(c, GAM_ERR_WEIGHTS, "missing tensor " + name);
+  const gam_tensor* g = it->second;
+  std::vector<int64_t> got(g->shape, g->shape + std::max(0, std::min(g->ndim, 4)));
+  if (allow_trailing_one && got.size() == shape.size() + 1 && got.back() == 1) got.pop_back();
+  if (got != shape || g->data == nullptr) {
+    std::string s = "tensor " + name + " has shape [";
+    for (auto v : got) s += std::to_string(v) + ",";
+    s += "], expected [";
+    for (auto v : shape) s += std::to_string(v) + ",";
+    return fail(c, GAM_ERR_WEIGHTS, s + "]");
+  }
+  *out = g;
+  return GAM_OK;
+}
+
+// Reads a float tensor (f32 or f16) into doubles.
+gam_status read_f(gam_ctx* c, const gam_tensor* g, std::vector<double>& v) {
+  int64_t n = 1;
+  for (int i = 0; i < g->ndim; ++i) n *= g->shape[i];
+  v.resize(n);
+  if (g->dtype == GAM_DTYPE_F32) {
+    const float* p = (const float*)g->data;
+    for (int64_t i = 0; i < n; ++i) v[i] = p[i];
+  } else if (g->dtype == GAM_DTYPE_F16) {
+    const __half* p = (const __half*)g->data;
+    for (int64_t i = 0; i < n; ++i) v[i] = (double)__half2float(p[i]);
+  } else {
+    return fail(c, GAM_ERR_WEIGHTS, std::string("tensor ") + g->name + " must be f32 or f16");
+  }
+  return GAM_OK;
+}
+
+gam_status get_vec(gam_ctx* c, const WeightTable& t, const std::string& name, int64_t n, std::vector<double>& v) {
+  const gam_tensor* g;
+  GAM_TRY(find(c, t, name, {n}, &g));
+  return read_f(c, g, v);
+}
+
+gam_status upload_f32(gam_ctx* c, float** dst, const std::vector<double>& v) {
+  std::vector<float> f(v.begin(), v.end());
+  return upload(c, dst, f.data(), f.size() * sizeof(float));
+}
+
+gam_status load_ln(gam_ctx* c, const WeightTable& t, const std::string& name, int d, DevLN& ln) {
+  std::vector<double> g, b;
+  GAM_TRY(get_vec(c, t, name + ".weight", d, g));
+  GAM_TRY(get_vec(c, t, name + ".bias", d, b));
+  GAM_TRY(upload_f32(c, &ln.g, g));
+  return upload_f32(c, &ln.b, b);
+}
+
+// Host copy of a linear weight in its device format, rows possibly permuted.
+struct HostLinear {
+  int N = 0, K = 0, dtype = 0;
+  std::vector<double> w;        // f32 / f16 modes: [N, K] values
+  std::vector<int8_t> q;        // int8 mode
+  std::vector<__half> s;        // int8 mode [N, K/64]
+  std::vector<double> b;
+};
+
+gam_status read_linear(gam_ctx* c, const WeightTable& t, const std::string& name, int N, int K, bool quantized,
+                       HostLinear& out) {
+  out.N = N;
+  out.K = K;
+  GAM_TRY(get_vec(c, t, name + ".bias", N, out.b));
+  if (quantized) {
+    const gam_tensor *gq, *gs;
+    GAM_TRY(find(c, t, name + ".weight_q", {N, K}, &gq, true));
+    GAM_TRY(find(c, t, name + ".weight_scale", {N, K / 64}, &gs));
+    if (gq->dtype != GAM_DTYPE_I8 || gs->dtype != GAM_DTYPE_F16)
+      return fail(c, GAM_ERR_WEIGHTS, name + ": weight_q must be int8 and weight_scale f16");
+    out.dtype = 2;
+    out.q.assign((const int8_t*)gq->data, (const int8_t*)gq->data + (size_t)N * K);
+    out.s.assign((const __half*)gs->data, (const __half*)gs->data + (size_t)N * (K / 64));
+    return GAM_OK;
+  }
+  const gam_tensor* gw;
+  GAM_TRY(find(c, t, name + ".weight", {N, K}, &gw, true));
+  out.dtype = c->wdtype == 0 ? 0 : 1;
+  return read_f(c, gw, out.w);
+}
+
+// Row permutation: new row i takes old row perm[i].
+void permute_rows(HostLinear& l, const std::vector<int>& perm) {
+  HostLinear o = l;
+  for (int i = 0; i < l.N; ++i) {
+    const int j = perm[i];
+    o.b[i] = l.b[j];
+    if (l.dtype == 2) {
+      std::memcpy(&o.q[(size_t)i * l.K], &l.q[(size_t)j * l.K], l.K);
+      std::memcpy(&o.s[(size_t)i * (l.K / 64)], &l.s[(size_t)j * (l.K / 64)], (l.K / 64) * sizeof(__half));
+    } else {
+      std::memcpy(&o.w[(size_t)i * l.K], &l.w[(size_t)j * l.K], l.K * sizeof(double));
+    }
+  }
+  l = std::move(o);
+}
+
+gam_status upload_linear(gam_ctx* c, const HostLinear& l, DevLinear& d) {
+  d.N = l.N;
+  d.K = l.K;
+  d.dtype = l.dtype;
+  GAM_TRY(upload_f32(c, &d.b, l.b));
+  if (l.dtype == 2) {
+    GAM_TRY(upload(c, (int8_t**)&d.w, l.q.data(), l.q.size()));
+    return upload(c, &d.scale, l.s.data(), l.s.size() * sizeof(__half));
+  }
+  if (l.dtype == 0) {
+    std::vector<float> f(l.w.begin(), l.w.end());
+    return upload(c, (float**)&d.w, f.data(), f.size() * sizeof(float));
+  }
+  std::vector<__half> h(l.w.size());
+  for (size_t i = 0; i < h.size(); ++i) h[i] = __float2half_rn((float)l.w[i]);
+  return upload(c, (__half**)&d.w, h.data(), h.size() * sizeof(__half));
+}
+
+// Conv1d [out, in, K] -> GEMM weight [out, K * in] (tap-major rows).
+gam_status load_conv(gam_ctx* c, const WeightTable& t, const std::string& name, int cout, int cin, int k,
+                     DevLinear& d) {
+  const gam_tensor* gw;
+  GAM_TRY(find(c, t, name + ".weight", {cout, cin, k}, &gw));
+  std::vector<double> w;
+  GAM_TRY(read_f(c, gw, w));
+  HostLinear l;
+  l.N = cout;
+  l.K = cin * k;
+  l.dtype = c->wdtype == 0 ? 0 : 1;
+  l.w.resize((size_t)cout * cin * k);
+  for (int o = 0; o < cout; ++o)
+    for (int ci = 0; ci < cin; ++ci)
+      for (int kk = 0; kk < k; ++kk)
+        l.w[((size_t)o * k + kk) * cin + ci] = w[((size_t)o * cin + ci) * k + kk];
+  GAM_TRY(get_vec(c, t, name + ".bias", cout, l.b));
+  return upload_linear(c, l, d);
+}
+
+gam_status validate_config(const gam_config* cfg) {
+  if (!cfg) return fail(nullptr, GAM_ERR_INVALID_ARG, "null config");
+  const gam_config& c = *cfg;
+  if (c.n_fft != 320 || c.win != 320 || c.hop != 160 || c.n_mels != 64)
+    return fail(nullptr, GAM_ERR_INVALID_ARG, "frontend must be n_fft = win = 320, hop = 160, n_mels = 64");
+  if (c.sub_kernel != 5) return fail(nullptr, GAM_ERR_INVALID_ARG, "sub_kernel must be 5");
+  if (c.n_layers < 1 || c.d_model <= 0 || c.d_model % 256 || c.d_model > 1024)
+    return fail(nullptr, GAM_ERR_INVALID_ARG, "d_model must be a multiple of 256, at most 1024");
+  if (c.n_heads <= 0 || c.d_model % c.n_heads ||
+      (c.d_model / c.n_heads != 48 && c.d_model / c.n_heads != 64))
+    return fail(nullptr, GAM_ERR_INVALID_ARG, "d_model / n_heads must be 48 or 64");
+  if (c.ffn_dim <= 0 || c.ffn_dim % 256) return fail(nullptr, GAM_ERR_INVALID_ARG, "ffn_dim must be a multiple of 256");
+  if (c.conv_kernel < 1 || c.conv_kernel > 63 || c.conv_kernel % 2 == 0)
+    return fail(nullptr, GAM_ERR_INVALID_ARG, "conv_kernel must be odd and <= 63");
+  if (c.n_classes < 2 || c.n_classes > 1024) return fail(nullptr, GAM_ERR_INVALID_ARG, "n_classes must be 2..1024");
+  if (c.precision < GAM_FP32 || c.precision > GAM_INT8_G64) return fail(nullptr, GAM_ERR_INVALID_ARG, "bad precision");
+  if (!(c.rope_base > 0) || !(c.ln_eps > 0) || !(c.bn_eps > 0))
+    return fail(nullptr, GAM_ERR_INVALID_ARG, "rope_base / eps must be positive");
+  if (c.max_batch < 1 || c.max_batch > 4096) return fail(nullptr, GAM_ERR_INVALID_ARG, "max_batch must be 1..4096");
+  if (c.max_samples < 1280 || c.max_samples > (int64_t)16000 * 3600)
+    return fail(nullptr, GAM_ERR_INVALID_ARG, "max_samples must be 1280 .. 1 hour");
+  return GAM_OK;
+}
+
+// Per-call plan.
+struct Plan {
+  int B = 0;
+  std::vector<ClipLen> len;
+  std::vector<int> e;  // B + 1
+  int E = 0, E_pad = 0, R1 = 0, R0 = 0, F_max = 0, T2_max = 0;
+};
+
+gam_status make_plan(gam_ctx* c, const gam_config& cfg, const int32_t* lengths, int batch, int64_t max_samples,
+                     Plan& p) {
+  if (!lengths || batch < 1) return fail(c, GAM_ERR_INVALID_ARG, "lengths must be non-null and batch >= 1");
+  p.B = batch;
+  p.len.resize(batch);
+  p.e.assign(batch + 1, 0);
+  for (int i = 0; i < batch; ++i) {
+    if (lengths[i] < 1280)
+      return fail(c, GAM_ERR_SHAPE, "clip " + std::to_string(i) + " has " + std::to_string(lengths[i]) +
+                                        " samples; at least 1280 are needed for one encoder frame");
+    if (max_samples > 0 && lengths[i] > max_samples)
+      return fail(c, GAM_ERR_SHAPE, "clip " + std::to_string(i) + " is longer than max_samples");
+    p.len[i] = clip_len(lengths[i], cfg);
+    p.e[i + 1] = p.e[i] + seg_rows(p.len[i]);
+    p.F_max = std::max(p.F_max, p.len[i].F);
+    p.T2_max = std::max(p.T2_max, p.len[i].T2);
+  }
+  p.E = p.e[batch];
+  p.E_pad = (int)round_up(p.E, 128);
+  p.R1 = (int)round_up(2 * (int64_t)p.E_pad + 4, 128);
+  p.R0 = 2 * p.R1 + 4;
+  return GAM_OK;
+}
+
+// Upload the clip table (and optional extra ints) through the pinned ring.
+gam_status upload_table(gam_ctx* c, const Plan& p, cudaStream_t s, Clips* out) {
+  const int slot = c->ring;
+  c->ring = (c->ring + 1) % kRing;
+  GAM_TRY(cuda_check(c, cudaEventSynchronize(c->tab_ev[slot]), "ring event"));
+  int* h = c->tab_host[slot];
+  const int B = p.B;
+  for (int i = 0; i <= B; ++i) h[i] = p.e[i];
+  for (int i = 0; i < B; ++i) {
+    h[(B + 1) + i] = p.len[i].F;
+    h[2 * (B + 1) + i] = p.len[i].L1;
+    h[3 * (B + 1) + i] = p.len[i].L2;
+    h[4 * (B + 1) + i] = 0;
+  }
+  const size_t bytes = 5 * (size_t)(B + 1) * sizeof(int);
+  GAM_TRY(cuda_check(c, cudaMemcpyAsync(c->tab_dev[slot], h, bytes, cudaMemcpyHostToDevice, s), "table upload"));
+  GAM_TRY(cuda_check(c, cudaEventRecord(c->tab_ev[slot], s), "ring event record"));
+  *out = Clips{c->tab_dev[slot], B};
+  return GAM_OK;
+}
+
+gam_status upload_ints(gam_ctx* c, const int32_t* src, int n, cudaStream_t s, const int** out) {
+  const int slot = c->ring;
+  c->ring = (c->ring + 1) % kRing;
+  GAM_TRY(cuda_check(c, cudaEventSynchronize(c->tab_ev[slot]), "ring event"));
+  std::memcpy(c->tab_host[slot], src, n * sizeof(int));
+  GAM_TRY(cuda_check(c, cudaMemcpyAsync(c->tab_dev[slot], c->tab_host[slot], n * sizeof(int), cudaMemcpyHostToDevice, s),
+                     "lengths upload"));
+  GAM_TRY(cuda_check(c, cudaEventRecord(c->tab_ev[slot], s), "ring event record"));
+  *out = c->tab_dev[slot];
+  return GAM_OK;
+}
+
+// ---- GEMM dispatch: tensor cores for fp16 / int8, CUDA cores for fp32 ----
+gam_status gemm(gam_ctx* c, int kind, cudaStream_t s, const void* A, const void* A2, int n_split, int lda,
+                const DevLinear& W, int M, int epi, float alpha, void* out, int ldo, const Clips& clips,
+                int a_f32 = 0) {
+  EpiParams ep{};
+  ep.out = out;
+  ep.x = (float*)out;
+  ep.bias = W.b;
+  ep.alpha = alpha;
+  ep.ldo = ldo;
+  ep.clips = clips;
+  ep.qk = c->qk;
+  ep.vt = c->vt;
+  ep.rows_pad = (int)c->E_cap;
+  ep.n_heads = c->cfg.n_heads;
+  ep.d_head = c->d_head;
+  ep.d_model = c->cfg.d_model;
+  const int a_dtype = a_f32 ? 0 : (c->act_half ? 1 : 0);
+  if (tc_supported(a_dtype, W.dtype, W.N, W.K, epi)) {
+    return run_kernel(c, kind, s, [&] {
+      return launch_gemm_tc(&c->tc, A, A2, n_split, lda, W.op(), M, W.N, W.K, epi, ep, s);
+    });
+  }
+  return run_kernel(c, kind, s, [&] {
+    return launch_gemm_simt(a_dtype, A, A2, n_split, lda, W.op(), M, W.N, W.K, epi, c->act_half, ep, s);
+  });
+}
+
+// The encoder up to (layer, stage); stage < 0 runs everything.  Leaves the
+// residual stream in c->x and scatters it to out.
+gam_status run_encoder(gam_ctx* c, const float* audio, const int32_t* lengths, int batch, int64_t max_samples,
+                       int stop_layer, int stop_stage, float* out, int32_t* enc_len_out, cudaStream_t s) {
+  const gam_config& cfg = c->cfg;
+  Plan p;
+  GAM_TRY(make_plan(c, cfg, lengths, batch, max_samples, p));
+  if (batch > cfg.max_batch) return fail(c, GAM_ERR_CAPACITY, "batch above max_batch");
+  if (max_samples > cfg.max_samples) return fail(c, GAM_ERR_CAPACITY, "max_samples above the context's capacity");
+  if (p.E_pad > c->E_cap || p.R1 > c->R1_cap || p.R0 > c->R0_cap || p.T2_max > c->T2_cap)
+    return fail(c, GAM_ERR_CAPACITY, "workspace too small for this batch");
+  if (!audio || !out) return fail(c, GAM_ERR_INVALID_ARG, "null audio or output pointer");
+  c->last_stream = s;
+  Clips clips;
+  GAM_TRY(upload_table(c, p, s, &clips));
+  const int d = cfg.d_model, f = cfg.ffn_dim, H = cfg.n_heads, dh = c->d_head;
+  const int ah = c->act_half;
+  const float eps = cfg.ln_eps;
+  const int M = p.E_pad;
+
+  GAM_TRY(run_kernel(c, PK_FRONTEND, s, [&] {
+    return launch_frontend(audio, max_samples, clips, p.R0, 1, 0, c->basis, c->fb, c->mel, ah, s);
+  }));
+  GAM_TRY(gemm(c, PK_GEMM_SUB, s, c->mel, nullptr, 0, 2 * cfg.n_mels, c->conv1, p.R1, EPI_CONV1, 1.f, c->c1, d,
+               clips));
+  GAM_TRY(gemm(c, PK_GEMM_SUB, s, c->c1, nullptr, 0, 2 * d, c->conv2, M, EPI_CONV2, 1.f, c->x, d, clips));
+
+  const int L = cfg.n_layers;
+  bool stopped = stop_stage == GAM_STAGE_SUBSAMPLING;
+  for (int l = 0; l < L && !stopped; ++l) {
+    DevLayer& w = c->layers[l];
+    if (l == 0)
+      GAM_TRY(run_kernel(c, PK_LAYERNORM, s, [&] {
+        return launch_layernorm(c->x, w.ln_ffn1.g, w.ln_ffn1.b, eps, c->u, ah, M, d, s);
+      }));
+    // FFN1 (half-step residual)
+    GAM_TRY(gemm(c, PK_GEMM_FFN_UP, s, c->u, nullptr, 0, d, w.ffn1_up, M, EPI_SWISH, 1.f, c->h, f, clips));
+    GAM_TRY(gemm(c, PK_GEMM_FFN_DOWN, s, c->h, nullptr, 0, f, w.ffn1_down, M, EPI_RESID, 0.5f, c->x, d, clips));
+    if (l == stop_layer && stop_stage == GAM_STAGE_FFN1) { stopped = true; break; }
+    // rotary MHSA
+    GAM_TRY(run_kernel(c, PK_LAYERNORM, s, [&] {
+      return launch_layernorm_rope(c->x, w.ln_attn.g, w.ln_attn.b, eps, c->rope_cos, c->rope_sin, clips, c->u,
+                                   c->urot, ah, M, d, dh, s);
+    }));
+    GAM_TRY(gemm(c, PK_GEMM_QKV, s, c->urot, c->u, 2 * d, d, w.qkv, M, EPI_QKV, 1.f, nullptr, 0, clips));
+    GAM_TRY(run_kernel(c, PK_ATTENTION, s, [&] {
+      return launch_attention(&c->tc, c->qk, c->vt, clips, c->urot, ah, (int)c->E_cap, H, dh, p.T2_max, s);
+    }));
+    GAM_TRY(gemm(c, PK_GEMM_OUT, s, c->urot, nullptr, 0, d, w.out, M, EPI_RESID, 1.f, c->x, d, clips));
+    if (l == stop_layer && stop_stage == GAM_STAGE_MHSA) { stopped = true; break; }
+    // convolution module
+    GAM_TRY(run_kernel(c, PK_LAYERNORM, s, [&] {
+      return launch_layernorm(c->x, w.ln_conv.g, w.ln_conv.b, eps, c->u, ah, M, d, s);
+    }));
+    GAM_TRY(gemm(c, PK_GEMM_PW1, s, c->u, nullptr, 0, d, w.pw1, M, EPI_GLU, 1.f, c->g, d, clips));
+    GAM_TRY(run_kernel(c, PK_DWCONV, s, [&] {
+      return launch_dwconv(c->g, w.dw_w, w.dw_b, clips, c->u, ah, M, d, cfg.conv_kernel, s);
+    }));
+    GAM_TRY(gemm(c, PK_GEMM_PW2, s, c->u, nullptr, 0, d, w.pw2, M, EPI_RESID, 1.f, c->x, d, clips));
+    if (l == stop_layer && stop_stage == GAM_STAGE_CONV) { stopped = true; break; }
+    // FFN2
+    GAM_TRY(run_kernel(c, PK_LAYERNORM, s, [&] {
+      return launch_layernorm(c->x, w.ln_ffn2.g, w.ln_ffn2.b, eps, c->u, ah, M, d, s);
+    }));
+    GAM_TRY(gemm(c, PK_GEMM_FFN_UP, s, c->u, nullptr, 0, d, w.ffn2_up, M, EPI_SWISH, 1.f, c->h, f, clips));
+    GAM_TRY(gemm(c, PK_GEMM_FFN_DOWN, s, c->h, nullptr, 0, f, w.ffn2_down, M, EPI_RESID, 0.5f, c->x, d, clips));
+    if (l == stop_layer && stop_stage == GAM_STAGE_FFN2) { stopped = true; break; }
+    // block-final LayerNorm, chained with the next block's first one
+    const bool last = (l == L - 1) || (l == stop_layer && stop_stage == GAM_STAGE_LAYER);
+    if (!last) {
+      DevLayer& nx = c->layers[l + 1];
+      GAM_TRY(run_kernel(c, PK_LAYERNORM, s, [&] {
+        return launch_layernorm_chain(c->x, w.ln_out.g, w.ln_out.b, nx.ln_ffn1.g, nx.ln_ffn1.b, eps, c->u, ah, M, d,
+                                      s);
+      }));
+    } else {
+      GAM_TRY(run_kernel(c, PK_LAYERNORM, s, [&] {
+        return launch_layernorm(c->x, w.ln_out.g, w.ln_out.b, eps, c->x, 0, M, d, s);
+      }));
+      stopped = (l == stop_layer);
+    }
+  }
+  GAM_TRY(run_kernel(c, PK_MISC, s, [&] { return launch_scatter_out(c->x, clips, out, p.T2_max, d, s); }));
+  if (enc_len_out)
+    for (int i = 0; i < batch; ++i) enc_len_out[i] = p.len[i].L2;
+  return GAM_OK;
+}
+
+gam_status run_ctc(gam_ctx* c, const float* enc, const int32_t* enc_len, int batch, int t_max, float* logp,
+                   int32_t* tokens, int32_t* counts, cudaStream_t s) {
+  const gam_config& cfg = c->cfg;
+  if (!enc || !enc_len || !tokens || !counts) return fail(c, GAM_ERR_INVALID_ARG, "null pointer");
+  if (batch < 1 || t_max < 1) return fail(c, GAM_ERR_INVALID_ARG, "batch and t_max must be >= 1");
+  if (batch > cfg.max_batch || t_max > c->T2_cap) return fail(c, GAM_ERR_CAPACITY, "batch or t_max above capacity");
+  for (int i = 0; i < batch; ++i)
+    if (enc_len[i] < 0 || enc_len[i] > t_max) return fail(c, GAM_ERR_SHAPE, "enc_len outside [0, t_max]");
+  c->last_stream = s;
+  const int* lens;
+  GAM_TRY(upload_ints(c, enc_len, batch, s, &lens));
+  const int C = cfg.n_classes, M = batch * t_max;
+  Clips none{nullptr, 0};
+  GAM_TRY(gemm(c, PK_CTC_GEMM, s, enc, nullptr, 0, cfg.d_model, c->head, M, EPI_F32, 1.f, c->logits, C, none, 1));
+  GAM_TRY(run_kernel(c, PK_CTC_SOFTMAX, s, [&] {
+    return launch_logsoftmax_argmax(c->logits, C, lens, batch, t_max, C, logp, c->argmax, s);
+  }));
+  return run_kernel(c, PK_CTC_COLLAPSE, s, [&] {
+    return launch_collapse(c->argmax, lens, batch, t_max, C - 1, tokens, counts, s);
+  });
+}
+
+gam_status build_weights(gam_ctx* c, const gam_tensor* tensors, int n) {
+  const gam_config& cfg = c->cfg;
+  WeightTable t;
+  for (int i = 0; i < n; ++i) {
+    if (!tensors[i].name) return fail(c, GAM_ERR_WEIGHTS, "tensor without a name");
+    t.by_name[tensors[i].name] = &tensors[i];
+  }
+  const int d = cfg.d_model, f = cfg.ffn_dim, K = cfg.conv_kernel;
+  const bool q8 = cfg.precision == GAM_INT8_G64;
+  // frontend: window folded into the DFT basis
+  {
+    std::vector<double> win, fbv;
+    GAM_TRY(get_vec(c, t, "frontend.window", cfg.win, win));
+    const gam_tensor* g;
+    GAM_TRY(find(c, t, "frontend.mel_fb", {cfg.n_fft / 2 + 1, cfg.n_mels}, &g));
+    GAM_TRY(read_f(c, g, fbv));
+    const int N = cfg.n_fft;
+    std::vector<double> basis((size_t)N * N, 0.0);
+    const double two_pi = 6.283185307179586476925286766559;
+    for (int nn = 0; nn < N; ++nn)
+      for (int k = 0; k <= N / 2; ++k) {
+        const double a = two_pi * (double)((int64_t)k * nn % N) / N;
+        basis[(size_t)nn * N + k] = win[nn] * std::cos(a);
+        if (k >= 1 && k < N / 2) basis[(size_t)nn * N + N / 2 + k] = win[nn] * std::sin(a);
+      }
+    GAM_TRY(upload_f32(c, &c->basis, basis));
+    GAM_TRY(upload_f32(c, &c->fb, fbv));
+  }
+  GAM_TRY(load_conv(c, t, "subsampling.conv1", d, cfg.n_mels, cfg.sub_kernel, c->conv1));
+  GAM_TRY(load_conv(c, t, "subsampling.conv2", d, d, cfg.sub_kernel, c->conv2));
+  c->layers.resize(cfg.n_layers);
+  for (int l = 0; l < cfg.n_layers; ++l) {
+    const std::string p = "layers." + std::to_string(l) + ".";
+    DevLayer& w = c->layers[l];
+    GAM_TRY(load_ln(c, t, p + "ffn1.norm", d, w.ln_ffn1));
+    GAM_TRY(load_ln(c, t, p + "attn.norm", d, w.ln_attn));
+    GAM_TRY(load_ln(c, t, p + "conv.norm", d, w.ln_conv));
+    GAM_TRY(load_ln(c, t, p + "ffn2.norm", d, w.ln_ffn2));
+    GAM_TRY(load_ln(c, t, p + "norm_out", d, w.ln_out));
+    HostLinear hl;
+    GAM_TRY(read_linear(c, t, p + "ffn1.linear1", f, d, q8, hl));
+    GAM_TRY(upload_linear(c, hl, w.ffn1_up));
+    GAM_TRY(read_linear(c, t, p + "ffn1.linear2", d, f, q8, hl));
+    GAM_TRY(upload_linear(c, hl, w.ffn1_down));
+    GAM_TRY(read_linear(c, t, p + "ffn2.linear1", f, d, q8, hl));
+    GAM_TRY(upload_linear(c, hl, w.ffn2_up));
+    GAM_TRY(read_linear(c, t, p + "ffn2.linear2", d, f, q8, hl));
+    GAM_TRY(upload_linear(c, hl, w.ffn2_down));
+    // Q, K, V concatenated along the output dim
+    {
+      HostLinear q, k, v;
+      GAM_TRY(read_linear(c, t, p + "attn.linear_q", d, d, q8, q));
+      GAM_TRY(read_linear(c, t, p + "attn.linear_k", d, d, q8, k));
+      GAM_TRY(read_linear(c, t, p + "attn.linear_v", d, d, q8, v));
+      HostLinear all = q;
+      all.N = 3 * d;
+      all.b.insert(all.b.end(), k.b.begin(), k.b.end());
+      all.b.insert(all.b.end(), v.b.begin(), v.b.end());
+      if (q8) {
+        all.q.insert(all.q.end(), k.q.begin(), k.q.end());
+        all.q.insert(all.q.end(), v.q.begin(), v.q.end());
+        all.s.insert(all.s.end(), k.s.begin(), k.s.end());
+        all.s.insert(all.s.end(), v.s.begin(), v.s.end());
+      } else {
+        all.w.insert(all.w.end(), k.w.begin(), k.w.end());
+        all.w.insert(all.w.end(), v.w.begin(), v.w.end());
+      }
+      GAM_TRY(upload_linear(c, all, w.qkv));
+    }
+    GAM_TRY(read_linear(c, t, p + "attn.linear_out", d, d, q8, hl));
+    GAM_TRY(upload_linear(c, hl, w.out));
+    // pointwise1: interleave value / gate rows in blocks of 64 for the GLU epilogue
+    GAM_TRY(read_linear(c, t, p + "conv.pointwise1", 2 * d, d, q8, hl));
+    {
+      std::vector<int> perm(2 * d);
+      for (int i = 0; i < 2 * d; ++i) {
+        const int blk = i / 128, within = i % 128;
+        perm[i] = within < 64 ? blk * 64 + within : d + blk * 64 + (within - 64);
+      }
+      permute_rows(hl, perm);
+    }
+    GAM_TRY(upload_linear(c, hl, w.pw1));
+    GAM_TRY(read_linear(c, t, p + "conv.pointwise2", d, d, q8, hl));
+    GAM_TRY(upload_linear(c, hl, w.pw2));
+    // depthwise + BatchNorm folded: y = s * (sum w x + b - mean) + beta, s = gamma / sqrt(var + eps)
+    {
+      const gam_tensor* gw;
+      GAM_TRY(find(c, t, p + "conv.depthwise.weight", {d, 1, K}, &gw));
+      std::vector<double> dw, db, gm, bt, mu, var;
+      GAM_TRY(read_f(c, gw, dw));
+      GAM_TRY(get_vec(c, t, p + "conv.depthwise.bias", d, db));
+      GAM_TRY(get_vec(c, t, p + "conv.bn.weight", d, gm));
+      GAM_TRY(get_vec(c, t, p + "conv.bn.bias", d, bt));
+      GAM_TRY(get_vec(c, t, p + "conv.bn.running_mean", d, mu));
+      GAM_TRY(get_vec(c, t, p + "conv.bn.running_var", d, var));
+      std::vector<double> wf((size_t)K * d), bf(d);
+      for (int ch = 0; ch < d; ++ch) {
+        const double sc = gm[ch] / std::sqrt(var[ch] + (double)cfg.bn_eps);
+        for (int k = 0; k < K; ++k) wf[(size_t)k * d + ch] = dw[(size_t)ch * K + k] * sc;
+        bf[ch] = (db[ch] - mu[ch]) * sc + bt[ch];
+      }
+      GAM_TRY(upload_f32(c, &w.dw_w, wf));
+      GAM_TRY(upload_f32(c, &w.dw_b, bf));
+    }
+  }
+  {
+    HostLinear hl;
+    GAM_TRY(read_linear(c, t, "head", cfg.n_classes, d, q8, hl));
+    GAM_TRY(upload_linear(c, hl, c->head));
+  }
+  // RoPE tables, base rope_base, positions 0 .. T2_cap - 1
+  {
+    const int half = c->d_head / 2;
+    std::vector<double> cs((size_t)c->T2_cap * half), sn((size_t)c->T2_cap * half);
+    for (int tt = 0; tt < c->T2_cap; ++tt)
+      for (int i = 0; i < half; ++i) {
+        const double inv = std::pow((double)cfg.rope_base, -2.0 * i / c->d_head);
+        cs[(size_t)tt * half + i] = std::cos(tt * inv);
+        sn[(size_t)tt * half + i] = std::sin(tt * inv);
+      }
+    GAM_TRY(upload_f32(c, &c->rope_cos, cs));
+    GAM_TRY(upload_f32(c, &c->rope_sin, sn));
+  }
+  return GAM_OK;
+}
+
+gam_status alloc_workspace(gam_ctx* c) {
+  const gam_config& cfg = c->cfg;
+  ClipLen lmax = clip_len(cfg.max_samples, cfg);
+  c->F_cap = lmax.F;
+  c->T2_cap = lmax.T2;
+  c->E_cap = round_up((int64_t)cfg.max_batch * seg_rows(lmax), 128);
+  c->R1_cap = round_up(2 * c->E_cap + 4, 128);
+  c->R0_cap = 2 * c->R1_cap + 4;
+  const size_t es = c->act_half ? 2 : 4;
+  const int d = cfg.d_model, f = cfg.ffn_dim, H = cfg.n_heads;
+  const int64_t E = c->E_cap;
+  GAM_TRY(dev_alloc(c, &c->mel, (size_t)c->R0_cap * cfg.n_mels * es));
+  GAM_TRY(dev_alloc(c, &c->c1, (size_t)c->R1_cap * d * es));
+  GAM_TRY(dev_alloc(c, (void**)&c->x, (size_t)E * d * 4));
+  GAM_TRY(dev_alloc(c, &c->u, (size_t)E * d * es));
+  GAM_TRY(dev_alloc(c, &c->urot, (size_t)E * d * es));
+  GAM_TRY(dev_alloc(c, &c->g, (size_t)E * d * es));
+  GAM_TRY(dev_alloc(c, &c->h, (size_t)E * f * es));
+  GAM_TRY(dev_alloc(c, &c->qk, (size_t)2 * H * E * 64 * es));
+  GAM_TRY(dev_alloc(c, &c->vt, (size_t)H * 64 * E * es));
+  const int64_t ctc_rows = (int64_t)cfg.max_batch * c->T2_cap;
+  GAM_TRY(dev_alloc(c, (void**)&c->logits, (size_t)ctc_rows * cfg.n_classes * 4));
+  GAM_TRY(dev_alloc(c, (void**)&c->argmax, (size_t)ctc_rows * 4));
+  GAM_TRY(dev_alloc(c, (void**)&c->audio_stage, (size_t)cfg.max_batch * cfg.max_samples * 4));
+  GAM_TRY(dev_alloc(c, (void**)&c->enc_stage, (size_t)ctc_rows * d * 4));
+  GAM_TRY(dev_alloc(c, (void**)&c->tokens_stage, (size_t)ctc_rows * 4));
+  GAM_TRY(dev_alloc(c, (void**)&c->counts_stage, (size_t)cfg.max_batch * 4));
+  GAM_TRY(dev_alloc(c, (void**)&c->dev_status, 16));
+  // zero once: the padded head-dim columns and every buffer read before written
+  GAM_TRY(cuda_check(c, cudaMemset(c->qk, 0, (size_t)2 * H * E * 64 * es), "memset"));
+  GAM_TRY(cuda_check(c, cudaMemset(c->vt, 0, (size_t)H * 64 * E * es), "memset"));
+  GAM_TRY(cuda_check(c, cudaMemset(c->dev_status, 0, 16), "memset"));
+  const size_t tab_ints = 5 * (size_t)(cfg.max_batch + 1) + 16;
+  for (int i = 0; i < kRing; ++i) {
+    GAM_TRY(cuda_check(c, cudaMallocHost((void**)&c->tab_host[i], tab_ints * 4), "cudaMallocHost"));
+    GAM_TRY(dev_alloc(c, (void**)&c->tab_dev[i], tab_ints * 4));
+    GAM_TRY(cuda_check(c, cudaEventCreateWithFlags(&c->tab_ev[i], cudaEventDisableTiming), "event"));
+  }
+  c->prof.ev.resize(2 * 16384);
+  for (auto& e : c->prof.ev) GAM_TRY(cuda_check(c, cudaEventCreate(&e), "event"));
+  return GAM_OK;
+}
+
+void destroy(gam_ctx* c) {
+  if (!c) return;
+  cudaSetDevice(c->device);
+  cudaDeviceSynchronize();
+  tc_release(&c->tc);
+  for (void* p : c->allocs) cudaFree(p);
+  for (int i = 0; i < kRing; ++i) {
+    if (c->tab_host[i]) cudaFreeHost(c->tab_host[i]);
+    if (c->tab_ev[i]) cudaEventDestroy(c->tab_ev[i]);
+  }
+  for (auto& e : c->prof.ev)
+    if (e) cudaEventDestroy(e);
+  delete c;
+}
+
+gam_status enter(gam_ctx* c) {
+  if (!c) return GAM_ERR_INVALID_ARG;
+  c->err.clear();
+  return cuda_check(c, cudaSetDevice(c->device), "cudaSetDevice");
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* gam_status_string(gam_status s) {
+  switch (s) {
+    case GAM_OK: return "GAM_OK";
+    case GAM_ERR_INVALID_ARG: return "GAM_ERR_INVALID_ARG";
+    case GAM_ERR_SHAPE: return "GAM_ERR_SHAPE";
+    case GAM_ERR_CAPACITY: return "GAM_ERR_CAPACITY";
+    case GAM_ERR_WEIGHTS: return "GAM_ERR_WEIGHTS";
+    case GAM_ERR_UNSUPPORTED_DEVICE: return "GAM_ERR_UNSUPPORTED_DEVICE";
+    case GAM_ERR_CUDA: return "GAM_ERR_CUDA";
+    case GAM_ERR_DEVICE_TIMEOUT: return "GAM_ERR_DEVICE_TIMEOUT";
+  }
+  return "GAM_ERR_UNKNOWN";
+}
+
+const char* gam_last_error(const gam_ctx* ctx) { return ctx ? ctx->err.c_str() : g_create_error.c_str(); }
+
+gam_status gam_plan_lengths(const gam_config* cfg, const int32_t* lengths, int batch, int32_t* frames_out,
+                            int32_t* enc_len_out, int32_t* dims_out) {
+  g_create_error.clear();
+  GAM_TRY(validate_config(cfg));
+  Plan p;
+  GAM_TRY(make_plan(nullptr, *cfg, lengths, batch, 0, p));
+  for (int i = 0; i < batch; ++i) {
+    if (frames_out) frames_out[i] = p.len[i].F;
+    if (enc_len_out) enc_len_out[i] = p.len[i].L2;
+  }
+  if (dims_out) {
+    dims_out[0] = p.F_max;
+    dims_out[1] = p.T2_max;
+  }
+  return GAM_OK;
+}
+
+gam_status gam_create(const gam_config* cfg, const gam_tensor* tensors, int n_tensors, int device, gam_ctx** out) {
+  g_create_error.clear();
+  if (!out) return fail(nullptr, GAM_ERR_INVALID_ARG, "null output pointer");
+  *out = nullptr;
+  GAM_TRY(validate_config(cfg));
+  if (!tensors || n_tensors <= 0) return fail(nullptr, GAM_ERR_INVALID_ARG, "no weight tensors");
+  int ndev = 0;
+  cudaError_t e = cudaGetDeviceCount(&ndev);
+  if (e != cudaSuccess || device < 0 || device >= ndev)
+    return fail(nullptr, GAM_ERR_UNSUPPORTED_DEVICE, std::string("no CUDA device ") + std::to_string(device) + ": " +
+                                                          cudaGetErrorString(e));
+  cudaDeviceProp prop;
+  if (cudaGetDeviceProperties(&prop, device) != cudaSuccess || prop.major != 10 || prop.minor != 0)
+    return fail(nullptr, GAM_ERR_UNSUPPORTED_DEVICE, "device is not compute capability 10.0 (B200 / sm_100a)");
+  gam_ctx* c = new gam_ctx();
+  c->cfg = *cfg;
+  c->device = device;
+  c->act_half = cfg->precision == GAM_FP32 ? 0 : 1;
+  c->wdtype = cfg->precision == GAM_FP32 ? 0 : (cfg->precision == GAM_FP16 ? 1 : 2);
+  c->d_head = cfg->d_model / cfg->n_heads;
+  gam_status s = cuda_check(c, cudaSetDevice(device), "cudaSetDevice");
+  if (s == GAM_OK) s = alloc_workspace(c);
+  if (s == GAM_OK) s = build_weights(c, tensors, n_tensors);
+  if (s == GAM_OK) s = cuda_check(c, cudaDeviceSynchronize(), "create sync");
+  if (s != GAM_OK) {
+    g_create_error = c->err;
+    destroy(c);
+    return s;
+  }
+  *out = c;
+  return GAM_OK;
+}
+
+gam_status gam_destroy(gam_ctx* ctx) {
+  destroy(ctx);
+  return GAM_OK;
+}
+
+gam_status gam_logmel(gam_ctx* c, const float* audio, const int32_t* lengths, int batch, int64_t max_samples,
+                      float* mel, int32_t* frames_out, void* stream) {
+  GAM_TRY(enter(c));
+  if (!audio || !mel) return fail(c, GAM_ERR_INVALID_ARG, "null pointer");
+  if (batch > c->cfg.max_batch) return fail(c, GAM_ERR_CAPACITY, "batch above max_batch");
+  Plan p;
+  GAM_TRY(make_plan(c, c->cfg, lengths, batch, max_samples, p));
+  cudaStream_t s = (cudaStream_t)stream;
+  c->last_stream = s;
+  Clips clips;
+  GAM_TRY(upload_table(c, p, s, &clips));
+  GAM_TRY(run_kernel(c, PK_FRONTEND, s, [&] {
+    return launch_frontend(audio, max_samples, clips, batch * p.F_max, 0, p.F_max, c->basis, c->fb, mel, 0, s);
+  }));
+  if (frames_out)
+    for (int i = 0; i < batch; ++i) frames_out[i] = p.len[i].F;
+  return GAM_OK;
+}
+
+gam_status gam_encode(gam_ctx* c, const float* audio, const int32_t* lengths, int batch, int64_t max_samples,
+                      float* enc, int32_t* enc_len_out, void* stream) {
+  GAM_TRY(enter(c));
+  return run_encoder(c, audio, lengths, batch, max_samples, -1, -1, enc, enc_len_out, (cudaStream_t)stream);
+}
+
+gam_status gam_encode_stage(gam_ctx* c, const float* audio, const int32_t* lengths, int batch, int64_t max_samples,
+                            int layer, int stage, float* out, void* stream) {
+  GAM_TRY(enter(c));
+  if (stage < GAM_STAGE_SUBSAMPLING || stage > GAM_STAGE_LAYER) return fail(c, GAM_ERR_INVALID_ARG, "bad stage");
+  if (stage != GAM_STAGE_SUBSAMPLING && (layer < 0 || layer >= c->cfg.n_layers))
+    return fail(c, GAM_ERR_INVALID_ARG, "layer out of range");
+  return run_encoder(c, audio, lengths, batch, max_samples, layer, stage, out, nullptr, (cudaStream_t)stream);
+}
+
+gam_status gam_ctc_greedy(gam_ctx* c, const float* enc, const int32_t* enc_len, int batch, int t_max, float* logp,
+                          int32_t* tokens, int32_t* counts, void* stream) {
+  GAM_TRY(enter(c));
+  return run_ctc(c, enc, enc_len, batch, t_max, logp, tokens, counts, (cudaStream_t)stream);
+}
+
+gam_status gam_ctc_collapse(gam_ctx* c, const float* logits, const int32_t* lengths, int batch, int t_max,
+                            int n_classes, int32_t* tokens, int32_t* counts, void* stream) {
+  GAM_TRY(enter(c));
+  if (!logits || !lengths || !tokens || !counts) return fail(c, GAM_ERR_INVALID_ARG, "null pointer");
+  if (batch < 1 || t_max < 1 || n_classes < 2) return fail(c, GAM_ERR_INVALID_ARG, "bad sizes");
+  if ((int64_t)batch * t_max > (int64_t)c->cfg.max_batch * c->T2_cap)
+    return fail(c, GAM_ERR_CAPACITY, "batch * t_max above the context's capacity");
+  for (int i = 0; i < batch; ++i)
+    if (lengths[i] < 0 || lengths[i] > t_max) return fail(c, GAM_ERR_SHAPE, "length outside [0, t_max]");
+  cudaStream_t s = (cudaStream_t)stream;
+  c->last_stream = s;
+  const int* lens;
+  GAM_TRY(upload_ints(c, lengths, batch, s, &lens));
+  GAM_TRY(run_kernel(c, PK_CTC_SOFTMAX, s, [&] {
+    return launch_logsoftmax_argmax(logits, n_classes, lens, batch, t_max, n_classes, nullptr, c->argmax, s);
+  }));
+  return run_kernel(c, PK_CTC_COLLAPSE, s, [&] {
+    return launch_collapse(c->argmax, lens, batch, t_max, n_classes - 1, tokens, counts, s);
+  });
+}
+
+gam_status gam_transcribe(gam_ctx* c, const float* audio_host, const int32_t* lengths, int batch, int64_t max_samples,
+                          int32_t* tokens_host, int32_t* counts_host, void* stream) {
+  GAM_TRY(enter(c));
+  if (!audio_host || !tokens_host || !counts_host) return fail(c, GAM_ERR_INVALID_ARG, "null pointer");
+  if (batch > c->cfg.max_batch || max_samples > c->cfg.max_samples)
+    return fail(c, GAM_ERR_CAPACITY, "batch or max_samples above capacity");
+  Plan p;
+  GAM_TRY(make_plan(c, c->cfg, lengths, batch, max_samples, p));
+  cudaStream_t s = (cudaStream_t)stream;
+  GAM_TRY(cuda_check(c, cudaMemcpyAsync(c->audio_stage, audio_host, (size_t)batch * max_samples * 4,
+                                        cudaMemcpyHostToDevice, s), "audio upload"));
+  std::vector<int32_t> enc_len(batch);
+  GAM_TRY(run_encoder(c, c->audio_stage, lengths, batch, max_samples, -1, -1, c->enc_stage, enc_len.data(), s));
+  GAM_TRY(run_ctc(c, c->enc_stage, enc_len.data(), batch, p.T2_max, nullptr, c->tokens_stage, c->counts_stage, s));
+  GAM_TRY(cuda_check(c, cudaMemcpyAsync(tokens_host, c->tokens_stage, (size_t)batch * p.T2_max * 4,
+                                        cudaMemcpyDeviceToHost, s), "tokens download"));
+  GAM_TRY(cuda_check(c, cudaMemcpyAsync(counts_host, c->counts_stage, (size_t)batch * 4, cudaMemcpyDeviceToHost, s),
+                     "counts download"));
+  return cuda_check(c, cudaStreamSynchronize(s), "transcribe sync");
+}
+
+gam_status gam_device_status(gam_ctx* c) {
+  GAM_TRY(enter(c));
+  GAM_TRY(cuda_check(c, cudaStreamSynchronize(c->last_stream), "stream sync"));
+  int st[4] = {0, 0, 0, 0};
+  GAM_TRY(cuda_check(c, cudaMemcpy(st, c->dev_status, 16, cudaMemcpyDeviceToHost), "status read"));
+  int tc_st = 0;
+  GAM_TRY(cuda_check(c, tc_read_status(&c->tc, &tc_st), "status read"));
+  if (st[0] != 0 || tc_st != 0) return fail(c, GAM_ERR_DEVICE_TIMEOUT, "a device-side wait gave up");
+  return GAM_OK;
+}
+
+gam_status gam_profile_enable(gam_ctx* c, int on) {
+  GAM_TRY(enter(c));
+  GAM_TRY(gam_profile_reset(c));
+  c->prof.mask = (uint32_t)on & ((1u << PK_COUNT) - 1u);
+  return GAM_OK;
+}
+
+gam_status gam_profile_reset(gam_ctx* c) {
+  GAM_TRY(enter(c));
+  GAM_TRY(cuda_check(c, cudaDeviceSynchronize(), "profile sync"));
+  for (int k = 0; k < PK_COUNT; ++k) {
+    c->prof.launches[k] = 0;
+    c->prof.ms[k] = 0.0;
+  }
+  c->prof.kind.clear();
+  c->prof.used = 0;
+  GAM_TRY(cuda_check(c, cudaMemset(c->dev_status, 0, 16), "status reset"));
+  return cuda_check(c, tc_reset_status(&c->tc), "status reset");
+}
+
+int gam_profile_kinds(void) { return PK_COUNT; }
+
+const char* gam_profile_kind_name(int kind) { return (kind >= 0 && kind < PK_COUNT) ? kKindNames[kind] : ""; }
+
+gam_status gam_profile_read(gam_ctx* c, int kind, double* total_ms, int64_t* launches) {
+  GAM_TRY(enter(c));
+  if (kind < 0 || kind >= PK_COUNT) return fail(c, GAM_ERR_INVALID_ARG, "bad kind");
+  Prof& p = c->prof;
+  if (p.used) {
+    GAM_TRY(cuda_check(c, cudaEventSynchronize(p.ev[p.used - 1]), "profile sync"));
+    for (size_t i = 0; i < p.kind.size(); ++i) {
+      float ms = 0.f;
+      GAM_TRY(cuda_check(c, cudaEventElapsedTime(&ms, p.ev[2 * i], p.ev[2 * i + 1]), "event time"));
+      p.ms[p.kind[i]] += ms;
+    }
+    p.kind.clear();
+    p.used = 0;
+  }
+  if (total_ms) *total_ms = p.ms[kind];
+  if (launches) *launches = p.launches[kind];
+  return GAM_OK;
+}
+
+gam_status gam_debug_inject_cuda_error(gam_ctx* c, int cuda_error, int count) {
+  if (!c) return GAM_ERR_INVALID_ARG;
+  c->inject_err = cuda_error;
+  c->inject_count = count;
+  return GAM_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,217 @@
+/*
+ * gam.h -- C ABI of the GigaAM Conformer encoder + CTC hot path on B200 (sm_100a).
+ *
+ * The path (audio -> log-mel -> Conv1d 4x subsampling -> N Conformer blocks ->
+ * CTC head -> greedy collapse) follows these pages:
+ *   - "GigaAM v3 MLX", sections "Runtime pipeline", "Frontend configuration"
+ *     and "Architecture details";
+ *   - "GigaAM on MLX: the transcripts matched, but the model was broken",
+ *     sections "What we're porting", "Trap 1" (RoPE base 5000), "Trap 2"
+ *     (RoPE on the raw input before linear_q / linear_k), "Trap 3" (stored
+ *     window and filterbank) and "Trap 4" (PyTorch weight layouts, fp16);
+ *   - "GigaAM v3 RNNT -- MLX (Apple Silicon)", section "Notes for other
+ *     runtimes" (center=False, log(clip(x, 1e-9, 1e9)), blank = len(vocab));
+ *   - "GigaAM MLX port for Mac", sections "What is inside the model" and
+ *     "How precision affects size and speed" (INT8 weights, one scale per
+ *     group of 64).
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ * - Plain C types only.  "device pointer" means memory the caller allocated
+ *   on the context's GPU (cudaMalloc, torch, ...); "host pointer" means CPU
+ *   memory.  `stream` is a cudaStream_t passed as void* (NULL = legacy
+ *   default stream).  All GPU work of a call is enqueued on that stream; no
+ *   call synchronises it except gam_transcribe and gam_device_status.
+ * - The caller owns every buffer it passes.  A context owns its weights and
+ *   one workspace sized at creation for (max_batch, max_samples); calls do no
+ *   device allocation.  One context serves one stream at a time.
+ * - Errors are returned, never thrown and never abort the process.  Arguments
+ *   are checked before any launch.  An asynchronous device error shows up as
+ *   GAM_ERR_CUDA on a later call.  Device-side waits are bounded; a wait that
+ *   gives up sets a status word read by gam_device_status
+ *   (GAM_ERR_DEVICE_TIMEOUT).
+ * - Lengths are host arrays so the host plans every shape without reading
+ *   device memory.  A clip of N samples has F = 1 + (N - 320) / 160 mel
+ *   frames (center=false), tensor lengths T1 = (F - 1) / 2 + 1 and
+ *   T' = (T1 - 1) / 2 + 1 after the two stride-2 convs, and valid lengths
+ *   L1 = (F - 1) / 2 and L' = (L1 - 1) / 2 (integer division).  Every clip
+ *   needs L' >= 1, i.e. N >= 1280 samples, else GAM_ERR_SHAPE.
+ * - Batched outputs are right-padded: frames at or beyond a clip's length are
+ *   written as zeros (token ids as -1).
+ */
+#ifndef GAM_H
+#define GAM_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  GAM_OK = 0,
+  GAM_ERR_INVALID_ARG = 1,        /* null pointer, bad enum, non-positive size   */
+  GAM_ERR_SHAPE = 2,              /* a clip too short / inconsistent sizes        */
+  GAM_ERR_CAPACITY = 3,           /* batch or samples above the context's limits  */
+  GAM_ERR_WEIGHTS = 4,            /* missing tensor, wrong shape or dtype         */
+  GAM_ERR_UNSUPPORTED_DEVICE = 5, /* not a compute capability 10.0 GPU           */
+  GAM_ERR_CUDA = 6,               /* a CUDA runtime / driver call failed          */
+  GAM_ERR_DEVICE_TIMEOUT = 7      /* a bounded device-side wait gave up           */
+} gam_status;
+
+/* gam_config.precision */
+enum { GAM_FP32 = 0, GAM_FP16 = 1, GAM_INT8_G64 = 2 };
+
+/* gam_tensor.dtype */
+enum { GAM_DTYPE_F32 = 0, GAM_DTYPE_F16 = 1, GAM_DTYPE_I8 = 2 };
+
+/* Stage ids of gam_encode_stage (the residual stream after each step). */
+enum {
+  GAM_STAGE_SUBSAMPLING = 0, /* layer ignored: output of the two convs      */
+  GAM_STAGE_FFN1 = 1,        /* x + 1/2 FFN1(LN x)                          */
+  GAM_STAGE_MHSA = 2,        /* + rotary MHSA                               */
+  GAM_STAGE_CONV = 3,        /* + convolution module                        */
+  GAM_STAGE_FFN2 = 4,        /* + 1/2 FFN2                                  */
+  GAM_STAGE_LAYER = 5        /* block output after its final LayerNorm      */
+};
+
+/* Model and capacity.  Field names follow the pages' notation. */
+typedef struct {
+  int n_layers;      /* Conformer blocks (16 for v3, 24 multilingual large)   */
+  int d_model;       /* model width d (768 / 1024); d % 256 == 0              */
+  int n_heads;       /* H; d_head = d / H must be 48 or 64                    */
+  int ffn_dim;       /* FFN hidden width (4 d); % 256 == 0                    */
+  int conv_kernel;   /* depthwise kernel K_dw (odd, <= 63)                    */
+  int n_mels;        /* 64                                                    */
+  int n_fft;         /* 320                                                   */
+  int win;           /* 320                                                   */
+  int hop;           /* 160                                                   */
+  int sub_kernel;    /* subsampling Conv1d kernel, 5 (stride 2, padding 2)    */
+  int n_classes;     /* vocabulary + 1; blank id = n_classes - 1; <= 1024     */
+  float rope_base;   /* 5000 (pos_emb_max_len), not 10000                     */
+  float ln_eps;      /* LayerNorm eps (1e-5)                                  */
+  float bn_eps;      /* BatchNorm eps (1e-5)                                  */
+  int precision;     /* GAM_FP32, GAM_FP16 or GAM_INT8_G64                    */
+  int max_batch;     /* capacity: clips per call                              */
+  int64_t max_samples; /* capacity: samples per clip                          */
+} gam_config;
+
+/* One named weight tensor, HOST memory, PyTorch layout (Linear [out, in],
+ * Conv1d [out, in, K]).  gam_create copies it; the caller may free it after. */
+typedef struct {
+  const char* name;
+  const void* data;
+  int dtype;         /* GAM_DTYPE_*                                           */
+  int ndim;
+  int64_t shape[4];
+} gam_tensor;
+
+typedef struct gam_ctx gam_ctx;
+
+/* Human-readable name of a status code (static storage). */
+const char* gam_status_string(gam_status status);
+
+/* Text of the last error seen by this context ("" if none; NULL ctx gives the
+ * last error of a failed gam_create on this thread). */
+const char* gam_last_error(const gam_ctx* ctx);
+
+/* Host-only length planning for `batch` clips of `lengths_host[i]` samples.
+ * Writes (each optional, may be NULL) frames_out[i] = F_i, enc_len_out[i] =
+ * L'_i, and dims_out[0..1] = (F_max, T'_max), the padded sizes of the mel and
+ * encoder outputs.  Fails with GAM_ERR_SHAPE for a clip shorter than 1280. */
+gam_status gam_plan_lengths(const gam_config* cfg, const int32_t* lengths_host, int batch,
+                            int32_t* frames_out, int32_t* enc_len_out, int32_t* dims_out);
+
+/* Build a context on CUDA device `device`: checks the device (sm_100),
+ * validates every tensor the config needs by name/shape/dtype, repacks the
+ * weights (fold the window into a DFT basis, fold BatchNorm into the depthwise
+ * conv, reorder GLU halves, transpose conv weights, quantised layouts), and
+ * allocates the workspace.  Tensors: "frontend.window" [win] f32,
+ * "frontend.mel_fb" [n_fft/2+1, n_mels] f32, "subsampling.conv{1,2}.{weight,
+ * bias}", per layer l "layers.l.{ffn1,ffn2}.{norm,linear1,linear2}.*",
+ * "layers.l.attn.{norm,linear_q,linear_k,linear_v,linear_out}.*",
+ * "layers.l.conv.{norm,pointwise1,depthwise,bn,pointwise2}.*",
+ * "layers.l.norm_out.*", "head.{weight,bias}" ([C, d] or [C, d, 1]).  In
+ * GAM_INT8_G64 precision the eleven linear weights of a block and the head's
+ * are given as "<name>.weight_q" (int8, same shape) and "<name>.weight_scale"
+ * (f16 [out, in/64]); all other tensors f16 or f32.  On success *out owns
+ * device memory until gam_destroy. */
+gam_status gam_create(const gam_config* cfg, const gam_tensor* tensors, int n_tensors, int device,
+                      gam_ctx** out);
+
+/* Free everything the context owns.  NULL is accepted. */
+gam_status gam_destroy(gam_ctx* ctx);
+
+/* Log-mel frontend only ("GigaAM v3 MLX", "Frontend configuration").
+ * audio_dev: device f32 [batch, max_samples] (row stride max_samples), clip i
+ * valid on its first lengths_host[i] samples.  mel_dev: device f32
+ * [batch, F_max, n_mels], time-major (the pages print [n_mels, F]); frames at
+ * or beyond F_i are zero.  frames_host_out (optional): F_i. */
+gam_status gam_logmel(gam_ctx* ctx, const float* audio_dev, const int32_t* lengths_host, int batch,
+                      int64_t max_samples, float* mel_dev, int32_t* frames_host_out, void* stream);
+
+/* Frontend + subsampling + all Conformer blocks.  enc_dev: device f32
+ * [batch, T'_max, d]; frames at or beyond L'_i are zero.  enc_len_host_out
+ * (optional): L'_i. */
+gam_status gam_encode(gam_ctx* ctx, const float* audio_dev, const int32_t* lengths_host, int batch,
+                      int64_t max_samples, float* enc_dev, int32_t* enc_len_host_out, void* stream);
+
+/* Debug tap for layer-by-layer localisation ("GigaAM on MLX ...", "Trap 1"):
+ * runs the same path as gam_encode up to `stage` of block `layer` and writes
+ * the f32 residual stream there to out_dev [batch, T'_max, d] (zero padded). */
+gam_status gam_encode_stage(gam_ctx* ctx, const float* audio_dev, const int32_t* lengths_host, int batch,
+                            int64_t max_samples, int layer, int stage, float* out_dev, void* stream);
+
+/* CTC head + greedy decoding.  enc_dev: device f32 [batch, t_max, d] with
+ * clip i valid on its first enc_len_host[i] <= t_max frames.  logp_dev
+ * (optional, device f32 [batch, t_max, n_classes]): log-softmax of the head's
+ * logits, zero beyond a clip.  tokens_dev: device i32 [batch, t_max], the
+ * collapsed ids (runs merged, then blanks dropped; argmax = lowest index of
+ * the fp32 maximum), -1 after the last token.  counts_dev: device i32 [batch]. */
+gam_status gam_ctc_greedy(gam_ctx* ctx, const float* enc_dev, const int32_t* enc_len_host, int batch,
+                          int t_max, float* logp_dev, int32_t* tokens_dev, int32_t* counts_dev,
+                          void* stream);
+
+/* Greedy decoding from given scores (test entry for the collapse kernel):
+ * logits_dev device f32 [batch, t_max, n_classes]; blank = n_classes - 1;
+ * outputs as gam_ctc_greedy.  Uses the context's workspace for the per-frame
+ * argmax, so batch * t_max must fit its capacity. */
+gam_status gam_ctc_collapse(gam_ctx* ctx, const float* logits_dev, const int32_t* lengths_host, int batch,
+                            int t_max, int n_classes, int32_t* tokens_dev, int32_t* counts_dev, void* stream);
+
+/* End-to-end call on HOST buffers: copies audio_host [batch, max_samples] f32
+ * to the device, runs gam_encode and gam_ctc_greedy, copies tokens_host
+ * [batch, T'_max] and counts_host [batch] back, and synchronises `stream`
+ * before returning.  Pinned host memory makes the copies asynchronous. */
+gam_status gam_transcribe(gam_ctx* ctx, const float* audio_host, const int32_t* lengths_host, int batch,
+                          int64_t max_samples, int32_t* tokens_host, int32_t* counts_host, void* stream);
+
+/* Synchronises the context's last stream and reports GAM_ERR_DEVICE_TIMEOUT
+ * if a device-side bounded wait gave up since the last gam_profile_reset. */
+gam_status gam_device_status(gam_ctx* ctx);
+
+/* ---- profiling (per kernel family, CUDA events on the launching stream) ---- */
+
+/* Choose which kernel families get an event pair recorded around every
+ * launch: 0 = none, -1 = all, else a bit mask (bit k = family k).  Each
+ * timed launch costs about a microsecond of stream time.  Resets the counters. */
+gam_status gam_profile_enable(gam_ctx* ctx, int on);
+gam_status gam_profile_reset(gam_ctx* ctx);
+/* Number of kernel families and the name of family `kind`. */
+int gam_profile_kinds(void);
+const char* gam_profile_kind_name(int kind);
+/* Totals since the last reset for family `kind` (synchronises the recorded
+ * events).  Launch counts are kept even when timing is off. */
+gam_status gam_profile_read(gam_ctx* ctx, int kind, double* total_ms, int64_t* launches);
+
+/* ---- host-side fault injection (tests) ---- */
+
+/* Make the next `count` CUDA-error checks of this context report
+ * `cuda_error` (a cudaError_t value) as if the runtime had returned it. */
+gam_status gam_debug_inject_cuda_error(gam_ctx* ctx, int cuda_error, int count);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GAM_H */

@@ -1,0 +1,89 @@
+"""GPU parity of the log-mel frontend and of the CTC decoder, through the C ABI."""
+import numpy as np
+import pytest
+
+import oracle
+from conformer_speech_recognition_b200 import gam, synth
+from gpu_common import TOL_LOGMEL, config_and_weights, max_abs, small_model, to_torch
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def small_ctx():
+    cfg, W = config_and_weights(small_model(), 34, "fp32")
+    ctx = gam.gam_create(cfg, W, 8, 200000)
+    yield cfg, W, ctx
+    ctx.close()
+
+
+def test_logmel_parity_ragged(small_ctx):
+    cfg, W, ctx = small_ctx
+    lengths = [16000, 1280, 16159, 4321, 48000, 160001]
+    audio, lens = synth.random_audio(lengths, seed=7)
+    mel, frames = gam.gam_logmel(ctx, to_torch(audio), lens)
+    mel = mel.cpu().numpy()
+    for i, n in enumerate(lens):
+        ref = oracle.log_mel(audio[i, :n].astype(np.float64), W["frontend.window"], W["frontend.mel_fb"], cfg)
+        assert frames[i] == ref.shape[0]
+        assert max_abs(mel[i, :frames[i]], ref) <= TOL_LOGMEL, i
+        assert np.all(mel[i, frames[i]:] == 0)
+
+
+def test_logmel_shape_printed_on_pages(small_ctx):
+    cfg, W, ctx = small_ctx
+    audio, lens = synth.random_audio([16000], seed=8)
+    mel, frames = gam.gam_logmel(ctx, to_torch(audio), lens)
+    assert tuple(mel.shape) == (1, 99, 64) and frames[0] == 99
+
+
+def _crafted_logits(rng, B, T, C):
+    z = rng.normal(size=(B, T, C)).astype(np.float32)
+    blank = C - 1
+    # runs of the same winner, blank runs and exact ties between two classes
+    for b in range(B):
+        for t in range(0, T, 7):
+            z[b, t:t + 3, 5 % C] += 10.0
+        for t in range(3, T, 11):
+            z[b, t, blank] += 20.0
+        for t in range(2, T, 13):
+            m = z[b, t].max() + 1.0
+            z[b, t, 1] = m
+            z[b, t, 4] = m  # tie: lowest index (1) must win
+    return z
+
+
+@pytest.mark.parametrize("C", [34, 257, 1025])
+def test_ctc_collapse_bit_exact(small_ctx, C):
+    cfg, W, ctx = small_ctx
+    rng = np.random.default_rng(C)
+    B, T = 6, 300
+    z = _crafted_logits(rng, B, T, C)
+    lens = np.array([300, 0, 1, 299, 150, 17], np.int32)
+    tok, cnt = gam.gam_ctc_collapse(ctx, to_torch(z), lens)
+    tok, cnt = tok.cpu().numpy(), cnt.cpu().numpy()
+    for b in range(B):
+        a = np.argmax(z[b, :lens[b]], axis=1)
+        ref = oracle.greedy_collapse(a, C - 1)
+        assert cnt[b] == len(ref)
+        assert tok[b, :cnt[b]].tolist() == ref
+        assert np.all(tok[b, cnt[b]:] == -1)
+
+
+def test_ctc_greedy_head_parity(small_ctx):
+    cfg, W, ctx = small_ctx
+    rng = np.random.default_rng(3)
+    B, T, d = 4, 37, cfg["d_model"]
+    enc = rng.normal(size=(B, T, d)).astype(np.float32)
+    lens = np.array([37, 1, 20, 36], np.int32)
+    tok, cnt, logp = gam.gam_ctc_greedy(ctx, to_torch(enc), lens, want_logp=True)
+    tok, cnt, logp = tok.cpu().numpy(), cnt.cpu().numpy(), logp.cpu().numpy()
+    for b in range(B):
+        z, lp, a = oracle.ctc_head(enc[b, :lens[b]].astype(np.float64), W)
+        assert max_abs(logp[b, :lens[b]], lp) < 1e-4
+        assert np.all(logp[b, lens[b]:] == 0)
+        zs = np.sort(z, axis=1)
+        clear = (zs[:, -1] - zs[:, -2]) > 1e-3
+        ref = oracle.greedy_collapse(a, cfg["n_classes"] - 1)
+        if clear.all():
+            assert tok[b, :cnt[b]].tolist() == ref
