@@ -32,13 +32,15 @@ struct Clips {
   __device__ __forceinline__ int L1(int i) const { return __ldg(tab + 2 * (B + 1) + i); }
   __device__ __forceinline__ int L2(int i) const { return __ldg(tab + 3 * (B + 1) + i); }
   __device__ __forceinline__ int N(int i) const { return __ldg(tab + 4 * (B + 1) + i); }
-  // Largest clip i with scale * e_i <= r (r >= 0): the clip whose segment at
-  // resolution `scale` (1 encoder, 2 conv1, 4 mel) contains row r.
-  __device__ __forceinline__ int find(int r, int scale) const {
+  // Largest clip i whose first row at this resolution, scale * e_i + off,
+  // is <= r (0 if none): (scale, off) = (1, 0) encoder, (2, 2) conv1,
+  // (4, 6) mel rows.  Row r belongs to that clip iff r - (scale e_i + off) is
+  // below the clip's length at this resolution.
+  __device__ __forceinline__ int find(int r, int scale, int off) const {
     int lo = 0, hi = B - 1;
     while (lo < hi) {
       int mid = (lo + hi + 1) >> 1;
-      if (scale * e(mid) <= r) lo = mid; else hi = mid - 1;
+      if (scale * e(mid) + off <= r) lo = mid; else hi = mid - 1;
     }
     return lo;
   }

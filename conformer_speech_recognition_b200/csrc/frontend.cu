@@ -46,7 +46,7 @@ frontend_kernel(const float* __restrict__ audio, int64_t stride, Clips clips, in
     int ci = -1, f = -1;
     if (r < rows) {
       if (packed) {
-        ci = clips.find(r, 4);
+        ci = clips.find(r, 4, 6);
         f = r - (4 * clips.e(ci) + 6);
       } else {
         ci = r / f_max;
@@ -78,6 +78,12 @@ frontend_kernel(const float* __restrict__ audio, int64_t stride, Clips clips, in
     __syncthreads();
     for (int idx = tid; idx < NCH * NFFT; idx += 256) bs[idx] = __ldg(basis + (size_t)n0 * NFFT + idx);
     __syncthreads();
+    // blocked summation: partial sums over 32 samples, then added to the totals
+    float pre[4][6], pim[4][6];
+#pragma unroll
+    for (int a = 0; a < 4; ++a)
+#pragma unroll
+      for (int q = 0; q < 6; ++q) pre[a][q] = pim[a][q] = 0.f;
 #pragma unroll 4
     for (int nn = 0; nn < NCH; ++nn) {
       float xv[4];
@@ -92,12 +98,19 @@ frontend_kernel(const float* __restrict__ audio, int64_t stride, Clips clips, in
           const float s = (k >= 1 && k <= 159) ? brow[160 + k] : 0.f;
 #pragma unroll
           for (int a = 0; a < 4; ++a) {
-            re[a][q] = fmaf(xv[a], c, re[a][q]);
-            im[a][q] = fmaf(xv[a], s, im[a][q]);
+            pre[a][q] = fmaf(xv[a], c, pre[a][q]);
+            pim[a][q] = fmaf(xv[a], s, pim[a][q]);
           }
         }
       }
     }
+#pragma unroll
+    for (int a = 0; a < 4; ++a)
+#pragma unroll
+      for (int q = 0; q < 6; ++q) {
+        re[a][q] += pre[a][q];
+        im[a][q] += pim[a][q];
+      }
   }
   __syncthreads();
   // power spectrum into fr as [FT][NBIN]

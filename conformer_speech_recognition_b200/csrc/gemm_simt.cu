@@ -154,7 +154,7 @@ gemm_simt_kernel(const TA* __restrict__ A, const TA* __restrict__ A2, int n_spli
         }
         break;
       case EPI_CONV1: {
-        const int ci = ep.clips.find(r, 2);
+        const int ci = ep.clips.find(r, 2, 2);
         const int t = r - (2 * ep.clips.e(ci) + 2);
         const bool valid = t >= 0 && t < ep.clips.L1(ci);
 #pragma unroll
@@ -164,7 +164,7 @@ gemm_simt_kernel(const TA* __restrict__ A, const TA* __restrict__ A2, int n_spli
         }
       } break;
       case EPI_CONV2: {
-        const int ci = ep.clips.find(r, 1);
+        const int ci = ep.clips.find(r, 1, 0);
         const int t = r - ep.clips.e(ci);
         const bool valid = t >= 0 && t < ep.clips.L2(ci);
 #pragma unroll

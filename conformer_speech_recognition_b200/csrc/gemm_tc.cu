@@ -1,17 +1,416 @@
-// Tensor-core kernels (placeholder dispatch: CUDA-core path until the tcgen05 kernels are enabled).
+// Tensor-core GEMM for sm_100a: C = A . B^T with fused epilogues.
+//
+// A [M, K] fp16 (row stride lda; a strided view for the subsampling convs),
+// B [N, K] fp16 weight (PyTorch Linear layout), fp32 accumulation in TMEM.
+//
+// Persistent, warp-specialised CTA of 192 threads, one CTA per SM:
+//   warp 0      one thread issues TMA loads of 128x64 A and BNx64 B tiles
+//               (128-byte swizzle) into a STAGES-deep shared-memory ring;
+//   warp 1      allocates 2*BN TMEM columns (two accumulators) and one thread
+//               issues tcgen05.mma (M=128, N=BN, K=16) per 16-wide K slice,
+//               committing stage releases and accumulator-ready barriers;
+//   warps 2..5  epilogue: tcgen05.ld of the accumulator (warp w reads TMEM
+//               lanes 32*(w%4) .. +31 = its 32 output rows), bias + activation
+//               / residual / scatter, global stores; then hand the
+//               accumulator back so the next tile's MMAs overlap this epilogue.
+// Tiles are visited n-fastest so the CTAs in flight share each A row block
+// through L2 and the weight (a few MB) stays L2-resident.
+// Every mbarrier wait is bounded (tc_common.cuh); a wait that gives up raises
+// a CTA abort flag, the other roles stop at their next wait, in-flight copies
+// and MMAs are drained with bounded waits, TMEM is freed, and a device status
+// word is set for the host.
+#include <cudaTypedefs.h>
+
+#include <climits>
+
 #include "gemm_tc.cuh"
+#include "tc_common.cuh"
 
 namespace gam {
+namespace {
 
-bool tc_supported(int, int, int, int, int) { return false; }
+using namespace tc;
 
-cudaError_t launch_gemm_tc(TcGemmCache*, const void*, const void*, int, int, WeightOp, int, int, int, int,
-                           const EpiParams&, cudaStream_t) {
-  return cudaErrorNotSupported;
+constexpr int BM = 128, BK = 64;
+constexpr int A_TILE = BM * BK * 2;  // 16 KB
+
+struct TcArgs {
+  int M, N, K;
+  int m_blocks, n_blocks, tiles;
+  int n_split;  // output columns >= n_split read A from the second map
+  int conv_c;   // 0: plain A [M, K]; else A row r = input rows 2r .. 2r+taps-1 of C = conv_c channels
+  int epi;
+  EpiParams ep;
+  int* status;
+};
+
+template <int BN, int STAGES>
+struct Cfg {
+  static constexpr int B_TILE = BN * BK * 2;
+  static constexpr int STAGE = A_TILE + B_TILE;
+  static constexpr int TMEM_COLS = 2 * BN;  // power of two for BN in {128, 256}
+  static constexpr size_t SMEM = (size_t)STAGES * STAGE + 1024 + 256;
+};
+
+__device__ __forceinline__ float sigm(float v) { return 1.f / (1.f + __expf(-v)); }
+
+__device__ __forceinline__ void store_half16(__half* dst, const float* v) {
+  uint4 w[2];
+  uint32_t* pw = reinterpret_cast<uint32_t*>(w);
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    __half2 h = __floats2half2_rn(v[2 * j], v[2 * j + 1]);
+    pw[j] = *reinterpret_cast<uint32_t*>(&h);
+  }
+  reinterpret_cast<uint4*>(dst)[0] = w[0];
+  reinterpret_cast<uint4*>(dst)[1] = w[1];
 }
 
-cudaError_t launch_attention(TcGemmCache*, const void* qk, const void* vt, Clips clips, void* o, int t_half,
+// Epilogue of one 32-column accumulator chunk of row r (columns n .. n+31).
+__device__ __forceinline__ void epi_chunk(const TcArgs& p, int r, int n, bool valid, const uint32_t (&u)[32]) {
+  const EpiParams& ep = p.ep;
+  float v[32];
+#pragma unroll
+  for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(u[j]) + __ldg(ep.bias + n + j);
+  switch (p.epi) {
+    case EPI_SWISH: {
+#pragma unroll
+      for (int j = 0; j < 32; ++j) v[j] = v[j] * sigm(v[j]);
+      __half* o = reinterpret_cast<__half*>(ep.out) + (size_t)r * ep.ldo + n;
+      store_half16(o, v);
+      store_half16(o + 16, v + 16);
+    } break;
+    case EPI_RESID: {
+      float4* px = reinterpret_cast<float4*>(ep.x + (size_t)r * ep.ldo + n);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        float4 a = px[j];
+        a.x += ep.alpha * v[4 * j];
+        a.y += ep.alpha * v[4 * j + 1];
+        a.z += ep.alpha * v[4 * j + 2];
+        a.w += ep.alpha * v[4 * j + 3];
+        px[j] = a;
+      }
+    } break;
+    case EPI_CONV1: {
+#pragma unroll
+      for (int j = 0; j < 32; ++j) v[j] = valid ? fmaxf(v[j], 0.f) : 0.f;
+      __half* o = reinterpret_cast<__half*>(ep.out) + (size_t)r * ep.ldo + n;
+      store_half16(o, v);
+      store_half16(o + 16, v + 16);
+    } break;
+    case EPI_CONV2: {
+      float4* px = reinterpret_cast<float4*>(ep.x + (size_t)r * ep.ldo + n);
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+        px[j] = valid ? make_float4(fmaxf(v[4 * j], 0.f), fmaxf(v[4 * j + 1], 0.f), fmaxf(v[4 * j + 2], 0.f),
+                                    fmaxf(v[4 * j + 3], 0.f))
+                      : make_float4(0.f, 0.f, 0.f, 0.f);
+    } break;
+    case EPI_QKV: {
+#pragma unroll
+      for (int g = 0; g < 2; ++g) {
+        const int nn = n + 16 * g;
+        const int which = nn / ep.d_model;
+        const int rem = nn - which * ep.d_model;
+        const int h = rem / ep.d_head, cc = rem - h * ep.d_head;
+        if (which < 2) {
+          __half* o = reinterpret_cast<__half*>(ep.qk) + (((size_t)which * ep.n_heads + h) * ep.rows_pad + r) * 64 + cc;
+          store_half16(o, v + 16 * g);
+        } else {
+          __half* o = reinterpret_cast<__half*>(ep.vt) + ((size_t)h * 64 + cc) * ep.rows_pad + r;
+#pragma unroll
+          for (int j = 0; j < 16; ++j) o[(size_t)j * ep.rows_pad] = __float2half_rn(v[16 * g + j]);
+        }
+      }
+    } break;
+    default:
+      break;
+  }
+}
+
+template <int BN>
+__device__ __forceinline__ void epilogue_tile(const TcArgs& p, int r, int n0, uint32_t tbase) {
+  const EpiParams& ep = p.ep;
+  const bool in_m = r < p.M;
+  bool valid = in_m;
+  if (in_m && (p.epi == EPI_CONV1 || p.epi == EPI_CONV2)) {
+    const int scale = p.epi == EPI_CONV1 ? 2 : 1;
+    const int ci = ep.clips.find(r, scale, scale == 2 ? 2 : 0);
+    const int t = r - (p.epi == EPI_CONV1 ? 2 * ep.clips.e(ci) + 2 : ep.clips.e(ci));
+    valid = t >= 0 && t < (p.epi == EPI_CONV1 ? ep.clips.L1(ci) : ep.clips.L2(ci));
+  }
+  if (p.epi == EPI_GLU) {
+    // weight rows interleaved in blocks of 64: [value 64 | gate 64] per 128 columns
+#pragma unroll 1
+    for (int blk = 0; blk < BN; blk += 128) {
+#pragma unroll 1
+      for (int hh = 0; hh < 64; hh += 32) {
+        uint32_t a[32], g[32];
+        tmem_ld32(tbase + blk + hh, a);
+        tmem_ld32(tbase + blk + 64 + hh, g);
+        tmem_ld_wait();
+        if (!in_m) continue;
+        const int nv = n0 + blk + hh, ng = nv + 64;
+        float y[32];
+#pragma unroll
+        for (int j = 0; j < 32; ++j)
+          y[j] = (__uint_as_float(a[j]) + __ldg(ep.bias + nv + j)) *
+                 sigm(__uint_as_float(g[j]) + __ldg(ep.bias + ng + j));
+        __half* o = reinterpret_cast<__half*>(ep.out) + (size_t)r * ep.ldo + (n0 + blk) / 2 + hh;
+        store_half16(o, y);
+        store_half16(o + 16, y + 16);
+      }
+    }
+    return;
+  }
+#pragma unroll 1
+  for (int c = 0; c < BN; c += 32) {
+    uint32_t u[32];
+    tmem_ld32(tbase + c, u);
+    tmem_ld_wait();
+    if (in_m) epi_chunk(p, r, n0 + c, valid, u);
+  }
+}
+
+template <int BN, int STAGES>
+__global__ void __launch_bounds__(192, 1)
+gemm_tc_kernel(const __grid_constant__ CUtensorMap mA, const __grid_constant__ CUtensorMap mA2,
+               const __grid_constant__ CUtensorMap mB, const TcArgs p) {
+  using C = Cfg<BN, STAGES>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+  uint8_t* sA = base;
+  uint8_t* sB = base + STAGES * A_TILE;
+  uint64_t* full = reinterpret_cast<uint64_t*>(base + STAGES * C::STAGE);
+  uint64_t* empty = full + STAGES;
+  uint64_t* tfull = empty + STAGES;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* drain = tempty + 2;
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tslot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&tfull[a], 1);
+      mbar_init(&tempty[a], 4);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&mA);
+    prefetch_tmap(&mA2);
+    prefetch_tmap(&mB);
+  }
+  if (warp == 1) tmem_alloc(tslot, C::TMEM_COLS);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tslot;
+  const int KB = p.K / BK;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      int it = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < p.tiles && ok; tile += gridDim.x) {
+        const int nb = tile % p.n_blocks, mb = tile / p.n_blocks;
+        const int m0 = mb * BM, n0 = nb * BN;
+        const CUtensorMap* ma = (n0 >= p.n_split) ? &mA2 : &mA;
+        for (int kb = 0; kb < KB; ++kb) {
+          const int s = it % STAGES;
+          if (!mbar_wait(&empty[s], ((it / STAGES) & 1) ^ 1, abort_flag)) {
+            ok = false;
+            break;
+          }
+          // A coordinates: plain GEMM, or tap t / channel c0 of the strided conv view,
+          // read from the [pairs of input rows, 2C] map: row 2r + t = pair r + t/2, half t%2
+          int ax = kb * BK, ay = m0;
+          if (p.conv_c) {
+            const int t = (kb * BK) / p.conv_c, c0 = kb * BK - t * p.conv_c;
+            ax = (t & 1) * p.conv_c + c0;
+            ay = m0 + (t >> 1);
+          }
+          mbar_arrive_expect_tx(&full[s], C::STAGE);
+          tma_load_2d(sA + s * A_TILE, ma, &full[s], ax, ay);
+          tma_load_2d(sB + s * C::B_TILE, &mB, &full[s], kb * BK, n0);
+          ++it;
+        }
+      }
+      // every issued copy has landed before the CTA can exit (bounded)
+      const int first = it > STAGES ? it - STAGES : 0;
+      for (int j = first; j < it; ++j) {
+        const uint64_t t0 = globaltimer_ns();
+        while (!mbar_try_wait(&full[j % STAGES], (j / STAGES) & 1))
+          if (globaltimer_ns() - t0 > kWaitLimitNs) {
+            *abort_flag = 1;
+            break;
+          }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_f16_f32(BM, BN);
+      int it = 0, local = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < p.tiles && ok; tile += gridDim.x, ++local) {
+        const int acc = local & 1;
+        const uint32_t use = (uint32_t)(local >> 1);
+        if (!mbar_wait(&tempty[acc], (use & 1) ^ 1, abort_flag)) break;
+        tc_fence_after();
+        const uint32_t d = tmem + (uint32_t)(acc * BN);
+        for (int kb = 0; kb < KB; ++kb) {
+          const int s = it % STAGES;
+          if (!mbar_wait(&full[s], (it / STAGES) & 1, abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint64_t da = sdesc_k_sw128(smem_u32(sA + s * A_TILE));
+          const uint64_t db = sdesc_k_sw128(smem_u32(sB + s * C::B_TILE));
+#pragma unroll
+          for (int k = 0; k < BK / 16; ++k) umma_f16(d, da + 2 * k, db + 2 * k, idesc, (kb | k) != 0 ? 1u : 0u);
+          umma_commit(&empty[s]);
+          ++it;
+        }
+        if (ok) umma_commit(&tfull[acc]);
+      }
+      // drain: all MMAs issued by this thread complete before TMEM is freed (bounded)
+      umma_commit(drain);
+      const uint64_t t0 = globaltimer_ns();
+      while (!mbar_try_wait(drain, 0))
+        if (globaltimer_ns() - t0 > kWaitLimitNs) {
+          *abort_flag = 1;
+          break;
+        }
+    }
+  } else {
+    const int q = warp & 3;
+    int local = 0;
+    for (int tile = blockIdx.x; tile < p.tiles; tile += gridDim.x, ++local) {
+      const int acc = local & 1;
+      const uint32_t use = (uint32_t)(local >> 1);
+      if (!mbar_wait(&tfull[acc], use & 1, abort_flag)) break;
+      tc_fence_after();
+      const int nb = tile % p.n_blocks, mb = tile / p.n_blocks;
+      const int r = mb * BM + q * 32 + lane;
+      const uint32_t tbase = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN);
+      epilogue_tile<BN>(p, r, nb * BN, tbase);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tempty[acc]);
+    }
+  }
+  __syncthreads();
+  if (threadIdx.x == 0 && *abort_flag) atomicExch(p.status, 1);
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// host side
+// ---------------------------------------------------------------------------
+
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+
+cudaError_t get_encoder() {
+  if (g_encode) return cudaSuccess;
+  cudaDriverEntryPointQueryResult q;
+  void* fn = nullptr;
+  cudaError_t e = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q);
+  if (e != cudaSuccess) return e;
+  if (q != cudaDriverEntryPointSuccess || !fn) return cudaErrorNotSupported;
+  g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  return cudaSuccess;
+}
+
+// 2D fp16 tensor map: `outer` rows of `inner` elements, rows `stride_bytes`
+// apart, box box_inner x box_outer, 128-byte swizzle, zero fill out of bounds.
+cudaError_t make_map_f16(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t outer, uint64_t stride_bytes,
+                         uint32_t box_inner, uint32_t box_outer) {
+  if ((reinterpret_cast<uintptr_t>(ptr) & 15) || (stride_bytes & 15)) return cudaErrorInvalidValue;
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {stride_bytes};
+  cuuint32_t box[2] = {box_inner, box_outer};
+  cuuint32_t es[2] = {1, 1};
+  CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void*>(ptr), dims, strides, box, es,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+template <int BN, int STAGES>
+cudaError_t launch_bn(TcGemmCache* cache, const CUtensorMap& mA, const CUtensorMap& mA2, const CUtensorMap& mB,
+                      const TcArgs& args, cudaStream_t s) {
+  using C = Cfg<BN, STAGES>;
+  auto kern = gemm_tc_kernel<BN, STAGES>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::SMEM);
+  if (e != cudaSuccess) return e;
+  const int grid = args.tiles < cache->sm_count ? args.tiles : cache->sm_count;
+  kern<<<grid, 192, C::SMEM, s>>>(mA, mA2, mB, args);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+bool tc_supported(int a_dtype, int b_dtype, int N, int K, int epi) {
+  return a_dtype == 1 && b_dtype == 1 && N % 256 == 0 && K % 64 == 0 && K >= 64 &&
+         (epi == EPI_SWISH || epi == EPI_GLU || epi == EPI_RESID || epi == EPI_QKV || epi == EPI_CONV1 ||
+          epi == EPI_CONV2);
+}
+
+cudaError_t tc_init(TcGemmCache* cache, int device) {
+  cudaError_t e = get_encoder();
+  if (e != cudaSuccess) return e;
+  e = cudaDeviceGetAttribute(&cache->sm_count, cudaDevAttrMultiProcessorCount, device);
+  if (e != cudaSuccess) return e;
+  e = cudaMalloc(&cache->status, sizeof(int));
+  if (e != cudaSuccess) return e;
+  return cudaMemset(cache->status, 0, sizeof(int));
+}
+
+cudaError_t launch_gemm_tc(TcGemmCache* cache, const void* A, const void* A2, int n_split, int lda, WeightOp B, int M,
+                           int N, int K, int epi, const EpiParams& ep, cudaStream_t s) {
+  if (!tc_supported(1, B.dtype, N, K, epi) || M <= 0) return cudaErrorInvalidValue;
+  constexpr int BN = 256;
+  // lda < K: stride-2 convolution view (lda = 2C, K = taps * C, C % 64 == 0); the
+  // buffer behind it holds (M + 2) * lda elements, mapped as M + 2 rows of 2C.
+  const bool conv = lda < K;
+  if (conv && ((lda & 1) || (lda / 2) % BK || K % (lda / 2))) return cudaErrorInvalidValue;
+  CUtensorMap mA, mA2, mB;
+  cudaError_t e = conv ? make_map_f16(&mA, A, lda, (uint64_t)M + 2, (uint64_t)lda * 2, BK, BM)
+                       : make_map_f16(&mA, A, K, M, (uint64_t)lda * 2, BK, BM);
+  if (e == cudaSuccess && !conv) e = make_map_f16(&mA2, A2 ? A2 : A, K, M, (uint64_t)lda * 2, BK, BM);
+  if (conv) mA2 = mA;
+  if (e == cudaSuccess) e = make_map_f16(&mB, B.w, K, N, (uint64_t)K * 2, BK, BN);
+  if (e != cudaSuccess) return e;
+  TcArgs args;
+  args.M = M;
+  args.N = N;
+  args.K = K;
+  args.m_blocks = (M + BM - 1) / BM;
+  args.n_blocks = N / BN;
+  args.tiles = args.m_blocks * args.n_blocks;
+  args.n_split = A2 ? n_split : INT_MAX;
+  args.conv_c = conv ? lda / 2 : 0;
+  args.epi = epi;
+  args.ep = ep;
+  args.status = cache->status;
+  return launch_bn<BN, 4>(cache, mA, mA2, mB, args, s);
+}
+
+cudaError_t launch_attention(TcGemmCache* cache, const void* qk, const void* vt, Clips clips, void* o, int t_half,
                              int rows_pad, int n_heads, int d_head, int t_max, cudaStream_t s) {
+  if (t_half) return launch_attention_tc(cache, qk, vt, clips, o, rows_pad, n_heads, d_head, t_max, s);
   return launch_attention_simt(qk, vt, clips, o, t_half, rows_pad, n_heads, d_head, t_max, s);
 }
 

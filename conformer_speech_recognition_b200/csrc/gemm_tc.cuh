@@ -9,13 +9,21 @@ namespace gam {
 // Per-context state of the tensor-core kernels (tensor-map cache, status word).
 struct TcGemmCache {
   int* status = nullptr;  // device word set when a bounded wait gives up
+  int sm_count = 148;
 };
+
+// Resolves the driver's tensor-map encoder and allocates the status word.
+cudaError_t tc_init(TcGemmCache* cache, int device);
 
 // True when the tensor-core GEMM handles this operand / shape / epilogue combination.
 bool tc_supported(int a_dtype, int b_dtype, int N, int K, int epi);
 
 cudaError_t launch_gemm_tc(TcGemmCache* cache, const void* A, const void* A2, int n_split, int lda, WeightOp B,
                            int M, int N, int K, int epi, const EpiParams& ep, cudaStream_t s);
+
+// Masked multi-head attention on tensor cores (fp16 Q/K/V^T, see attention_tc.cu).
+cudaError_t launch_attention_tc(TcGemmCache* cache, const void* qk, const void* vt, Clips clips, void* o,
+                                int rows_pad, int n_heads, int d_head, int t_max, cudaStream_t s);
 
 // Masked multi-head attention: tensor cores for fp16 activations, CUDA cores for fp32.
 cudaError_t launch_attention(TcGemmCache* cache, const void* qk, const void* vt, Clips clips, void* o, int t_half,

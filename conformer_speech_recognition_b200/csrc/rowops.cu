@@ -133,7 +133,7 @@ ln_rope_kernel(const float* __restrict__ x, const float* __restrict__ g, const f
       *reinterpret_cast<float4*>(sr + c) = v[j];
     }
   __syncwarp();
-  const int ci = clips.find(row, 1);
+  const int ci = clips.find(row, 1, 0);
   int t = row - clips.e(ci);
   if (t < 0 || t >= clips.L2(ci)) t = 0;  // gap row: any finite rotation
   const int half = dh >> 1;
@@ -177,7 +177,7 @@ dwconv_kernel(const T* __restrict__ g, const float* __restrict__ w, const float*
   for (int j = threadIdx.x >> 7; j < 32; j += 2) {
     const int r = r0 + j;
     if (r >= rows) break;
-    const int ci = clips.find(r, 1);
+    const int ci = clips.find(r, 1, 0);
     const int lo = clips.e(ci), hi = lo + clips.L2(ci);
     float v = 0.f;
     if (r >= lo && r < hi) {

@@ -71,9 +71,9 @@ struct Prof {
   uint32_t mask = 0;  // families whose launches are timed
   int64_t launches[PK_COUNT] = {};
   double ms[PK_COUNT] = {};
-  std::vector<cudaEvent_t> ev;  // pairs
-  std::vector<int> kind;        // per recorded pair
-  size_t used = 0;
+  std::vector<cudaEvent_t> ev;  // event pair i = (ev[2i], ev[2i+1])
+  std::vector<int> pair_kind;   // family of pair i (-1: recording failed)
+  int npairs = 0;               // pairs recorded since the last read
 };
 
 constexpr int kRing = 8;
@@ -154,14 +154,13 @@ template <class F>
 gam_status run_kernel(gam_ctx* c, int kind, cudaStream_t s, F&& launch) {
   Prof& p = c->prof;
   p.launches[kind]++;
-  const bool timed = ((p.mask >> kind) & 1u) && p.used + 2 <= p.ev.size();
-  if (timed) cudaEventRecord(p.ev[p.used], s);
-  cudaError_t e = launch();
-  if (timed) {
-    cudaEventRecord(p.ev[p.used + 1], s);
-    p.kind.push_back(kind);
-    p.used += 2;
+  int slot = -1;
+  if (((p.mask >> kind) & 1u) && p.npairs < (int)p.pair_kind.size()) {
+    slot = p.npairs++;
+    p.pair_kind[slot] = cudaEventRecord(p.ev[2 * slot], s) == cudaSuccess ? kind : -1;
   }
+  const cudaError_t e = launch();
+  if (slot >= 0 && cudaEventRecord(p.ev[2 * slot + 1], s) != cudaSuccess) p.pair_kind[slot] = -1;
   return cuda_check(c, e, kKindNames[kind]);
 }
 
@@ -714,6 +713,7 @@ gam_status alloc_workspace(gam_ctx* c) {
     GAM_TRY(cuda_check(c, cudaEventCreateWithFlags(&c->tab_ev[i], cudaEventDisableTiming), "event"));
   }
   c->prof.ev.resize(2 * 16384);
+  c->prof.pair_kind.assign(16384, -1);
   for (auto& e : c->prof.ev) GAM_TRY(cuda_check(c, cudaEventCreate(&e), "event"));
   return GAM_OK;
 }
@@ -797,6 +797,7 @@ gam_status gam_create(const gam_config* cfg, const gam_tensor* tensors, int n_te
   c->wdtype = cfg->precision == GAM_FP32 ? 0 : (cfg->precision == GAM_FP16 ? 1 : 2);
   c->d_head = cfg->d_model / cfg->n_heads;
   gam_status s = cuda_check(c, cudaSetDevice(device), "cudaSetDevice");
+  if (s == GAM_OK) s = cuda_check(c, tc_init(&c->tc, device), "tensor-core init");
   if (s == GAM_OK) s = alloc_workspace(c);
   if (s == GAM_OK) s = build_weights(c, tensors, n_tensors);
   if (s == GAM_OK) s = cuda_check(c, cudaDeviceSynchronize(), "create sync");
@@ -921,8 +922,7 @@ gam_status gam_profile_reset(gam_ctx* c) {
     c->prof.launches[k] = 0;
     c->prof.ms[k] = 0.0;
   }
-  c->prof.kind.clear();
-  c->prof.used = 0;
+  c->prof.npairs = 0;
   GAM_TRY(cuda_check(c, cudaMemset(c->dev_status, 0, 16), "status reset"));
   return cuda_check(c, tc_reset_status(&c->tc), "status reset");
 }
@@ -935,19 +935,41 @@ gam_status gam_profile_read(gam_ctx* c, int kind, double* total_ms, int64_t* lau
   GAM_TRY(enter(c));
   if (kind < 0 || kind >= PK_COUNT) return fail(c, GAM_ERR_INVALID_ARG, "bad kind");
   Prof& p = c->prof;
-  if (p.used) {
-    GAM_TRY(cuda_check(c, cudaEventSynchronize(p.ev[p.used - 1]), "profile sync"));
-    for (size_t i = 0; i < p.kind.size(); ++i) {
-      float ms = 0.f;
-      GAM_TRY(cuda_check(c, cudaEventElapsedTime(&ms, p.ev[2 * i], p.ev[2 * i + 1]), "event time"));
-      p.ms[p.kind[i]] += ms;
+  if (p.npairs > 0) {
+    GAM_TRY(cuda_check(c, cudaEventSynchronize(p.ev[2 * p.npairs - 1]), "profile sync"));
+    for (int i = 0; i < p.npairs; ++i) {
+      if (p.pair_kind[i] < 0) continue;
+      float t = 0.f;
+      GAM_TRY(cuda_check(c, cudaEventElapsedTime(&t, p.ev[2 * i], p.ev[2 * i + 1]), "event time"));
+      p.ms[p.pair_kind[i]] += (double)t;
     }
-    p.kind.clear();
-    p.used = 0;
+    p.npairs = 0;
   }
   if (total_ms) *total_ms = p.ms[kind];
   if (launches) *launches = p.launches[kind];
   return GAM_OK;
+}
+
+gam_status gam_debug_gemm(gam_ctx* c, int impl, const void* a, int lda, const void* w, const float* bias, int m, int n,
+                          int k, float* out, int ldo, void* stream) {
+  GAM_TRY(enter(c));
+  if (!a || !w || !bias || !out || m < 1 || n < 1 || k < 1 || lda < 1 || ldo < n)
+    return fail(c, GAM_ERR_INVALID_ARG, "bad gemm arguments");
+  cudaStream_t s = (cudaStream_t)stream;
+  c->last_stream = s;
+  EpiParams ep{};
+  ep.x = out;
+  ep.out = out;
+  ep.bias = bias;
+  ep.alpha = 1.f;
+  ep.ldo = ldo;
+  WeightOp W{w, nullptr, 1};
+  if (impl == 0) {
+    if (!tc_supported(1, 1, n, k, EPI_RESID)) return fail(c, GAM_ERR_SHAPE, "tensor-core GEMM needs N % 256 == 0, K % 64 == 0");
+    return run_kernel(c, PK_MISC, s, [&] { return launch_gemm_tc(&c->tc, a, nullptr, 0, lda, W, m, n, k, EPI_RESID, ep, s); });
+  }
+  if (k % 16 || n % 128) return fail(c, GAM_ERR_SHAPE, "CUDA-core GEMM needs N % 128 == 0, K % 16 == 0");
+  return run_kernel(c, PK_MISC, s, [&] { return launch_gemm_simt(1, a, nullptr, 0, lda, W, m, n, k, EPI_RESID, 0, ep, s); });
 }
 
 gam_status gam_debug_inject_cuda_error(gam_ctx* c, int cuda_error, int count) {

@@ -28,7 +28,7 @@ STATUS = {0: "GAM_OK", 1: "GAM_ERR_INVALID_ARG", 2: "GAM_ERR_SHAPE", 3: "GAM_ERR
 EXPORTS = ("gam_status_string", "gam_last_error", "gam_plan_lengths", "gam_create", "gam_destroy", "gam_logmel",
            "gam_encode", "gam_encode_stage", "gam_ctc_greedy", "gam_ctc_collapse", "gam_transcribe",
            "gam_device_status", "gam_profile_enable", "gam_profile_reset", "gam_profile_kinds",
-           "gam_profile_kind_name", "gam_profile_read", "gam_debug_inject_cuda_error")
+           "gam_profile_kind_name", "gam_profile_read", "gam_debug_gemm", "gam_debug_inject_cuda_error")
 
 
 class GamConfig(ctypes.Structure):
@@ -85,6 +85,8 @@ def lib() -> ctypes.CDLL:
         L.gam_profile_kind_name.restype = ctypes.c_char_p
         L.gam_profile_kind_name.argtypes = [ctypes.c_int]
         L.gam_profile_read.argtypes = [vp, ctypes.c_int, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_int64)]
+        L.gam_debug_gemm.argtypes = [vp, ctypes.c_int, vp, ctypes.c_int, vp, vp, ctypes.c_int, ctypes.c_int,
+                                     ctypes.c_int, vp, ctypes.c_int, vp]
         L.gam_debug_inject_cuda_error.argtypes = [vp, ctypes.c_int, ctypes.c_int]
         for name in EXPORTS:
             if name not in ("gam_status_string", "gam_last_error", "gam_profile_kind_name"):
@@ -306,6 +308,15 @@ def gam_profile_read(ctx: Context, kind: int) -> Tuple[float, int]:
 
 def gam_profile_all(ctx: Context) -> Dict[str, Tuple[float, int]]:
     return {gam_profile_kind_name(k): gam_profile_read(ctx, k) for k in range(gam_profile_kinds())}
+
+
+def gam_debug_gemm(ctx: Context, impl: int, a, w, bias, out, stream=None):
+    """out += a . w^T + bias (a, w fp16 CUDA tensors; bias, out fp32)."""
+    M, K = a.shape
+    N = w.shape[0]
+    _check(lib().gam_debug_gemm(ctx.handle, impl, a.data_ptr(), a.stride(0), w.data_ptr(), bias.data_ptr(), M, N, K,
+                                out.data_ptr(), out.stride(0), _stream(stream)), ctx)
+    return out
 
 
 def gam_debug_inject_cuda_error(ctx: Context, cuda_error: int, count: int = 1):

@@ -204,6 +204,19 @@ const char* gam_profile_kind_name(int kind);
  * events).  Launch counts are kept even when timing is off. */
 gam_status gam_profile_read(gam_ctx* ctx, int kind, double* total_ms, int64_t* launches);
 
+/* ---- kernel unit test (tests) ---- */
+
+/* One GEMM of the encoder's kind through the chosen implementation
+ * (impl 0 = tensor cores (tcgen05), 1 = CUDA cores): out[M, N] (device f32,
+ * row stride ldo) += A[M, K] . W[N, K]^T + bias[N], where A (row stride lda)
+ * and W are device fp16 and bias device f32.  N % 256 == 0 and K % 64 == 0
+ * for impl 0.  lda < k selects the strided convolution view of the
+ * subsampling convs: row r of A is rows 2r .. 2r+k/C-1 of a [rows, C] buffer
+ * with lda = 2C (C % 64 == 0), and the buffer must hold (m + 2) * lda
+ * elements.  Uses the residual-update epilogue of the encoder (alpha 1). */
+gam_status gam_debug_gemm(gam_ctx* ctx, int impl, const void* a_dev, int lda, const void* w_dev,
+                          const float* bias_dev, int m, int n, int k, float* out_dev, int ldo, void* stream);
+
 /* ---- host-side fault injection (tests) ---- */
 
 /* Make the next `count` CUDA-error checks of this context report

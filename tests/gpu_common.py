@@ -9,8 +9,13 @@ from conformer_speech_recognition_b200 import gam, synth
 
 # fp32 build mode: max |delta| per layer output (and per stage).
 TOL_FP32_LAYER = 1e-4
-# fp32 frontend: max |delta| of the log-mel features.
-TOL_LOGMEL = 1e-4
+# fp32 frontend: max |delta| of the log-mel features.  The DFT runs in fp32 with
+# blocked summation (10 partial sums of 32 samples): first-order error of a DFT
+# coefficient <= (32 + 10) u sum|x w cos|, u = 2^-24, so the relative error of a
+# power bin is <= 2 * 42 u * rho with rho = sum|x w cos| / |X| (<= ~40 for the
+# synthetic tones + noise floor): 2 * 42 * 6e-8 * 40 = 2.0e-4 on the log scale.
+# (The pages' own frontend ports report 3e-5 and 4.2e-4 against PyTorch fp32.)
+TOL_LOGMEL = 2e-4
 # fp16 / INT8 product modes: relative Frobenius error, max |delta|, argmax agreement.
 TOL_REL_FRO = 1e-2
 TOL_MAX_ABS = 5e-2

@@ -161,3 +161,21 @@ def test_transcribe_host_buffers_match_device_path():
     assert np.array_equal(cnt.cpu().numpy(), cnt_h)
     assert np.array_equal(tok.cpu().numpy(), tok_h)
     ctx.close()
+
+
+def test_fp32_subsampling_every_length_residue():
+    """Clips of F = 7 .. 22 frames (every F mod 4 and every L' mod 8, so the
+    segment layout is packed with and without slack) back to back: the
+    subsampling output of each clip matches the oracle."""
+    model = small_model(d=256, heads=4, ffn=512, layers=1, K=5)
+    cfg, W = config_and_weights(model, 34, "fp32")
+    lengths = [320 + 160 * (F - 1) + (F % 3) * 40 for F in range(7, 23)]
+    audio, lens = synth.random_audio(lengths, seed=13)
+    ctx = gam.gam_create(cfg, W, len(lens), int(max(lens)))
+    out = gam.gam_encode_stage(ctx, to_torch(audio), lens, 0, gam.STAGE_SUBSAMPLING).cpu().numpy()
+    _, el, _, _ = gam.gam_plan_lengths(cfg, lens)
+    for i in range(len(lens)):
+        _, dump = oracle_clip(audio[i], lens[i], W, cfg, dump=True, n_layers=0)
+        assert out[i, :el[i]].shape == dump["x0"].shape
+        assert max_abs(out[i, :el[i]], dump["x0"]) <= TOL_FP32_LAYER, i
+    ctx.close()

@@ -1,0 +1,48 @@
+"""Unit parity of the encoder's GEMM kernels through the C ABI (gam_debug_gemm):
+out += A . W^T + bias with fp16 operands and fp32 accumulation, for the
+tensor-core (tcgen05) and CUDA-core implementations, against NumPy in fp64."""
+import numpy as np
+import pytest
+
+from conformer_speech_recognition_b200 import gam
+from gpu_common import config_and_weights, small_model
+
+pytestmark = pytest.mark.gpu
+
+# fp32 accumulation of K fp16 products: relative to the largest output
+TOL_GEMM_REL = 2e-4
+
+
+@pytest.fixture(scope="module")
+def ctx():
+    cfg, W = config_and_weights(small_model(layers=1), 34, "fp16")
+    c = gam.gam_create(cfg, W, 1, 16000)
+    yield c
+    c.close()
+
+
+@pytest.mark.parametrize("impl", [0, 1], ids=["tcgen05", "cuda_cores"])
+@pytest.mark.parametrize("M,N,K,lda", [(128, 256, 64, 64), (300, 512, 320, 320), (1000, 768, 768, 768),
+                                       (5000, 3072, 768, 768), (2100, 256, 3072, 3072),
+                                       (777, 768, 320, 128)],
+                         ids=["one_tile", "ragged_m", "d768", "many_tiles", "deep_k", "strided_view"])
+def test_gemm_parity(ctx, impl, M, N, K, lda):
+    import torch
+    rng = np.random.default_rng(M + N + K)
+    rows_needed = (M - 1) * lda + K if lda >= K else (M + 2) * lda
+    flat = rng.normal(size=rows_needed).astype(np.float16)
+    A = np.lib.stride_tricks.as_strided(flat, shape=(M, K), strides=(lda * 2, 2))
+    Wt = rng.normal(size=(N, K)).astype(np.float16)
+    b = rng.normal(size=N).astype(np.float32)
+    out0 = rng.normal(size=(M, N)).astype(np.float32)
+    ta = torch.from_numpy(flat).cuda()
+    a_view = torch.as_strided(ta, (M, K), (lda, 1))
+    tw = torch.from_numpy(Wt).cuda()
+    tb = torch.from_numpy(b).cuda()
+    to = torch.from_numpy(out0.copy()).cuda()
+    gam.gam_debug_gemm(ctx, impl, a_view, tw, tb, to)
+    got = to.cpu().numpy()
+    ref = out0.astype(np.float64) + A.astype(np.float64) @ Wt.astype(np.float64).T + b
+    err = np.abs(got - ref).max() / np.abs(ref).max()
+    assert err <= TOL_GEMM_REL, err
+    gam.gam_device_status(ctx)
