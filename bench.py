@@ -90,6 +90,21 @@ def algorithmic_work(cfg, lens):
     return fl, by, launches
 
 
+def reduce_max_over_ranks(values, device=None):
+    """Element-wise max over all ranks (torch.distributed all_reduce MAX)."""
+    import torch
+    import torch.distributed as td
+    t = torch.tensor(list(values), dtype=torch.float64, device=device)
+    td.all_reduce(t, op=td.ReduceOp.MAX)
+    return [float(v) for v in t.tolist()]
+
+
+def job_throughput(world, audio_seconds_per_rank_step, steps, elapsed_ms):
+    """Whole-job audio-s/s: every rank processed its own batch each step; the job
+    took the slowest rank's time."""
+    return world * audio_seconds_per_rank_step * steps / (elapsed_ms / 1e3)
+
+
 class ClockSampler:
     """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
 
@@ -301,15 +316,13 @@ def run_ours(args, rank, world, local_rank):
     e2e_ms = e0.elapsed_time(e1)
 
     if dist:
-        t = torch.tensor([elapsed_ms, e2e_ms], dtype=torch.float64, device=dev)
-        td.all_reduce(t, op=td.ReduceOp.MAX)
-        elapsed_ms, e2e_ms = float(t[0]), float(t[1])
+        elapsed_ms, e2e_ms = reduce_max_over_ranks([elapsed_ms, e2e_ms], device=dev)
 
     if rank == 0:
         peaks = load_peaks()
         fl, by, _ = algorithmic_work(cfg, lens)
-        value = world * audio_seconds * args.steps / (elapsed_ms / 1e3)
-        e2e_value = world * audio_seconds * args.steps / (e2e_ms / 1e3)
+        value = job_throughput(world, audio_seconds, args.steps, elapsed_ms)
+        e2e_value = job_throughput(world, audio_seconds, args.steps, e2e_ms)
         avg_launch_ms = dom_ms / max(dom_n, 1)
         per_step_launches_dom = dom_n / args.steps
         if dominant in fl and dominant != "frontend":

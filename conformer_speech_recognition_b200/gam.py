@@ -283,8 +283,13 @@ def gam_device_status(ctx: Context):
     _check(lib().gam_device_status(ctx.handle), ctx)
 
 
-def gam_profile_enable(ctx: Context, on: bool = True):
-    _check(lib().gam_profile_enable(ctx.handle, 1 if on else 0), ctx)
+def gam_profile_enable(ctx: Context, mask=True):
+    """mask: True / -1 = every kernel family, False / 0 = none, else a bit mask of families."""
+    if mask is True:
+        mask = -1
+    elif mask is False:
+        mask = 0
+    _check(lib().gam_profile_enable(ctx.handle, int(mask)), ctx)
 
 
 def gam_profile_reset(ctx: Context):
