@@ -119,3 +119,12 @@ cudaError_t launch_collapse(const int* argmax, const int* lens, int batch, int t
 cudaError_t launch_f32_to_f16(const float* in, __half* out, int64_t n, cudaStream_t s);
 
 }  // namespace gam
+
+#include <string>
+
+namespace gam {
+
+// Error text of calls that take no context, returned by gam_last_error(NULL).
+void set_context_free_error(const std::string& msg);
+
+}  // namespace gam

@@ -741,6 +741,8 @@ gam_status enter(gam_ctx* c) {
 
 }  // namespace
 
+void gam::set_context_free_error(const std::string& msg) { g_create_error = msg; }
+
 extern "C" {
 
 const char* gam_status_string(gam_status s) {

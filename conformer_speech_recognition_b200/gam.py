@@ -28,7 +28,10 @@ STATUS = {0: "GAM_OK", 1: "GAM_ERR_INVALID_ARG", 2: "GAM_ERR_SHAPE", 3: "GAM_ERR
 EXPORTS = ("gam_status_string", "gam_last_error", "gam_plan_lengths", "gam_create", "gam_destroy", "gam_logmel",
            "gam_encode", "gam_encode_stage", "gam_ctc_greedy", "gam_ctc_collapse", "gam_transcribe",
            "gam_device_status", "gam_profile_enable", "gam_profile_reset", "gam_profile_kinds",
-           "gam_profile_kind_name", "gam_profile_read", "gam_debug_gemm", "gam_debug_inject_cuda_error")
+           "gam_profile_kind_name", "gam_profile_read", "gam_ctc_collapse_noalloc", "gam_debug_gemm",
+           "gam_debug_inject_cuda_error")
+
+GAM_NOALLOC_MAX_FRAMES = 1 << 20
 
 
 class GamConfig(ctypes.Structure):
@@ -85,6 +88,7 @@ def lib() -> ctypes.CDLL:
         L.gam_profile_kind_name.restype = ctypes.c_char_p
         L.gam_profile_kind_name.argtypes = [ctypes.c_int]
         L.gam_profile_read.argtypes = [vp, ctypes.c_int, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_int64)]
+        L.gam_ctc_collapse_noalloc.argtypes = [vp, vp, ctypes.c_int, ctypes.c_int, ctypes.c_int, vp, vp, vp]
         L.gam_debug_gemm.argtypes = [vp, ctypes.c_int, vp, ctypes.c_int, vp, vp, ctypes.c_int, ctypes.c_int,
                                      ctypes.c_int, vp, ctypes.c_int, vp]
         L.gam_debug_inject_cuda_error.argtypes = [vp, ctypes.c_int, ctypes.c_int]
@@ -313,6 +317,18 @@ def gam_profile_read(ctx: Context, kind: int) -> Tuple[float, int]:
 
 def gam_profile_all(ctx: Context) -> Dict[str, Tuple[float, int]]:
     return {gam_profile_kind_name(k): gam_profile_read(ctx, k) for k in range(gam_profile_kinds())}
+
+
+def gam_ctc_collapse_noalloc(logits, lengths_dev, tokens, counts, stream=None):
+    """Greedy decoding with no context and no allocation inside the call.
+
+    logits: CUDA f32 [B, T, C]; lengths_dev: CUDA int32 [B]; tokens (CUDA int32
+    [B, T]) and counts (CUDA int32 [B]) are written.  The caller allocates all
+    four; the library keeps its per-frame scratch in a fixed device array."""
+    B, T, C = logits.shape
+    _check(lib().gam_ctc_collapse_noalloc(logits.data_ptr(), lengths_dev.data_ptr(), B, T, C, tokens.data_ptr(),
+                                          counts.data_ptr(), _stream(stream)))
+    return tokens, counts
 
 
 def gam_debug_gemm(ctx: Context, impl: int, a, w, bias, out, stream=None):

@@ -111,8 +111,9 @@ typedef struct gam_ctx gam_ctx;
 /* Human-readable name of a status code (static storage). */
 const char* gam_status_string(gam_status status);
 
-/* Text of the last error seen by this context ("" if none; NULL ctx gives the
- * last error of a failed gam_create on this thread). */
+/* Text of the last error seen by this context ("" if none).  A NULL ctx gives
+ * the last error on this thread of the calls that take no context
+ * (gam_create, gam_plan_lengths, gam_ctc_collapse_noalloc). */
 const char* gam_last_error(const gam_ctx* ctx);
 
 /* Host-only length planning for `batch` clips of `lengths_host[i]` samples.
@@ -203,6 +204,33 @@ const char* gam_profile_kind_name(int kind);
 /* Totals since the last reset for family `kind` (synchronises the recorded
  * events).  Launch counts are kept even when timing is off. */
 gam_status gam_profile_read(gam_ctx* ctx, int kind, double* total_ms, int64_t* launches);
+
+/* ---- greedy decoding without any allocation ---- */
+
+/* Frames of the fixed scratch array behind gam_ctc_collapse_noalloc. */
+#define GAM_NOALLOC_MAX_FRAMES (1 << 20)
+
+/* The pages have no counterpart of this call: it is a service for callers
+ * that must not allocate device memory -- code that cannot afford the device
+ * synchronisation a cudaMalloc may cause, plug-ins whose host framework owns
+ * all device memory, or callers without a gam_ctx.  Same result as
+ * gam_ctc_collapse (argmax = lowest index of the fp32 maximum, runs merged,
+ * then blanks dropped; tokens -1 after the last one), but it takes no context
+ * and allocates nothing: the per-frame argmax it needs lives in a file-scope
+ * device array of GAM_NOALLOC_MAX_FRAMES ints (4 MiB) that every GPU loading
+ * the library keeps until the process exits.
+ *   logits_dev  device f32 [batch, t_max, n_classes]; blank = n_classes - 1
+ *   lengths_dev device i32 [batch]: valid frames per clip, clamped to [0, t_max]
+ *   tokens_dev  device i32 [batch, t_max]; counts_dev device i32 [batch]
+ * batch * t_max above GAM_NOALLOC_MAX_FRAMES fails with GAM_ERR_CAPACITY
+ * before any launch (text in gam_last_error(NULL)).  The first call on a
+ * device (that device current) looks up the array's device address once;
+ * make that first call before any stream capture.  All calls on a device
+ * share the array and each fully rewrites the part it reads, so nothing needs
+ * clearing, but calls whose GPU work overlaps (other streams or threads) race
+ * on it.  Runs on the current device and on `stream`. */
+gam_status gam_ctc_collapse_noalloc(const float* logits_dev, const int32_t* lengths_dev, int batch, int t_max,
+                                    int n_classes, int32_t* tokens_dev, int32_t* counts_dev, void* stream);
 
 /* ---- kernel unit test (tests) ---- */
 
