@@ -3,16 +3,18 @@
 // A [M, K] fp16 (row stride lda; a strided view for the subsampling convs),
 // B [N, K] fp16 weight (PyTorch Linear layout), fp32 accumulation in TMEM.
 //
-// Persistent, warp-specialised CTA of 192 threads, one CTA per SM:
+// Persistent, warp-specialised CTA of 320 threads, one CTA per SM:
 //   warp 0      one thread issues TMA loads of 128x64 A and BNx64 B tiles
 //               (128-byte swizzle) into a STAGES-deep shared-memory ring;
 //   warp 1      allocates 2*BN TMEM columns (two accumulators) and one thread
 //               issues tcgen05.mma (M=128, N=BN, K=16) per 16-wide K slice,
 //               committing stage releases and accumulator-ready barriers;
-//   warps 2..5  epilogue: tcgen05.ld of the accumulator (warp w reads TMEM
-//               lanes 32*(w%4) .. +31 = its 32 output rows), bias + activation
-//               / residual / scatter, global stores; then hand the
-//               accumulator back so the next tile's MMAs overlap this epilogue.
+//   warps 2..9  epilogue: tcgen05.ld of the accumulator (warp w reads TMEM
+//               lanes 32*(w%4) .. +31 = its 32 output rows, and one half of
+//               the tile's columns, so two warps share each sub-partition and
+//               hide each other's latency), bias + activation / residual /
+//               scatter, global stores; then hand the accumulator back so the
+//               next tile's MMAs overlap this epilogue.
 // Tiles are visited n-fastest so the CTAs in flight share each A row block
 // through L2 and the weight (a few MB) stays L2-resident.
 // Every mbarrier wait is bounded (tc_common.cuh); a wait that gives up raises
@@ -52,7 +54,21 @@ struct Cfg {
   static constexpr size_t SMEM = (size_t)STAGES * STAGE + 1024 + 256;
 };
 
-__device__ __forceinline__ float sigm(float v) { return 1.f / (1.f + __expf(-v)); }
+// Logistic function with the fast exp / divide intrinsics (|rel err| ~ 1e-6,
+// far below the fp16 rounding of the stored result).
+__device__ __forceinline__ float sigm(float v) { return __fdividef(1.f, 1.f + __expf(-v)); }
+
+__device__ __forceinline__ void load_bias32(const float* b, float (&v)[32]) {
+  const float4* p = reinterpret_cast<const float4*>(b);
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    const float4 t = __ldg(p + j);
+    v[4 * j] = t.x;
+    v[4 * j + 1] = t.y;
+    v[4 * j + 2] = t.z;
+    v[4 * j + 3] = t.w;
+  }
+}
 
 __device__ __forceinline__ void store_half16(__half* dst, const float* v) {
   uint4 w[2];
@@ -67,15 +83,17 @@ __device__ __forceinline__ void store_half16(__half* dst, const float* v) {
 }
 
 // Epilogue of one 32-column accumulator chunk of row r (columns n .. n+31).
+template <int EPI>
 __device__ __forceinline__ void epi_chunk(const TcArgs& p, int r, int n, bool valid, const uint32_t (&u)[32]) {
   const EpiParams& ep = p.ep;
   float v[32];
+  load_bias32(ep.bias + n, v);
 #pragma unroll
-  for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(u[j]) + __ldg(ep.bias + n + j);
-  switch (p.epi) {
+  for (int j = 0; j < 32; ++j) v[j] += __uint_as_float(u[j]);
+  switch (EPI) {
     case EPI_SWISH: {
 #pragma unroll
-      for (int j = 0; j < 32; ++j) v[j] = v[j] * sigm(v[j]);
+      for (int j = 0; j < 32; ++j) v[j] = __fdividef(v[j], 1.f + __expf(-v[j]));
       __half* o = reinterpret_cast<__half*>(ep.out) + (size_t)r * ep.ldo + n;
       store_half16(o, v);
       store_half16(o + 16, v + 16);
@@ -129,21 +147,24 @@ __device__ __forceinline__ void epi_chunk(const TcArgs& p, int r, int n, bool va
   }
 }
 
-template <int BN>
-__device__ __forceinline__ void epilogue_tile(const TcArgs& p, int r, int n0, uint32_t tbase) {
+// Epilogue of columns [c_lo, c_hi) of a tile for row r (this warp's half).
+template <int BN, int EPI>
+__device__ __forceinline__ void epilogue_tile(const TcArgs& p, int r, int n0, uint32_t tbase, int c_lo, int c_hi) {
   const EpiParams& ep = p.ep;
   const bool in_m = r < p.M;
   bool valid = in_m;
-  if (in_m && (p.epi == EPI_CONV1 || p.epi == EPI_CONV2)) {
-    const int scale = p.epi == EPI_CONV1 ? 2 : 1;
-    const int ci = ep.clips.find(r, scale, scale == 2 ? 2 : 0);
-    const int t = r - (p.epi == EPI_CONV1 ? 2 * ep.clips.e(ci) + 2 : ep.clips.e(ci));
-    valid = t >= 0 && t < (p.epi == EPI_CONV1 ? ep.clips.L1(ci) : ep.clips.L2(ci));
+  if (EPI == EPI_CONV1 || EPI == EPI_CONV2) {
+    if (in_m) {
+      constexpr int scale = EPI == EPI_CONV1 ? 2 : 1;
+      const int ci = ep.clips.find(r, scale, scale == 2 ? 2 : 0);
+      const int t = r - (scale * ep.clips.e(ci) + (scale == 2 ? 2 : 0));
+      valid = t >= 0 && t < (EPI == EPI_CONV1 ? ep.clips.L1(ci) : ep.clips.L2(ci));
+    }
   }
-  if (p.epi == EPI_GLU) {
+  if (EPI == EPI_GLU) {
     // weight rows interleaved in blocks of 64: [value 64 | gate 64] per 128 columns
 #pragma unroll 1
-    for (int blk = 0; blk < BN; blk += 128) {
+    for (int blk = c_lo; blk < c_hi; blk += 128) {
 #pragma unroll 1
       for (int hh = 0; hh < 64; hh += 32) {
         uint32_t a[32], g[32];
@@ -152,11 +173,12 @@ __device__ __forceinline__ void epilogue_tile(const TcArgs& p, int r, int n0, ui
         tmem_ld_wait();
         if (!in_m) continue;
         const int nv = n0 + blk + hh, ng = nv + 64;
-        float y[32];
+        float bv[32], bg[32], y[32];
+        load_bias32(ep.bias + nv, bv);
+        load_bias32(ep.bias + ng, bg);
 #pragma unroll
         for (int j = 0; j < 32; ++j)
-          y[j] = (__uint_as_float(a[j]) + __ldg(ep.bias + nv + j)) *
-                 sigm(__uint_as_float(g[j]) + __ldg(ep.bias + ng + j));
+          y[j] = (__uint_as_float(a[j]) + bv[j]) * sigm(__uint_as_float(g[j]) + bg[j]);
         __half* o = reinterpret_cast<__half*>(ep.out) + (size_t)r * ep.ldo + (n0 + blk) / 2 + hh;
         store_half16(o, y);
         store_half16(o + 16, y + 16);
@@ -165,16 +187,19 @@ __device__ __forceinline__ void epilogue_tile(const TcArgs& p, int r, int n0, ui
     return;
   }
 #pragma unroll 1
-  for (int c = 0; c < BN; c += 32) {
+  for (int c = c_lo; c < c_hi; c += 32) {
     uint32_t u[32];
     tmem_ld32(tbase + c, u);
     tmem_ld_wait();
-    if (in_m) epi_chunk(p, r, n0 + c, valid, u);
+    if (in_m) epi_chunk<EPI>(p, r, n0 + c, valid, u);
   }
 }
 
-template <int BN, int STAGES>
-__global__ void __launch_bounds__(192, 1)
+constexpr int kEpiWarps = 8;
+constexpr int kThreads = 64 + 32 * kEpiWarps;
+
+template <int BN, int STAGES, int EPI>
+__global__ void __launch_bounds__(kThreads, 1)
 gemm_tc_kernel(const __grid_constant__ CUtensorMap mA, const __grid_constant__ CUtensorMap mA2,
                const __grid_constant__ CUtensorMap mB, const TcArgs p) {
   using C = Cfg<BN, STAGES>;
@@ -198,7 +223,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap mA, const __grid_constant__ C
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&tfull[a], 1);
-      mbar_init(&tempty[a], 4);
+      mbar_init(&tempty[a], kEpiWarps);
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -292,7 +317,8 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap mA, const __grid_constant__ C
         }
     }
   } else {
-    const int q = warp & 3;
+    const int q = warp & 3;                       // TMEM lane quarter of this warp
+    const int half = (warp - 2) / 4;              // which half of the tile's columns
     int local = 0;
     for (int tile = blockIdx.x; tile < p.tiles; tile += gridDim.x, ++local) {
       const int acc = local & 1;
@@ -302,7 +328,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap mA, const __grid_constant__ C
       const int nb = tile % p.n_blocks, mb = tile / p.n_blocks;
       const int r = mb * BM + q * 32 + lane;
       const uint32_t tbase = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN);
-      epilogue_tile<BN>(p, r, nb * BN, tbase);
+      epilogue_tile<BN, EPI>(p, r, nb * BN, tbase, half * (BN / 2), (half + 1) * (BN / 2));
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&tempty[acc]);
@@ -348,16 +374,30 @@ cudaError_t make_map_f16(CUtensorMap* m, const void* ptr, uint64_t inner, uint64
   return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
-template <int BN, int STAGES>
-cudaError_t launch_bn(TcGemmCache* cache, const CUtensorMap& mA, const CUtensorMap& mA2, const CUtensorMap& mB,
-                      const TcArgs& args, cudaStream_t s) {
+template <int BN, int STAGES, int EPI>
+cudaError_t launch_epi(TcGemmCache* cache, const CUtensorMap& mA, const CUtensorMap& mA2, const CUtensorMap& mB,
+                       const TcArgs& args, cudaStream_t s) {
   using C = Cfg<BN, STAGES>;
-  auto kern = gemm_tc_kernel<BN, STAGES>;
+  auto kern = gemm_tc_kernel<BN, STAGES, EPI>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::SMEM);
   if (e != cudaSuccess) return e;
   const int grid = args.tiles < cache->sm_count ? args.tiles : cache->sm_count;
-  kern<<<grid, 192, C::SMEM, s>>>(mA, mA2, mB, args);
+  kern<<<grid, kThreads, C::SMEM, s>>>(mA, mA2, mB, args);
   return cudaGetLastError();
+}
+
+template <int BN, int STAGES>
+cudaError_t launch_bn(TcGemmCache* cache, const CUtensorMap& mA, const CUtensorMap& mA2, const CUtensorMap& mB,
+                      const TcArgs& args, cudaStream_t s) {
+  switch (args.epi) {
+    case EPI_SWISH: return launch_epi<BN, STAGES, EPI_SWISH>(cache, mA, mA2, mB, args, s);
+    case EPI_GLU: return launch_epi<BN, STAGES, EPI_GLU>(cache, mA, mA2, mB, args, s);
+    case EPI_RESID: return launch_epi<BN, STAGES, EPI_RESID>(cache, mA, mA2, mB, args, s);
+    case EPI_QKV: return launch_epi<BN, STAGES, EPI_QKV>(cache, mA, mA2, mB, args, s);
+    case EPI_CONV1: return launch_epi<BN, STAGES, EPI_CONV1>(cache, mA, mA2, mB, args, s);
+    case EPI_CONV2: return launch_epi<BN, STAGES, EPI_CONV2>(cache, mA, mA2, mB, args, s);
+    default: return cudaErrorInvalidValue;
+  }
 }
 
 }  // namespace

@@ -156,41 +156,134 @@ ln_rope_kernel(const float* __restrict__ x, const float* __restrict__ g, const f
     }
 }
 
-// Depthwise conv: CTA = 32 rows x 128 channels; input rows [r0 - pad, r0 + 32 + pad)
-// staged in shared memory; w is tap-major [K][d] with BatchNorm folded in.
-template <typename T>
+// Depthwise conv + folded BatchNorm + Swish.  CTA = 64 rows x 128 channels,
+// 256 threads: thread (channel c, row half h) produces rows 32h .. 32h+31 of
+// channel c in 4 groups of 8, sliding over the staged input rows so each
+// shared-memory value feeds up to 8 outputs.  Weights (tap-major [K][d], BN
+// folded) live in registers.  Clip bounds are looked up once per row; rows
+// whose whole window lies inside their clip skip the per-tap checks.
+template <typename T, int K>
 __global__ void __launch_bounds__(256)
 dwconv_kernel(const T* __restrict__ g, const float* __restrict__ w, const float* __restrict__ bias, Clips clips,
-              T* __restrict__ out, int rows, int d, int K) {
-  __shared__ float tile[94][128];
-  const int pad = (K - 1) / 2;
-  const int r0 = blockIdx.x * 32, c0 = blockIdx.y * 128;
-  const int nrow = 32 + 2 * pad;
-  for (int idx = threadIdx.x; idx < nrow * 128; idx += 256) {
-    const int rr = idx >> 7, cc = idx & 127;
-    const int src = r0 - pad + rr;
-    tile[rr][cc] = (src >= 0 && src < rows) ? ld1(g + (size_t)src * d + c0 + cc) : 0.f;
+              T* __restrict__ out, int rows, int d) {
+  constexpr int PAD = (K - 1) / 2, R = 64, HALO = R + 2 * PAD;
+  __shared__ float tile[HALO][128];
+  __shared__ int s_lo[R], s_hi[R];
+  const int r0 = blockIdx.x * R, c0 = blockIdx.y * 128;
+  for (int idx = threadIdx.x; idx < HALO * 16; idx += 256) {  // 16 x 8 channels per row
+    const int rr = idx >> 4, c8 = (idx & 15) * 8;
+    const int src = r0 - PAD + rr;
+    float v[8];
+    if (src >= 0 && src < rows) {
+      if constexpr (sizeof(T) == 2) {
+        const uint4 raw = *reinterpret_cast<const uint4*>(g + (size_t)src * d + c0 + c8);
+        const __half2* h2 = reinterpret_cast<const __half2*>(&raw);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float2 f = __half22float2(h2[e]);
+          v[2 * e] = f.x;
+          v[2 * e + 1] = f.y;
+        }
+      } else {
+        const float4 a = *reinterpret_cast<const float4*>(g + (size_t)src * d + c0 + c8);
+        const float4 b = *reinterpret_cast<const float4*>(g + (size_t)src * d + c0 + c8 + 4);
+        v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w; v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+      }
+    } else {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) v[e] = 0.f;
+    }
+#pragma unroll
+    for (int e = 0; e < 8; ++e) tile[rr][c8 + e] = v[e];
+  }
+  if (threadIdx.x < R) {
+    const int r = r0 + threadIdx.x;
+    int lo = 0, hi = 0;
+    if (r < rows) {
+      const int ci = clips.find(r, 1, 0);
+      lo = clips.e(ci);
+      hi = lo + clips.L2(ci);
+    }
+    s_lo[threadIdx.x] = lo;
+    s_hi[threadIdx.x] = hi;
   }
   __syncthreads();
   const int cc = threadIdx.x & 127, c = c0 + cc;
+  float wk[K];
+#pragma unroll
+  for (int k = 0; k < K; ++k) wk[k] = __ldg(w + (size_t)k * d + c);
   const float bv = __ldg(bias + c);
-  for (int j = threadIdx.x >> 7; j < 32; j += 2) {
-    const int r = r0 + j;
-    if (r >= rows) break;
-    const int ci = clips.find(r, 1, 0);
-    const int lo = clips.e(ci), hi = lo + clips.L2(ci);
-    float v = 0.f;
-    if (r >= lo && r < hi) {
-      float acc = bv;
-      for (int k = 0; k < K; ++k) {
-        const int src = r + k - pad;
-        if (src >= lo && src < hi) acc = fmaf(__ldg(w + (size_t)k * d + c), tile[j + k][cc], acc);
+  const int rbase = (threadIdx.x >> 7) * 32;
+#pragma unroll 1
+  for (int grp = 0; grp < 4; ++grp) {
+    const int j0 = rbase + grp * 8;  // first tile row of this group
+    const int lo = s_lo[j0], hi = s_hi[j0];
+    const bool same = s_lo[j0 + 7] == lo;
+    const int r = r0 + j0;
+    float acc[8];
+    if (same && r - PAD >= lo && r + 7 + PAD < hi) {
+      // interior: every tap of the 8 rows is inside the clip
+#pragma unroll
+      for (int i = 0; i < 8; ++i) acc[i] = bv;
+#pragma unroll
+      for (int t = 0; t < K + 7; ++t) {
+        const float x = tile[j0 + t][cc];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const int k = t - i;
+          if (k >= 0 && k < K) acc[i] = fmaf(wk[k], x, acc[i]);
+        }
       }
-      v = acc / (1.f + __expf(-acc));
+#pragma unroll
+      for (int i = 0; i < 8; ++i) acc[i] = __fdividef(acc[i], 1.f + __expf(-acc[i]));
+    } else {
+#pragma unroll 1
+      for (int i = 0; i < 8; ++i) {
+        const int ri = r + i, li = s_lo[j0 + i], hiI = s_hi[j0 + i];
+        float a = 0.f;
+        if (ri >= li && ri < hiI) {
+          a = bv;
+#pragma unroll
+          for (int k = 0; k < K; ++k) {
+            const int src = ri + k - PAD;
+            if (src >= li && src < hiI) a = fmaf(wk[k], tile[j0 + i + k][cc], a);
+          }
+          a = __fdividef(a, 1.f + __expf(-a));
+        }
+        acc[i] = a;
+      }
     }
-    if constexpr (sizeof(T) == 2) out[(size_t)r * d + c] = __float2half_rn(v);
-    else out[(size_t)r * d + c] = v;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      if (r + i >= rows) break;
+      if constexpr (sizeof(T) == 2) out[(size_t)(r + i) * d + c] = __float2half_rn(acc[i]);
+      else out[(size_t)(r + i) * d + c] = acc[i];
+    }
   }
+}
+
+// Any other odd kernel size (<= 63): one output per thread and tap loop.
+template <typename T>
+__global__ void __launch_bounds__(256)
+dwconv_generic_kernel(const T* __restrict__ g, const float* __restrict__ w, const float* __restrict__ bias,
+                      Clips clips, T* __restrict__ out, int rows, int d, int K) {
+  const int pad = (K - 1) / 2;
+  const size_t idx = (size_t)blockIdx.x * 256 + threadIdx.x;
+  if (idx >= (size_t)rows * d) return;
+  const int r = (int)(idx / d), c = (int)(idx % d);
+  const int ci = clips.find(r, 1, 0);
+  const int lo = clips.e(ci), hi = lo + clips.L2(ci);
+  float a = 0.f;
+  if (r >= lo && r < hi) {
+    a = __ldg(bias + c);
+    for (int k = 0; k < K; ++k) {
+      const int src = r + k - pad;
+      if (src >= lo && src < hi) a = fmaf(__ldg(w + (size_t)k * d + c), ld1(g + (size_t)src * d + c), a);
+    }
+    a = __fdividef(a, 1.f + __expf(-a));
+  }
+  if constexpr (sizeof(T) == 2) out[idx] = __float2half_rn(a);
+  else out[idx] = a;
 }
 
 __global__ void scatter_kernel(const float* __restrict__ x, Clips clips, float* __restrict__ out, int t_max, int d) {
@@ -323,13 +416,27 @@ cudaError_t launch_layernorm_rope(const float* x, const float* g, const float* b
   return cudaGetLastError();
 }
 
+template <typename T>
+cudaError_t dwconv_t(const void* g, const float* w, const float* bias, Clips clips, void* out, int rows, int d, int K,
+                     cudaStream_t s) {
+  dim3 grid((rows + 63) / 64, d / 128);
+  const T* gi = (const T*)g;
+  T* o = (T*)out;
+  if (K == 31) dwconv_kernel<T, 31><<<grid, 256, 0, s>>>(gi, w, bias, clips, o, rows, d);
+  else if (K == 5) dwconv_kernel<T, 5><<<grid, 256, 0, s>>>(gi, w, bias, clips, o, rows, d);
+  else if (K == 15) dwconv_kernel<T, 15><<<grid, 256, 0, s>>>(gi, w, bias, clips, o, rows, d);
+  else {
+    const size_t n = (size_t)rows * d;
+    dwconv_generic_kernel<T><<<(unsigned)((n + 255) / 256), 256, 0, s>>>(gi, w, bias, clips, o, rows, d, K);
+  }
+  return cudaGetLastError();
+}
+
 cudaError_t launch_dwconv(const void* g, const float* w, const float* bias, Clips clips, void* out, int t_half,
                           int rows, int d, int K, cudaStream_t s) {
   if (d % 128 || K > 63 || (K & 1) == 0) return cudaErrorInvalidValue;
-  dim3 grid((rows + 31) / 32, d / 128);
-  if (t_half) dwconv_kernel<__half><<<grid, 256, 0, s>>>((const __half*)g, w, bias, clips, (__half*)out, rows, d, K);
-  else dwconv_kernel<float><<<grid, 256, 0, s>>>((const float*)g, w, bias, clips, (float*)out, rows, d, K);
-  return cudaGetLastError();
+  if (t_half) return dwconv_t<__half>(g, w, bias, clips, out, rows, d, K, s);
+  return dwconv_t<float>(g, w, bias, clips, out, rows, d, K, s);
 }
 
 cudaError_t launch_scatter_out(const float* x, Clips clips, float* out, int t_max, int d, cudaStream_t s) {
