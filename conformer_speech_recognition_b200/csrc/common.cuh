@@ -81,9 +81,10 @@ enum ProfKind {
 
 // Weight operand of a GEMM: [N, K] row-major (PyTorch Linear layout).
 struct WeightOp {
-  const void* w;       // float / __half / int8 [N, K]
-  const __half* scale; // int8 only: [N, K/64]
-  int dtype;           // 0 f32, 1 f16, 2 int8-g64
+  const void* w;         // float / __half / int8 [N, K]
+  const __half* scale;   // int8 only: [N, K/64]
+  int dtype;             // 0 f32, 1 f16, 2 int8-g64
+  const __half* scale_t; // int8 only: the same scales transposed to [K/64, N]
 };
 
 // --- launchers (return cudaGetLastError()) ---------------------------------

@@ -43,13 +43,16 @@ struct TcArgs {
   int conv_c;   // 0: plain A [M, K]; else A row r = input rows 2r .. 2r+taps-1 of C = conv_c channels
   int epi;
   EpiParams ep;
+  const __half* scale_t;  // INT8 weights: fp16 scales transposed to [K/64][N]
   int* status;
 };
 
-template <int BN, int STAGES>
+template <int BN, int STAGES, bool QB>
 struct Cfg {
-  static constexpr int B_TILE = BN * BK * 2;
-  static constexpr int STAGE = A_TILE + B_TILE;
+  static constexpr int B_TILE = BN * BK * 2;                 // fp16 B operand (128-byte swizzle)
+  static constexpr int RAW_TILE = QB ? BN * BK : 0;          // INT8 weights as loaded (64-byte rows)
+  static constexpr int TX = A_TILE + (QB ? RAW_TILE : B_TILE);  // bytes landed by TMA per stage
+  static constexpr int STAGE = A_TILE + B_TILE + RAW_TILE;
   static constexpr int TMEM_COLS = 2 * BN;  // power of two for BN in {128, 256}
   static constexpr size_t SMEM = (size_t)STAGES * STAGE + 1024 + 256;
 };
@@ -161,7 +164,7 @@ __device__ __forceinline__ void epilogue_tile(const TcArgs& p, int r, int n0, ui
       valid = t >= 0 && t < (EPI == EPI_CONV1 ? ep.clips.L1(ci) : ep.clips.L2(ci));
     }
   }
-  if (EPI == EPI_GLU) {
+  if constexpr (EPI == EPI_GLU) {
     // weight rows interleaved in blocks of 64: [value 64 | gate 64] per 128 columns
 #pragma unroll 1
     for (int blk = c_lo; blk < c_hi; blk += 128) {
@@ -184,35 +187,61 @@ __device__ __forceinline__ void epilogue_tile(const TcArgs& p, int r, int n0, ui
         store_half16(o + 16, y + 16);
       }
     }
-    return;
-  }
+  } else {
 #pragma unroll 1
-  for (int c = c_lo; c < c_hi; c += 32) {
-    uint32_t u[32];
-    tmem_ld32(tbase + c, u);
-    tmem_ld_wait();
-    if (in_m) epi_chunk<EPI>(p, r, n0 + c, valid, u);
+    for (int c = c_lo; c < c_hi; c += 32) {
+      uint32_t u[32];
+      tmem_ld32(tbase + c, u);
+      tmem_ld_wait();
+      if (in_m) epi_chunk<EPI>(p, r, n0 + c, valid, u);
+    }
   }
 }
 
 constexpr int kEpiWarps = 8;
-constexpr int kThreads = 64 + 32 * kEpiWarps;
+constexpr int kCvtWarps = 4;  // INT8 variant: warps that dequantise the weight tile
+template <bool QB>
+constexpr int threads_of() { return 64 + 32 * kEpiWarps + (QB ? 32 * kCvtWarps : 0); }
 
-template <int BN, int STAGES, int EPI>
-__global__ void __launch_bounds__(kThreads, 1)
+// INT8 -> fp16 dequantisation of one 16-byte chunk (16 weights of one row)
+// into two 16-byte chunks of the swizzled fp16 operand.  An int8 x becomes
+// exactly x in fp16 by writing the byte x + 128 into the low mantissa bits of
+// 1024.0 (fp16 0x6400, where the spacing is exactly 1) and subtracting 1152;
+// the product with the group scale is then rounded once to fp16.
+__device__ __forceinline__ void dequant16(uint4 raw, __half2 s2, uint4& out0, uint4& out1) {
+  const __half2 off = __floats2half2_rn(1152.f, 1152.f);
+  const uint32_t w[4] = {raw.x ^ 0x80808080u, raw.y ^ 0x80808080u, raw.z ^ 0x80808080u, raw.w ^ 0x80808080u};
+  uint32_t o[8];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    uint32_t lo = __byte_perm(w[i], 0x64646464u, 0x4140);
+    uint32_t hi = __byte_perm(w[i], 0x64646464u, 0x4342);
+    __half2 hl = __hmul2(__hsub2(*reinterpret_cast<__half2*>(&lo), off), s2);
+    __half2 hh = __hmul2(__hsub2(*reinterpret_cast<__half2*>(&hi), off), s2);
+    o[2 * i] = *reinterpret_cast<uint32_t*>(&hl);
+    o[2 * i + 1] = *reinterpret_cast<uint32_t*>(&hh);
+  }
+  out0 = make_uint4(o[0], o[1], o[2], o[3]);
+  out1 = make_uint4(o[4], o[5], o[6], o[7]);
+}
+
+template <int BN, int STAGES, int EPI, bool QB>
+__global__ void __launch_bounds__(threads_of<QB>(), 1)
 gemm_tc_kernel(const __grid_constant__ CUtensorMap mA, const __grid_constant__ CUtensorMap mA2,
                const __grid_constant__ CUtensorMap mB, const TcArgs p) {
-  using C = Cfg<BN, STAGES>;
+  using C = Cfg<BN, STAGES, QB>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
   uint8_t* sA = base;
   uint8_t* sB = base + STAGES * A_TILE;
+  uint8_t* sRaw = sB + STAGES * C::B_TILE;  // INT8 variant only
   uint64_t* full = reinterpret_cast<uint64_t*>(base + STAGES * C::STAGE);
   uint64_t* empty = full + STAGES;
   uint64_t* tfull = empty + STAGES;
   uint64_t* tempty = tfull + 2;
   uint64_t* drain = tempty + 2;
-  uint32_t* tslot = reinterpret_cast<uint32_t*>(drain + 1);
+  uint64_t* bready = drain + 1;  // [STAGES], INT8 variant: dequantised B tile written
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(bready + STAGES);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tslot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -226,6 +255,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap mA, const __grid_constant__ C
       mbar_init(&tempty[a], kEpiWarps);
     }
     mbar_init(drain, 1);
+    for (int st = 0; st < STAGES; ++st) mbar_init(&bready[st], kCvtWarps);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -263,9 +293,10 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap mA, const __grid_constant__ C
             ax = (t & 1) * p.conv_c + c0;
             ay = m0 + (t >> 1);
           }
-          mbar_arrive_expect_tx(&full[s], C::STAGE);
+          mbar_arrive_expect_tx(&full[s], C::TX);
           tma_load_2d(sA + s * A_TILE, ma, &full[s], ax, ay);
-          tma_load_2d(sB + s * C::B_TILE, &mB, &full[s], kb * BK, n0);
+          if (QB) tma_load_2d(sRaw + s * C::RAW_TILE, &mB, &full[s], kb * BK, n0);
+          else tma_load_2d(sB + s * C::B_TILE, &mB, &full[s], kb * BK, n0);
           ++it;
         }
       }
@@ -293,7 +324,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap mA, const __grid_constant__ C
         const uint32_t d = tmem + (uint32_t)(acc * BN);
         for (int kb = 0; kb < KB; ++kb) {
           const int s = it % STAGES;
-          if (!mbar_wait(&full[s], (it / STAGES) & 1, abort_flag)) {
+          if (!mbar_wait(QB ? &bready[s] : &full[s], (it / STAGES) & 1, abort_flag)) {
             ok = false;
             break;
           }
@@ -315,6 +346,40 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap mA, const __grid_constant__ C
           *abort_flag = 1;
           break;
         }
+    }
+  } else if (QB && warp >= 2 + kEpiWarps) {
+    // converter warps: INT8 tile (BN rows x 64 B) -> fp16 swizzled operand (BN rows x 128 B)
+    const int t = threadIdx.x - 32 * (2 + kEpiWarps);  // 0 .. 127
+    const int ch = t & 3;                              // 16-byte chunk of a 64-byte INT8 row
+    int it = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; tile < p.tiles && ok; tile += gridDim.x) {
+      const int n0 = (tile % p.n_blocks) * BN;
+      for (int kb = 0; kb < KB; ++kb) {
+        const int s = it % STAGES;
+        if (!mbar_wait(&full[s], (it / STAGES) & 1, abort_flag)) {
+          ok = false;
+          break;
+        }
+        const uint8_t* raw = sRaw + s * C::RAW_TILE;
+        uint8_t* dst = sB + s * C::B_TILE;
+        const __half* sc = p.scale_t + (size_t)kb * p.N + n0;
+#pragma unroll 4
+        for (int pass = 0; pass < BN / 32; ++pass) {
+          const int row = pass * 32 + (t >> 2);
+          const uint4 q = *reinterpret_cast<const uint4*>(raw + row * 64 + ch * 16);
+          const __half sv = __ldg(sc + row);
+          uint4 o0, o1;
+          dequant16(q, __half2(sv, sv), o0, o1);
+          uint8_t* drow = dst + (row >> 3) * 1024 + (row & 7) * 128;
+          *reinterpret_cast<uint4*>(drow + (((2 * ch) ^ (row & 7)) << 4)) = o0;
+          *reinterpret_cast<uint4*>(drow + (((2 * ch + 1) ^ (row & 7)) << 4)) = o1;
+        }
+        fence_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bready[s]);
+        ++it;
+      }
     }
   } else {
     const int q = warp & 3;                       // TMEM lane quarter of this warp
@@ -374,28 +439,42 @@ cudaError_t make_map_f16(CUtensorMap* m, const void* ptr, uint64_t inner, uint64
   return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
-template <int BN, int STAGES, int EPI>
+// 2D INT8 tensor map, no swizzle (64-byte rows of the raw weight tile).
+cudaError_t make_map_i8(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t outer, uint32_t box_inner,
+                        uint32_t box_outer) {
+  if ((reinterpret_cast<uintptr_t>(ptr) & 15) || (inner & 15)) return cudaErrorInvalidValue;
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {inner};
+  cuuint32_t box[2] = {box_inner, box_outer};
+  cuuint32_t es[2] = {1, 1};
+  CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(ptr), dims, strides, box, es,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+template <int BN, int STAGES, int EPI, bool QB>
 cudaError_t launch_epi(TcGemmCache* cache, const CUtensorMap& mA, const CUtensorMap& mA2, const CUtensorMap& mB,
                        const TcArgs& args, cudaStream_t s) {
-  using C = Cfg<BN, STAGES>;
-  auto kern = gemm_tc_kernel<BN, STAGES, EPI>;
+  using C = Cfg<BN, STAGES, QB>;
+  auto kern = gemm_tc_kernel<BN, STAGES, EPI, QB>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::SMEM);
   if (e != cudaSuccess) return e;
   const int grid = args.tiles < cache->sm_count ? args.tiles : cache->sm_count;
-  kern<<<grid, kThreads, C::SMEM, s>>>(mA, mA2, mB, args);
+  kern<<<grid, threads_of<QB>(), C::SMEM, s>>>(mA, mA2, mB, args);
   return cudaGetLastError();
 }
 
-template <int BN, int STAGES>
+template <int BN, int STAGES, bool QB>
 cudaError_t launch_bn(TcGemmCache* cache, const CUtensorMap& mA, const CUtensorMap& mA2, const CUtensorMap& mB,
                       const TcArgs& args, cudaStream_t s) {
   switch (args.epi) {
-    case EPI_SWISH: return launch_epi<BN, STAGES, EPI_SWISH>(cache, mA, mA2, mB, args, s);
-    case EPI_GLU: return launch_epi<BN, STAGES, EPI_GLU>(cache, mA, mA2, mB, args, s);
-    case EPI_RESID: return launch_epi<BN, STAGES, EPI_RESID>(cache, mA, mA2, mB, args, s);
-    case EPI_QKV: return launch_epi<BN, STAGES, EPI_QKV>(cache, mA, mA2, mB, args, s);
-    case EPI_CONV1: return launch_epi<BN, STAGES, EPI_CONV1>(cache, mA, mA2, mB, args, s);
-    case EPI_CONV2: return launch_epi<BN, STAGES, EPI_CONV2>(cache, mA, mA2, mB, args, s);
+    case EPI_SWISH: return launch_epi<BN, STAGES, EPI_SWISH, QB>(cache, mA, mA2, mB, args, s);
+    case EPI_GLU: return launch_epi<BN, STAGES, EPI_GLU, QB>(cache, mA, mA2, mB, args, s);
+    case EPI_RESID: return launch_epi<BN, STAGES, EPI_RESID, QB>(cache, mA, mA2, mB, args, s);
+    case EPI_QKV: return launch_epi<BN, STAGES, EPI_QKV, QB>(cache, mA, mA2, mB, args, s);
+    case EPI_CONV1: return launch_epi<BN, STAGES, EPI_CONV1, QB>(cache, mA, mA2, mB, args, s);
+    case EPI_CONV2: return launch_epi<BN, STAGES, EPI_CONV2, QB>(cache, mA, mA2, mB, args, s);
     default: return cudaErrorInvalidValue;
   }
 }
@@ -403,7 +482,7 @@ cudaError_t launch_bn(TcGemmCache* cache, const CUtensorMap& mA, const CUtensorM
 }  // namespace
 
 bool tc_supported(int a_dtype, int b_dtype, int N, int K, int epi) {
-  return a_dtype == 1 && b_dtype == 1 && N % 256 == 0 && K % 64 == 0 && K >= 64 &&
+  return a_dtype == 1 && (b_dtype == 1 || b_dtype == 2) && N % 256 == 0 && K % 64 == 0 && K >= 64 &&
          (epi == EPI_SWISH || epi == EPI_GLU || epi == EPI_RESID || epi == EPI_QKV || epi == EPI_CONV1 ||
           epi == EPI_CONV2);
 }
@@ -421,6 +500,8 @@ cudaError_t tc_init(TcGemmCache* cache, int device) {
 cudaError_t launch_gemm_tc(TcGemmCache* cache, const void* A, const void* A2, int n_split, int lda, WeightOp B, int M,
                            int N, int K, int epi, const EpiParams& ep, cudaStream_t s) {
   if (!tc_supported(1, B.dtype, N, K, epi) || M <= 0) return cudaErrorInvalidValue;
+  const bool qb = B.dtype == 2;
+  if (qb && !B.scale_t) return cudaErrorInvalidValue;
   constexpr int BN = 256;
   // lda < K: stride-2 convolution view (lda = 2C, K = taps * C, C % 64 == 0); the
   // buffer behind it holds (M + 2) * lda elements, mapped as M + 2 rows of 2C.
@@ -431,7 +512,7 @@ cudaError_t launch_gemm_tc(TcGemmCache* cache, const void* A, const void* A2, in
                        : make_map_f16(&mA, A, K, M, (uint64_t)lda * 2, BK, BM);
   if (e == cudaSuccess && !conv) e = make_map_f16(&mA2, A2 ? A2 : A, K, M, (uint64_t)lda * 2, BK, BM);
   if (conv) mA2 = mA;
-  if (e == cudaSuccess) e = make_map_f16(&mB, B.w, K, N, (uint64_t)K * 2, BK, BN);
+  if (e == cudaSuccess) e = qb ? make_map_i8(&mB, B.w, K, N, BK, BN) : make_map_f16(&mB, B.w, K, N, (uint64_t)K * 2, BK, BN);
   if (e != cudaSuccess) return e;
   TcArgs args;
   args.M = M;
@@ -444,8 +525,10 @@ cudaError_t launch_gemm_tc(TcGemmCache* cache, const void* A, const void* A2, in
   args.conv_c = conv ? lda / 2 : 0;
   args.epi = epi;
   args.ep = ep;
+  args.scale_t = B.scale_t;
   args.status = cache->status;
-  return launch_bn<BN, 4>(cache, mA, mA2, mB, args, s);
+  if (qb) return launch_bn<BN, 3, true>(cache, mA, mA2, mB, args, s);
+  return launch_bn<BN, 4, false>(cache, mA, mA2, mB, args, s);
 }
 
 cudaError_t launch_attention(TcGemmCache* cache, const void* qk, const void* vt, Clips clips, void* o, int t_half,

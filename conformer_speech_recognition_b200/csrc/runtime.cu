@@ -50,11 +50,12 @@ int seg_rows(const ClipLen& l) {
 }
 
 struct DevLinear {
-  void* w = nullptr;        // [N, K] f32 / f16 / int8
-  __half* scale = nullptr;  // int8: [N, K/64]
-  float* b = nullptr;       // [N]
+  void* w = nullptr;          // [N, K] f32 / f16 / int8
+  __half* scale = nullptr;    // int8: [N, K/64]
+  __half* scale_t = nullptr;  // int8: [K/64, N]
+  float* b = nullptr;         // [N]
   int N = 0, K = 0, dtype = 0;
-  WeightOp op() const { return WeightOp{w, scale, dtype}; }
+  WeightOp op() const { return WeightOp{w, scale, dtype, scale_t}; }
 };
 struct DevLN {
   float* g = nullptr;
@@ -290,6 +291,11 @@ gam_status upload_linear(gam_ctx* c, const HostLinear& l, DevLinear& d) {
   GAM_TRY(upload_f32(c, &d.b, l.b));
   if (l.dtype == 2) {
     GAM_TRY(upload(c, (int8_t**)&d.w, l.q.data(), l.q.size()));
+    const int G = l.K / 64;
+    std::vector<__half> st((size_t)G * l.N);
+    for (int n = 0; n < l.N; ++n)
+      for (int g = 0; g < G; ++g) st[(size_t)g * l.N + n] = l.s[(size_t)n * G + g];
+    GAM_TRY(upload(c, &d.scale_t, st.data(), st.size() * sizeof(__half)));
     return upload(c, &d.scale, l.s.data(), l.s.size() * sizeof(__half));
   }
   if (l.dtype == 0) {
@@ -965,7 +971,7 @@ gam_status gam_debug_gemm(gam_ctx* c, int impl, const void* a, int lda, const vo
   ep.bias = bias;
   ep.alpha = 1.f;
   ep.ldo = ldo;
-  WeightOp W{w, nullptr, 1};
+  WeightOp W{w, nullptr, 1, nullptr};
   if (impl == 0) {
     if (!tc_supported(1, 1, n, k, EPI_RESID)) return fail(c, GAM_ERR_SHAPE, "tensor-core GEMM needs N % 256 == 0, K % 64 == 0");
     return run_kernel(c, PK_MISC, s, [&] { return launch_gemm_tc(&c->tc, a, nullptr, 0, lda, W, m, n, k, EPI_RESID, ep, s); });
