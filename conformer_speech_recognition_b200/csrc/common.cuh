@@ -55,7 +55,7 @@ enum EpiKind {
   EPI_QKV = 3,       // scatter to Q/K head-major (padded to 64) and V^T
   EPI_CONV1 = 4,     // out_t = relu(acc + b), zero outside conv1 clip rows
   EPI_CONV2 = 5,     // x (fp32) = relu(acc + b), zero outside encoder clip rows
-  EPI_F32 = 6        // out_f32[r, n] = acc + b[n] (n < N)
+  EPI_F32 = 6        // out_f32[r, n] = acc + b[n] (n < n_valid, or N when n_valid == 0)
 };
 
 struct EpiParams {
@@ -69,6 +69,7 @@ struct EpiParams {
   void* qk;           // [2][H][rows_pad][64]
   void* vt;           // [H][64][rows_pad]
   int rows_pad, n_heads, d_head, d_model;
+  int n_valid;        // EPI_F32: columns stored (the padded weight rows beyond it are skipped)
 };
 
 // Kernel families for profiling (order = gam_profile_kind_name order).
@@ -113,8 +114,14 @@ cudaError_t launch_dwconv(const void* g, const float* w, const float* bias, Clip
 cudaError_t launch_scatter_out(const float* x, Clips clips, float* out, int t_max, int d, cudaStream_t s);
 cudaError_t launch_attention_simt(const void* qk, const void* vt, Clips clips, void* o, int t_half,
                                   int rows_pad, int n_heads, int d_head, int t_max, cudaStream_t s);
+// logits row of frame (b, t): b * t_max + t, or off[b] + t when off (per-clip
+// offsets of the compacted valid frames, B + 1 entries) is given.
 cudaError_t launch_logsoftmax_argmax(const float* logits, int ld, const int* lens, int batch, int t_max,
-                                     int C, float* logp, int* argmax, cudaStream_t s);
+                                     int C, float* logp, int* argmax, cudaStream_t s, const int* off = nullptr);
+// Valid frames of enc [B, t_max, d] (fp32) compacted to rows off[b] + t and
+// split into fp16 hi and lo parts: a[v, c] = hi, a[v, d + c] = lo (x ~= hi + lo).
+cudaError_t launch_split_hi_lo(const float* enc, const int* off, int batch, int t_max, int d, int rows,
+                               __half* a, cudaStream_t s);
 cudaError_t launch_collapse(const int* argmax, const int* lens, int batch, int t_max, int blank,
                             int* tokens, int* counts, cudaStream_t s);
 cudaError_t launch_f32_to_f16(const float* in, __half* out, int64_t n, cudaStream_t s);

@@ -145,6 +145,13 @@ __device__ __forceinline__ void epi_chunk(const TcArgs& p, int r, int n, bool va
         }
       }
     } break;
+    case EPI_F32: {
+      float* o = reinterpret_cast<float*>(ep.out) + (size_t)r * ep.ldo + n;
+      const int lim = ep.n_valid - n;
+#pragma unroll
+      for (int j = 0; j < 32; ++j)
+        if (j < lim) o[j] = v[j];
+    } break;
     default:
       break;
   }
@@ -475,6 +482,7 @@ cudaError_t launch_bn(TcGemmCache* cache, const CUtensorMap& mA, const CUtensorM
     case EPI_QKV: return launch_epi<BN, STAGES, EPI_QKV, QB>(cache, mA, mA2, mB, args, s);
     case EPI_CONV1: return launch_epi<BN, STAGES, EPI_CONV1, QB>(cache, mA, mA2, mB, args, s);
     case EPI_CONV2: return launch_epi<BN, STAGES, EPI_CONV2, QB>(cache, mA, mA2, mB, args, s);
+    case EPI_F32: return launch_epi<BN, STAGES, EPI_F32, QB>(cache, mA, mA2, mB, args, s);
     default: return cudaErrorInvalidValue;
   }
 }
@@ -484,7 +492,7 @@ cudaError_t launch_bn(TcGemmCache* cache, const CUtensorMap& mA, const CUtensorM
 bool tc_supported(int a_dtype, int b_dtype, int N, int K, int epi) {
   return a_dtype == 1 && (b_dtype == 1 || b_dtype == 2) && N % 256 == 0 && K % 64 == 0 && K >= 64 &&
          (epi == EPI_SWISH || epi == EPI_GLU || epi == EPI_RESID || epi == EPI_QKV || epi == EPI_CONV1 ||
-          epi == EPI_CONV2);
+          epi == EPI_CONV2 || epi == EPI_F32);
 }
 
 cudaError_t tc_init(TcGemmCache* cache, int device) {

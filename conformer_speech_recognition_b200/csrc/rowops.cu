@@ -302,7 +302,7 @@ __global__ void scatter_kernel(const float* __restrict__ x, Clips clips, float* 
 
 __global__ void logsoftmax_argmax_kernel(const float* __restrict__ logits, int ld, const int* __restrict__ lens,
                                          int batch, int t_max, int C, float* __restrict__ logp,
-                                         int* __restrict__ argmax) {
+                                         int* __restrict__ argmax, const int* __restrict__ off) {
   const int row = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
   if (row >= batch * t_max) return;
   const int b = row / t_max, t = row - b * t_max;
@@ -312,7 +312,7 @@ __global__ void logsoftmax_argmax_kernel(const float* __restrict__ logits, int l
     if (lane == 0) argmax[row] = -1;
     return;
   }
-  const float* z = logits + (size_t)row * ld;
+  const float* z = logits + (size_t)(off ? __ldg(off + b) + t : row) * ld;
   float best = -INFINITY;
   int bi = 0x7fffffff;
   for (int c = lane; c < C; c += 32) {
@@ -375,6 +375,32 @@ collapse_kernel(const int* __restrict__ argmax, const int* __restrict__ lens, in
   const int total = s_total;
   for (int t = total + tid; t < t_max; t += 256) tok[t] = -1;
   if (tid == 0) counts[b] = total;
+}
+
+// One warp per valid frame v: find its clip b (largest b with off[b] <= v),
+// read enc[b, v - off[b], :] and write the fp16 hi / lo split.
+__global__ void split_hi_lo_kernel(const float* __restrict__ enc, const int* __restrict__ off, int batch, int t_max,
+                                   int d, int rows, __half* __restrict__ a) {
+  const int v = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+  if (v >= rows) return;
+  int lo = 0, hi = batch - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (__ldg(off + mid) <= v) lo = mid; else hi = mid - 1;
+  }
+  const int t = v - __ldg(off + lo);
+  const float* x = enc + ((size_t)lo * t_max + t) * d;
+  __half* ah = a + (size_t)v * 2 * d;
+  for (int c = lane * 4; c < d; c += 128) {
+    const float4 f = *reinterpret_cast<const float4*>(x + c);
+    const __half2 h0 = __floats2half2_rn(f.x, f.y), h1 = __floats2half2_rn(f.z, f.w);
+    const float2 b0 = __half22float2(h0), b1 = __half22float2(h1);
+    const __half2 l0 = __floats2half2_rn(f.x - b0.x, f.y - b0.y), l1 = __floats2half2_rn(f.z - b1.x, f.w - b1.y);
+    *reinterpret_cast<__half2*>(ah + c) = h0;
+    *reinterpret_cast<__half2*>(ah + c + 2) = h1;
+    *reinterpret_cast<__half2*>(ah + d + c) = l0;
+    *reinterpret_cast<__half2*>(ah + d + c + 2) = l1;
+  }
 }
 
 __global__ void f32_to_f16_kernel(const float* __restrict__ in, __half* __restrict__ out, int64_t n) {
@@ -446,9 +472,17 @@ cudaError_t launch_scatter_out(const float* x, Clips clips, float* out, int t_ma
 }
 
 cudaError_t launch_logsoftmax_argmax(const float* logits, int ld, const int* lens, int batch, int t_max, int C,
-                                     float* logp, int* argmax, cudaStream_t s) {
+                                     float* logp, int* argmax, cudaStream_t s, const int* off) {
   const int rows = batch * t_max;
-  logsoftmax_argmax_kernel<<<(rows + 7) / 8, 256, 0, s>>>(logits, ld, lens, batch, t_max, C, logp, argmax);
+  logsoftmax_argmax_kernel<<<(rows + 7) / 8, 256, 0, s>>>(logits, ld, lens, batch, t_max, C, logp, argmax, off);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_split_hi_lo(const float* enc, const int* off, int batch, int t_max, int d, int rows, __half* a,
+                               cudaStream_t s) {
+  if (rows <= 0) return cudaSuccess;
+  if (d % 128) return cudaErrorInvalidValue;
+  split_hi_lo_kernel<<<(rows + 7) / 8, 256, 0, s>>>(enc, off, batch, t_max, d, rows, a);
   return cudaGetLastError();
 }
 

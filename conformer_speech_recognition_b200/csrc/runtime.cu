@@ -93,6 +93,8 @@ struct gam_ctx {
   float* basis = nullptr;  // [320][320]
   float* fb = nullptr;     // [161][64]
   DevLinear conv1, conv2, head;
+  DevLinear head2;         // tensor-core CTC head: [W | W] padded to a multiple of 256 rows, K = 2d
+  __half* ctc_a = nullptr; // [rows, 2d] fp16 hi / lo split of the valid encoder frames
   std::vector<DevLayer> layers;
   float* rope_cos = nullptr;  // [T2_cap][d_head/2]
   float* rope_sin = nullptr;
@@ -419,7 +421,7 @@ gam_status upload_ints(gam_ctx* c, const int32_t* src, int n, cudaStream_t s, co
 // ---- GEMM dispatch: tensor cores for fp16 / int8, CUDA cores for fp32 ----
 gam_status gemm(gam_ctx* c, int kind, cudaStream_t s, const void* A, const void* A2, int n_split, int lda,
                 const DevLinear& W, int M, int epi, float alpha, void* out, int ldo, const Clips& clips,
-                int a_f32 = 0) {
+                int a_f32 = 0, int n_valid = 0) {
   EpiParams ep{};
   ep.out = out;
   ep.x = (float*)out;
@@ -433,6 +435,7 @@ gam_status gemm(gam_ctx* c, int kind, cudaStream_t s, const void* A, const void*
   ep.n_heads = c->cfg.n_heads;
   ep.d_head = c->d_head;
   ep.d_model = c->cfg.d_model;
+  ep.n_valid = n_valid ? n_valid : W.N;
   const int a_dtype = a_f32 ? 0 : (c->act_half ? 1 : 0);
   if (tc_supported(a_dtype, W.dtype, W.N, W.K, epi)) {
     return run_kernel(c, kind, s, [&] {
@@ -541,14 +544,36 @@ gam_status run_ctc(gam_ctx* c, const float* enc, const int32_t* enc_len, int bat
   for (int i = 0; i < batch; ++i)
     if (enc_len[i] < 0 || enc_len[i] > t_max) return fail(c, GAM_ERR_SHAPE, "enc_len outside [0, t_max]");
   c->last_stream = s;
-  const int* lens;
-  GAM_TRY(upload_ints(c, enc_len, batch, s, &lens));
+  // lengths and the offsets of the compacted valid frames, one upload
+  std::vector<int32_t> lo(2 * batch + 1);
+  for (int i = 0; i < batch; ++i) lo[i] = enc_len[i];
+  lo[batch] = 0;
+  for (int i = 0; i < batch; ++i) lo[batch + 1 + i] = lo[batch + i] + enc_len[i];
+  const int M_valid = lo[2 * batch];
+  const int* dev;
+  GAM_TRY(upload_ints(c, lo.data(), 2 * batch + 1, s, &dev));
+  const int* lens = dev;
+  const int* off = dev + batch;
   const int C = cfg.n_classes, M = batch * t_max;
   Clips none{nullptr, 0};
-  GAM_TRY(gemm(c, PK_CTC_GEMM, s, enc, nullptr, 0, cfg.d_model, c->head, M, EPI_F32, 1.f, c->logits, C, none, 1));
-  GAM_TRY(run_kernel(c, PK_CTC_SOFTMAX, s, [&] {
-    return launch_logsoftmax_argmax(c->logits, C, lens, batch, t_max, C, logp, c->argmax, s);
-  }));
+  if (c->head2.w) {
+    // tensor cores: logits = [hi | lo] . [W | W]^T on the valid frames only
+    if (M_valid > 0) {
+      GAM_TRY(run_kernel(c, PK_CTC_GEMM, s, [&] {
+        return launch_split_hi_lo(enc, off, batch, t_max, cfg.d_model, M_valid, c->ctc_a, s);
+      }));
+      GAM_TRY(gemm(c, PK_CTC_GEMM, s, c->ctc_a, nullptr, 0, 2 * cfg.d_model, c->head2, M_valid, EPI_F32, 1.f,
+                   c->logits, C, none, 0, C));
+    }
+    GAM_TRY(run_kernel(c, PK_CTC_SOFTMAX, s, [&] {
+      return launch_logsoftmax_argmax(c->logits, C, lens, batch, t_max, C, logp, c->argmax, s, off);
+    }));
+  } else {
+    GAM_TRY(gemm(c, PK_CTC_GEMM, s, enc, nullptr, 0, cfg.d_model, c->head, M, EPI_F32, 1.f, c->logits, C, none, 1));
+    GAM_TRY(run_kernel(c, PK_CTC_SOFTMAX, s, [&] {
+      return launch_logsoftmax_argmax(c->logits, C, lens, batch, t_max, C, logp, c->argmax, s);
+    }));
+  }
   return run_kernel(c, PK_CTC_COLLAPSE, s, [&] {
     return launch_collapse(c->argmax, lens, batch, t_max, C - 1, tokens, counts, s);
   });
@@ -663,6 +688,34 @@ gam_status build_weights(gam_ctx* c, const gam_tensor* tensors, int n) {
     HostLinear hl;
     GAM_TRY(read_linear(c, t, "head", cfg.n_classes, d, q8, hl));
     GAM_TRY(upload_linear(c, hl, c->head));
+    if (cfg.precision != GAM_FP32) {
+      // [W | W] with zero rows up to a multiple of 256: one fp16 tensor-core GEMM of
+      // the hi / lo split activations gives fp32-grade logits
+      const int Cp = (int)round_up(cfg.n_classes, 256);
+      HostLinear h2;
+      h2.N = Cp;
+      h2.K = 2 * d;
+      h2.dtype = hl.dtype;
+      h2.b.assign(Cp, 0.0);
+      for (int n = 0; n < cfg.n_classes; ++n) h2.b[n] = hl.b[n];
+      if (hl.dtype == 2) {
+        h2.q.assign((size_t)Cp * 2 * d, 0);
+        h2.s.assign((size_t)Cp * (2 * d / 64), __float2half(1.f));
+        const int G = d / 64;
+        for (int n = 0; n < cfg.n_classes; ++n) {
+          for (int h = 0; h < 2; ++h) {
+            std::memcpy(&h2.q[(size_t)n * 2 * d + h * d], &hl.q[(size_t)n * d], d);
+            for (int g = 0; g < G; ++g) h2.s[(size_t)n * 2 * G + h * G + g] = hl.s[(size_t)n * G + g];
+          }
+        }
+      } else {
+        h2.w.assign((size_t)Cp * 2 * d, 0.0);
+        for (int n = 0; n < cfg.n_classes; ++n)
+          for (int h = 0; h < 2; ++h)
+            std::memcpy(&h2.w[(size_t)n * 2 * d + h * d], &hl.w[(size_t)n * d], d * sizeof(double));
+      }
+      GAM_TRY(upload_linear(c, h2, c->head2));
+    }
   }
   // RoPE tables, base rope_base, positions 0 .. T2_cap - 1
   {
@@ -703,6 +756,7 @@ gam_status alloc_workspace(gam_ctx* c) {
   const int64_t ctc_rows = (int64_t)cfg.max_batch * c->T2_cap;
   GAM_TRY(dev_alloc(c, (void**)&c->logits, (size_t)ctc_rows * cfg.n_classes * 4));
   GAM_TRY(dev_alloc(c, (void**)&c->argmax, (size_t)ctc_rows * 4));
+  if (cfg.precision != GAM_FP32) GAM_TRY(dev_alloc(c, (void**)&c->ctc_a, (size_t)ctc_rows * 2 * cfg.d_model * 2));
   GAM_TRY(dev_alloc(c, (void**)&c->audio_stage, (size_t)cfg.max_batch * cfg.max_samples * 4));
   GAM_TRY(dev_alloc(c, (void**)&c->enc_stage, (size_t)ctc_rows * d * 4));
   GAM_TRY(dev_alloc(c, (void**)&c->tokens_stage, (size_t)ctc_rows * 4));
@@ -712,7 +766,7 @@ gam_status alloc_workspace(gam_ctx* c) {
   GAM_TRY(cuda_check(c, cudaMemset(c->qk, 0, (size_t)2 * H * E * 64 * es), "memset"));
   GAM_TRY(cuda_check(c, cudaMemset(c->vt, 0, (size_t)H * 64 * E * es), "memset"));
   GAM_TRY(cuda_check(c, cudaMemset(c->dev_status, 0, 16), "memset"));
-  const size_t tab_ints = 5 * (size_t)(cfg.max_batch + 1) + 16;
+  const size_t tab_ints = 5 * (size_t)(cfg.max_batch + 1) + 16;  // also >= 2 * max_batch + 1
   for (int i = 0; i < kRing; ++i) {
     GAM_TRY(cuda_check(c, cudaMallocHost((void**)&c->tab_host[i], tab_ints * 4), "cudaMallocHost"));
     GAM_TRY(dev_alloc(c, (void**)&c->tab_dev[i], tab_ints * 4));

@@ -87,3 +87,30 @@ def test_ctc_greedy_head_parity(small_ctx):
         ref = oracle.greedy_collapse(a, cfg["n_classes"] - 1)
         if clear.all():
             assert tok[b, :cnt[b]].tolist() == ref
+
+
+@pytest.mark.parametrize("precision,C", [("fp16", 34), ("fp16", 257), ("int8_g64", 257)])
+def test_ctc_greedy_tensor_core_head(precision, C):
+    """fp16 / INT8 contexts run the head on tensor cores with the fp32 frames
+    split into fp16 hi + lo parts, so the activations keep ~22 bits.  fp16
+    weights are exact: log-probs within 1e-4 of the oracle.  INT8 weights are
+    dequantised in the mainloop and q*s is rounded once to fp16 (rms relative
+    error 2^-11/sqrt(3) ~ 2.8e-4 per weight): here |z| ~ sqrt(256) * 0.02 = 0.32,
+    so the logit error has sigma ~ 9e-5 and its maximum over the 38k values of
+    this test stays below ~5 sigma: bound 1e-3 for INT8."""
+    cfg, W = config_and_weights(small_model(layers=1), C, precision)
+    ctx = gam.gam_create(cfg, W, 6, 100000)
+    rng = np.random.default_rng(C)
+    B, T, d = 5, 150, cfg["d_model"]
+    enc = rng.normal(size=(B, T, d)).astype(np.float32)
+    lens = np.array([150, 0, 1, 77, 149], np.int32)
+    tok, cnt, logp = gam.gam_ctc_greedy(ctx, to_torch(enc), lens, want_logp=True)
+    tok, cnt, logp = tok.cpu().numpy(), cnt.cpu().numpy(), logp.cpu().numpy()
+    for b in range(B):
+        z, lp, a = oracle.ctc_head(enc[b, :lens[b]].astype(np.float64), W)
+        assert max_abs(logp[b, :lens[b]], lp) < (1e-3 if precision == "int8_g64" else 1e-4)
+        assert np.all(logp[b, lens[b]:] == 0)
+        zs = np.sort(z, axis=1) if lens[b] else np.zeros((0, 2))
+        if np.all(zs[:, -1] - zs[:, -2] > 2e-3):
+            assert tok[b, :cnt[b]].tolist() == oracle.greedy_collapse(a, C - 1)
+    ctx.close()
