@@ -90,6 +90,24 @@ def algorithmic_work(cfg, lens):
     return fl, by, launches
 
 
+def measured_traffic(workload, family):
+    """DRAM bytes per launch of `family` from the committed ncu summary
+    (profiles/traffic.json), or None when there is none for this workload or the
+    kernel source changed since the counters were taken."""
+    import hashlib
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            entry = json.load(f)[workload][family]
+        src = os.path.join(ROOT, entry["kernel_source"])
+        with open(src, "rb") as f:
+            if hashlib.sha256(f.read()).hexdigest()[:16] != entry["kernel_source_sha256_16"]:
+                return None
+        return entry["bytes_per_launch"]
+    except (OSError, KeyError, ValueError):
+        return None
+
+
 def reduce_max_over_ranks(values, device=None):
     """Element-wise max over all ranks (torch.distributed all_reduce MAX)."""
     import torch
@@ -336,14 +354,15 @@ def run_ours(args, rank, world, local_rank):
             achieved = per_launch / (avg_launch_ms / 1e3) / 1e12
             peak = peaks["bf16_tflops_sustained"]
             roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                    "frac": achieved / peak, "traffic": None, "kernel": dominant,
+                    "frac": achieved / peak, "traffic": measured_traffic(name, dominant), "kernel": dominant,
                     "peak_source": f"{peaks['source']} bf16 sustained (fp16 dense rate equal to bf16)"}
         else:
             per_launch = by.get(dominant, 0.0) / max(per_step_launches_dom, 1)
             achieved = per_launch / (avg_launch_ms / 1e3) / 1e9
             peak = peaks["hbm_gbs"]
             roof = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
-                    "traffic": None, "kernel": dominant, "peak_source": f"{peaks['source']} HBM copy"}
+                    "traffic": measured_traffic(name, dominant), "kernel": dominant,
+                    "peak_source": f"{peaks['source']} HBM copy"}
         gemm_flops = sum(v for k, v in fl.items() if k.startswith("gemm_"))
         # GEMM kernel time per step from the profiled steps (every family timed there)
         gemm_ms = sum(v[0] for k, v in warm.items() if k.startswith("gemm_")) / n_prof
