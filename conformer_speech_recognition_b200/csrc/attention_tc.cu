@@ -12,10 +12,13 @@
 //   warp 1      TMEM allocation; one thread issues S = Q K^T (M=128, N=128,
 //               K=d_head) into TMEM, then O_blk = P V (M=128, N=d_head,
 //               K=128) with P read from shared memory;
-//   warps 2..5  softmax, one query row per thread (TMEM lane): two passes
-//               over the S row (max, then exp2 / row sum / fp16 P written
-//               into the swizzled shared-memory operand layout), then
-//               O = O * corr + O_blk in registers.
+//   warps 2..5  softmax, one query row per thread (TMEM lane): pass 1 takes
+//               the row max of S (overlapping the previous block's P.V),
+//               pass 2 writes exp2 / fp16 P into the swizzled shared-memory
+//               operand layout.  O accumulates in TMEM across key blocks; it
+//               is rescaled in place (tcgen05.ld / st) only when the running
+//               max rises by more than 2^8, and divided by the row sum at the
+//               end.
 // Q, K come from the head-major buffer [2][H][rows][64] (head dim padded to
 // 64) and V from V^T [H][64][rows]; clip starts are multiples of 8 rows so
 // every TMA x coordinate is 16-byte aligned.  All waits are bounded.
@@ -46,14 +49,29 @@ struct AttnArgs {
   int* status;
 };
 
-__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
   asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
-      "%15}, [%16];"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
-        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
-      : "r"(taddr));
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+      "%15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]),
+      "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]),
+      "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]),
+      "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31]));
 }
+__device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+// 2^x with the hardware approximation (ex2.approx, relative error ~2^-22),
+// plenty for softmax weights that are rounded to fp16 afterwards.
+__device__ __forceinline__ float fast_exp2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// Lazy rescaling threshold (log2 units): the running max used for the
+// exponentials is only raised when a new score exceeds it by more than this,
+// so P <= 2^8 stays well inside fp16 and O in TMEM is rarely rescaled.
+constexpr float kRescaleThreshold = 8.f;
 
 __global__ void __launch_bounds__(192, 2)
 attn_tc_kernel(const __grid_constant__ CUtensorMap mQK, const __grid_constant__ CUtensorMap mVT, const AttnArgs p) {
@@ -79,7 +97,6 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap mQK, const __grid_constant__ 
   uint64_t* s_full = bars + 7;
   uint64_t* p_full = bars + 8;
   uint64_t* o_full = bars + 9;
-  uint64_t* o_free = bars + 10;
   uint64_t* drain = bars + 11;
   uint32_t* tslot = reinterpret_cast<uint32_t*>(bars + 12);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tslot + 1);
@@ -96,7 +113,6 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap mQK, const __grid_constant__ 
     mbar_init(s_full, 1);
     mbar_init(p_full, 4);
     mbar_init(o_full, 1);
-    mbar_init(o_free, 4);
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -158,7 +174,6 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap mQK, const __grid_constant__ 
         umma_commit(s_full);
         umma_commit(&k_empty[s]);
         if (!mbar_wait(p_full, j & 1, abort_flag)) break;
-        if (j > 0 && !mbar_wait(o_free, (j - 1) & 1, abort_flag)) break;
         if (!mbar_wait(v_full, j & 1, abort_flag)) break;
         tc_fence_after();
         const uint32_t pbase = smem_u32(sP), vbase = smem_u32(sV);
@@ -166,7 +181,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap mQK, const __grid_constant__ 
         for (int kk = 0; kk < BKV / 16; ++kk) {
           const uint64_t da = sdesc_k_sw128(pbase + (kk >> 2) * (P_BYTES / 2)) + 2 * (kk & 3);
           const uint64_t db = sdesc_k_sw128(vbase + (kk >> 2) * (V_BYTES / 2)) + 2 * (kk & 3);
-          umma_f16(tO, da, db, idesc_o, kk != 0 ? 1u : 0u);
+          umma_f16(tO, da, db, idesc_o, (j | kk) != 0 ? 1u : 0u);  // O accumulates across key blocks
         }
         umma_commit(o_full);
         umma_commit(v_empty);
@@ -184,32 +199,59 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap mQK, const __grid_constant__ 
     const int q = warp & 3;
     const int r = q * 32 + lane;
     const uint32_t lane_off = (uint32_t)(q * 32) << 16;
-    float acc[64];
-#pragma unroll
-    for (int c = 0; c < 64; ++c) acc[c] = 0.f;
-    float m = -INFINITY, l = 0.f;
-    uint8_t* prow = sP + r * 128;  // row r inside each 64-key atom
+    float m_used = -INFINITY, l = 0.f;  // exponent offset in use (log2 units), row sum
+    uint8_t* prow = sP + r * 128;        // row r inside each 64-key atom
     const int sw = r & 7;
     bool ok = true;
     for (int j = 0; j < nblk && ok; ++j) {
-      if (!mbar_wait(s_full, j & 1, abort_flag)) {
+      // wait outcomes are made warp-uniform: the tcgen05 loads below are .sync.aligned
+      if (!__all_sync(0xffffffffu, mbar_wait(s_full, j & 1, abort_flag))) {
         ok = false;
         break;
       }
       tc_fence_after();
       const int kvalid = L - j * BKV;  // keys [0, kvalid) of this block are valid
+      // pass 1: row max of the raw scores (scale > 0 commutes with max)
       float mx = -INFINITY;
 #pragma unroll 1
       for (int c = 0; c < BKV; c += 32) {
         uint32_t u[32];
         tmem_ld32(tS + lane_off + c, u);
         tmem_ld_wait();
+        if (c + 32 <= kvalid) {
 #pragma unroll
-        for (int t = 0; t < 32; ++t)
-          if (c + t < kvalid) mx = fmaxf(mx, __uint_as_float(u[t]) * p.scale_log2);
+          for (int t = 0; t < 32; ++t) mx = fmaxf(mx, __uint_as_float(u[t]));
+        } else {
+#pragma unroll
+          for (int t = 0; t < 32; ++t)
+            if (c + t < kvalid) mx = fmaxf(mx, __uint_as_float(u[t]));
+        }
       }
-      const float m_new = fmaxf(m, mx);
-      const float corr = exp2f(m - m_new);
+      mx *= p.scale_log2;
+      // P and O of the previous block: P.V(j-1) must have finished reading P and writing O
+      if (j > 0 && !__all_sync(0xffffffffu, mbar_wait(o_full, (j - 1) & 1, abort_flag))) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      if (mx > m_used + kRescaleThreshold) {
+        const float corr = fast_exp2(m_used - mx);  // 0 for the first block
+        if (j > 0) {
+#pragma unroll 1
+          for (int c = 0; c < dh; c += 32) {  // dh in {48, 64}: rescale columns [c, c+32) (the tail is unused)
+            uint32_t o[32];
+            tmem_ld32(tO + lane_off + c, o);
+            tmem_ld_wait();
+#pragma unroll
+            for (int t = 0; t < 32; ++t) o[t] = __float_as_uint(__uint_as_float(o[t]) * corr);
+            tmem_st32(tO + lane_off + c, o);
+          }
+          tmem_st_wait();
+        }
+        l *= corr;
+        m_used = mx;
+      }
+      // pass 2: exponentials, row sum, fp16 P into the swizzled operand layout
       float sum = 0.f;
 #pragma unroll 1
       for (int c = 0; c < BKV; c += 32) {
@@ -217,12 +259,16 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap mQK, const __grid_constant__ 
         tmem_ld32(tS + lane_off + c, u);
         tmem_ld_wait();
         float pv[32];
+        if (c + 32 <= kvalid) {
 #pragma unroll
-        for (int t = 0; t < 32; ++t) {
-          pv[t] = (c + t < kvalid) ? exp2f(__uint_as_float(u[t]) * p.scale_log2 - m_new) : 0.f;
-          sum += pv[t];
+          for (int t = 0; t < 32; ++t) pv[t] = fast_exp2(fmaf(__uint_as_float(u[t]), p.scale_log2, -m_used));
+        } else {
+#pragma unroll
+          for (int t = 0; t < 32; ++t)
+            pv[t] = (c + t < kvalid) ? fast_exp2(fmaf(__uint_as_float(u[t]), p.scale_log2, -m_used)) : 0.f;
         }
-        // 32 keys = four 16-byte chunks of the row, 128-byte swizzle within each 64-key atom
+#pragma unroll
+        for (int t = 0; t < 32; ++t) sum += pv[t];
         uint8_t* atom = prow + (c >> 6) * (P_BYTES / 2);
 #pragma unroll
         for (int ch = 0; ch < 4; ++ch) {
@@ -237,41 +283,19 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap mQK, const __grid_constant__ 
           *reinterpret_cast<uint4*>(atom + ((logical ^ sw) << 4)) = w;
         }
       }
-      l = l * corr + sum;
-      m = m_new;
+      l += sum;
       fence_async_smem();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(p_full);
-      if (!mbar_wait(o_full, j & 1, abort_flag)) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
-      uint32_t o0[32];
-      tmem_ld32(tO + lane_off, o0);
-      if (dh == 64) {
-        uint32_t o1[32];
-        tmem_ld32(tO + lane_off + 32, o1);
-        tmem_ld_wait();
-#pragma unroll
-        for (int c = 0; c < 32; ++c) {
-          acc[c] = acc[c] * corr + __uint_as_float(o0[c]);
-          acc[32 + c] = acc[32 + c] * corr + __uint_as_float(o1[c]);
-        }
-      } else {
-        uint32_t o1[16];
-        tmem_ld16(tO + lane_off + 32, o1);
-        tmem_ld_wait();
-#pragma unroll
-        for (int c = 0; c < 32; ++c) acc[c] = acc[c] * corr + __uint_as_float(o0[c]);
-#pragma unroll
-        for (int c = 0; c < 16; ++c) acc[32 + c] = acc[32 + c] * corr + __uint_as_float(o1[c]);
-      }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(o_free);
     }
+    // epilogue: O / l after the last P.V
+    if (ok && !__all_sync(0xffffffffu, mbar_wait(o_full, (nblk - 1) & 1, abort_flag))) ok = false;
+    tc_fence_after();
+    uint32_t o0[32], o1[32];
+    tmem_ld32(tO + lane_off, o0);
+    tmem_ld32(tO + lane_off + 32, o1);
+    tmem_ld_wait();
     if (ok && q0 + r < L) {
       const float inv = 1.f / l;
       __half* o = p.out + (size_t)(e0 + q0 + r) * (p.n_heads * dh) + h * dh;
@@ -282,7 +306,10 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap mQK, const __grid_constant__ 
           uint32_t* pw = reinterpret_cast<uint32_t*>(&w);
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
-            __half2 hv = __floats2half2_rn(acc[c + 2 * e] * inv, acc[c + 2 * e + 1] * inv);
+            const int k0 = c + 2 * e;
+            const float a0 = __uint_as_float(k0 < 32 ? o0[k0] : o1[k0 - 32]);
+            const float a1 = __uint_as_float(k0 + 1 < 32 ? o0[k0 + 1] : o1[k0 + 1 - 32]);
+            __half2 hv = __floats2half2_rn(a0 * inv, a1 * inv);
             pw[e] = *reinterpret_cast<uint32_t*>(&hv);
           }
           *reinterpret_cast<uint4*>(o + c) = w;
