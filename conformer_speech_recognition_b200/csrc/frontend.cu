@@ -140,7 +140,93 @@ frontend_kernel(const float* __restrict__ audio, int64_t stride, Clips clips, in
   }
 }
 
+// fp16 frames for the tensor-core DFT: row r of the packed mel rows holds
+// audio[clip, 160 f .. 160 f + 319] (zeros for rows outside every clip).
+template <bool VEC>
+__global__ void __launch_bounds__(256)
+frames_kernel(const float* __restrict__ audio, int64_t stride, Clips clips, int rows, __half* __restrict__ frames) {
+  const int r = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+  if (r >= rows) return;
+  const int ci = clips.find(r, 4, 6);
+  const int f = r - (4 * clips.e(ci) + 6);
+  const bool valid = f >= 0 && f < clips.F(ci);
+  __half* dst = frames + (size_t)r * NFFT;
+  const float* src = audio + (int64_t)ci * stride + (int64_t)f * HOP;
+  for (int c = lane * 4; c < NFFT; c += 128) {  // 80 float4 per frame
+    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (valid) {
+      if (VEC) v = __ldg(reinterpret_cast<const float4*>(src + c));
+      else v = make_float4(__ldg(src + c), __ldg(src + c + 1), __ldg(src + c + 2), __ldg(src + c + 3));
+    }
+    const __half2 a = __floats2half2_rn(v.x, v.y), b = __floats2half2_rn(v.z, v.w);
+    uint2 w;
+    w.x = *reinterpret_cast<const uint32_t*>(&a);
+    w.y = *reinterpret_cast<const uint32_t*>(&b);
+    *reinterpret_cast<uint2*>(dst + c) = w;
+  }
+}
+
+// mel = power[:, :161] . fb, then log(clip(mel, 1e-9, 1e9)); 32 rows per CTA.
+constexpr size_t MEL_SMEM = (size_t)(FT * NBIN + NBIN * NMEL) * sizeof(float);
+
+__global__ void __launch_bounds__(256)
+mel_log_kernel(const float* __restrict__ power, int ld, const float* __restrict__ fb, Clips clips, int rows,
+               void* __restrict__ mel, int out_half) {
+  extern __shared__ float dyn[];
+  float (*sp)[NBIN] = reinterpret_cast<float (*)[NBIN]>(dyn);  // [FT][NBIN]
+  float* sfb = dyn + FT * NBIN;                                // [NBIN][NMEL]
+  __shared__ int s_valid[FT];
+  const int tid = threadIdx.x, row0 = blockIdx.x * FT;
+  if (tid < FT) {
+    const int r = row0 + tid;
+    int ok = 0;
+    if (r < rows) {
+      const int ci = clips.find(r, 4, 6);
+      const int f = r - (4 * clips.e(ci) + 6);
+      ok = f >= 0 && f < clips.F(ci);
+    }
+    s_valid[tid] = ok;
+  }
+  for (int idx = tid; idx < NBIN * NMEL; idx += 256) sfb[idx] = __ldg(fb + idx);
+  for (int idx = tid; idx < FT * NBIN; idx += 256) {
+    const int j = idx / NBIN, k = idx - j * NBIN;
+    const int r = row0 + j;
+    sp[j][k] = r < rows ? __ldg(power + (size_t)r * ld + k) : 0.f;
+  }
+  __syncthreads();
+  const int m = tid & 63;
+#pragma unroll
+  for (int j = 0; j < FT / 4; ++j) {
+    const int a = (tid >> 6) + 4 * j;
+    float acc = 0.f;
+    for (int k = 0; k < NBIN; ++k) acc = fmaf(sp[a][k], sfb[k * NMEL + m], acc);
+    const int r = row0 + a;
+    if (r >= rows) continue;
+    const float v = s_valid[a] ? logf(fminf(fmaxf(acc, 1e-9f), 1e9f)) : 0.f;
+    if (out_half) reinterpret_cast<__half*>(mel)[(size_t)r * NMEL + m] = __float2half_rn(v);
+    else reinterpret_cast<float*>(mel)[(size_t)r * NMEL + m] = v;
+  }
+}
+
 }  // namespace
+
+cudaError_t launch_frames(const float* audio, int64_t audio_stride, Clips clips, int rows, __half* frames,
+                          cudaStream_t s) {
+  if (rows <= 0) return cudaSuccess;
+  const bool vec = audio_stride % 4 == 0 && (reinterpret_cast<uintptr_t>(audio) & 15) == 0;
+  if (vec) frames_kernel<true><<<(rows + 7) / 8, 256, 0, s>>>(audio, audio_stride, clips, rows, frames);
+  else frames_kernel<false><<<(rows + 7) / 8, 256, 0, s>>>(audio, audio_stride, clips, rows, frames);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_mel_log(const float* power, int ld_power, const float* fb, Clips clips, int rows, void* mel,
+                           int out_half, cudaStream_t s) {
+  if (rows <= 0) return cudaSuccess;
+  cudaError_t e = cudaFuncSetAttribute(mel_log_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)MEL_SMEM);
+  if (e != cudaSuccess) return e;
+  mel_log_kernel<<<(rows + FT - 1) / FT, 256, MEL_SMEM, s>>>(power, ld_power, fb, clips, rows, mel, out_half);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_frontend(const float* audio, int64_t audio_stride, Clips clips, int rows, int packed, int f_max,
                             const float* basis, const float* fb, void* out, int out_half, cudaStream_t s) {

@@ -53,7 +53,7 @@ struct Cfg {
   static constexpr int RAW_TILE = QB ? BN * BK : 0;          // INT8 weights as loaded (64-byte rows)
   static constexpr int TX = A_TILE + (QB ? RAW_TILE : B_TILE);  // bytes landed by TMA per stage
   static constexpr int STAGE = A_TILE + B_TILE + RAW_TILE;
-  static constexpr int TMEM_COLS = 2 * BN;  // power of two for BN in {128, 256}
+  static constexpr int TMEM_COLS = BN == 128 ? 256 : 512;  // two accumulators, rounded to a power of two
   static constexpr size_t SMEM = (size_t)STAGES * STAGE + 1024 + 256;
 };
 
@@ -157,9 +157,12 @@ __device__ __forceinline__ void epi_chunk(const TcArgs& p, int r, int n, bool va
   }
 }
 
-// Epilogue of columns [c_lo, c_hi) of a tile for row r (this warp's half).
+// Epilogue of this warp's half of a tile for row r: columns [half BN/2, (half+1) BN/2),
+// or for the paired epilogues (GLU, power: 128-column blocks [first 64 | second 64])
+// the (first, second) pairs of 32-column chunks number half * BN/128 .. (half+1) * BN/128 - 1.
 template <int BN, int EPI>
-__device__ __forceinline__ void epilogue_tile(const TcArgs& p, int r, int n0, uint32_t tbase, int c_lo, int c_hi) {
+__device__ __forceinline__ void epilogue_tile(const TcArgs& p, int r, int n0, uint32_t tbase, int half) {
+  const int c_lo = half * (BN / 2), c_hi = (half + 1) * (BN / 2);
   const EpiParams& ep = p.ep;
   const bool in_m = r < p.M;
   bool valid = in_m;
@@ -171,12 +174,35 @@ __device__ __forceinline__ void epilogue_tile(const TcArgs& p, int r, int n0, ui
       valid = t >= 0 && t < (EPI == EPI_CONV1 ? ep.clips.L1(ci) : ep.clips.L2(ci));
     }
   }
-  if constexpr (EPI == EPI_GLU) {
+  if constexpr (EPI == EPI_POWER) {
+    // DFT basis rows interleaved in blocks of 64: [cos 64 bins | sin 64 bins] per 128 columns
+#pragma unroll 1
+    for (int pr = half * (BN / 128); pr < (half + 1) * (BN / 128); ++pr) {
+      const int blk = (pr >> 1) * 128, hh = (pr & 1) * 32;
+      {
+        uint32_t a[32], g[32];
+        tmem_ld32(tbase + blk + hh, a);
+        tmem_ld32(tbase + blk + 64 + hh, g);
+        tmem_ld_wait();
+        if (!in_m) continue;
+        float4* o = reinterpret_cast<float4*>(reinterpret_cast<float*>(ep.out) + (size_t)r * ep.ldo + (n0 + blk) / 2 + hh);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          float4 w;
+          w.x = __uint_as_float(a[4 * j]) * __uint_as_float(a[4 * j]) + __uint_as_float(g[4 * j]) * __uint_as_float(g[4 * j]);
+          w.y = __uint_as_float(a[4 * j + 1]) * __uint_as_float(a[4 * j + 1]) + __uint_as_float(g[4 * j + 1]) * __uint_as_float(g[4 * j + 1]);
+          w.z = __uint_as_float(a[4 * j + 2]) * __uint_as_float(a[4 * j + 2]) + __uint_as_float(g[4 * j + 2]) * __uint_as_float(g[4 * j + 2]);
+          w.w = __uint_as_float(a[4 * j + 3]) * __uint_as_float(a[4 * j + 3]) + __uint_as_float(g[4 * j + 3]) * __uint_as_float(g[4 * j + 3]);
+          o[j] = w;
+        }
+      }
+    }
+  } else if constexpr (EPI == EPI_GLU) {
     // weight rows interleaved in blocks of 64: [value 64 | gate 64] per 128 columns
 #pragma unroll 1
-    for (int blk = c_lo; blk < c_hi; blk += 128) {
-#pragma unroll 1
-      for (int hh = 0; hh < 64; hh += 32) {
+    for (int pr = half * (BN / 128); pr < (half + 1) * (BN / 128); ++pr) {
+      const int blk = (pr >> 1) * 128, hh = (pr & 1) * 32;
+      {
         uint32_t a[32], g[32];
         tmem_ld32(tbase + blk + hh, a);
         tmem_ld32(tbase + blk + 64 + hh, g);
@@ -400,7 +426,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap mA, const __grid_constant__ C
       const int nb = tile % p.n_blocks, mb = tile / p.n_blocks;
       const int r = mb * BM + q * 32 + lane;
       const uint32_t tbase = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN);
-      epilogue_tile<BN, EPI>(p, r, nb * BN, tbase, half * (BN / 2), (half + 1) * (BN / 2));
+      epilogue_tile<BN, EPI>(p, r, nb * BN, tbase, half);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&tempty[acc]);
@@ -483,6 +509,7 @@ cudaError_t launch_bn(TcGemmCache* cache, const CUtensorMap& mA, const CUtensorM
     case EPI_CONV1: return launch_epi<BN, STAGES, EPI_CONV1, QB>(cache, mA, mA2, mB, args, s);
     case EPI_CONV2: return launch_epi<BN, STAGES, EPI_CONV2, QB>(cache, mA, mA2, mB, args, s);
     case EPI_F32: return launch_epi<BN, STAGES, EPI_F32, QB>(cache, mA, mA2, mB, args, s);
+    case EPI_POWER: return launch_epi<BN, STAGES, EPI_POWER, QB>(cache, mA, mA2, mB, args, s);
     default: return cudaErrorInvalidValue;
   }
 }
@@ -492,7 +519,7 @@ cudaError_t launch_bn(TcGemmCache* cache, const CUtensorMap& mA, const CUtensorM
 bool tc_supported(int a_dtype, int b_dtype, int N, int K, int epi) {
   return a_dtype == 1 && (b_dtype == 1 || b_dtype == 2) && N % 256 == 0 && K % 64 == 0 && K >= 64 &&
          (epi == EPI_SWISH || epi == EPI_GLU || epi == EPI_RESID || epi == EPI_QKV || epi == EPI_CONV1 ||
-          epi == EPI_CONV2 || epi == EPI_F32);
+          epi == EPI_CONV2 || epi == EPI_F32 || epi == EPI_POWER);
 }
 
 cudaError_t tc_init(TcGemmCache* cache, int device) {
@@ -505,12 +532,33 @@ cudaError_t tc_init(TcGemmCache* cache, int device) {
   return cudaMemset(cache->status, 0, sizeof(int));
 }
 
+// Tile width: the BN in {128, 192, 256} dividing N (GLU / power epilogues need
+// 128-column blocks) that minimises (waves of tiles over the SMs) x (tile cost),
+// counting a fixed per-tile overhead of 32 columns.
+int choose_bn(int M, int N, int epi, int sms) {
+  const int mt = (M + BM - 1) / BM;
+  int best = 0;
+  double best_cost = 1e30;
+  for (int bn : {256, 192, 128}) {
+    if (N % bn) continue;
+    if ((epi == EPI_GLU || epi == EPI_POWER) && bn % 128) continue;
+    const int tiles = mt * (N / bn);
+    const double cost = (double)((tiles + sms - 1) / sms) * (bn + 32);
+    if (cost < best_cost - 1e-9) {
+      best_cost = cost;
+      best = bn;
+    }
+  }
+  return best;
+}
+
 cudaError_t launch_gemm_tc(TcGemmCache* cache, const void* A, const void* A2, int n_split, int lda, WeightOp B, int M,
                            int N, int K, int epi, const EpiParams& ep, cudaStream_t s) {
   if (!tc_supported(1, B.dtype, N, K, epi) || M <= 0) return cudaErrorInvalidValue;
   const bool qb = B.dtype == 2;
   if (qb && !B.scale_t) return cudaErrorInvalidValue;
-  constexpr int BN = 256;
+  const int BN = choose_bn(M, N, epi, cache->sm_count);
+  if (!BN) return cudaErrorInvalidValue;
   // lda < K: stride-2 convolution view (lda = 2C, K = taps * C, C % 64 == 0); the
   // buffer behind it holds (M + 2) * lda elements, mapped as M + 2 rows of 2C.
   const bool conv = lda < K;
@@ -535,8 +583,15 @@ cudaError_t launch_gemm_tc(TcGemmCache* cache, const void* A, const void* A2, in
   args.ep = ep;
   args.scale_t = B.scale_t;
   args.status = cache->status;
-  if (qb) return launch_bn<BN, 3, true>(cache, mA, mA2, mB, args, s);
-  return launch_bn<BN, 4, false>(cache, mA, mA2, mB, args, s);
+  // stages: as many as fit in ~200 KB of shared memory
+  if (qb) {
+    if (BN == 256) return launch_bn<256, 3, true>(cache, mA, mA2, mB, args, s);
+    if (BN == 192) return launch_bn<192, 4, true>(cache, mA, mA2, mB, args, s);
+    return launch_bn<128, 5, true>(cache, mA, mA2, mB, args, s);
+  }
+  if (BN == 256) return launch_bn<256, 4, false>(cache, mA, mA2, mB, args, s);
+  if (BN == 192) return launch_bn<192, 5, false>(cache, mA, mA2, mB, args, s);
+  return launch_bn<128, 6, false>(cache, mA, mA2, mB, args, s);
 }
 
 cudaError_t launch_attention(TcGemmCache* cache, const void* qk, const void* vt, Clips clips, void* o, int t_half,

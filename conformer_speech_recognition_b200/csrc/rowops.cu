@@ -75,32 +75,35 @@ __device__ __forceinline__ void load_row(const float* x, float4 (&v)[8], int nv,
     if (j < nv) v[j] = *reinterpret_cast<const float4*>(x + (j * 32 + lane) * 4);
 }
 
+// Plain LayerNorm: each warp normalises rows (16 w + i) and (16 w + i + 8) of its
+// CTA's 16-row block together, so two rows' loads are in flight per lane.
 template <typename T>
 __global__ void __launch_bounds__(256)
 ln_kernel(const float* __restrict__ x, const float* __restrict__ g, const float* __restrict__ b, float eps,
           T* __restrict__ u, int rows, int d) {
-  const int row = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
-  if (row >= rows) return;
+  const int r0 = blockIdx.x * 16 + (threadIdx.x >> 5), r1 = r0 + 8, lane = threadIdx.x & 31;
   const int nv = d >> 7;
-  float4 v[8];
-  load_row(x + (size_t)row * d, v, nv, lane);
-  ln_row(v, nv, d, eps, g, b, lane);
+  float4 v0[8], v1[8];
+  if (r0 < rows) load_row(x + (size_t)r0 * d, v0, nv, lane);
+  if (r1 < rows) load_row(x + (size_t)r1 * d, v1, nv, lane);
+  if (r0 < rows) {
+    ln_row(v0, nv, d, eps, g, b, lane);
 #pragma unroll
-  for (int j = 0; j < 8; ++j)
-    if (j < nv) store4<T>(u + (size_t)row * d + (j * 32 + lane) * 4, v[j]);
+    for (int j = 0; j < 8; ++j)
+      if (j < nv) store4<T>(u + (size_t)r0 * d + (j * 32 + lane) * 4, v0[j]);
+  }
+  if (r1 < rows) {
+    ln_row(v1, nv, d, eps, g, b, lane);
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+      if (j < nv) store4<T>(u + (size_t)r1 * d + (j * 32 + lane) * 4, v1[j]);
+  }
 }
 
 template <typename T>
-__global__ void __launch_bounds__(256)
-ln_chain_kernel(float* __restrict__ x, const float* __restrict__ g1, const float* __restrict__ b1,
-                const float* __restrict__ g2, const float* __restrict__ b2, float eps, T* __restrict__ u, int rows,
-                int d) {
-  const int row = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
-  if (row >= rows) return;
-  const int nv = d >> 7;
-  float4 v[8];
-  float* xr = x + (size_t)row * d;
-  load_row(xr, v, nv, lane);
+__device__ __forceinline__ void ln_chain_row(float* xr, T* ur, float4 (&v)[8], int nv, int d, float eps,
+                                             const float* g1, const float* b1, const float* g2, const float* b2,
+                                             int lane) {
   ln_row(v, nv, d, eps, g1, b1, lane);
 #pragma unroll
   for (int j = 0; j < 8; ++j)
@@ -108,14 +111,29 @@ ln_chain_kernel(float* __restrict__ x, const float* __restrict__ g1, const float
   ln_row(v, nv, d, eps, g2, b2, lane);
 #pragma unroll
   for (int j = 0; j < 8; ++j)
-    if (j < nv) store4<T>(u + (size_t)row * d + (j * 32 + lane) * 4, v[j]);
+    if (j < nv) store4<T>(ur + (j * 32 + lane) * 4, v[j]);
 }
 
 template <typename T>
 __global__ void __launch_bounds__(256)
+ln_chain_kernel(float* __restrict__ x, const float* __restrict__ g1, const float* __restrict__ b1,
+                const float* __restrict__ g2, const float* __restrict__ b2, float eps, T* __restrict__ u, int rows,
+                int d) {
+  const int r0 = blockIdx.x * 16 + (threadIdx.x >> 5), r1 = r0 + 8, lane = threadIdx.x & 31;
+  const int nv = d >> 7;
+  float4 v0[8], v1[8];
+  if (r0 < rows) load_row(x + (size_t)r0 * d, v0, nv, lane);
+  if (r1 < rows) load_row(x + (size_t)r1 * d, v1, nv, lane);
+  if (r0 < rows) ln_chain_row<T>(x + (size_t)r0 * d, u + (size_t)r0 * d, v0, nv, d, eps, g1, b1, g2, b2, lane);
+  if (r1 < rows) ln_chain_row<T>(x + (size_t)r1 * d, u + (size_t)r1 * d, v1, nv, d, eps, g1, b1, g2, b2, lane);
+}
+
+template <typename T, int DH>
+__global__ void __launch_bounds__(256)
 ln_rope_kernel(const float* __restrict__ x, const float* __restrict__ g, const float* __restrict__ b, float eps,
                const float* __restrict__ cos_tab, const float* __restrict__ sin_tab, Clips clips, T* __restrict__ u,
-               T* __restrict__ urot, int rows, int d, int dh) {
+               T* __restrict__ urot, int rows, int d) {
+  constexpr int dh = DH;
   __shared__ __align__(16) float srow[8][1024];
   const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int row = blockIdx.x * 8 + w;
@@ -167,34 +185,34 @@ __global__ void __launch_bounds__(256)
 dwconv_kernel(const T* __restrict__ g, const float* __restrict__ w, const float* __restrict__ bias, Clips clips,
               T* __restrict__ out, int rows, int d) {
   constexpr int PAD = (K - 1) / 2, R = 64, HALO = R + 2 * PAD;
-  __shared__ float tile[HALO][128];
+  __shared__ __align__(16) float tile[HALO][128];
   __shared__ int s_lo[R], s_hi[R];
   const int r0 = blockIdx.x * R, c0 = blockIdx.y * 128;
-  for (int idx = threadIdx.x; idx < HALO * 16; idx += 256) {  // 16 x 8 channels per row
-    const int rr = idx >> 4, c8 = (idx & 15) * 8;
+  // staging: one warp per row, 4 channels per lane, one 16-byte shared store each
+  // (conflict-free); every load of the thread is issued before the first store
+  constexpr int ITEMS = (HALO * 32 + 255) / 256;
+  float4 v[ITEMS];
+#pragma unroll
+  for (int it = 0; it < ITEMS; ++it) {
+    const int idx = threadIdx.x + it * 256;
+    const int rr = idx >> 5, c4 = (idx & 31) * 4;
     const int src = r0 - PAD + rr;
-    float v[8];
-    if (src >= 0 && src < rows) {
+    v[it] = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (idx < HALO * 32 && src >= 0 && src < rows) {
       if constexpr (sizeof(T) == 2) {
-        const uint4 raw = *reinterpret_cast<const uint4*>(g + (size_t)src * d + c0 + c8);
-        const __half2* h2 = reinterpret_cast<const __half2*>(&raw);
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float2 f = __half22float2(h2[e]);
-          v[2 * e] = f.x;
-          v[2 * e + 1] = f.y;
-        }
+        const uint2 raw = __ldg(reinterpret_cast<const uint2*>(g + (size_t)src * d + c0 + c4));
+        const float2 a = __half22float2(*reinterpret_cast<const __half2*>(&raw.x));
+        const float2 b = __half22float2(*reinterpret_cast<const __half2*>(&raw.y));
+        v[it] = make_float4(a.x, a.y, b.x, b.y);
       } else {
-        const float4 a = *reinterpret_cast<const float4*>(g + (size_t)src * d + c0 + c8);
-        const float4 b = *reinterpret_cast<const float4*>(g + (size_t)src * d + c0 + c8 + 4);
-        v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w; v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+        v[it] = __ldg(reinterpret_cast<const float4*>(g + (size_t)src * d + c0 + c4));
       }
-    } else {
-#pragma unroll
-      for (int e = 0; e < 8; ++e) v[e] = 0.f;
     }
+  }
 #pragma unroll
-    for (int e = 0; e < 8; ++e) tile[rr][c8 + e] = v[e];
+  for (int it = 0; it < ITEMS; ++it) {
+    const int idx = threadIdx.x + it * 256;
+    if (idx < HALO * 32) *reinterpret_cast<float4*>(&tile[idx >> 5][(idx & 31) * 4]) = v[it];
   }
   if (threadIdx.x < R) {
     const int r = r0 + threadIdx.x;
@@ -413,7 +431,7 @@ __global__ void f32_to_f16_kernel(const float* __restrict__ in, __half* __restri
 cudaError_t launch_layernorm(const float* x, const float* g, const float* b, float eps, void* u, int u_half, int rows,
                              int d, cudaStream_t s) {
   if (d % 128 || d > 1024) return cudaErrorInvalidValue;
-  const int grid = (rows + 7) / 8;
+  const int grid = (rows + 15) / 16;
   if (u_half) ln_kernel<__half><<<grid, 256, 0, s>>>(x, g, b, eps, (__half*)u, rows, d);
   else ln_kernel<float><<<grid, 256, 0, s>>>(x, g, b, eps, (float*)u, rows, d);
   return cudaGetLastError();
@@ -422,7 +440,7 @@ cudaError_t launch_layernorm(const float* x, const float* g, const float* b, flo
 cudaError_t launch_layernorm_chain(float* x, const float* g1, const float* b1, const float* g2, const float* b2,
                                    float eps, void* u, int u_half, int rows, int d, cudaStream_t s) {
   if (d % 128 || d > 1024) return cudaErrorInvalidValue;
-  const int grid = (rows + 7) / 8;
+  const int grid = (rows + 15) / 16;
   if (u_half) ln_chain_kernel<__half><<<grid, 256, 0, s>>>(x, g1, b1, g2, b2, eps, (__half*)u, rows, d);
   else ln_chain_kernel<float><<<grid, 256, 0, s>>>(x, g1, b1, g2, b2, eps, (float*)u, rows, d);
   return cudaGetLastError();
@@ -433,12 +451,22 @@ cudaError_t launch_layernorm_rope(const float* x, const float* g, const float* b
                                   int d_head, cudaStream_t s) {
   if (d % 128 || d > 1024 || d_head % 4) return cudaErrorInvalidValue;
   const int grid = (rows + 7) / 8;
-  if (u_half)
-    ln_rope_kernel<__half><<<grid, 256, 0, s>>>(x, g, b, eps, cos_tab, sin_tab, clips, (__half*)u, (__half*)urot,
-                                                rows, d, d_head);
-  else
-    ln_rope_kernel<float><<<grid, 256, 0, s>>>(x, g, b, eps, cos_tab, sin_tab, clips, (float*)u, (float*)urot, rows,
-                                               d, d_head);
+  if (d_head != 48 && d_head != 64) return cudaErrorInvalidValue;
+  if (u_half) {
+    if (d_head == 48)
+      ln_rope_kernel<__half, 48><<<grid, 256, 0, s>>>(x, g, b, eps, cos_tab, sin_tab, clips, (__half*)u,
+                                                      (__half*)urot, rows, d);
+    else
+      ln_rope_kernel<__half, 64><<<grid, 256, 0, s>>>(x, g, b, eps, cos_tab, sin_tab, clips, (__half*)u,
+                                                      (__half*)urot, rows, d);
+  } else {
+    if (d_head == 48)
+      ln_rope_kernel<float, 48><<<grid, 256, 0, s>>>(x, g, b, eps, cos_tab, sin_tab, clips, (float*)u, (float*)urot,
+                                                     rows, d);
+    else
+      ln_rope_kernel<float, 64><<<grid, 256, 0, s>>>(x, g, b, eps, cos_tab, sin_tab, clips, (float*)u, (float*)urot,
+                                                     rows, d);
+  }
   return cudaGetLastError();
 }
 

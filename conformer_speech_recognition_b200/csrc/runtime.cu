@@ -92,6 +92,10 @@ struct gam_ctx {
   // weights
   float* basis = nullptr;  // [320][320]
   float* fb = nullptr;     // [161][64]
+  DevLinear dft;           // fp16 modes: windowed DFT basis as a [512, 320] GEMM weight,
+                           // rows [cos 64 bins | sin 64 bins] per 128 (bins 0..255, zero past 160)
+  __half* frames = nullptr;  // [R0_cap, 320] fp16 frames
+  float* power = nullptr;    // [R0_cap, 256] power spectrum
   DevLinear conv1, conv2, head;
   DevLinear head2;         // tensor-core CTC head: [W | W] padded to a multiple of 256 rows, K = 2d
   __half* ctc_a = nullptr; // [rows, 2d] fp16 hi / lo split of the valid encoder frames
@@ -467,9 +471,19 @@ gam_status run_encoder(gam_ctx* c, const float* audio, const int32_t* lengths, i
   const float eps = cfg.ln_eps;
   const int M = p.E_pad;
 
-  GAM_TRY(run_kernel(c, PK_FRONTEND, s, [&] {
-    return launch_frontend(audio, max_samples, clips, p.R0, 1, 0, c->basis, c->fb, c->mel, ah, s);
-  }));
+  if (c->dft.w) {
+    // tensor-core frontend: fp16 frames -> DFT GEMM with the power epilogue -> mel + log
+    GAM_TRY(run_kernel(c, PK_FRONTEND, s, [&] { return launch_frames(audio, max_samples, clips, p.R0, c->frames, s); }));
+    GAM_TRY(gemm(c, PK_FRONTEND, s, c->frames, nullptr, 0, cfg.n_fft, c->dft, p.R0, EPI_POWER, 1.f, c->power, 256,
+                 clips));
+    GAM_TRY(run_kernel(c, PK_FRONTEND, s, [&] {
+      return launch_mel_log(c->power, 256, c->fb, clips, p.R0, c->mel, ah, s);
+    }));
+  } else {
+    GAM_TRY(run_kernel(c, PK_FRONTEND, s, [&] {
+      return launch_frontend(audio, max_samples, clips, p.R0, 1, 0, c->basis, c->fb, c->mel, ah, s);
+    }));
+  }
   GAM_TRY(gemm(c, PK_GEMM_SUB, s, c->mel, nullptr, 0, 2 * cfg.n_mels, c->conv1, p.R1, EPI_CONV1, 1.f, c->c1, d,
                clips));
   GAM_TRY(gemm(c, PK_GEMM_SUB, s, c->c1, nullptr, 0, 2 * d, c->conv2, M, EPI_CONV2, 1.f, c->x, d, clips));
@@ -606,6 +620,25 @@ gam_status build_weights(gam_ctx* c, const gam_tensor* tensors, int n) {
       }
     GAM_TRY(upload_f32(c, &c->basis, basis));
     GAM_TRY(upload_f32(c, &c->fb, fbv));
+    if (cfg.precision != GAM_FP32) {
+      HostLinear hd;
+      hd.N = 512;
+      hd.K = N;
+      hd.dtype = 1;
+      hd.b.assign(512, 0.0);
+      hd.w.assign((size_t)512 * N, 0.0);
+      for (int row = 0; row < 512; ++row) {
+        const int tile = row / 256, blk = (row % 256) / 128, within = row % 128;
+        const bool is_sin = within >= 64;
+        const int bin = tile * 128 + blk * 64 + (within % 64);
+        if (bin > N / 2 || (is_sin && (bin == 0 || bin == N / 2))) continue;
+        for (int nn = 0; nn < N; ++nn) {
+          const double a = two_pi * (double)((int64_t)bin * nn % N) / N;
+          hd.w[(size_t)row * N + nn] = win[nn] * (is_sin ? std::sin(a) : std::cos(a));
+        }
+      }
+      GAM_TRY(upload_linear(c, hd, c->dft));
+    }
   }
   GAM_TRY(load_conv(c, t, "subsampling.conv1", d, cfg.n_mels, cfg.sub_kernel, c->conv1));
   GAM_TRY(load_conv(c, t, "subsampling.conv2", d, d, cfg.sub_kernel, c->conv2));
@@ -745,6 +778,10 @@ gam_status alloc_workspace(gam_ctx* c) {
   const int d = cfg.d_model, f = cfg.ffn_dim, H = cfg.n_heads;
   const int64_t E = c->E_cap;
   GAM_TRY(dev_alloc(c, &c->mel, (size_t)c->R0_cap * cfg.n_mels * es));
+  if (cfg.precision != GAM_FP32) {
+    GAM_TRY(dev_alloc(c, (void**)&c->frames, (size_t)c->R0_cap * cfg.n_fft * 2));
+    GAM_TRY(dev_alloc(c, (void**)&c->power, (size_t)c->R0_cap * 256 * 4));
+  }
   GAM_TRY(dev_alloc(c, &c->c1, (size_t)c->R1_cap * d * es));
   GAM_TRY(dev_alloc(c, (void**)&c->x, (size_t)E * d * 4));
   GAM_TRY(dev_alloc(c, &c->u, (size_t)E * d * es));

@@ -46,3 +46,10 @@ def test_gemm_parity(ctx, impl, M, N, K, lda):
     err = np.abs(got - ref).max() / np.abs(ref).max()
     assert err <= TOL_GEMM_REL, err
     gam.gam_device_status(ctx)
+
+
+@pytest.mark.parametrize("M,N,K", [(300, 768, 768), (9000, 768, 3072), (4000, 2304, 768), (1200, 1024, 1024)],
+                         ids=["bn192_small", "bn192_deep", "qkv_width", "bn128_d1024"])
+def test_gemm_tile_widths(ctx, M, N, K):
+    """Shapes for which the tensor-core GEMM picks a 192- or 128-column tile."""
+    test_gemm_parity(ctx, 0, M, N, K, K)
