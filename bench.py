@@ -108,6 +108,44 @@ def measured_traffic(workload, family):
         return None
 
 
+def time_workload(name, steps=5, warmup=3, weights=None, device=0):
+    """×realtime of one workload on this GPU: gam_encode + gam_ctc_greedy with the
+    audio resident, CUDA events over `steps` steps after `warmup` steps."""
+    import torch
+    from conformer_speech_recognition_b200 import gam
+    cfg = synth.workload_config(name)
+    W = weights if weights is not None else synth.random_weights(cfg, seed=0)
+    audio_np, lens = synth.workload_audio(name)
+    B, nmax = audio_np.shape
+    ctx = gam.gam_create(cfg, W, B, nmax, device=device)
+    try:
+        dev = torch.device("cuda", device)
+        audio = torch.from_numpy(audio_np).to(dev)
+        _, el, _, tmax = gam.gam_plan_lengths(cfg, lens)
+        enc = torch.empty((B, tmax, cfg["d_model"]), dtype=torch.float32, device=dev)
+        stream = torch.cuda.current_stream(dev)
+
+        def step():
+            gam.gam_encode(ctx, audio, lens, out=enc, stream=stream)
+            gam.gam_ctc_greedy(ctx, enc, el, stream=stream)
+
+        for _ in range(warmup):
+            step()
+        torch.cuda.synchronize(dev)
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        t0.record(stream)
+        for _ in range(steps):
+            step()
+        t1.record(stream)
+        torch.cuda.synchronize(dev)
+        ms = t0.elapsed_time(t1) / steps
+        audio_s = float(np.sum(lens)) / synth.SAMPLE_RATE
+        return {"value": audio_s / (ms / 1e3), "unit": UNIT, "ms_per_step": ms, "steps": steps, "warmup": warmup,
+                "batch": int(B), "audio_seconds_per_step": audio_s, "precision": cfg["precision"]}
+    finally:
+        ctx.close()
+
+
 def reduce_max_over_ranks(values, device=None):
     """Element-wise max over all ranks (torch.distributed all_reduce MAX)."""
     import torch
@@ -370,6 +408,14 @@ def run_ours(args, rank, world, local_rank):
         if not args.no_cpu_baseline and world == 1:
             v, desc, threads = oracle_throughput(name, args.cpu_budget)
             cpu = {"value": v, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": desc}
+        per_workload = None
+        if world == 1 and not args.no_per_workload:
+            per_workload = {}
+            for other in sorted(synth.WORKLOADS):
+                if other == name:
+                    continue
+                same_model = synth.workload_config(other) == cfg
+                per_workload[other] = time_workload(other, weights=W if same_model else None, device=local_rank)
         h2d = int(B * nmax * 4 + 5 * (B + 1) * 4 + B * 4)
         d2h = int(B * tmax * 4 + B * 4)
         line = {
@@ -392,6 +438,7 @@ def run_ours(args, rank, world, local_rank):
             "gpu_launches": int(launches),
             "clocks": clock_info,
             "profile_ms_per_step": {k: round(v[0] / n_prof, 4) for k, v in warm.items() if v[1]},
+            "per_workload": per_workload,
         }
         print(json.dumps(line), flush=True)
     ctx.close()
@@ -406,6 +453,7 @@ def main():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(synth.WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-per-workload", action="store_true", help="skip the ×realtime of the other workloads")
     ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle CPU time for cpu_baseline")
     args = ap.parse_args()
     if args.warmup < 3:
