@@ -57,9 +57,19 @@ struct Cfg {
   static constexpr size_t SMEM = (size_t)STAGES * STAGE + 1024 + 256;
 };
 
-// Logistic function with the fast exp / divide intrinsics (|rel err| ~ 1e-6,
-// far below the fp16 rounding of the stored result).
-__device__ __forceinline__ float sigm(float v) { return __fdividef(1.f, 1.f + __expf(-v)); }
+// Hardware tanh (tanh.approx, one special-function op, relative error about
+// 2^-11 -- the size of the fp16 rounding the results get next).
+__device__ __forceinline__ float tanh_fast(float x) {
+  float y;
+  asm("tanh.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+// Logistic function sigma(v) = (1 + tanh(v / 2)) / 2 and Swish v sigma(v).
+__device__ __forceinline__ float sigm(float v) { return fmaf(0.5f, tanh_fast(0.5f * v), 0.5f); }
+__device__ __forceinline__ float swish_fast(float v) {
+  const float h = 0.5f * v;
+  return fmaf(h, tanh_fast(h), h);
+}
 
 __device__ __forceinline__ void load_bias32(const float* b, float (&v)[32]) {
   const float4* p = reinterpret_cast<const float4*>(b);
@@ -96,7 +106,7 @@ __device__ __forceinline__ void epi_chunk(const TcArgs& p, int r, int n, bool va
   switch (EPI) {
     case EPI_SWISH: {
 #pragma unroll
-      for (int j = 0; j < 32; ++j) v[j] = __fdividef(v[j], 1.f + __expf(-v[j]));
+      for (int j = 0; j < 32; ++j) v[j] = swish_fast(v[j]);
       __half* o = reinterpret_cast<__half*>(ep.out) + (size_t)r * ep.ldo + n;
       store_half16(o, v);
       store_half16(o + 16, v + 16);

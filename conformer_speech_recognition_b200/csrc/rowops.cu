@@ -40,25 +40,24 @@ __device__ __forceinline__ void store4<__half>(__half* p, float4 v) {
 __device__ __forceinline__ float ld1(const float* p) { return *p; }
 __device__ __forceinline__ float ld1(const __half* p) { return __half2float(*p); }
 
-// Normalise the row held in v[0..nv) (float4 chunks, chunk j at column 4(32 j + lane)).
-__device__ __forceinline__ void ln_row(float4 (&v)[8], int nv, int d, float eps, const float* g, const float* b,
-                                       int lane) {
+// Normalise the row held in v[0..NV) (float4 chunks, chunk j at column 4(32 j + lane)),
+// NV = d / 128 fixed at compile time so only the registers of one row are live.
+template <int NV>
+__device__ __forceinline__ void ln_row(float4 (&v)[NV], int d, float eps, const float* g, const float* b, int lane) {
+  constexpr int nv = NV;
   float s = 0.f;
 #pragma unroll
-  for (int j = 0; j < 8; ++j)
-    if (j < nv) s += v[j].x + v[j].y + v[j].z + v[j].w;
+  for (int j = 0; j < nv; ++j) s += v[j].x + v[j].y + v[j].z + v[j].w;
   const float mean = warp_sum(s) / d;
   float q = 0.f;
 #pragma unroll
-  for (int j = 0; j < 8; ++j)
-    if (j < nv) {
+  for (int j = 0; j < nv; ++j) {
       v[j].x -= mean; v[j].y -= mean; v[j].z -= mean; v[j].w -= mean;
       q += v[j].x * v[j].x + v[j].y * v[j].y + v[j].z * v[j].z + v[j].w * v[j].w;
     }
   const float rstd = rsqrtf(warp_sum(q) / d + eps);
 #pragma unroll
-  for (int j = 0; j < 8; ++j)
-    if (j < nv) {
+  for (int j = 0; j < nv; ++j) {
       const int c = (j * 32 + lane) * 4;
       const float4 gg = *reinterpret_cast<const float4*>(g + c);
       const float4 bb = *reinterpret_cast<const float4*>(b + c);
@@ -69,83 +68,76 @@ __device__ __forceinline__ void ln_row(float4 (&v)[8], int nv, int d, float eps,
     }
 }
 
-__device__ __forceinline__ void load_row(const float* x, float4 (&v)[8], int nv, int lane) {
+template <int NV>
+__device__ __forceinline__ void load_row(const float* x, float4 (&v)[NV], int lane) {
 #pragma unroll
-  for (int j = 0; j < 8; ++j)
-    if (j < nv) v[j] = *reinterpret_cast<const float4*>(x + (j * 32 + lane) * 4);
+  for (int j = 0; j < NV; ++j) v[j] = *reinterpret_cast<const float4*>(x + (j * 32 + lane) * 4);
 }
 
 // Plain LayerNorm: each warp normalises rows (16 w + i) and (16 w + i + 8) of its
 // CTA's 16-row block together, so two rows' loads are in flight per lane.
-template <typename T>
+template <typename T, int NV>
 __global__ void __launch_bounds__(256)
 ln_kernel(const float* __restrict__ x, const float* __restrict__ g, const float* __restrict__ b, float eps,
-          T* __restrict__ u, int rows, int d) {
+          T* __restrict__ u, int rows) {
+  constexpr int d = NV * 128;
   const int r0 = blockIdx.x * 16 + (threadIdx.x >> 5), r1 = r0 + 8, lane = threadIdx.x & 31;
-  const int nv = d >> 7;
-  float4 v0[8], v1[8];
-  if (r0 < rows) load_row(x + (size_t)r0 * d, v0, nv, lane);
-  if (r1 < rows) load_row(x + (size_t)r1 * d, v1, nv, lane);
+  float4 v0[NV], v1[NV];
+  if (r0 < rows) load_row<NV>(x + (size_t)r0 * d, v0, lane);
+  if (r1 < rows) load_row<NV>(x + (size_t)r1 * d, v1, lane);
   if (r0 < rows) {
-    ln_row(v0, nv, d, eps, g, b, lane);
+    ln_row<NV>(v0, d, eps, g, b, lane);
 #pragma unroll
-    for (int j = 0; j < 8; ++j)
-      if (j < nv) store4<T>(u + (size_t)r0 * d + (j * 32 + lane) * 4, v0[j]);
+    for (int j = 0; j < NV; ++j) store4<T>(u + (size_t)r0 * d + (j * 32 + lane) * 4, v0[j]);
   }
   if (r1 < rows) {
-    ln_row(v1, nv, d, eps, g, b, lane);
+    ln_row<NV>(v1, d, eps, g, b, lane);
 #pragma unroll
-    for (int j = 0; j < 8; ++j)
-      if (j < nv) store4<T>(u + (size_t)r1 * d + (j * 32 + lane) * 4, v1[j]);
+    for (int j = 0; j < NV; ++j) store4<T>(u + (size_t)r1 * d + (j * 32 + lane) * 4, v1[j]);
   }
 }
 
-template <typename T>
-__device__ __forceinline__ void ln_chain_row(float* xr, T* ur, float4 (&v)[8], int nv, int d, float eps,
-                                             const float* g1, const float* b1, const float* g2, const float* b2,
-                                             int lane) {
-  ln_row(v, nv, d, eps, g1, b1, lane);
+template <typename T, int NV>
+__device__ __forceinline__ void ln_chain_row(float* xr, T* ur, float4 (&v)[NV], float eps, const float* g1,
+                                             const float* b1, const float* g2, const float* b2, int lane) {
+  constexpr int d = NV * 128;
+  ln_row<NV>(v, d, eps, g1, b1, lane);
 #pragma unroll
-  for (int j = 0; j < 8; ++j)
-    if (j < nv) *reinterpret_cast<float4*>(xr + (j * 32 + lane) * 4) = v[j];
-  ln_row(v, nv, d, eps, g2, b2, lane);
+  for (int j = 0; j < NV; ++j) *reinterpret_cast<float4*>(xr + (j * 32 + lane) * 4) = v[j];
+  ln_row<NV>(v, d, eps, g2, b2, lane);
 #pragma unroll
-  for (int j = 0; j < 8; ++j)
-    if (j < nv) store4<T>(ur + (j * 32 + lane) * 4, v[j]);
+  for (int j = 0; j < NV; ++j) store4<T>(ur + (j * 32 + lane) * 4, v[j]);
 }
 
-template <typename T>
+template <typename T, int NV>
 __global__ void __launch_bounds__(256)
 ln_chain_kernel(float* __restrict__ x, const float* __restrict__ g1, const float* __restrict__ b1,
-                const float* __restrict__ g2, const float* __restrict__ b2, float eps, T* __restrict__ u, int rows,
-                int d) {
+                const float* __restrict__ g2, const float* __restrict__ b2, float eps, T* __restrict__ u, int rows) {
+  constexpr int d = NV * 128;
   const int r0 = blockIdx.x * 16 + (threadIdx.x >> 5), r1 = r0 + 8, lane = threadIdx.x & 31;
-  const int nv = d >> 7;
-  float4 v0[8], v1[8];
-  if (r0 < rows) load_row(x + (size_t)r0 * d, v0, nv, lane);
-  if (r1 < rows) load_row(x + (size_t)r1 * d, v1, nv, lane);
-  if (r0 < rows) ln_chain_row<T>(x + (size_t)r0 * d, u + (size_t)r0 * d, v0, nv, d, eps, g1, b1, g2, b2, lane);
-  if (r1 < rows) ln_chain_row<T>(x + (size_t)r1 * d, u + (size_t)r1 * d, v1, nv, d, eps, g1, b1, g2, b2, lane);
+  float4 v0[NV], v1[NV];
+  if (r0 < rows) load_row<NV>(x + (size_t)r0 * d, v0, lane);
+  if (r1 < rows) load_row<NV>(x + (size_t)r1 * d, v1, lane);
+  if (r0 < rows) ln_chain_row<T, NV>(x + (size_t)r0 * d, u + (size_t)r0 * d, v0, eps, g1, b1, g2, b2, lane);
+  if (r1 < rows) ln_chain_row<T, NV>(x + (size_t)r1 * d, u + (size_t)r1 * d, v1, eps, g1, b1, g2, b2, lane);
 }
 
-template <typename T, int DH>
+template <typename T, int DH, int NV>
 __global__ void __launch_bounds__(256)
 ln_rope_kernel(const float* __restrict__ x, const float* __restrict__ g, const float* __restrict__ b, float eps,
                const float* __restrict__ cos_tab, const float* __restrict__ sin_tab, Clips clips, T* __restrict__ u,
-               T* __restrict__ urot, int rows, int d) {
-  constexpr int dh = DH;
+               T* __restrict__ urot, int rows) {
+  constexpr int dh = DH, d = NV * 128, nv = NV;
   __shared__ __align__(16) float srow[8][1024];
   const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int row = blockIdx.x * 8 + w;
   if (row >= rows) return;
-  const int nv = d >> 7;
-  float4 v[8];
-  load_row(x + (size_t)row * d, v, nv, lane);
-  ln_row(v, nv, d, eps, g, b, lane);
+  float4 v[NV];
+  load_row<NV>(x + (size_t)row * d, v, lane);
+  ln_row<NV>(v, d, eps, g, b, lane);
   float* sr = srow[w];
 #pragma unroll
-  for (int j = 0; j < 8; ++j)
-    if (j < nv) {
+  for (int j = 0; j < nv; ++j) {
       const int c = (j * 32 + lane) * 4;
       store4<T>(u + (size_t)row * d + c, v[j]);
       *reinterpret_cast<float4*>(sr + c) = v[j];
@@ -158,8 +150,7 @@ ln_rope_kernel(const float* __restrict__ x, const float* __restrict__ g, const f
   const float* ct = cos_tab + (size_t)t * half;
   const float* st = sin_tab + (size_t)t * half;
 #pragma unroll
-  for (int j = 0; j < 8; ++j)
-    if (j < nv) {
+  for (int j = 0; j < nv; ++j) {
       const int c0 = (j * 32 + lane) * 4;
       float o[4];
 #pragma unroll
@@ -172,6 +163,20 @@ ln_rope_kernel(const float* __restrict__ x, const float* __restrict__ g, const f
       }
       store4<T>(urot + (size_t)row * d + c0, make_float4(o[0], o[1], o[2], o[3]));
     }
+}
+
+// Swish: exact form for the fp32 build mode; in the fp16 modes one hardware
+// tanh (relative error ~2^-11, the size of the fp16 rounding of the result).
+template <typename T>
+__device__ __forceinline__ float swish_t(float v) {
+  if constexpr (sizeof(T) == 2) {
+    const float h = 0.5f * v;
+    float t;
+    asm("tanh.approx.f32 %0, %1;" : "=f"(t) : "f"(h));
+    return fmaf(h, t, h);
+  } else {
+    return v / (1.f + expf(-v));
+  }
 }
 
 // Depthwise conv + folded BatchNorm + Swish.  CTA = 64 rows x 128 channels,
@@ -253,7 +258,7 @@ dwconv_kernel(const T* __restrict__ g, const float* __restrict__ w, const float*
         }
       }
 #pragma unroll
-      for (int i = 0; i < 8; ++i) acc[i] = __fdividef(acc[i], 1.f + __expf(-acc[i]));
+      for (int i = 0; i < 8; ++i) acc[i] = swish_t<T>(acc[i]);
     } else {
 #pragma unroll 1
       for (int i = 0; i < 8; ++i) {
@@ -266,7 +271,7 @@ dwconv_kernel(const T* __restrict__ g, const float* __restrict__ w, const float*
             const int src = ri + k - PAD;
             if (src >= li && src < hiI) a = fmaf(wk[k], tile[j0 + i + k][cc], a);
           }
-          a = __fdividef(a, 1.f + __expf(-a));
+          a = swish_t<T>(a);
         }
         acc[i] = a;
       }
@@ -298,7 +303,7 @@ dwconv_generic_kernel(const T* __restrict__ g, const float* __restrict__ w, cons
       const int src = r + k - pad;
       if (src >= lo && src < hi) a = fmaf(__ldg(w + (size_t)k * d + c), ld1(g + (size_t)src * d + c), a);
     }
-    a = __fdividef(a, 1.f + __expf(-a));
+    a = swish_t<T>(a);
   }
   if constexpr (sizeof(T) == 2) out[idx] = __float2half_rn(a);
   else out[idx] = a;
@@ -428,12 +433,21 @@ __global__ void f32_to_f16_kernel(const float* __restrict__ in, __half* __restri
 
 }  // namespace
 
+#define GAM_NV_DISPATCH(d, CALL) \
+  switch ((d) >> 7) {              \
+    case 2: { constexpr int NV = 2; CALL; } break; \
+    case 4: { constexpr int NV = 4; CALL; } break; \
+    case 6: { constexpr int NV = 6; CALL; } break; \
+    case 8: { constexpr int NV = 8; CALL; } break; \
+    default: return cudaErrorInvalidValue; \
+  }
+
 cudaError_t launch_layernorm(const float* x, const float* g, const float* b, float eps, void* u, int u_half, int rows,
                              int d, cudaStream_t s) {
   if (d % 128 || d > 1024) return cudaErrorInvalidValue;
   const int grid = (rows + 15) / 16;
-  if (u_half) ln_kernel<__half><<<grid, 256, 0, s>>>(x, g, b, eps, (__half*)u, rows, d);
-  else ln_kernel<float><<<grid, 256, 0, s>>>(x, g, b, eps, (float*)u, rows, d);
+  if (u_half) GAM_NV_DISPATCH(d, (ln_kernel<__half, NV><<<grid, 256, 0, s>>>(x, g, b, eps, (__half*)u, rows)))
+  else GAM_NV_DISPATCH(d, (ln_kernel<float, NV><<<grid, 256, 0, s>>>(x, g, b, eps, (float*)u, rows)))
   return cudaGetLastError();
 }
 
@@ -441,33 +455,31 @@ cudaError_t launch_layernorm_chain(float* x, const float* g1, const float* b1, c
                                    float eps, void* u, int u_half, int rows, int d, cudaStream_t s) {
   if (d % 128 || d > 1024) return cudaErrorInvalidValue;
   const int grid = (rows + 15) / 16;
-  if (u_half) ln_chain_kernel<__half><<<grid, 256, 0, s>>>(x, g1, b1, g2, b2, eps, (__half*)u, rows, d);
-  else ln_chain_kernel<float><<<grid, 256, 0, s>>>(x, g1, b1, g2, b2, eps, (float*)u, rows, d);
+  if (u_half) GAM_NV_DISPATCH(d, (ln_chain_kernel<__half, NV><<<grid, 256, 0, s>>>(x, g1, b1, g2, b2, eps, (__half*)u, rows)))
+  else GAM_NV_DISPATCH(d, (ln_chain_kernel<float, NV><<<grid, 256, 0, s>>>(x, g1, b1, g2, b2, eps, (float*)u, rows)))
+  return cudaGetLastError();
+}
+
+template <typename T, int DH>
+cudaError_t rope_t(const float* x, const float* g, const float* b, float eps, const float* cos_tab,
+                   const float* sin_tab, Clips clips, void* u, void* urot, int rows, int d, cudaStream_t s) {
+  const int grid = (rows + 7) / 8;
+  GAM_NV_DISPATCH(d, (ln_rope_kernel<T, DH, NV><<<grid, 256, 0, s>>>(x, g, b, eps, cos_tab, sin_tab, clips, (T*)u,
+                                                                       (T*)urot, rows)))
   return cudaGetLastError();
 }
 
 cudaError_t launch_layernorm_rope(const float* x, const float* g, const float* b, float eps, const float* cos_tab,
                                   const float* sin_tab, Clips clips, void* u, void* urot, int u_half, int rows, int d,
                                   int d_head, cudaStream_t s) {
-  if (d % 128 || d > 1024 || d_head % 4) return cudaErrorInvalidValue;
-  const int grid = (rows + 7) / 8;
+  if (d % 128 || d > 1024) return cudaErrorInvalidValue;
   if (d_head != 48 && d_head != 64) return cudaErrorInvalidValue;
   if (u_half) {
-    if (d_head == 48)
-      ln_rope_kernel<__half, 48><<<grid, 256, 0, s>>>(x, g, b, eps, cos_tab, sin_tab, clips, (__half*)u,
-                                                      (__half*)urot, rows, d);
-    else
-      ln_rope_kernel<__half, 64><<<grid, 256, 0, s>>>(x, g, b, eps, cos_tab, sin_tab, clips, (__half*)u,
-                                                      (__half*)urot, rows, d);
-  } else {
-    if (d_head == 48)
-      ln_rope_kernel<float, 48><<<grid, 256, 0, s>>>(x, g, b, eps, cos_tab, sin_tab, clips, (float*)u, (float*)urot,
-                                                     rows, d);
-    else
-      ln_rope_kernel<float, 64><<<grid, 256, 0, s>>>(x, g, b, eps, cos_tab, sin_tab, clips, (float*)u, (float*)urot,
-                                                     rows, d);
+    if (d_head == 48) return rope_t<__half, 48>(x, g, b, eps, cos_tab, sin_tab, clips, u, urot, rows, d, s);
+    return rope_t<__half, 64>(x, g, b, eps, cos_tab, sin_tab, clips, u, urot, rows, d, s);
   }
-  return cudaGetLastError();
+  if (d_head == 48) return rope_t<float, 48>(x, g, b, eps, cos_tab, sin_tab, clips, u, urot, rows, d, s);
+  return rope_t<float, 64>(x, g, b, eps, cos_tab, sin_tab, clips, u, urot, rows, d, s);
 }
 
 template <typename T>
