@@ -24,6 +24,8 @@
 #include <cudaTypedefs.h>
 
 #include <climits>
+#include <cstdlib>
+#include <cstring>
 
 #include "gemm_tc.cuh"
 #include "tc_common.cuh"
@@ -451,6 +453,224 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap mA, const __grid_constant__ C
 }
 
 // ---------------------------------------------------------------------------
+// 2-SM variant: a cluster of two CTAs computes a 256 x 256 tile with
+// tcgen05.mma.cta_group::2 (M = 256 split as 128 rows per CTA, B split as 128
+// rows per CTA).  Each CTA loads only its own 128 A rows and half of B per
+// k-block (32 KB instead of 48 KB per 128x256 of output), which is what lets
+// the mainloop run faster than L2 can feed the 1-SM tiles.  Both CTAs issue
+// their TMA loads with completion on the leader CTA's full barrier (the
+// leader expects the bytes of both); the leader alone issues the MMAs and
+// commits with a two-CTA multicast to the stage / accumulator barriers of
+// both CTAs; each CTA's epilogue reads its own TMEM rows and releases the
+// accumulator on the leader's barrier.  No TMA load uses multicast.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ uint32_t map_to_cta(const void* p, uint32_t cta) {
+  uint32_t out;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(out) : "r"(smem_u32(p)), "r"(cta));
+  return out;
+}
+__device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tma_load_2d_pair(void* dst, const CUtensorMap* map, uint32_t mbar_cluster, int x, int y) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], "
+      "[%2];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(mbar_cluster), "r"(x), "r"(y)
+      : "memory");
+}
+__device__ __forceinline__ void umma_f16_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                              uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, {%5, %6, %7, %8, %9, %10, %11, %12}, p;\n\t}\n" ::"r"(
+          d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(0), "r"(0), "r"(0), "r"(0), "r"(0), "r"(0), "r"(0),
+      "r"(0));
+}
+// Arrive once on the barrier at this offset in both CTAs of the pair when the MMAs complete.
+__device__ __forceinline__ void umma_commit_pair(uint64_t* bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
+          smem_u32(bar)),
+      "h"((uint16_t)3)
+      : "memory");
+}
+__device__ __forceinline__ void umma_commit_pair_local(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+               : "memory");
+}
+
+constexpr int kPairStages = 6;
+constexpr int kPairBH = 128;                      // B rows per CTA
+constexpr int kPairBTile = kPairBH * BK * 2;      // 16 KB
+constexpr int kPairStage = A_TILE + kPairBTile;   // 32 KB
+constexpr size_t kPairSmem = (size_t)kPairStages * kPairStage + 1024 + 256;
+
+template <int EPI>
+__global__ void __launch_bounds__(threads_of<false>(), 1)
+gemm_tc_pair_kernel(const __grid_constant__ CUtensorMap mA, const __grid_constant__ CUtensorMap mA2,
+                    const __grid_constant__ CUtensorMap mB, const TcArgs p) {
+  constexpr int BN = 256, STAGES = kPairStages;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+  uint8_t* sA = base;
+  uint8_t* sB = base + STAGES * A_TILE;
+  uint64_t* full = reinterpret_cast<uint64_t*>(base + STAGES * kPairStage);
+  uint64_t* empty = full + STAGES;
+  uint64_t* tfull = empty + STAGES;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* drain = tempty + 2;
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tslot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_rank();
+  const bool leader = rank == 0;
+  const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
+  if (threadIdx.x == 0) {
+    for (int st = 0; st < STAGES; ++st) {
+      mbar_init(&full[st], 1);
+      mbar_init(&empty[st], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&tfull[a], 1);
+      mbar_init(&tempty[a], 2 * kEpiWarps);  // epilogue warps of both CTAs
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&mA);
+    prefetch_tmap(&mA2);
+    prefetch_tmap(&mB);
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tslot)), "r"(512));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;");
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync_all();  // barriers of both CTAs initialised before any remote arrive / TMA completion
+  tc_fence_after();
+  const uint32_t tmem = *tslot;
+  const int KB = p.K / BK;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      int it = 0;
+      bool ok = true;
+      for (int tile = pair; tile < p.tiles && ok; tile += npairs) {
+        const int nb = tile % p.n_blocks, mb = tile / p.n_blocks;
+        const int m0 = mb * 256 + (int)rank * 128, n0 = nb * BN;
+        const CUtensorMap* ma = (n0 >= p.n_split) ? &mA2 : &mA;
+        for (int kb = 0; kb < KB; ++kb) {
+          const int s = it % STAGES;
+          if (!mbar_wait(&empty[s], ((it / STAGES) & 1) ^ 1, abort_flag)) {
+            ok = false;
+            break;
+          }
+          int ax = kb * BK, ay = m0;
+          if (p.conv_c) {
+            const int t = (kb * BK) / p.conv_c, c0 = kb * BK - t * p.conv_c;
+            ax = (t & 1) * p.conv_c + c0;
+            ay = m0 + (t >> 1);
+          }
+          if (leader) mbar_arrive_expect_tx(&full[s], 2 * kPairStage);
+          const uint32_t fb = map_to_cta(&full[s], 0);
+          tma_load_2d_pair(sA + s * A_TILE, ma, fb, ax, ay);
+          tma_load_2d_pair(sB + s * kPairBTile, &mB, fb, kb * BK, n0 + (int)rank * kPairBH);
+          ++it;
+        }
+      }
+      // the leader's full barriers count both CTAs' bytes: every issued copy of
+      // the pair has landed before either CTA passes the final cluster barrier
+      if (leader) {
+        const int first = it > STAGES ? it - STAGES : 0;
+        for (int j = first; j < it; ++j) {
+          const uint64_t t0 = globaltimer_ns();
+          while (!mbar_try_wait(&full[j % STAGES], (j / STAGES) & 1))
+            if (globaltimer_ns() - t0 > kWaitLimitNs) {
+              *abort_flag = 1;
+              break;
+            }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (leader && lane == 0) {
+      constexpr uint32_t idesc = idesc_f16_f32(256, BN);
+      int it = 0, local = 0;
+      bool ok = true;
+      for (int tile = pair; tile < p.tiles && ok; tile += npairs, ++local) {
+        const int acc = local & 1;
+        const uint32_t use = (uint32_t)(local >> 1);
+        if (!mbar_wait(&tempty[acc], (use & 1) ^ 1, abort_flag)) break;
+        tc_fence_after();
+        const uint32_t d = tmem + (uint32_t)(acc * BN);
+        for (int kb = 0; kb < KB; ++kb) {
+          const int s = it % STAGES;
+          if (!mbar_wait(&full[s], (it / STAGES) & 1, abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint64_t da = sdesc_k_sw128(smem_u32(sA + s * A_TILE));
+          const uint64_t db = sdesc_k_sw128(smem_u32(sB + s * kPairBTile));
+#pragma unroll
+          for (int k = 0; k < BK / 16; ++k)
+            umma_f16_pair(d, da + 2 * k, db + 2 * k, idesc, (kb | k) != 0 ? 1u : 0u);
+          umma_commit_pair(&empty[s]);
+          ++it;
+        }
+        if (ok) umma_commit_pair(&tfull[acc]);
+      }
+      umma_commit_pair_local(drain);
+      const uint64_t t0 = globaltimer_ns();
+      while (!mbar_try_wait(drain, 0))
+        if (globaltimer_ns() - t0 > kWaitLimitNs) {
+          *abort_flag = 1;
+          break;
+        }
+    }
+  } else {
+    const int q = warp & 3, half = (warp - 2) / 4;
+    int local = 0;
+    for (int tile = pair; tile < p.tiles; tile += npairs, ++local) {
+      const int acc = local & 1;
+      const uint32_t use = (uint32_t)(local >> 1);
+      if (!mbar_wait(&tfull[acc], use & 1, abort_flag)) break;
+      tc_fence_after();
+      const int nb = tile % p.n_blocks, mb = tile / p.n_blocks;
+      const int r = mb * 256 + (int)rank * 128 + q * 32 + lane;
+      const uint32_t tbase = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN);
+      epilogue_tile<BN, EPI>(p, r, nb * BN, tbase, half);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_remote(map_to_cta(&tempty[acc], 0));
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync_all();  // the leader's MMAs (reading both CTAs' shared memory) and remote arrives are done
+  if (threadIdx.x == 0 && *abort_flag) atomicExch(p.status, 1);
+  if (warp == 1) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(512));
+  }
+}
+
+// ---------------------------------------------------------------------------
 // host side
 // ---------------------------------------------------------------------------
 
@@ -508,6 +728,64 @@ cudaError_t launch_epi(TcGemmCache* cache, const CUtensorMap& mA, const CUtensor
   return cudaGetLastError();
 }
 
+template <int EPI>
+cudaError_t launch_pair_epi(TcGemmCache* cache, const CUtensorMap& mA, const CUtensorMap& mA2, const CUtensorMap& mB,
+                            const TcArgs& args, cudaStream_t s) {
+  auto kern = gemm_tc_pair_kernel<EPI>;
+  static int max_clusters = 0;  // co-resident clusters of two (per process; one device model)
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kPairSmem);
+  if (e != cudaSuccess) return e;
+  if (!max_clusters) {
+    cudaLaunchConfig_t q = {};
+    cudaLaunchAttribute qa[1];
+    qa[0].id = cudaLaunchAttributeClusterDimension;
+    qa[0].val.clusterDim.x = 2;
+    qa[0].val.clusterDim.y = 1;
+    qa[0].val.clusterDim.z = 1;
+    q.gridDim = dim3(2 * (cache->sm_count / 2));
+    q.blockDim = dim3(threads_of<false>());
+    q.dynamicSmemBytes = kPairSmem;
+    q.attrs = qa;
+    q.numAttrs = 1;
+    int n = 0;
+    e = cudaOccupancyMaxActiveClusters(&n, kern, &q);
+    if (e != cudaSuccess) return e;
+    if (n < 1) return cudaErrorInvalidConfiguration;
+    max_clusters = n;
+  }
+  const int pairs = args.tiles < max_clusters ? args.tiles : max_clusters;
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.gridDim = dim3(2 * pairs);
+  cfg.blockDim = dim3(threads_of<false>());
+  cfg.dynamicSmemBytes = kPairSmem;
+  cfg.stream = s;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, kern, mA, mA2, mB, args);
+  if (e != cudaSuccess) return e;
+  return cudaGetLastError();
+}
+
+cudaError_t launch_pair(TcGemmCache* cache, const CUtensorMap& mA, const CUtensorMap& mA2, const CUtensorMap& mB,
+                        const TcArgs& args, cudaStream_t s) {
+  switch (args.epi) {
+    case EPI_SWISH: return launch_pair_epi<EPI_SWISH>(cache, mA, mA2, mB, args, s);
+    case EPI_GLU: return launch_pair_epi<EPI_GLU>(cache, mA, mA2, mB, args, s);
+    case EPI_RESID: return launch_pair_epi<EPI_RESID>(cache, mA, mA2, mB, args, s);
+    case EPI_QKV: return launch_pair_epi<EPI_QKV>(cache, mA, mA2, mB, args, s);
+    case EPI_CONV1: return launch_pair_epi<EPI_CONV1>(cache, mA, mA2, mB, args, s);
+    case EPI_CONV2: return launch_pair_epi<EPI_CONV2>(cache, mA, mA2, mB, args, s);
+    case EPI_F32: return launch_pair_epi<EPI_F32>(cache, mA, mA2, mB, args, s);
+    case EPI_POWER: return launch_pair_epi<EPI_POWER>(cache, mA, mA2, mB, args, s);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
 template <int BN, int STAGES, bool QB>
 cudaError_t launch_bn(TcGemmCache* cache, const CUtensorMap& mA, const CUtensorMap& mA2, const CUtensorMap& mB,
                       const TcArgs& args, cudaStream_t s) {
@@ -537,6 +815,12 @@ cudaError_t tc_init(TcGemmCache* cache, int device) {
   if (e != cudaSuccess) return e;
   e = cudaDeviceGetAttribute(&cache->sm_count, cudaDevAttrMultiProcessorCount, device);
   if (e != cudaSuccess) return e;
+  // GAM_GEMM_TILES=single|pair|auto (default auto): tile-shape policy of the fp16 GEMMs
+  if (const char* v = std::getenv("GAM_GEMM_TILES")) {
+    if (!std::strcmp(v, "single")) cache->pair_mode = 0;
+    else if (!std::strcmp(v, "pair")) cache->pair_mode = 2;
+    else cache->pair_mode = 1;
+  }
   e = cudaMalloc(&cache->status, sizeof(int));
   if (e != cudaSuccess) return e;
   return cudaMemset(cache->status, 0, sizeof(int));
@@ -562,12 +846,29 @@ int choose_bn(int M, int N, int epi, int sms) {
   return best;
 }
 
+// Paired-CTA tiles (256 x 256 per two SMs) for fp16 weights when there are
+// enough of them to fill the GPU at least twice over; otherwise the single-CTA
+// tile chosen by choose_bn.
+bool choose_pair(const TcGemmCache* cache, int M, int N) {
+  if (N % 256 || cache->pair_mode == 0) return false;
+  if (cache->pair_mode == 2) return true;
+  const int tiles = ((M + 255) / 256) * (N / 256);
+  return tiles >= cache->sm_count;
+}
+
 cudaError_t launch_gemm_tc(TcGemmCache* cache, const void* A, const void* A2, int n_split, int lda, WeightOp B, int M,
-                           int N, int K, int epi, const EpiParams& ep, cudaStream_t s) {
+                           int N, int K, int epi, const EpiParams& ep, cudaStream_t s, int variant) {
   if (!tc_supported(1, B.dtype, N, K, epi) || M <= 0) return cudaErrorInvalidValue;
   const bool qb = B.dtype == 2;
   if (qb && !B.scale_t) return cudaErrorInvalidValue;
-  const int BN = choose_bn(M, N, epi, cache->sm_count);
+  bool pair = false;
+  if (variant == 1) {
+    if (qb || N % 256) return cudaErrorInvalidValue;
+    pair = true;
+  } else if (variant < 0) {
+    pair = !qb && choose_pair(cache, M, N);
+  }
+  const int BN = pair ? 256 : choose_bn(M, N, epi, cache->sm_count);
   if (!BN) return cudaErrorInvalidValue;
   // lda < K: stride-2 convolution view (lda = 2C, K = taps * C, C % 64 == 0); the
   // buffer behind it holds (M + 2) * lda elements, mapped as M + 2 rows of 2C.
@@ -578,13 +879,15 @@ cudaError_t launch_gemm_tc(TcGemmCache* cache, const void* A, const void* A2, in
                        : make_map_f16(&mA, A, K, M, (uint64_t)lda * 2, BK, BM);
   if (e == cudaSuccess && !conv) e = make_map_f16(&mA2, A2 ? A2 : A, K, M, (uint64_t)lda * 2, BK, BM);
   if (conv) mA2 = mA;
-  if (e == cudaSuccess) e = qb ? make_map_i8(&mB, B.w, K, N, BK, BN) : make_map_f16(&mB, B.w, K, N, (uint64_t)K * 2, BK, BN);
+  if (e == cudaSuccess)
+    e = qb ? make_map_i8(&mB, B.w, K, N, BK, BN)
+           : make_map_f16(&mB, B.w, K, N, (uint64_t)K * 2, BK, pair ? (uint32_t)kPairBH : (uint32_t)BN);
   if (e != cudaSuccess) return e;
   TcArgs args;
   args.M = M;
   args.N = N;
   args.K = K;
-  args.m_blocks = (M + BM - 1) / BM;
+  args.m_blocks = pair ? (M + 255) / 256 : (M + BM - 1) / BM;
   args.n_blocks = N / BN;
   args.tiles = args.m_blocks * args.n_blocks;
   args.n_split = A2 ? n_split : INT_MAX;
@@ -593,6 +896,7 @@ cudaError_t launch_gemm_tc(TcGemmCache* cache, const void* A, const void* A2, in
   args.ep = ep;
   args.scale_t = B.scale_t;
   args.status = cache->status;
+  if (pair) return launch_pair(cache, mA, mA2, mB, args, s);
   // stages: as many as fit in ~200 KB of shared memory
   if (qb) {
     if (BN == 256) return launch_bn<256, 3, true>(cache, mA, mA2, mB, args, s);

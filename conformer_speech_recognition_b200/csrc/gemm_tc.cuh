@@ -10,6 +10,9 @@ namespace gam {
 struct TcGemmCache {
   int* status = nullptr;  // device word set when a bounded wait gives up
   int sm_count = 148;
+  // fp16 GEMM tiles: 0 single-CTA only, 1 paired-CTA (cta_group::2) 256 x 256 tiles
+  // where they are cheaper, 2 paired-CTA tiles wherever N % 256 == 0
+  int pair_mode = 1;
 };
 
 // Resolves the driver's tensor-map encoder and allocates the status word.
@@ -18,8 +21,10 @@ cudaError_t tc_init(TcGemmCache* cache, int device);
 // True when the tensor-core GEMM handles this operand / shape / epilogue combination.
 bool tc_supported(int a_dtype, int b_dtype, int N, int K, int epi);
 
+// variant: -1 chooses the tile shape, 0 forces single-CTA tiles, 1 forces paired-CTA
+// 256 x 256 tiles (fp16 weights, N % 256 == 0).
 cudaError_t launch_gemm_tc(TcGemmCache* cache, const void* A, const void* A2, int n_split, int lda, WeightOp B,
-                           int M, int N, int K, int epi, const EpiParams& ep, cudaStream_t s);
+                           int M, int N, int K, int epi, const EpiParams& ep, cudaStream_t s, int variant = -1);
 
 // Masked multi-head attention on tensor cores (fp16 Q/K/V^T, see attention_tc.cu).
 cudaError_t launch_attention_tc(TcGemmCache* cache, const void* qk, const void* vt, Clips clips, void* o,

@@ -1063,10 +1063,13 @@ gam_status gam_debug_gemm(gam_ctx* c, int impl, const void* a, int lda, const vo
   ep.alpha = 1.f;
   ep.ldo = ldo;
   WeightOp W{w, nullptr, 1, nullptr};
-  if (impl == 0) {
+  if (impl == 0 || impl == 2 || impl == 3) {
     if (!tc_supported(1, 1, n, k, EPI_RESID)) return fail(c, GAM_ERR_SHAPE, "tensor-core GEMM needs N % 256 == 0, K % 64 == 0");
-    return run_kernel(c, PK_MISC, s, [&] { return launch_gemm_tc(&c->tc, a, nullptr, 0, lda, W, m, n, k, EPI_RESID, ep, s); });
+    const int variant = impl == 0 ? -1 : impl == 2 ? 0 : 1;
+    return run_kernel(c, PK_MISC, s,
+                      [&] { return launch_gemm_tc(&c->tc, a, nullptr, 0, lda, W, m, n, k, EPI_RESID, ep, s, variant); });
   }
+  if (impl != 1) return fail(c, GAM_ERR_INVALID_ARG, "impl must be 0, 1, 2 or 3");
   if (k % 16 || n % 128) return fail(c, GAM_ERR_SHAPE, "CUDA-core GEMM needs N % 128 == 0, K % 16 == 0");
   return run_kernel(c, PK_MISC, s, [&] { return launch_gemm_simt(1, a, nullptr, 0, lda, W, m, n, k, EPI_RESID, 0, ep, s); });
 }

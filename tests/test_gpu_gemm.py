@@ -1,6 +1,8 @@
 """Unit parity of the encoder's GEMM kernels through the C ABI (gam_debug_gemm):
 out += A . W^T + bias with fp16 operands and fp32 accumulation, for the
-tensor-core (tcgen05) and CUDA-core implementations, against NumPy in fp64."""
+tensor-core (tcgen05) and CUDA-core implementations, against NumPy in fp64.
+impl 0 lets the library choose the tile shape, 2 forces single-CTA tiles and
+3 forces paired-CTA (cta_group::2) 256 x 256 tiles."""
 import numpy as np
 import pytest
 
@@ -21,7 +23,7 @@ def ctx():
     c.close()
 
 
-@pytest.mark.parametrize("impl", [0, 1], ids=["tcgen05", "cuda_cores"])
+@pytest.mark.parametrize("impl", [0, 1, 2, 3], ids=["tcgen05", "cuda_cores", "tc_single_cta", "tc_cta_pair"])
 @pytest.mark.parametrize("M,N,K,lda", [(128, 256, 64, 64), (300, 512, 320, 320), (1000, 768, 768, 768),
                                        (5000, 3072, 768, 768), (2100, 256, 3072, 3072),
                                        (777, 768, 320, 128)],
@@ -53,3 +55,13 @@ def test_gemm_parity(ctx, impl, M, N, K, lda):
 def test_gemm_tile_widths(ctx, M, N, K):
     """Shapes for which the tensor-core GEMM picks a 192- or 128-column tile."""
     test_gemm_parity(ctx, 0, M, N, K, K)
+
+
+@pytest.mark.parametrize("M,N,K,lda", [(129, 256, 64, 64), (256, 512, 128, 128), (20000, 3072, 768, 768),
+                                       (4097, 768, 3072, 3072), (3001, 1536, 1536, 768)],
+                         ids=["peer_rows_empty", "one_pair_tile", "more_tiles_than_pairs", "deep_k_ragged",
+                              "strided_view_wide"])
+def test_gemm_cta_pair(ctx, M, N, K, lda):
+    """Paired-CTA tiles: a pair whose second CTA holds only padding rows, a single
+    pair tile, more tiles than co-resident pairs, and the convolution view."""
+    test_gemm_parity(ctx, 3, M, N, K, lda)
