@@ -12,9 +12,11 @@
 //   warps 2..9  epilogue: tcgen05.ld of the accumulator (warp w reads TMEM
 //               lanes 32*(w%4) .. +31 = its 32 output rows, and one half of
 //               the tile's columns, so two warps share each sub-partition and
-//               hide each other's latency), bias + activation / residual /
-//               scatter, global stores; then hand the accumulator back so the
-//               next tile's MMAs overlap this epilogue.
+//               hide each other's latency), bias + activation / scatter and
+//               global stores, or for the residual update x += alpha (acc + b)
+//               a 32 x 32 staging tile per warp that a TMA reduction adds into
+//               x at the L2; then hand the accumulator back so the next tile's
+//               MMAs overlap this epilogue.
 // Tiles are visited n-fastest so the CTAs in flight share each A row block
 // through L2 and the weight (a few MB) stays L2-resident.
 // Every mbarrier wait is bounded (tc_common.cuh); a wait that gives up raises
@@ -49,14 +51,26 @@ struct TcArgs {
   int* status;
 };
 
-template <int BN, int STAGES, bool QB>
+// Residual epilogue: per epilogue warp a 32 x 32 fp32 staging tile (4 KB, 128-byte
+// swizzle) that a TMA reduction adds into x.
+constexpr int kEpiWarps = 8;
+constexpr int kStageTile = 32 * 32 * 4;
+template <int EPI>
+__host__ __device__ constexpr int epi_smem() { return EPI == EPI_RESID ? kEpiWarps * kStageTile : 0; }
+// Shared memory for the operand ring: what is left of 227 KB after the epilogue
+// staging and 1.25 KB of alignment slack and barriers, at most 8 stages.
+template <int EPI>
+__host__ __device__ constexpr int ring_budget() { return 227 * 1024 - 1280 - epi_smem<EPI>(); }
+
+template <int BN, bool QB, int EPI>
 struct Cfg {
   static constexpr int B_TILE = BN * BK * 2;                 // fp16 B operand (128-byte swizzle)
   static constexpr int RAW_TILE = QB ? BN * BK : 0;          // INT8 weights as loaded (64-byte rows)
   static constexpr int TX = A_TILE + (QB ? RAW_TILE : B_TILE);  // bytes landed by TMA per stage
   static constexpr int STAGE = A_TILE + B_TILE + RAW_TILE;
+  static constexpr int STAGES = ring_budget<EPI>() / STAGE < 8 ? ring_budget<EPI>() / STAGE : 8;
   static constexpr int TMEM_COLS = BN == 128 ? 256 : 512;  // two accumulators, rounded to a power of two
-  static constexpr size_t SMEM = (size_t)STAGES * STAGE + 1024 + 256;
+  static constexpr size_t SMEM = (size_t)STAGES * STAGE + epi_smem<EPI>() + 1024 + 256;
 };
 
 // Hardware tanh (tanh.approx, one special-function op, relative error about
@@ -113,18 +127,6 @@ __device__ __forceinline__ void epi_chunk(const TcArgs& p, int r, int n, bool va
       store_half16(o, v);
       store_half16(o + 16, v + 16);
     } break;
-    case EPI_RESID: {
-      float4* px = reinterpret_cast<float4*>(ep.x + (size_t)r * ep.ldo + n);
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        float4 a = px[j];
-        a.x += ep.alpha * v[4 * j];
-        a.y += ep.alpha * v[4 * j + 1];
-        a.z += ep.alpha * v[4 * j + 2];
-        a.w += ep.alpha * v[4 * j + 3];
-        px[j] = a;
-      }
-    } break;
     case EPI_CONV1: {
 #pragma unroll
       for (int j = 0; j < 32; ++j) v[j] = valid ? fmaxf(v[j], 0.f) : 0.f;
@@ -173,7 +175,8 @@ __device__ __forceinline__ void epi_chunk(const TcArgs& p, int r, int n, bool va
 // or for the paired epilogues (GLU, power: 128-column blocks [first 64 | second 64])
 // the (first, second) pairs of 32-column chunks number half * BN/128 .. (half+1) * BN/128 - 1.
 template <int BN, int EPI>
-__device__ __forceinline__ void epilogue_tile(const TcArgs& p, int r, int n0, uint32_t tbase, int half) {
+__device__ __forceinline__ void epilogue_tile(const TcArgs& p, int r, int n0, uint32_t tbase, int half,
+                                              const CUtensorMap* mX, uint8_t* stage) {
   const int c_lo = half * (BN / 2), c_hi = (half + 1) * (BN / 2);
   const EpiParams& ep = p.ep;
   const bool in_m = r < p.M;
@@ -232,6 +235,35 @@ __device__ __forceinline__ void epilogue_tile(const TcArgs& p, int r, int n0, ui
         store_half16(o + 16, y + 16);
       }
     }
+  } else if constexpr (EPI == EPI_RESID) {
+    // x += alpha (acc + bias): this warp stages its 32 rows x 32 columns and one
+    // lane hands them to a TMA reduction, so the L2 does the read-modify-write
+    // of x (rows past M are clipped by the tensor map)
+    const int lane = threadIdx.x & 31, row0 = r - lane;
+#pragma unroll 1
+    for (int c = c_lo; c < c_hi; c += 32) {
+      uint32_t u[32];
+      tmem_ld32(tbase + c, u);
+      tmem_ld_wait();
+      if (row0 >= p.M) continue;
+      float v[32];
+      load_bias32(ep.bias + n0 + c, v);
+#pragma unroll
+      for (int j = 0; j < 32; ++j) v[j] = ep.alpha * (__uint_as_float(u[j]) + v[j]);
+      if (lane == 0) bulk_wait_read0();  // the previous reduction has read the staging tile
+      __syncwarp();
+      uint8_t* row = stage + lane * 128;
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+        *reinterpret_cast<float4*>(row + ((j ^ (lane & 7)) << 4)) =
+            make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+      fence_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        tma_reduce_add_2d(mX, stage, n0 + c, row0);
+        bulk_commit();
+      }
+    }
   } else {
 #pragma unroll 1
     for (int c = c_lo; c < c_hi; c += 32) {
@@ -243,7 +275,6 @@ __device__ __forceinline__ void epilogue_tile(const TcArgs& p, int r, int n0, ui
   }
 }
 
-constexpr int kEpiWarps = 8;
 constexpr int kCvtWarps = 4;  // INT8 variant: warps that dequantise the weight tile
 template <bool QB>
 constexpr int threads_of() { return 64 + 32 * kEpiWarps + (QB ? 32 * kCvtWarps : 0); }
@@ -270,17 +301,19 @@ __device__ __forceinline__ void dequant16(uint4 raw, __half2 s2, uint4& out0, ui
   out1 = make_uint4(o[4], o[5], o[6], o[7]);
 }
 
-template <int BN, int STAGES, int EPI, bool QB>
+template <int BN, int EPI, bool QB>
 __global__ void __launch_bounds__(threads_of<QB>(), 1)
 gemm_tc_kernel(const __grid_constant__ CUtensorMap mA, const __grid_constant__ CUtensorMap mA2,
-               const __grid_constant__ CUtensorMap mB, const TcArgs p) {
-  using C = Cfg<BN, STAGES, QB>;
+               const __grid_constant__ CUtensorMap mB, const __grid_constant__ CUtensorMap mX, const TcArgs p) {
+  using C = Cfg<BN, QB, EPI>;
+  constexpr int STAGES = C::STAGES;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
   uint8_t* sA = base;
   uint8_t* sB = base + STAGES * A_TILE;
   uint8_t* sRaw = sB + STAGES * C::B_TILE;  // INT8 variant only
-  uint64_t* full = reinterpret_cast<uint64_t*>(base + STAGES * C::STAGE);
+  uint8_t* sEpi = base + STAGES * C::STAGE;  // residual epilogue staging, kStageTile per warp
+  uint64_t* full = reinterpret_cast<uint64_t*>(sEpi + epi_smem<EPI>());
   uint64_t* empty = full + STAGES;
   uint64_t* tfull = empty + STAGES;
   uint64_t* tempty = tfull + 2;
@@ -438,11 +471,12 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap mA, const __grid_constant__ C
       const int nb = tile % p.n_blocks, mb = tile / p.n_blocks;
       const int r = mb * BM + q * 32 + lane;
       const uint32_t tbase = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN);
-      epilogue_tile<BN, EPI>(p, r, nb * BN, tbase, half);
+      epilogue_tile<BN, EPI>(p, r, nb * BN, tbase, half, &mX, sEpi + (warp - 2) * kStageTile);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&tempty[acc]);
     }
+    if (EPI == EPI_RESID && lane == 0) bulk_wait0();  // reductions complete before the CTA exits
   }
   __syncthreads();
   if (threadIdx.x == 0 && *abort_flag) atomicExch(p.status, 1);
@@ -510,22 +544,30 @@ __device__ __forceinline__ void umma_commit_pair_local(uint64_t* bar) {
                : "memory");
 }
 
-constexpr int kPairStages = 6;
-constexpr int kPairBH = 128;                      // B rows per CTA
-constexpr int kPairBTile = kPairBH * BK * 2;      // 16 KB
-constexpr int kPairStage = A_TILE + kPairBTile;   // 32 KB
-constexpr size_t kPairSmem = (size_t)kPairStages * kPairStage + 1024 + 256;
+// TN output columns per pair tile (128, 192 or 256): each CTA holds TN/2 rows of
+// B per stage; two accumulators of TN columns in TMEM.
+template <int TN, int EPI>
+struct PairCfg {
+  static constexpr int BH = TN / 2;                      // B rows per CTA
+  static constexpr int B_TILE = BH * BK * 2;
+  static constexpr int STAGE = A_TILE + B_TILE;
+  static constexpr int STAGES = ring_budget<EPI>() / STAGE < 8 ? ring_budget<EPI>() / STAGE : 8;
+  static constexpr int TMEM_COLS = TN == 128 ? 256 : 512;
+  static constexpr size_t SMEM = (size_t)STAGES * STAGE + epi_smem<EPI>() + 1024 + 256;
+};
 
-template <int EPI>
+template <int TN, int EPI>
 __global__ void __launch_bounds__(threads_of<false>(), 1)
 gemm_tc_pair_kernel(const __grid_constant__ CUtensorMap mA, const __grid_constant__ CUtensorMap mA2,
-                    const __grid_constant__ CUtensorMap mB, const TcArgs p) {
-  constexpr int BN = 256, STAGES = kPairStages;
+                    const __grid_constant__ CUtensorMap mB, const __grid_constant__ CUtensorMap mX, const TcArgs p) {
+  using C = PairCfg<TN, EPI>;
+  constexpr int BN = TN, STAGES = C::STAGES;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
   uint8_t* sA = base;
   uint8_t* sB = base + STAGES * A_TILE;
-  uint64_t* full = reinterpret_cast<uint64_t*>(base + STAGES * kPairStage);
+  uint8_t* sEpi = base + STAGES * C::STAGE;  // residual epilogue staging, kStageTile per warp
+  uint64_t* full = reinterpret_cast<uint64_t*>(sEpi + epi_smem<EPI>());
   uint64_t* empty = full + STAGES;
   uint64_t* tfull = empty + STAGES;
   uint64_t* tempty = tfull + 2;
@@ -556,7 +598,8 @@ gemm_tc_pair_kernel(const __grid_constant__ CUtensorMap mA, const __grid_constan
     prefetch_tmap(&mB);
   }
   if (warp == 1) {
-    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tslot)), "r"(512));
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tslot)),
+                 "r"(C::TMEM_COLS));
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;");
   }
   tc_fence_before();
@@ -586,10 +629,10 @@ gemm_tc_pair_kernel(const __grid_constant__ CUtensorMap mA, const __grid_constan
             ax = (t & 1) * p.conv_c + c0;
             ay = m0 + (t >> 1);
           }
-          if (leader) mbar_arrive_expect_tx(&full[s], 2 * kPairStage);
+          if (leader) mbar_arrive_expect_tx(&full[s], 2 * C::STAGE);
           const uint32_t fb = map_to_cta(&full[s], 0);
           tma_load_2d_pair(sA + s * A_TILE, ma, fb, ax, ay);
-          tma_load_2d_pair(sB + s * kPairBTile, &mB, fb, kb * BK, n0 + (int)rank * kPairBH);
+          tma_load_2d_pair(sB + s * C::B_TILE, &mB, fb, kb * BK, n0 + (int)rank * C::BH);
           ++it;
         }
       }
@@ -626,7 +669,7 @@ gemm_tc_pair_kernel(const __grid_constant__ CUtensorMap mA, const __grid_constan
           }
           tc_fence_after();
           const uint64_t da = sdesc_k_sw128(smem_u32(sA + s * A_TILE));
-          const uint64_t db = sdesc_k_sw128(smem_u32(sB + s * kPairBTile));
+          const uint64_t db = sdesc_k_sw128(smem_u32(sB + s * C::B_TILE));
 #pragma unroll
           for (int k = 0; k < BK / 16; ++k)
             umma_f16_pair(d, da + 2 * k, db + 2 * k, idesc, (kb | k) != 0 ? 1u : 0u);
@@ -654,11 +697,12 @@ gemm_tc_pair_kernel(const __grid_constant__ CUtensorMap mA, const __grid_constan
       const int nb = tile % p.n_blocks, mb = tile / p.n_blocks;
       const int r = mb * 256 + (int)rank * 128 + q * 32 + lane;
       const uint32_t tbase = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN);
-      epilogue_tile<BN, EPI>(p, r, nb * BN, tbase, half);
+      epilogue_tile<BN, EPI>(p, r, nb * BN, tbase, half, &mX, sEpi + (warp - 2) * kStageTile);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_remote(map_to_cta(&tempty[acc], 0));
     }
+    if (EPI == EPI_RESID && lane == 0) bulk_wait0();  // reductions complete before the CTA exits
   }
   tc_fence_before();
   __syncthreads();
@@ -666,7 +710,7 @@ gemm_tc_pair_kernel(const __grid_constant__ CUtensorMap mA, const __grid_constan
   if (threadIdx.x == 0 && *abort_flag) atomicExch(p.status, 1);
   if (warp == 1) {
     tc_fence_after();
-    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(512));
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(C::TMEM_COLS));
   }
 }
 
@@ -702,6 +746,21 @@ cudaError_t make_map_f16(CUtensorMap* m, const void* ptr, uint64_t inner, uint64
   return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
+// 2D fp32 tensor map with 128-byte swizzle (box_inner * 4 must be 128), used for
+// the residual reductions; out-of-bounds elements are neither read nor written.
+cudaError_t make_map_f32(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t outer, uint64_t stride_bytes,
+                         uint32_t box_inner, uint32_t box_outer) {
+  if ((reinterpret_cast<uintptr_t>(ptr) & 15) || (stride_bytes & 15)) return cudaErrorInvalidValue;
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {stride_bytes};
+  cuuint32_t box[2] = {box_inner, box_outer};
+  cuuint32_t es[2] = {1, 1};
+  CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<void*>(ptr), dims, strides, box, es,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
 // 2D INT8 tensor map, no swizzle (64-byte rows of the raw weight tile).
 cudaError_t make_map_i8(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t outer, uint32_t box_inner,
                         uint32_t box_outer) {
@@ -716,88 +775,80 @@ cudaError_t make_map_i8(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_
   return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
-template <int BN, int STAGES, int EPI, bool QB>
+template <int BN, int EPI, bool QB>
 cudaError_t launch_epi(TcGemmCache* cache, const CUtensorMap& mA, const CUtensorMap& mA2, const CUtensorMap& mB,
-                       const TcArgs& args, cudaStream_t s) {
-  using C = Cfg<BN, STAGES, QB>;
-  auto kern = gemm_tc_kernel<BN, STAGES, EPI, QB>;
+                       const CUtensorMap& mX, const TcArgs& args, cudaStream_t s) {
+  using C = Cfg<BN, QB, EPI>;
+  auto kern = gemm_tc_kernel<BN, EPI, QB>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::SMEM);
   if (e != cudaSuccess) return e;
   const int grid = args.tiles < cache->sm_count ? args.tiles : cache->sm_count;
-  kern<<<grid, threads_of<QB>(), C::SMEM, s>>>(mA, mA2, mB, args);
+  kern<<<grid, threads_of<QB>(), C::SMEM, s>>>(mA, mA2, mB, mX, args);
   return cudaGetLastError();
 }
 
-template <int EPI>
+template <int TN, int EPI>
 cudaError_t launch_pair_epi(TcGemmCache* cache, const CUtensorMap& mA, const CUtensorMap& mA2, const CUtensorMap& mB,
-                            const TcArgs& args, cudaStream_t s) {
-  auto kern = gemm_tc_pair_kernel<EPI>;
+                            const CUtensorMap& mX, const TcArgs& args, cudaStream_t s) {
+  using C = PairCfg<TN, EPI>;
+  auto kern = gemm_tc_pair_kernel<TN, EPI>;
   static int max_clusters = 0;  // co-resident clusters of two (per process; one device model)
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kPairSmem);
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::SMEM);
   if (e != cudaSuccess) return e;
-  if (!max_clusters) {
-    cudaLaunchConfig_t q = {};
-    cudaLaunchAttribute qa[1];
-    qa[0].id = cudaLaunchAttributeClusterDimension;
-    qa[0].val.clusterDim.x = 2;
-    qa[0].val.clusterDim.y = 1;
-    qa[0].val.clusterDim.z = 1;
-    q.gridDim = dim3(2 * (cache->sm_count / 2));
-    q.blockDim = dim3(threads_of<false>());
-    q.dynamicSmemBytes = kPairSmem;
-    q.attrs = qa;
-    q.numAttrs = 1;
-    int n = 0;
-    e = cudaOccupancyMaxActiveClusters(&n, kern, &q);
-    if (e != cudaSuccess) return e;
-    if (n < 1) return cudaErrorInvalidConfiguration;
-    max_clusters = n;
-  }
-  const int pairs = args.tiles < max_clusters ? args.tiles : max_clusters;
-  cudaLaunchConfig_t cfg = {};
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = 2;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
-  cfg.gridDim = dim3(2 * pairs);
+  cudaLaunchConfig_t cfg = {};
   cfg.blockDim = dim3(threads_of<false>());
-  cfg.dynamicSmemBytes = kPairSmem;
-  cfg.stream = s;
+  cfg.dynamicSmemBytes = C::SMEM;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  e = cudaLaunchKernelEx(&cfg, kern, mA, mA2, mB, args);
+  if (!max_clusters) {
+    cfg.gridDim = dim3(2 * (cache->sm_count / 2));
+    int n = 0;
+    e = cudaOccupancyMaxActiveClusters(&n, kern, &cfg);
+    if (e != cudaSuccess) return e;
+    if (n < 1) return cudaErrorInvalidConfiguration;
+    max_clusters = n;
+  }
+  const int pairs = args.tiles < max_clusters ? args.tiles : max_clusters;
+  cfg.gridDim = dim3(2 * pairs);
+  cfg.stream = s;
+  e = cudaLaunchKernelEx(&cfg, kern, mA, mA2, mB, mX, args);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
+template <int TN>
 cudaError_t launch_pair(TcGemmCache* cache, const CUtensorMap& mA, const CUtensorMap& mA2, const CUtensorMap& mB,
-                        const TcArgs& args, cudaStream_t s) {
+                        const CUtensorMap& mX, const TcArgs& args, cudaStream_t s) {
   switch (args.epi) {
-    case EPI_SWISH: return launch_pair_epi<EPI_SWISH>(cache, mA, mA2, mB, args, s);
-    case EPI_GLU: return launch_pair_epi<EPI_GLU>(cache, mA, mA2, mB, args, s);
-    case EPI_RESID: return launch_pair_epi<EPI_RESID>(cache, mA, mA2, mB, args, s);
-    case EPI_QKV: return launch_pair_epi<EPI_QKV>(cache, mA, mA2, mB, args, s);
-    case EPI_CONV1: return launch_pair_epi<EPI_CONV1>(cache, mA, mA2, mB, args, s);
-    case EPI_CONV2: return launch_pair_epi<EPI_CONV2>(cache, mA, mA2, mB, args, s);
-    case EPI_F32: return launch_pair_epi<EPI_F32>(cache, mA, mA2, mB, args, s);
-    case EPI_POWER: return launch_pair_epi<EPI_POWER>(cache, mA, mA2, mB, args, s);
+    case EPI_SWISH: return launch_pair_epi<TN, EPI_SWISH>(cache, mA, mA2, mB, mX, args, s);
+    case EPI_GLU: return launch_pair_epi<TN, EPI_GLU>(cache, mA, mA2, mB, mX, args, s);
+    case EPI_RESID: return launch_pair_epi<TN, EPI_RESID>(cache, mA, mA2, mB, mX, args, s);
+    case EPI_QKV: return launch_pair_epi<TN, EPI_QKV>(cache, mA, mA2, mB, mX, args, s);
+    case EPI_CONV1: return launch_pair_epi<TN, EPI_CONV1>(cache, mA, mA2, mB, mX, args, s);
+    case EPI_CONV2: return launch_pair_epi<TN, EPI_CONV2>(cache, mA, mA2, mB, mX, args, s);
+    case EPI_F32: return launch_pair_epi<TN, EPI_F32>(cache, mA, mA2, mB, mX, args, s);
+    case EPI_POWER: return launch_pair_epi<TN, EPI_POWER>(cache, mA, mA2, mB, mX, args, s);
     default: return cudaErrorInvalidValue;
   }
 }
 
-template <int BN, int STAGES, bool QB>
+template <int BN, bool QB>
 cudaError_t launch_bn(TcGemmCache* cache, const CUtensorMap& mA, const CUtensorMap& mA2, const CUtensorMap& mB,
-                      const TcArgs& args, cudaStream_t s) {
+                      const CUtensorMap& mX, const TcArgs& args, cudaStream_t s) {
   switch (args.epi) {
-    case EPI_SWISH: return launch_epi<BN, STAGES, EPI_SWISH, QB>(cache, mA, mA2, mB, args, s);
-    case EPI_GLU: return launch_epi<BN, STAGES, EPI_GLU, QB>(cache, mA, mA2, mB, args, s);
-    case EPI_RESID: return launch_epi<BN, STAGES, EPI_RESID, QB>(cache, mA, mA2, mB, args, s);
-    case EPI_QKV: return launch_epi<BN, STAGES, EPI_QKV, QB>(cache, mA, mA2, mB, args, s);
-    case EPI_CONV1: return launch_epi<BN, STAGES, EPI_CONV1, QB>(cache, mA, mA2, mB, args, s);
-    case EPI_CONV2: return launch_epi<BN, STAGES, EPI_CONV2, QB>(cache, mA, mA2, mB, args, s);
-    case EPI_F32: return launch_epi<BN, STAGES, EPI_F32, QB>(cache, mA, mA2, mB, args, s);
-    case EPI_POWER: return launch_epi<BN, STAGES, EPI_POWER, QB>(cache, mA, mA2, mB, args, s);
+    case EPI_SWISH: return launch_epi<BN, EPI_SWISH, QB>(cache, mA, mA2, mB, mX, args, s);
+    case EPI_GLU: return launch_epi<BN, EPI_GLU, QB>(cache, mA, mA2, mB, mX, args, s);
+    case EPI_RESID: return launch_epi<BN, EPI_RESID, QB>(cache, mA, mA2, mB, mX, args, s);
+    case EPI_QKV: return launch_epi<BN, EPI_QKV, QB>(cache, mA, mA2, mB, mX, args, s);
+    case EPI_CONV1: return launch_epi<BN, EPI_CONV1, QB>(cache, mA, mA2, mB, mX, args, s);
+    case EPI_CONV2: return launch_epi<BN, EPI_CONV2, QB>(cache, mA, mA2, mB, mX, args, s);
+    case EPI_F32: return launch_epi<BN, EPI_F32, QB>(cache, mA, mA2, mB, mX, args, s);
+    case EPI_POWER: return launch_epi<BN, EPI_POWER, QB>(cache, mA, mA2, mB, mX, args, s);
     default: return cudaErrorInvalidValue;
   }
 }
@@ -826,50 +877,52 @@ cudaError_t tc_init(TcGemmCache* cache, int device) {
   return cudaMemset(cache->status, 0, sizeof(int));
 }
 
-// Tile width: the BN in {128, 192, 256} dividing N (GLU / power epilogues need
-// 128-column blocks) that minimises (waves of tiles over the SMs) x (tile cost),
-// counting a fixed per-tile overhead of 32 columns.
-int choose_bn(int M, int N, int epi, int sms) {
-  const int mt = (M + BM - 1) / BM;
-  int best = 0;
+// Relative cost per output column of a paired-CTA tile against a single-CTA
+// tile of the same width: each SM of a pair loads half as much of B, which the
+// mainloop turns into speed because it is bound by the L2 -> shared memory feed.
+constexpr double kPairCost = 0.8;
+
+// Tile shape: over single-CTA tiles (128 rows) and paired-CTA tiles (256 rows
+// on two SMs) of width 256, 192 or 128 dividing N (GLU / power epilogues need
+// 128-column blocks), the one that minimises (waves of tiles over the SMs) x
+// (per-SM tile cost), counting a fixed per-tile overhead of 32 columns.
+// variant: -1 any, 0 single-CTA only, 1 paired-CTA only; width 0: any.  With a
+// second A operand from column n_split on (n_split > 0), tiles may not straddle it.
+TileShape choose_tile(const TcGemmCache* cache, int M, int N, int epi, bool qb, int variant, int width,
+                      int n_split) {
+  TileShape best{false, 0};
   double best_cost = 1e30;
-  for (int bn : {256, 192, 128}) {
-    if (N % bn) continue;
-    if ((epi == EPI_GLU || epi == EPI_POWER) && bn % 128) continue;
-    const int tiles = mt * (N / bn);
-    const double cost = (double)((tiles + sms - 1) / sms) * (bn + 32);
-    if (cost < best_cost - 1e-9) {
-      best_cost = cost;
-      best = bn;
+  const int sms = cache->sm_count;
+  for (int pair = 0; pair < 2; ++pair) {
+    if ((variant >= 0 && pair != variant) || (pair && qb)) continue;
+    if (variant < 0 && ((pair && cache->pair_mode == 0) || (!pair && cache->pair_mode == 2))) continue;
+    const int units = pair ? sms / 2 : sms;
+    const int mt = pair ? (M + 255) / 256 : (M + BM - 1) / BM;
+    for (int bn : {256, 192, 128}) {
+      if (N % bn || (width && bn != width) || (n_split > 0 && n_split % bn)) continue;
+      if ((epi == EPI_GLU || epi == EPI_POWER) && bn % 128) continue;
+      const int tiles = mt * (N / bn);
+      const double cost = (double)((tiles + units - 1) / units) * (bn + 32) * (pair ? kPairCost : 1.0);
+      if (cost < best_cost - 1e-9) {
+        best_cost = cost;
+        best = TileShape{pair != 0, bn};
+      }
     }
   }
+  // the "pair" policy falls back to single-CTA tiles where no paired tile applies
+  if (!best.width && variant < 0 && cache->pair_mode == 2) return choose_tile(cache, M, N, epi, qb, 0, width, n_split);
   return best;
 }
 
-// Paired-CTA tiles (256 x 256 per two SMs) for fp16 weights when there are
-// enough of them to fill the GPU at least twice over; otherwise the single-CTA
-// tile chosen by choose_bn.
-bool choose_pair(const TcGemmCache* cache, int M, int N) {
-  if (N % 256 || cache->pair_mode == 0) return false;
-  if (cache->pair_mode == 2) return true;
-  const int tiles = ((M + 255) / 256) * (N / 256);
-  return tiles >= cache->sm_count;
-}
-
 cudaError_t launch_gemm_tc(TcGemmCache* cache, const void* A, const void* A2, int n_split, int lda, WeightOp B, int M,
-                           int N, int K, int epi, const EpiParams& ep, cudaStream_t s, int variant) {
+                           int N, int K, int epi, const EpiParams& ep, cudaStream_t s, int variant, int width) {
   if (!tc_supported(1, B.dtype, N, K, epi) || M <= 0) return cudaErrorInvalidValue;
   const bool qb = B.dtype == 2;
   if (qb && !B.scale_t) return cudaErrorInvalidValue;
-  bool pair = false;
-  if (variant == 1) {
-    if (qb || N % 256) return cudaErrorInvalidValue;
-    pair = true;
-  } else if (variant < 0) {
-    pair = !qb && choose_pair(cache, M, N);
-  }
-  const int BN = pair ? 256 : choose_bn(M, N, epi, cache->sm_count);
-  if (!BN) return cudaErrorInvalidValue;
+  const TileShape t = choose_tile(cache, M, N, epi, qb, variant, width, A2 ? n_split : 0);
+  if (!t.width) return cudaErrorInvalidValue;
+  const bool pair = t.pair;
+  const int BN = t.width;
   // lda < K: stride-2 convolution view (lda = 2C, K = taps * C, C % 64 == 0); the
   // buffer behind it holds (M + 2) * lda elements, mapped as M + 2 rows of 2C.
   const bool conv = lda < K;
@@ -881,7 +934,7 @@ cudaError_t launch_gemm_tc(TcGemmCache* cache, const void* A, const void* A2, in
   if (conv) mA2 = mA;
   if (e == cudaSuccess)
     e = qb ? make_map_i8(&mB, B.w, K, N, BK, BN)
-           : make_map_f16(&mB, B.w, K, N, (uint64_t)K * 2, BK, pair ? (uint32_t)kPairBH : (uint32_t)BN);
+           : make_map_f16(&mB, B.w, K, N, (uint64_t)K * 2, BK, pair ? (uint32_t)(BN / 2) : (uint32_t)BN);
   if (e != cudaSuccess) return e;
   TcArgs args;
   args.M = M;
@@ -896,16 +949,25 @@ cudaError_t launch_gemm_tc(TcGemmCache* cache, const void* A, const void* A2, in
   args.ep = ep;
   args.scale_t = B.scale_t;
   args.status = cache->status;
-  if (pair) return launch_pair(cache, mA, mA2, mB, args, s);
-  // stages: as many as fit in ~200 KB of shared memory
-  if (qb) {
-    if (BN == 256) return launch_bn<256, 3, true>(cache, mA, mA2, mB, args, s);
-    if (BN == 192) return launch_bn<192, 4, true>(cache, mA, mA2, mB, args, s);
-    return launch_bn<128, 5, true>(cache, mA, mA2, mB, args, s);
+  // residual epilogue: fp32 map over x [M, N] (row stride ldo) for the TMA reduction
+  CUtensorMap mX = mB;
+  if (epi == EPI_RESID) {
+    e = make_map_f32(&mX, ep.x, N, M, (uint64_t)ep.ldo * 4, 32, 32);
+    if (e != cudaSuccess) return e;
   }
-  if (BN == 256) return launch_bn<256, 4, false>(cache, mA, mA2, mB, args, s);
-  if (BN == 192) return launch_bn<192, 5, false>(cache, mA, mA2, mB, args, s);
-  return launch_bn<128, 6, false>(cache, mA, mA2, mB, args, s);
+  if (pair) {
+    if (BN == 256) return launch_pair<256>(cache, mA, mA2, mB, mX, args, s);
+    if (BN == 192) return launch_pair<192>(cache, mA, mA2, mB, mX, args, s);
+    return launch_pair<128>(cache, mA, mA2, mB, mX, args, s);
+  }
+  if (qb) {
+    if (BN == 256) return launch_bn<256, true>(cache, mA, mA2, mB, mX, args, s);
+    if (BN == 192) return launch_bn<192, true>(cache, mA, mA2, mB, mX, args, s);
+    return launch_bn<128, true>(cache, mA, mA2, mB, mX, args, s);
+  }
+  if (BN == 256) return launch_bn<256, false>(cache, mA, mA2, mB, mX, args, s);
+  if (BN == 192) return launch_bn<192, false>(cache, mA, mA2, mB, mX, args, s);
+  return launch_bn<128, false>(cache, mA, mA2, mB, mX, args, s);
 }
 
 cudaError_t launch_attention(TcGemmCache* cache, const void* qk, const void* vt, Clips clips, void* o, int t_half,

@@ -10,8 +10,8 @@ namespace gam {
 struct TcGemmCache {
   int* status = nullptr;  // device word set when a bounded wait gives up
   int sm_count = 148;
-  // fp16 GEMM tiles: 0 single-CTA only, 1 paired-CTA (cta_group::2) 256 x 256 tiles
-  // where they are cheaper, 2 paired-CTA tiles wherever N % 256 == 0
+  // fp16 GEMM tiles: 0 single-CTA only, 1 single- or paired-CTA (cta_group::2)
+  // tiles, whichever is cheaper, 2 paired-CTA tiles wherever one applies
   int pair_mode = 1;
 };
 
@@ -21,10 +21,21 @@ cudaError_t tc_init(TcGemmCache* cache, int device);
 // True when the tensor-core GEMM handles this operand / shape / epilogue combination.
 bool tc_supported(int a_dtype, int b_dtype, int N, int K, int epi);
 
-// variant: -1 chooses the tile shape, 0 forces single-CTA tiles, 1 forces paired-CTA
-// 256 x 256 tiles (fp16 weights, N % 256 == 0).
+struct TileShape {
+  bool pair;  // paired-CTA (cta_group::2) tile of 256 rows, else 128 rows on one SM
+  int width;  // output columns per tile (256, 192 or 128); 0: no shape applies
+};
+
+// The tile shape launch_gemm_tc uses.  variant: -1 any, 0 single-CTA only,
+// 1 paired-CTA only (fp16 weights); width: 0 any, else 256, 192 or 128;
+// n_split > 0: output columns from n_split on read a second A operand, so a
+// tile's width must divide n_split.
+TileShape choose_tile(const TcGemmCache* cache, int M, int N, int epi, bool int8_weights, int variant, int width,
+                      int n_split = 0);
+
 cudaError_t launch_gemm_tc(TcGemmCache* cache, const void* A, const void* A2, int n_split, int lda, WeightOp B,
-                           int M, int N, int K, int epi, const EpiParams& ep, cudaStream_t s, int variant = -1);
+                           int M, int N, int K, int epi, const EpiParams& ep, cudaStream_t s, int variant = -1,
+                           int width = 0);
 
 // Masked multi-head attention on tensor cores (fp16 Q/K/V^T, see attention_tc.cu).
 cudaError_t launch_attention_tc(TcGemmCache* cache, const void* qk, const void* vt, Clips clips, void* o,

@@ -1063,13 +1063,18 @@ gam_status gam_debug_gemm(gam_ctx* c, int impl, const void* a, int lda, const vo
   ep.alpha = 1.f;
   ep.ldo = ldo;
   WeightOp W{w, nullptr, 1, nullptr};
-  if (impl == 0 || impl == 2 || impl == 3) {
+  const int kind = impl & 0xff, width = impl >> 8;
+  if (impl < 0 || kind > 3 || (kind == 1 && width) || (width && width != 128 && width != 192 && width != 256))
+    return fail(c, GAM_ERR_INVALID_ARG, "impl: kind 0 .. 3 plus (tile width 128, 192 or 256) << 8");
+  if (kind != 1) {
     if (!tc_supported(1, 1, n, k, EPI_RESID)) return fail(c, GAM_ERR_SHAPE, "tensor-core GEMM needs N % 256 == 0, K % 64 == 0");
-    const int variant = impl == 0 ? -1 : impl == 2 ? 0 : 1;
-    return run_kernel(c, PK_MISC, s,
-                      [&] { return launch_gemm_tc(&c->tc, a, nullptr, 0, lda, W, m, n, k, EPI_RESID, ep, s, variant); });
+    const int variant = kind == 0 ? -1 : kind == 2 ? 0 : 1;
+    if (!choose_tile(&c->tc, m, n, EPI_RESID, false, variant, width).width)
+      return fail(c, GAM_ERR_SHAPE, "no tile of that width divides N");
+    return run_kernel(c, PK_MISC, s, [&] {
+      return launch_gemm_tc(&c->tc, a, nullptr, 0, lda, W, m, n, k, EPI_RESID, ep, s, variant, width);
+    });
   }
-  if (impl != 1) return fail(c, GAM_ERR_INVALID_ARG, "impl must be 0, 1, 2 or 3");
   if (k % 16 || n % 128) return fail(c, GAM_ERR_SHAPE, "CUDA-core GEMM needs N % 128 == 0, K % 16 == 0");
   return run_kernel(c, PK_MISC, s, [&] { return launch_gemm_simt(1, a, nullptr, 0, lda, W, m, n, k, EPI_RESID, 0, ep, s); });
 }

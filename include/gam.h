@@ -138,8 +138,8 @@ gam_status gam_plan_lengths(const gam_config* cfg, const int32_t* lengths_host, 
  * (f16 [out, in/64]); all other tensors f16 or f32.  On success *out owns
  * device memory until gam_destroy.  The environment variable GAM_GEMM_TILES
  * (read here) sets the tile policy of the fp16 tensor-core GEMMs: "single"
- * (single-CTA tiles only), "pair" (paired-CTA 256 x 256 tiles wherever the
- * output width is a multiple of 256) or, by default, "auto". */
+ * (single-CTA tiles only), "pair" (paired-CTA tiles wherever one applies) or,
+ * by default, "auto" (the cheaper of the two by the library's cost model). */
 gam_status gam_create(const gam_config* cfg, const gam_tensor* tensors, int n_tensors, int device,
                       gam_ctx** out);
 
@@ -237,16 +237,21 @@ gam_status gam_ctc_collapse_noalloc(const float* logits_dev, const int32_t* leng
 
 /* ---- kernel unit test (tests) ---- */
 
-/* One GEMM of the encoder's kind through the chosen implementation
- * (impl 0 = tensor cores (tcgen05) with the tile shape the encoder would
- * choose, 1 = CUDA cores, 2 = tensor cores with single-CTA tiles, 3 = tensor
- * cores with paired-CTA 256 x 256 tiles): out[M, N] (device f32, row stride
- * ldo) += A[M, K] . W[N, K]^T + bias[N], where A (row stride lda) and W are
- * device fp16 and bias device f32.  N % 256 == 0 and K % 64 == 0 for impl 0,
- * 2 and 3; any other impl fails with GAM_ERR_INVALID_ARG.  lda < k selects the strided convolution view of the
- * subsampling convs: row r of A is rows 2r .. 2r+k/C-1 of a [rows, C] buffer
- * with lda = 2C (C % 64 == 0), and the buffer must hold (m + 2) * lda
- * elements.  Uses the residual-update epilogue of the encoder (alpha 1). */
+/* One GEMM of the encoder's kind through the chosen implementation:
+ * out[M, N] (device f32, row stride ldo) += A[M, K] . W[N, K]^T + bias[N],
+ * where A (row stride lda) and W are device fp16 and bias device f32.
+ * impl = kind | (width << 8).  kind 0 = tensor cores (tcgen05) with the tile
+ * shape the encoder would choose, 1 = CUDA cores, 2 = tensor cores with
+ * single-CTA tiles (128 rows), 3 = tensor cores with paired-CTA tiles (256
+ * rows on two SMs, cta_group::2); width 0 lets the library choose the tile
+ * width, else 128, 192 or 256 output columns (tensor-core kinds only).
+ * N % 256 == 0 and K % 64 == 0 for the tensor-core kinds, N % 128 == 0 and
+ * K % 16 == 0 for CUDA cores; a width that does not divide N fails with
+ * GAM_ERR_SHAPE, an impl outside these values with GAM_ERR_INVALID_ARG.
+ * lda < k selects the strided convolution view of the subsampling convs: row
+ * r of A is rows 2r .. 2r+k/C-1 of a [rows, C] buffer with lda = 2C
+ * (C % 64 == 0), and the buffer must hold (m + 2) * lda elements.  Uses the
+ * residual-update epilogue of the encoder (alpha 1). */
 gam_status gam_debug_gemm(gam_ctx* ctx, int impl, const void* a_dev, int lda, const void* w_dev,
                           const float* bias_dev, int m, int n, int k, float* out_dev, int ldo, void* stream);
 

@@ -2,7 +2,8 @@
 out += A . W^T + bias with fp16 operands and fp32 accumulation, for the
 tensor-core (tcgen05) and CUDA-core implementations, against NumPy in fp64.
 impl 0 lets the library choose the tile shape, 2 forces single-CTA tiles and
-3 forces paired-CTA (cta_group::2) 256 x 256 tiles."""
+3 paired-CTA (cta_group::2) tiles; a tile width (128, 192, 256) shifted left by
+8 bits forces the width too."""
 import numpy as np
 import pytest
 
@@ -57,11 +58,26 @@ def test_gemm_tile_widths(ctx, M, N, K):
     test_gemm_parity(ctx, 0, M, N, K, K)
 
 
-@pytest.mark.parametrize("M,N,K,lda", [(129, 256, 64, 64), (256, 512, 128, 128), (20000, 3072, 768, 768),
-                                       (4097, 768, 3072, 3072), (3001, 1536, 1536, 768)],
-                         ids=["peer_rows_empty", "one_pair_tile", "more_tiles_than_pairs", "deep_k_ragged",
+@pytest.mark.parametrize("M,N,K,lda", [(129, 768, 64, 64), (256, 768, 128, 128), (20000, 1536, 768, 768),
+                                       (4097, 768, 3072, 3072), (3001, 768, 1536, 768)],
+                         ids=["peer_rows_empty", "one_pair_row", "more_tiles_than_pairs", "deep_k_ragged",
                               "strided_view_wide"])
-def test_gemm_cta_pair(ctx, M, N, K, lda):
-    """Paired-CTA tiles: a pair whose second CTA holds only padding rows, a single
-    pair tile, more tiles than co-resident pairs, and the convolution view."""
-    test_gemm_parity(ctx, 3, M, N, K, lda)
+@pytest.mark.parametrize("kind", [2, 3], ids=["single_cta", "cta_pair"])
+@pytest.mark.parametrize("width", [128, 192, 256])
+def test_gemm_tile_shapes(ctx, M, N, K, lda, kind, width):
+    """Every tile shape: a pair whose second CTA holds only padding rows, a single
+    row of pair tiles, more tiles than co-resident pairs, a deep ragged K loop and
+    the convolution view, at each tile width."""
+    test_gemm_parity(ctx, kind | (width << 8), M, N, K, lda)
+
+
+def test_gemm_width_must_divide_n(ctx):
+    import torch
+    a = torch.zeros(256, 64, dtype=torch.float16, device="cuda")
+    w = torch.zeros(1024, 64, dtype=torch.float16, device="cuda")
+    b = torch.zeros(1024, dtype=torch.float32, device="cuda")
+    o = torch.zeros(256, 1024, dtype=torch.float32, device="cuda")
+    with pytest.raises(gam.GamError, match="SHAPE|shape"):
+        gam.gam_debug_gemm(ctx, 3 | (192 << 8), a, w, b, o)
+    with pytest.raises(gam.GamError):
+        gam.gam_debug_gemm(ctx, 3 | (100 << 8), a, w, b, o)
