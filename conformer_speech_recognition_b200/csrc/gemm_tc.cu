@@ -57,10 +57,22 @@ constexpr int kEpiWarps = 8;
 constexpr int kStageTile = 32 * 32 * 4;
 template <int EPI>
 __host__ __device__ constexpr int epi_smem() { return EPI == EPI_RESID ? kEpiWarps * kStageTile : 0; }
-// Shared memory for the operand ring: what is left of 227 KB after the epilogue
-// staging and 1.25 KB of alignment slack and barriers, at most 8 stages.
+// Bias of the tile's columns, one 128-float copy per epilogue warp, loaded one
+// tile ahead so the epilogue never waits on it.  Used by the fp16-weight kernels
+// (the INT8 mainloop is bound by its converters, the power epilogue has no bias),
+// and by the residual epilogue only where it costs no pipeline stage.
+constexpr int kBiasStage = 128 * 4;
+constexpr int kBiasSmem = kEpiWarps * kBiasStage;
+__host__ __device__ constexpr int min8(int n) { return n < 8 ? n : 8; }
+// Shared memory for the operand ring: 227 KB less the epilogue staging and
+// 1.25 KB of alignment slack and barriers; at most 8 stages.
 template <int EPI>
 __host__ __device__ constexpr int ring_budget() { return 227 * 1024 - 1280 - epi_smem<EPI>(); }
+template <int EPI, bool QB, int STAGE>
+__host__ __device__ constexpr bool staged_bias() {
+  return !QB && EPI != EPI_POWER &&
+         (EPI != EPI_RESID || min8((ring_budget<EPI>() - kBiasSmem) / STAGE) == min8(ring_budget<EPI>() / STAGE));
+}
 
 template <int BN, bool QB, int EPI>
 struct Cfg {
@@ -68,9 +80,11 @@ struct Cfg {
   static constexpr int RAW_TILE = QB ? BN * BK : 0;          // INT8 weights as loaded (64-byte rows)
   static constexpr int TX = A_TILE + (QB ? RAW_TILE : B_TILE);  // bytes landed by TMA per stage
   static constexpr int STAGE = A_TILE + B_TILE + RAW_TILE;
-  static constexpr int STAGES = ring_budget<EPI>() / STAGE < 8 ? ring_budget<EPI>() / STAGE : 8;
+  static constexpr bool SB = staged_bias<EPI, QB, STAGE>();
+  static constexpr int BIAS_SMEM = SB ? kBiasSmem : 0;
+  static constexpr int STAGES = min8((ring_budget<EPI>() - BIAS_SMEM) / STAGE);
   static constexpr int TMEM_COLS = BN == 128 ? 256 : 512;  // two accumulators, rounded to a power of two
-  static constexpr size_t SMEM = (size_t)STAGES * STAGE + epi_smem<EPI>() + 1024 + 256;
+  static constexpr size_t SMEM = (size_t)STAGES * STAGE + epi_smem<EPI>() + BIAS_SMEM + 1024 + 256;
 };
 
 // Hardware tanh (tanh.approx, one special-function op, relative error about
@@ -87,11 +101,14 @@ __device__ __forceinline__ float swish_fast(float v) {
   return fmaf(h, tanh_fast(h), h);
 }
 
+// 32 consecutive bias values: from the warp's shared-memory copy of the tile's
+// bias (SB) or from global memory through the read-only path.
+template <bool SB>
 __device__ __forceinline__ void load_bias32(const float* b, float (&v)[32]) {
   const float4* p = reinterpret_cast<const float4*>(b);
 #pragma unroll
   for (int j = 0; j < 8; ++j) {
-    const float4 t = __ldg(p + j);
+    const float4 t = SB ? p[j] : __ldg(p + j);
     v[4 * j] = t.x;
     v[4 * j + 1] = t.y;
     v[4 * j + 2] = t.z;
@@ -112,11 +129,12 @@ __device__ __forceinline__ void store_half16(__half* dst, const float* v) {
 }
 
 // Epilogue of one 32-column accumulator chunk of row r (columns n .. n+31).
-template <int EPI>
-__device__ __forceinline__ void epi_chunk(const TcArgs& p, int r, int n, bool valid, const uint32_t (&u)[32]) {
+template <int EPI, bool SB>
+__device__ __forceinline__ void epi_chunk(const TcArgs& p, int r, int n, bool valid, const uint32_t (&u)[32],
+                                          const float* bias) {
   const EpiParams& ep = p.ep;
   float v[32];
-  load_bias32(ep.bias + n, v);
+  load_bias32<SB>(bias, v);
 #pragma unroll
   for (int j = 0; j < 32; ++j) v[j] += __uint_as_float(u[j]);
   switch (EPI) {
@@ -174,9 +192,10 @@ __device__ __forceinline__ void epi_chunk(const TcArgs& p, int r, int n, bool va
 // Epilogue of this warp's half of a tile for row r: columns [half BN/2, (half+1) BN/2),
 // or for the paired epilogues (GLU, power: 128-column blocks [first 64 | second 64])
 // the (first, second) pairs of 32-column chunks number half * BN/128 .. (half+1) * BN/128 - 1.
-template <int BN, int EPI>
+// bt: bias of the tile's columns (bt[c] = bias[n0 + c]), in shared memory if SB.
+template <int BN, int EPI, bool SB>
 __device__ __forceinline__ void epilogue_tile(const TcArgs& p, int r, int n0, uint32_t tbase, int half,
-                                              const CUtensorMap* mX, uint8_t* stage) {
+                                              const CUtensorMap* mX, uint8_t* stage, const float* bt) {
   const int c_lo = half * (BN / 2), c_hi = (half + 1) * (BN / 2);
   const EpiParams& ep = p.ep;
   const bool in_m = r < p.M;
@@ -225,8 +244,8 @@ __device__ __forceinline__ void epilogue_tile(const TcArgs& p, int r, int n0, ui
         if (!in_m) continue;
         const int nv = n0 + blk + hh, ng = nv + 64;
         float bv[32], bg[32], y[32];
-        load_bias32(ep.bias + nv, bv);
-        load_bias32(ep.bias + ng, bg);
+        load_bias32<SB>(bt + blk + hh, bv);
+        load_bias32<SB>(bt + blk + 64 + hh, bg);
 #pragma unroll
         for (int j = 0; j < 32; ++j)
           y[j] = (__uint_as_float(a[j]) + bv[j]) * sigm(__uint_as_float(g[j]) + bg[j]);
@@ -240,16 +259,22 @@ __device__ __forceinline__ void epilogue_tile(const TcArgs& p, int r, int n0, ui
     // lane hands them to a TMA reduction, so the L2 does the read-modify-write
     // of x (rows past M are clipped by the tensor map)
     const int lane = threadIdx.x & 31, row0 = r - lane;
+    float bcur[32];
+    load_bias32<SB>(bt + c_lo, bcur);
 #pragma unroll 1
     for (int c = c_lo; c < c_hi; c += 32) {
       uint32_t u[32];
       tmem_ld32(tbase + c, u);
+      float bnext[32] = {};
+      if (c + 32 < c_hi) load_bias32<SB>(bt + c + 32, bnext);  // next chunk's bias while this one is read
       tmem_ld_wait();
-      if (row0 >= p.M) continue;
       float v[32];
-      load_bias32(ep.bias + n0 + c, v);
 #pragma unroll
-      for (int j = 0; j < 32; ++j) v[j] = ep.alpha * (__uint_as_float(u[j]) + v[j]);
+      for (int j = 0; j < 32; ++j) {
+        v[j] = ep.alpha * (__uint_as_float(u[j]) + bcur[j]);
+        bcur[j] = bnext[j];
+      }
+      if (row0 >= p.M) continue;
       if (lane == 0) bulk_wait_read0();  // the previous reduction has read the staging tile
       __syncwarp();
       uint8_t* row = stage + lane * 128;
@@ -270,10 +295,38 @@ __device__ __forceinline__ void epilogue_tile(const TcArgs& p, int r, int n0, ui
       uint32_t u[32];
       tmem_ld32(tbase + c, u);
       tmem_ld_wait();
-      if (in_m) epi_chunk<EPI>(p, r, n0 + c, valid, u);
+      if (in_m) epi_chunk<EPI, SB>(p, r, n0 + c, valid, u, bt + c);
     }
   }
 }
+
+// Per-warp bias of the columns this warp's epilogue reads (all 128 columns of a
+// 128-wide tile, else its half of the tile), held in registers one tile ahead
+// (a float4 per lane) and written to the warp's shared-memory copy when the
+// tile's accumulator is ready.  Without SB the epilogue reads global memory.
+template <int BN, bool SB>
+struct BiasPrefetch {
+  static constexpr int COLS = BN == 128 ? 128 : BN / 2;
+  float* smem;
+  int col0, lane;
+  float4 next;
+  __device__ __forceinline__ BiasPrefetch(const TcArgs& p, int half, float* s, int first_tile)
+      : smem(s), col0(BN == 128 ? 0 : half * (BN / 2)), lane(threadIdx.x & 31) {
+    load(p, first_tile);
+  }
+  __device__ __forceinline__ void load(const TcArgs& p, int tile) {
+    if (SB && tile < p.tiles && lane * 4 < COLS)
+      next = __ldg(reinterpret_cast<const float4*>(p.ep.bias + (tile % p.n_blocks) * BN + col0) + lane);
+  }
+  // bias of the tile at column n0 (bt[c] = bias[n0 + c]); starts the load for the tile after
+  __device__ __forceinline__ const float* tile(const TcArgs& p, int n0, int following) {
+    if (!SB) return p.ep.bias + n0;
+    if (lane * 4 < COLS) reinterpret_cast<float4*>(smem)[lane] = next;
+    __syncwarp();
+    load(p, following);
+    return smem - col0;
+  }
+};
 
 constexpr int kCvtWarps = 4;  // INT8 variant: warps that dequantise the weight tile
 template <bool QB>
@@ -313,7 +366,8 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap mA, const __grid_constant__ C
   uint8_t* sB = base + STAGES * A_TILE;
   uint8_t* sRaw = sB + STAGES * C::B_TILE;  // INT8 variant only
   uint8_t* sEpi = base + STAGES * C::STAGE;  // residual epilogue staging, kStageTile per warp
-  uint64_t* full = reinterpret_cast<uint64_t*>(sEpi + epi_smem<EPI>());
+  uint8_t* sBias = sEpi + epi_smem<EPI>();    // per-warp bias copies, kBiasStage each
+  uint64_t* full = reinterpret_cast<uint64_t*>(sBias + C::BIAS_SMEM);
   uint64_t* empty = full + STAGES;
   uint64_t* tfull = empty + STAGES;
   uint64_t* tempty = tfull + 2;
@@ -462,6 +516,8 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap mA, const __grid_constant__ C
   } else {
     const int q = warp & 3;                       // TMEM lane quarter of this warp
     const int half = (warp - 2) / 4;              // which half of the tile's columns
+    constexpr bool SB = C::SB;
+    BiasPrefetch<BN, SB> bias(p, half, reinterpret_cast<float*>(sBias + (warp - 2) * kBiasStage), blockIdx.x);
     int local = 0;
     for (int tile = blockIdx.x; tile < p.tiles; tile += gridDim.x, ++local) {
       const int acc = local & 1;
@@ -471,7 +527,8 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap mA, const __grid_constant__ C
       const int nb = tile % p.n_blocks, mb = tile / p.n_blocks;
       const int r = mb * BM + q * 32 + lane;
       const uint32_t tbase = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN);
-      epilogue_tile<BN, EPI>(p, r, nb * BN, tbase, half, &mX, sEpi + (warp - 2) * kStageTile);
+      const float* bt = bias.tile(p, nb * BN, tile + gridDim.x);
+      epilogue_tile<BN, EPI, SB>(p, r, nb * BN, tbase, half, &mX, sEpi + (warp - 2) * kStageTile, bt);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&tempty[acc]);
@@ -551,9 +608,11 @@ struct PairCfg {
   static constexpr int BH = TN / 2;                      // B rows per CTA
   static constexpr int B_TILE = BH * BK * 2;
   static constexpr int STAGE = A_TILE + B_TILE;
-  static constexpr int STAGES = ring_budget<EPI>() / STAGE < 8 ? ring_budget<EPI>() / STAGE : 8;
+  static constexpr bool SB = staged_bias<EPI, false, STAGE>();
+  static constexpr int BIAS_SMEM = SB ? kBiasSmem : 0;
+  static constexpr int STAGES = min8((ring_budget<EPI>() - BIAS_SMEM) / STAGE);
   static constexpr int TMEM_COLS = TN == 128 ? 256 : 512;
-  static constexpr size_t SMEM = (size_t)STAGES * STAGE + epi_smem<EPI>() + 1024 + 256;
+  static constexpr size_t SMEM = (size_t)STAGES * STAGE + epi_smem<EPI>() + BIAS_SMEM + 1024 + 256;
 };
 
 template <int TN, int EPI>
@@ -567,7 +626,8 @@ gemm_tc_pair_kernel(const __grid_constant__ CUtensorMap mA, const __grid_constan
   uint8_t* sA = base;
   uint8_t* sB = base + STAGES * A_TILE;
   uint8_t* sEpi = base + STAGES * C::STAGE;  // residual epilogue staging, kStageTile per warp
-  uint64_t* full = reinterpret_cast<uint64_t*>(sEpi + epi_smem<EPI>());
+  uint8_t* sBias = sEpi + epi_smem<EPI>();    // per-warp bias copies, kBiasStage each
+  uint64_t* full = reinterpret_cast<uint64_t*>(sBias + C::BIAS_SMEM);
   uint64_t* empty = full + STAGES;
   uint64_t* tfull = empty + STAGES;
   uint64_t* tempty = tfull + 2;
@@ -688,6 +748,8 @@ gemm_tc_pair_kernel(const __grid_constant__ CUtensorMap mA, const __grid_constan
     }
   } else {
     const int q = warp & 3, half = (warp - 2) / 4;
+    constexpr bool SB = C::SB;
+    BiasPrefetch<BN, SB> bias(p, half, reinterpret_cast<float*>(sBias + (warp - 2) * kBiasStage), pair);
     int local = 0;
     for (int tile = pair; tile < p.tiles; tile += npairs, ++local) {
       const int acc = local & 1;
@@ -697,7 +759,8 @@ gemm_tc_pair_kernel(const __grid_constant__ CUtensorMap mA, const __grid_constan
       const int nb = tile % p.n_blocks, mb = tile / p.n_blocks;
       const int r = mb * 256 + (int)rank * 128 + q * 32 + lane;
       const uint32_t tbase = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN);
-      epilogue_tile<BN, EPI>(p, r, nb * BN, tbase, half, &mX, sEpi + (warp - 2) * kStageTile);
+      const float* bt = bias.tile(p, nb * BN, tile + npairs);
+      epilogue_tile<BN, EPI, SB>(p, r, nb * BN, tbase, half, &mX, sEpi + (warp - 2) * kStageTile, bt);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_remote(map_to_cta(&tempty[acc], 0));
@@ -880,12 +943,19 @@ cudaError_t tc_init(TcGemmCache* cache, int device) {
 // Relative cost per output column of a paired-CTA tile against a single-CTA
 // tile of the same width: each SM of a pair loads half as much of B, which the
 // mainloop turns into speed because it is bound by the L2 -> shared memory feed.
-constexpr double kPairCost = 0.8;
+constexpr double kPairCost = 0.7;
+// Weight of the round-up to whole waves: with fp16 weights a partly filled last
+// wave runs faster per tile than a full one (fewer SMs share the L2 feed), so
+// tiles count for 0.75 x (tiles / units) + 0.25 x ceil(tiles / units) waves.
+// The INT8 mainloop is bound by its converter warps inside each SM instead, and
+// its waves count whole.
+constexpr double kWaveRoundUp = 0.25;
 
 // Tile shape: over single-CTA tiles (128 rows) and paired-CTA tiles (256 rows
 // on two SMs) of width 256, 192 or 128 dividing N (GLU / power epilogues need
 // 128-column blocks), the one that minimises (waves of tiles over the SMs) x
-// (per-SM tile cost), counting a fixed per-tile overhead of 32 columns.
+// (per-SM tile cost), counting a fixed per-tile overhead of 32 columns.  The
+// constants were fitted to measured times of the encoder's GEMM shapes on B200.
 // variant: -1 any, 0 single-CTA only, 1 paired-CTA only; width 0: any.  With a
 // second A operand from column n_split on (n_split > 0), tiles may not straddle it.
 TileShape choose_tile(const TcGemmCache* cache, int M, int N, int epi, bool qb, int variant, int width,
@@ -902,7 +972,9 @@ TileShape choose_tile(const TcGemmCache* cache, int M, int N, int epi, bool qb, 
       if (N % bn || (width && bn != width) || (n_split > 0 && n_split % bn)) continue;
       if ((epi == EPI_GLU || epi == EPI_POWER) && bn % 128) continue;
       const int tiles = mt * (N / bn);
-      const double cost = (double)((tiles + units - 1) / units) * (bn + 32) * (pair ? kPairCost : 1.0);
+      const double round_up = qb ? 1.0 : kWaveRoundUp;
+      const double waves = round_up * (double)((tiles + units - 1) / units) + (1.0 - round_up) * (double)tiles / units;
+      const double cost = waves * (bn + 32) * (pair ? kPairCost : 1.0);
       if (cost < best_cost - 1e-9) {
         best_cost = cost;
         best = TileShape{pair != 0, bn};
