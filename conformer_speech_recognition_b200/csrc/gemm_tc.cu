@@ -116,16 +116,18 @@ __device__ __forceinline__ void load_bias32(const float* b, float (&v)[32]) {
   }
 }
 
+// 16 values as fp16 to 32 bytes at dst (32-byte aligned) with one 256-bit store:
+// a full L2 sector per thread, where two 128-bit stores would each write half of one.
 __device__ __forceinline__ void store_half16(__half* dst, const float* v) {
-  uint4 w[2];
-  uint32_t* pw = reinterpret_cast<uint32_t*>(w);
+  uint32_t w[8];
 #pragma unroll
   for (int j = 0; j < 8; ++j) {
     __half2 h = __floats2half2_rn(v[2 * j], v[2 * j + 1]);
-    pw[j] = *reinterpret_cast<uint32_t*>(&h);
+    w[j] = *reinterpret_cast<uint32_t*>(&h);
   }
-  reinterpret_cast<uint4*>(dst)[0] = w[0];
-  reinterpret_cast<uint4*>(dst)[1] = w[1];
+  asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(dst), "r"(w[0]), "r"(w[1]),
+               "r"(w[2]), "r"(w[3]), "r"(w[4]), "r"(w[5]), "r"(w[6]), "r"(w[7])
+               : "memory");
 }
 
 // Epilogue of one 32-column accumulator chunk of row r (columns n .. n+31).
@@ -242,7 +244,6 @@ __device__ __forceinline__ void epilogue_tile(const TcArgs& p, int r, int n0, ui
         tmem_ld32(tbase + blk + 64 + hh, g);
         tmem_ld_wait();
         if (!in_m) continue;
-        const int nv = n0 + blk + hh, ng = nv + 64;
         float bv[32], bg[32], y[32];
         load_bias32<SB>(bt + blk + hh, bv);
         load_bias32<SB>(bt + blk + 64 + hh, bg);
@@ -989,6 +990,11 @@ TileShape choose_tile(const TcGemmCache* cache, int M, int N, int epi, bool qb, 
 cudaError_t launch_gemm_tc(TcGemmCache* cache, const void* A, const void* A2, int n_split, int lda, WeightOp B, int M,
                            int N, int K, int epi, const EpiParams& ep, cudaStream_t s, int variant, int width) {
   if (!tc_supported(1, B.dtype, N, K, epi) || M <= 0) return cudaErrorInvalidValue;
+  // fp16 outputs are written 32 bytes per thread: 32-byte aligned rows
+  if ((epi == EPI_SWISH || epi == EPI_GLU || epi == EPI_CONV1) &&
+      ((reinterpret_cast<uintptr_t>(ep.out) & 31) || ep.ldo % 16))
+    return cudaErrorInvalidValue;
+  if (epi == EPI_QKV && ((reinterpret_cast<uintptr_t>(ep.qk) & 31) || ep.d_head % 16)) return cudaErrorInvalidValue;
   const bool qb = B.dtype == 2;
   if (qb && !B.scale_t) return cudaErrorInvalidValue;
   const TileShape t = choose_tile(cache, M, N, epi, qb, variant, width, A2 ? n_split : 0);
