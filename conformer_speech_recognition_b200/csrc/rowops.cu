@@ -74,95 +74,110 @@ __device__ __forceinline__ void load_row(const float* x, float4 (&v)[NV], int la
   for (int j = 0; j < NV; ++j) v[j] = *reinterpret_cast<const float4*>(x + (j * 32 + lane) * 4);
 }
 
-// Plain LayerNorm: each warp normalises rows (16 w + i) and (16 w + i + 8) of its
-// CTA's 16-row block together, so two rows' loads are in flight per lane.
+// The LayerNorm kernels run one resident wave of CTAs (grid sized from the
+// occupancy); warp w of the grid takes rows w, w + W, w + 2W, ... (W warps in
+// the grid) and loads its next row while it normalises the current one, so
+// each SM keeps a row per warp in flight and no second, partly filled wave
+// follows the first.
+
+// Plain LayerNorm.
 template <typename T, int NV>
 __global__ void __launch_bounds__(256)
 ln_kernel(const float* __restrict__ x, const float* __restrict__ g, const float* __restrict__ b, float eps,
           T* __restrict__ u, int rows) {
   constexpr int d = NV * 128;
-  const int r0 = blockIdx.x * 16 + (threadIdx.x >> 5), r1 = r0 + 8, lane = threadIdx.x & 31;
-  float4 v0[NV], v1[NV];
-  if (r0 < rows) load_row<NV>(x + (size_t)r0 * d, v0, lane);
-  if (r1 < rows) load_row<NV>(x + (size_t)r1 * d, v1, lane);
-  if (r0 < rows) {
-    ln_row<NV>(v0, d, eps, g, b, lane);
+  const int lane = threadIdx.x & 31, nw = gridDim.x * 8;
+  int row = blockIdx.x * 8 + (threadIdx.x >> 5);
+  float4 cur[NV], nxt[NV];
+  if (row < rows) load_row<NV>(x + (size_t)row * d, cur, lane);
+  for (; row < rows; row += nw) {
+    if (row + nw < rows) load_row<NV>(x + (size_t)(row + nw) * d, nxt, lane);
+    ln_row<NV>(cur, d, eps, g, b, lane);
 #pragma unroll
-    for (int j = 0; j < NV; ++j) store4<T>(u + (size_t)r0 * d + (j * 32 + lane) * 4, v0[j]);
-  }
-  if (r1 < rows) {
-    ln_row<NV>(v1, d, eps, g, b, lane);
-#pragma unroll
-    for (int j = 0; j < NV; ++j) store4<T>(u + (size_t)r1 * d + (j * 32 + lane) * 4, v1[j]);
+    for (int j = 0; j < NV; ++j) {
+      store4<T>(u + (size_t)row * d + (j * 32 + lane) * 4, cur[j]);
+      cur[j] = nxt[j];
+    }
   }
 }
 
-template <typename T, int NV>
-__device__ __forceinline__ void ln_chain_row(float* xr, T* ur, float4 (&v)[NV], float eps, const float* g1,
-                                             const float* b1, const float* g2, const float* b2, int lane) {
-  constexpr int d = NV * 128;
-  ln_row<NV>(v, d, eps, g1, b1, lane);
-#pragma unroll
-  for (int j = 0; j < NV; ++j) *reinterpret_cast<float4*>(xr + (j * 32 + lane) * 4) = v[j];
-  ln_row<NV>(v, d, eps, g2, b2, lane);
-#pragma unroll
-  for (int j = 0; j < NV; ++j) store4<T>(ur + (j * 32 + lane) * 4, v[j]);
-}
-
+// Two LayerNorms in a row (a block's final norm, then the next block's first):
+// x <- LN1(x) in place, u = LN2(LN1(x)).
 template <typename T, int NV>
 __global__ void __launch_bounds__(256)
 ln_chain_kernel(float* __restrict__ x, const float* __restrict__ g1, const float* __restrict__ b1,
                 const float* __restrict__ g2, const float* __restrict__ b2, float eps, T* __restrict__ u, int rows) {
   constexpr int d = NV * 128;
-  const int r0 = blockIdx.x * 16 + (threadIdx.x >> 5), r1 = r0 + 8, lane = threadIdx.x & 31;
-  float4 v0[NV], v1[NV];
-  if (r0 < rows) load_row<NV>(x + (size_t)r0 * d, v0, lane);
-  if (r1 < rows) load_row<NV>(x + (size_t)r1 * d, v1, lane);
-  if (r0 < rows) ln_chain_row<T, NV>(x + (size_t)r0 * d, u + (size_t)r0 * d, v0, eps, g1, b1, g2, b2, lane);
-  if (r1 < rows) ln_chain_row<T, NV>(x + (size_t)r1 * d, u + (size_t)r1 * d, v1, eps, g1, b1, g2, b2, lane);
+  const int lane = threadIdx.x & 31, nw = gridDim.x * 8;
+  int row = blockIdx.x * 8 + (threadIdx.x >> 5);
+  float4 cur[NV], nxt[NV];
+  if (row < rows) load_row<NV>(x + (size_t)row * d, cur, lane);
+  for (; row < rows; row += nw) {
+    if (row + nw < rows) load_row<NV>(x + (size_t)(row + nw) * d, nxt, lane);
+    float* xr = x + (size_t)row * d;
+    T* ur = u + (size_t)row * d;
+    ln_row<NV>(cur, d, eps, g1, b1, lane);
+#pragma unroll
+    for (int j = 0; j < NV; ++j) *reinterpret_cast<float4*>(xr + (j * 32 + lane) * 4) = cur[j];
+    ln_row<NV>(cur, d, eps, g2, b2, lane);
+#pragma unroll
+    for (int j = 0; j < NV; ++j) {
+      store4<T>(ur + (j * 32 + lane) * 4, cur[j]);
+      cur[j] = nxt[j];
+    }
+  }
 }
 
+// LayerNorm, then RoPE on the normalised row: u = LN(x) and, per head,
+// urot = u cos(t w_i) + rotate_half(u) sin(t w_i) at the row's position t in
+// its clip.  The row goes through shared memory so each lane can read the
+// partner half of its columns; the cos / sin tables are [T][d_head / 2].
 template <typename T, int DH, int NV>
 __global__ void __launch_bounds__(256)
 ln_rope_kernel(const float* __restrict__ x, const float* __restrict__ g, const float* __restrict__ b, float eps,
                const float* __restrict__ cos_tab, const float* __restrict__ sin_tab, Clips clips, T* __restrict__ u,
                T* __restrict__ urot, int rows) {
-  constexpr int dh = DH, d = NV * 128, nv = NV;
-  __shared__ __align__(16) float srow[8][1024];
-  const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int row = blockIdx.x * 8 + w;
-  if (row >= rows) return;
-  float4 v[NV];
-  load_row<NV>(x + (size_t)row * d, v, lane);
-  ln_row<NV>(v, d, eps, g, b, lane);
+  constexpr int dh = DH, half = DH / 2, d = NV * 128;
+  static_assert(half % 4 == 0, "a float4 of columns never straddles a half head");
+  __shared__ __align__(16) float srow[8][d];
+  const int w = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = gridDim.x * 8;
   float* sr = srow[w];
+  int row = blockIdx.x * 8 + w;
+  float4 cur[NV], nxt[NV];
+  if (row < rows) load_row<NV>(x + (size_t)row * d, cur, lane);
+  for (; row < rows; row += nw) {
+    if (row + nw < rows) load_row<NV>(x + (size_t)(row + nw) * d, nxt, lane);
+    ln_row<NV>(cur, d, eps, g, b, lane);
 #pragma unroll
-  for (int j = 0; j < nv; ++j) {
+    for (int j = 0; j < NV; ++j) {
       const int c = (j * 32 + lane) * 4;
-      store4<T>(u + (size_t)row * d + c, v[j]);
-      *reinterpret_cast<float4*>(sr + c) = v[j];
+      store4<T>(u + (size_t)row * d + c, cur[j]);
+      *reinterpret_cast<float4*>(sr + c) = cur[j];
+      cur[j] = nxt[j];
     }
-  __syncwarp();
-  const int ci = clips.find(row, 1, 0);
-  int t = row - clips.e(ci);
-  if (t < 0 || t >= clips.L2(ci)) t = 0;  // gap row: any finite rotation
-  const int half = dh >> 1;
-  const float* ct = cos_tab + (size_t)t * half;
-  const float* st = sin_tab + (size_t)t * half;
+    __syncwarp();
+    const int ci = clips.find(row, 1, 0);
+    int t = row - clips.e(ci);
+    if (t < 0 || t >= clips.L2(ci)) t = 0;  // gap row: any finite rotation
+    const float* ct = cos_tab + (size_t)t * half;
+    const float* st = sin_tab + (size_t)t * half;
 #pragma unroll
-  for (int j = 0; j < nv; ++j) {
+    for (int j = 0; j < NV; ++j) {
       const int c0 = (j * 32 + lane) * 4;
-      float o[4];
-#pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        const int c = c0 + k;
-        const int cc = c % dh;
-        const int i = cc < half ? cc : cc - half;
-        const float cs = __ldg(ct + i), sn = __ldg(st + i);
-        o[k] = cc < half ? sr[c] * cs - sr[c + half] * sn : sr[c] * cs + sr[c - half] * sn;
-      }
-      store4<T>(urot + (size_t)row * d + c0, make_float4(o[0], o[1], o[2], o[3]));
+      const int cc = c0 % dh;
+      const bool first = cc < half;
+      const int i = first ? cc : cc - half;
+      const float4 cs = __ldg(reinterpret_cast<const float4*>(ct + i));
+      const float4 sn = __ldg(reinterpret_cast<const float4*>(st + i));
+      const float4 a = *reinterpret_cast<const float4*>(sr + c0);
+      const float4 q = *reinterpret_cast<const float4*>(sr + (first ? c0 + half : c0 - half));
+      const float sg = first ? -1.f : 1.f;  // rotate_half: [-x2, x1]
+      store4<T>(urot + (size_t)row * d + c0,
+                make_float4(fmaf(sg * q.x, sn.x, a.x * cs.x), fmaf(sg * q.y, sn.y, a.y * cs.y),
+                            fmaf(sg * q.z, sn.z, a.z * cs.z), fmaf(sg * q.w, sn.w, a.w * cs.w)));
     }
+    __syncwarp();  // the row buffer is rewritten by the next iteration
+  }
 }
 
 // Swish: exact form for the fp32 build mode; in the fp16 modes one hardware
@@ -442,31 +457,66 @@ __global__ void f32_to_f16_kernel(const float* __restrict__ in, __half* __restri
     default: return cudaErrorInvalidValue; \
   }
 
+// CTAs of 256 threads that fit on the device at once (per kernel, looked up once;
+// a process drives one GPU model), capped by the 8-row groups there is work for.
+template <auto KERNEL>
+int resident_grid(int rows) {
+  static const int resident = [] {
+    int dev = 0, sms = 148, per_sm = 1;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, KERNEL, 256, 0) != cudaSuccess || per_sm < 1) per_sm = 1;
+    return sms * per_sm;
+  }();
+  const int groups = (rows + 7) / 8;
+  return groups < resident ? groups : resident;
+}
+
+template <typename T, int NV>
+cudaError_t ln_t(const float* x, const float* g, const float* b, float eps, void* u, int rows, cudaStream_t s) {
+  ln_kernel<T, NV><<<resident_grid<ln_kernel<T, NV>>(rows), 256, 0, s>>>(x, g, b, eps, (T*)u, rows);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_layernorm(const float* x, const float* g, const float* b, float eps, void* u, int u_half, int rows,
                              int d, cudaStream_t s) {
   if (d % 128 || d > 1024) return cudaErrorInvalidValue;
-  const int grid = (rows + 15) / 16;
-  if (u_half) GAM_NV_DISPATCH(d, (ln_kernel<__half, NV><<<grid, 256, 0, s>>>(x, g, b, eps, (__half*)u, rows)))
-  else GAM_NV_DISPATCH(d, (ln_kernel<float, NV><<<grid, 256, 0, s>>>(x, g, b, eps, (float*)u, rows)))
+  if (rows <= 0) return cudaSuccess;
+  if (u_half) GAM_NV_DISPATCH(d, return (ln_t<__half, NV>(x, g, b, eps, u, rows, s)))
+  else GAM_NV_DISPATCH(d, return (ln_t<float, NV>(x, g, b, eps, u, rows, s)))
+  return cudaErrorInvalidValue;
+}
+
+template <typename T, int NV>
+cudaError_t ln_chain_t(float* x, const float* g1, const float* b1, const float* g2, const float* b2, float eps, void* u,
+                       int rows, cudaStream_t s) {
+  ln_chain_kernel<T, NV><<<resident_grid<ln_chain_kernel<T, NV>>(rows), 256, 0, s>>>(x, g1, b1, g2, b2, eps, (T*)u,
+                                                                                        rows);
   return cudaGetLastError();
 }
 
 cudaError_t launch_layernorm_chain(float* x, const float* g1, const float* b1, const float* g2, const float* b2,
                                    float eps, void* u, int u_half, int rows, int d, cudaStream_t s) {
   if (d % 128 || d > 1024) return cudaErrorInvalidValue;
-  const int grid = (rows + 15) / 16;
-  if (u_half) GAM_NV_DISPATCH(d, (ln_chain_kernel<__half, NV><<<grid, 256, 0, s>>>(x, g1, b1, g2, b2, eps, (__half*)u, rows)))
-  else GAM_NV_DISPATCH(d, (ln_chain_kernel<float, NV><<<grid, 256, 0, s>>>(x, g1, b1, g2, b2, eps, (float*)u, rows)))
+  if (rows <= 0) return cudaSuccess;
+  if (u_half) GAM_NV_DISPATCH(d, return (ln_chain_t<__half, NV>(x, g1, b1, g2, b2, eps, u, rows, s)))
+  else GAM_NV_DISPATCH(d, return (ln_chain_t<float, NV>(x, g1, b1, g2, b2, eps, u, rows, s)))
+  return cudaErrorInvalidValue;
+}
+
+template <typename T, int DH, int NV>
+cudaError_t rope_nv(const float* x, const float* g, const float* b, float eps, const float* cos_tab,
+                    const float* sin_tab, Clips clips, void* u, void* urot, int rows, cudaStream_t s) {
+  ln_rope_kernel<T, DH, NV><<<resident_grid<ln_rope_kernel<T, DH, NV>>(rows), 256, 0, s>>>(
+      x, g, b, eps, cos_tab, sin_tab, clips, (T*)u, (T*)urot, rows);
   return cudaGetLastError();
 }
 
 template <typename T, int DH>
 cudaError_t rope_t(const float* x, const float* g, const float* b, float eps, const float* cos_tab,
                    const float* sin_tab, Clips clips, void* u, void* urot, int rows, int d, cudaStream_t s) {
-  const int grid = (rows + 7) / 8;
-  GAM_NV_DISPATCH(d, (ln_rope_kernel<T, DH, NV><<<grid, 256, 0, s>>>(x, g, b, eps, cos_tab, sin_tab, clips, (T*)u,
-                                                                       (T*)urot, rows)))
-  return cudaGetLastError();
+  if (rows <= 0) return cudaSuccess;
+  GAM_NV_DISPATCH(d, return (rope_nv<T, DH, NV>(x, g, b, eps, cos_tab, sin_tab, clips, u, urot, rows, s)))
+  return cudaErrorInvalidValue;
 }
 
 cudaError_t launch_layernorm_rope(const float* x, const float* g, const float* b, float eps, const float* cos_tab,
