@@ -10,8 +10,9 @@
 //   warp 0      TMA: Q tile once, then K tiles of 128 keys into a 2-stage
 //               ring and V^T tiles into a single buffer (128-byte swizzle);
 //   warp 1      TMEM allocation; one thread issues S = Q K^T (M=128, N=128,
-//               K=d_head) into TMEM, then O_blk = P V (M=128, N=d_head,
-//               K=128) with P read from shared memory;
+//               K=d_head) into TMEM and, once the softmax has turned S into
+//               P, first the next block's S and then O_blk = P V (M=128,
+//               N=d_head, K=128) with P read from shared memory;
 //   warps 2..5  softmax, one query row per thread (TMEM lane): pass 1 takes
 //               the row max of S (overlapping the previous block's P.V),
 //               pass 2 writes exp2 / fp16 P into the swizzled shared-memory
@@ -165,15 +166,23 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap mQK, const __grid_constant__ 
       const int ksteps_s = dh / 16;
       bool ok = mbar_wait(q_full, 0, abort_flag);
       const uint64_t dq = sdesc_k_sw128(smem_u32(sQ));
-      for (int j = 0; j < nblk && ok; ++j) {
+      // S(j) = Q K(j)^T into TMEM, then release the K stage
+      auto issue_s = [&](int j) {
         const int s = j & 1;
-        if (!mbar_wait(&k_full[s], (j >> 1) & 1, abort_flag)) break;
+        if (!mbar_wait(&k_full[s], (j >> 1) & 1, abort_flag)) return false;
         tc_fence_after();
         const uint64_t dk = sdesc_k_sw128(smem_u32(sK + s * K_BYTES));
         for (int k = 0; k < ksteps_s; ++k) umma_f16(tS, dq + 2 * k, dk + 2 * k, idesc_s, k != 0 ? 1u : 0u);
         umma_commit(s_full);
         umma_commit(&k_empty[s]);
+        return true;
+      };
+      if (ok) ok = issue_s(0);
+      for (int j = 0; j < nblk && ok; ++j) {
+        // once the softmax has consumed S(j) (P(j) written), S(j+1) goes first so the
+        // next softmax pass starts while P(j).V(j) runs
         if (!mbar_wait(p_full, j & 1, abort_flag)) break;
+        if (j + 1 < nblk && !issue_s(j + 1)) break;
         if (!mbar_wait(v_full, j & 1, abort_flag)) break;
         tc_fence_after();
         const uint32_t pbase = smem_u32(sP), vbase = smem_u32(sV);
@@ -211,20 +220,21 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap mQK, const __grid_constant__ 
       }
       tc_fence_after();
       const int kvalid = L - j * BKV;  // keys [0, kvalid) of this block are valid
-      // pass 1: row max of the raw scores (scale > 0 commutes with max)
+      // pass 1: row max of the raw scores (scale > 0 commutes with max), 64 columns per TMEM wait
       float mx = -INFINITY;
 #pragma unroll 1
-      for (int c = 0; c < BKV; c += 32) {
-        uint32_t u[32];
-        tmem_ld32(tS + lane_off + c, u);
+      for (int c = 0; c < BKV; c += 64) {
+        uint32_t u[2][32];
+        tmem_ld32(tS + lane_off + c, u[0]);
+        tmem_ld32(tS + lane_off + c + 32, u[1]);
         tmem_ld_wait();
-        if (c + 32 <= kvalid) {
+        if (c + 64 <= kvalid) {
 #pragma unroll
-          for (int t = 0; t < 32; ++t) mx = fmaxf(mx, __uint_as_float(u[t]));
+          for (int t = 0; t < 64; ++t) mx = fmaxf(mx, __uint_as_float(u[t >> 5][t & 31]));
         } else {
 #pragma unroll
-          for (int t = 0; t < 32; ++t)
-            if (c + t < kvalid) mx = fmaxf(mx, __uint_as_float(u[t]));
+          for (int t = 0; t < 64; ++t)
+            if (c + t < kvalid) mx = fmaxf(mx, __uint_as_float(u[t >> 5][t & 31]));
         }
       }
       mx *= p.scale_log2;
@@ -251,28 +261,31 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap mQK, const __grid_constant__ 
         l *= corr;
         m_used = mx;
       }
-      // pass 2: exponentials, row sum, fp16 P into the swizzled operand layout
+      // pass 2: exponentials, row sum, fp16 P into the swizzled operand layout; one
+      // 64-key swizzle atom (64 columns) per TMEM wait
       float sum = 0.f;
 #pragma unroll 1
-      for (int c = 0; c < BKV; c += 32) {
-        uint32_t u[32];
-        tmem_ld32(tS + lane_off + c, u);
+      for (int c = 0; c < BKV; c += 64) {
+        uint32_t u[2][32];
+        tmem_ld32(tS + lane_off + c, u[0]);
+        tmem_ld32(tS + lane_off + c + 32, u[1]);
         tmem_ld_wait();
-        float pv[32];
-        if (c + 32 <= kvalid) {
+        float pv[64];
+        if (c + 64 <= kvalid) {
 #pragma unroll
-          for (int t = 0; t < 32; ++t) pv[t] = fast_exp2(fmaf(__uint_as_float(u[t]), p.scale_log2, -m_used));
+          for (int t = 0; t < 64; ++t)
+            pv[t] = fast_exp2(fmaf(__uint_as_float(u[t >> 5][t & 31]), p.scale_log2, -m_used));
         } else {
 #pragma unroll
-          for (int t = 0; t < 32; ++t)
-            pv[t] = (c + t < kvalid) ? fast_exp2(fmaf(__uint_as_float(u[t]), p.scale_log2, -m_used)) : 0.f;
+          for (int t = 0; t < 64; ++t)
+            pv[t] = (c + t < kvalid) ? fast_exp2(fmaf(__uint_as_float(u[t >> 5][t & 31]), p.scale_log2, -m_used))
+                                     : 0.f;
         }
 #pragma unroll
-        for (int t = 0; t < 32; ++t) sum += pv[t];
+        for (int t = 0; t < 64; ++t) sum += pv[t];
         uint8_t* atom = prow + (c >> 6) * (P_BYTES / 2);
 #pragma unroll
-        for (int ch = 0; ch < 4; ++ch) {
-          const int logical = ((c & 63) >> 3) + ch;
+        for (int ch = 0; ch < 8; ++ch) {
           uint4 w;
           uint32_t* pw = reinterpret_cast<uint32_t*>(&w);
 #pragma unroll
@@ -280,7 +293,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap mQK, const __grid_constant__ 
             __half2 hv = __floats2half2_rn(pv[8 * ch + 2 * e], pv[8 * ch + 2 * e + 1]);
             pw[e] = *reinterpret_cast<uint32_t*>(&hv);
           }
-          *reinterpret_cast<uint4*>(atom + ((logical ^ sw) << 4)) = w;
+          *reinterpret_cast<uint4*>(atom + ((ch ^ sw) << 4)) = w;
         }
       }
       l += sum;
