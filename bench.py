@@ -123,11 +123,13 @@ def time_workload(name, steps=5, warmup=3, weights=None, device=0):
         audio = torch.from_numpy(audio_np).to(dev)
         _, el, _, tmax = gam.gam_plan_lengths(cfg, lens)
         enc = torch.empty((B, tmax, cfg["d_model"]), dtype=torch.float32, device=dev)
+        tok = torch.empty((B, tmax), dtype=torch.int32, device=dev)
+        cnt = torch.empty((B,), dtype=torch.int32, device=dev)
         stream = torch.cuda.current_stream(dev)
 
         def step():
             gam.gam_encode(ctx, audio, lens, out=enc, stream=stream)
-            gam.gam_ctc_greedy(ctx, enc, el, stream=stream)
+            gam.gam_ctc_greedy(ctx, enc, el, stream=stream, tokens=tok, counts=cnt)
 
         for _ in range(warmup):
             step()
@@ -314,12 +316,14 @@ def run_ours(args, rank, world, local_rank):
     audio = torch.from_numpy(audio_np).to(dev)
     fr, el, fmax, tmax = gam.gam_plan_lengths(cfg, lens)
     enc = torch.empty((B, tmax, cfg["d_model"]), dtype=torch.float32, device=dev)
+    tok = torch.empty((B, tmax), dtype=torch.int32, device=dev)
+    cnt = torch.empty((B,), dtype=torch.int32, device=dev)
     stream = torch.cuda.current_stream(dev)
     audio_seconds = float(np.sum(lens)) / synth.SAMPLE_RATE
 
     def step():
         gam.gam_encode(ctx, audio, lens, out=enc, stream=stream)
-        return gam.gam_ctc_greedy(ctx, enc, el, stream=stream)
+        return gam.gam_ctc_greedy(ctx, enc, el, stream=stream, tokens=tok, counts=cnt)
 
     # warm-up (untimed), then two profiled steps with every kernel family timed:
     # the per-family table and the dominant family come from steady-state steps

@@ -3,8 +3,10 @@
 // (segment layout, see common.cuh), the launch sequence of the encoder and of
 // the CTC decoder, launch counting / CUDA-event profiling and host-side fault
 // injection.
+#include <algorithm>
 #include <cmath>
 #include <cstdio>
+#include <cstdlib>
 #include <cstring>
 #include <map>
 #include <string>
@@ -79,6 +81,27 @@ struct Prof {
 
 constexpr int kRing = 8;
 
+// CUDA graphs for repeated calls.  A call is identified by everything its
+// kernel sequence depends on besides buffer contents: the entry point, the
+// clip lengths (hence the plan and every launch shape) and the caller's
+// pointers.  The first call with a key runs eagerly; the second is captured
+// (on a private stream) into a graph together with a private device copy of
+// its clip table, and every later call replays it with one cudaGraphLaunch.
+struct GraphEntry {
+  std::vector<int64_t> key;
+  cudaGraphExec_t exec = nullptr;
+  int* table = nullptr;  // device: the call's table, read by the captured kernels
+  uint64_t used = 0;
+};
+struct GraphCache {
+  bool enabled = true;
+  cudaStream_t cap = nullptr;
+  std::vector<GraphEntry> entries;
+  std::vector<std::vector<int64_t>> seen;  // keys met once
+  uint64_t tick = 0;
+};
+constexpr size_t kGraphCap = 16, kSeenCap = 64;
+
 }  // namespace
 
 struct gam_ctx {
@@ -131,6 +154,7 @@ struct gam_ctx {
   // tcgen05 GEMM plans
   TcGemmCache tc;
   Prof prof;
+  GraphCache graphs;
   int inject_err = 0, inject_count = 0;
 };
 
@@ -389,12 +413,10 @@ gam_status make_plan(gam_ctx* c, const gam_config& cfg, const int32_t* lengths, 
   return GAM_OK;
 }
 
-// Upload the clip table (and optional extra ints) through the pinned ring.
-gam_status upload_table(gam_ctx* c, const Plan& p, cudaStream_t s, Clips* out) {
-  const int slot = c->ring;
-  c->ring = (c->ring + 1) % kRing;
-  GAM_TRY(cuda_check(c, cudaEventSynchronize(c->tab_ev[slot]), "ring event"));
-  int* h = c->tab_host[slot];
+// The clip table read by the kernels (Clips): segment starts e[0..B], then F, L1,
+// L2 and a zero row, B + 1 ints each.
+int table_ints(const Plan& p) { return 5 * (p.B + 1); }
+void fill_table(const Plan& p, int* h) {
   const int B = p.B;
   for (int i = 0; i <= B; ++i) h[i] = p.e[i];
   for (int i = 0; i < B; ++i) {
@@ -403,7 +425,17 @@ gam_status upload_table(gam_ctx* c, const Plan& p, cudaStream_t s, Clips* out) {
     h[3 * (B + 1) + i] = p.len[i].L2;
     h[4 * (B + 1) + i] = 0;
   }
-  const size_t bytes = 5 * (size_t)(B + 1) * sizeof(int);
+}
+
+// Upload the clip table (and optional extra ints) through the pinned ring.
+gam_status upload_table(gam_ctx* c, const Plan& p, cudaStream_t s, Clips* out) {
+  const int slot = c->ring;
+  c->ring = (c->ring + 1) % kRing;
+  GAM_TRY(cuda_check(c, cudaEventSynchronize(c->tab_ev[slot]), "ring event"));
+  int* h = c->tab_host[slot];
+  const int B = p.B;
+  fill_table(p, h);
+  const size_t bytes = table_ints(p) * sizeof(int);
   GAM_TRY(cuda_check(c, cudaMemcpyAsync(c->tab_dev[slot], h, bytes, cudaMemcpyHostToDevice, s), "table upload"));
   GAM_TRY(cuda_check(c, cudaEventRecord(c->tab_ev[slot], s), "ring event record"));
   *out = Clips{c->tab_dev[slot], B};
@@ -419,6 +451,75 @@ gam_status upload_ints(gam_ctx* c, const int32_t* src, int n, cudaStream_t s, co
                      "lengths upload"));
   GAM_TRY(cuda_check(c, cudaEventRecord(c->tab_ev[slot], s), "ring event record"));
   *out = c->tab_dev[slot];
+  return GAM_OK;
+}
+
+// ---- CUDA graphs ----
+bool graphs_usable(const gam_ctx* c) { return c->graphs.enabled && c->prof.mask == 0 && c->inject_count == 0; }
+
+GraphEntry* graph_find(gam_ctx* c, const std::vector<int64_t>& key) {
+  for (GraphEntry& e : c->graphs.entries)
+    if (e.key == key) {
+      e.used = ++c->graphs.tick;
+      return &e;
+    }
+  return nullptr;
+}
+
+// True on the second call with this key (capture now); the first call only records it.
+bool graph_second_sighting(gam_ctx* c, const std::vector<int64_t>& key) {
+  auto& seen = c->graphs.seen;
+  for (size_t i = 0; i < seen.size(); ++i)
+    if (seen[i] == key) {
+      seen.erase(seen.begin() + i);
+      return true;
+    }
+  if (seen.size() >= kSeenCap) seen.erase(seen.begin());
+  seen.push_back(key);
+  return false;
+}
+
+void graph_free(GraphEntry& e) {
+  if (e.exec) cudaGraphExecDestroy(e.exec);
+  if (e.table) cudaFree(e.table);  // synchronises the device: no replay still reads it
+  e.exec = nullptr;
+  e.table = nullptr;
+}
+
+// Capture body(device table, capture stream) into a graph for key, with a private
+// device copy of table_host (n ints).  On success *out is the new cache entry.
+template <class F>
+gam_status graph_capture(gam_ctx* c, const std::vector<int64_t>& key, const int* table_host, int n, F&& body,
+                         GraphEntry** out) {
+  GraphCache& gc = c->graphs;
+  if (!gc.cap) GAM_TRY(cuda_check(c, cudaStreamCreateWithFlags(&gc.cap, cudaStreamNonBlocking), "capture stream"));
+  GraphEntry e;
+  e.key = key;
+  GAM_TRY(cuda_check(c, cudaMalloc((void**)&e.table, (size_t)n * sizeof(int)), "graph table"));
+  gam_status st = cuda_check(c, cudaMemcpy(e.table, table_host, (size_t)n * sizeof(int), cudaMemcpyHostToDevice),
+                             "graph table upload");
+  cudaGraph_t g = nullptr;
+  if (st == GAM_OK) st = cuda_check(c, cudaStreamBeginCapture(gc.cap, cudaStreamCaptureModeThreadLocal), "capture");
+  if (st == GAM_OK) {
+    st = body(e.table, gc.cap);
+    const gam_status end = cuda_check(c, cudaStreamEndCapture(gc.cap, &g), "end capture");
+    if (st == GAM_OK) st = end;
+  }
+  if (st == GAM_OK) st = cuda_check(c, cudaGraphInstantiate(&e.exec, g, 0), "graph instantiate");
+  if (g) cudaGraphDestroy(g);
+  if (st != GAM_OK) {
+    graph_free(e);
+    return st;
+  }
+  if (gc.entries.size() >= kGraphCap) {
+    auto lru = std::min_element(gc.entries.begin(), gc.entries.end(),
+                                [](const GraphEntry& a, const GraphEntry& b) { return a.used < b.used; });
+    graph_free(*lru);
+    gc.entries.erase(lru);
+  }
+  e.used = ++gc.tick;
+  gc.entries.push_back(e);
+  *out = &gc.entries.back();
   return GAM_OK;
 }
 
@@ -451,8 +552,12 @@ gam_status gemm(gam_ctx* c, int kind, cudaStream_t s, const void* A, const void*
   });
 }
 
+gam_status encoder_kernels(gam_ctx* c, const Plan& p, const Clips& clips, const float* audio, int64_t max_samples,
+                           int stop_layer, int stop_stage, float* out, cudaStream_t s);
+
 // The encoder up to (layer, stage); stage < 0 runs everything.  Leaves the
-// residual stream in c->x and scatters it to out.
+// residual stream in c->x and scatters it to out.  Repeated identical calls
+// replay a CUDA graph (see GraphCache).
 gam_status run_encoder(gam_ctx* c, const float* audio, const int32_t* lengths, int batch, int64_t max_samples,
                        int stop_layer, int stop_stage, float* out, int32_t* enc_len_out, cudaStream_t s) {
   const gam_config& cfg = c->cfg;
@@ -464,8 +569,31 @@ gam_status run_encoder(gam_ctx* c, const float* audio, const int32_t* lengths, i
     return fail(c, GAM_ERR_CAPACITY, "workspace too small for this batch");
   if (!audio || !out) return fail(c, GAM_ERR_INVALID_ARG, "null audio or output pointer");
   c->last_stream = s;
+  if (enc_len_out)
+    for (int i = 0; i < batch; ++i) enc_len_out[i] = p.len[i].L2;
+  if (graphs_usable(c)) {
+    std::vector<int64_t> key = {0, stop_layer, stop_stage, (int64_t)(uintptr_t)audio, max_samples,
+                                (int64_t)(uintptr_t)out, batch};
+    key.insert(key.end(), lengths, lengths + batch);
+    GraphEntry* e = graph_find(c, key);
+    if (!e && graph_second_sighting(c, key)) {
+      std::vector<int> tab(table_ints(p));
+      fill_table(p, tab.data());
+      GAM_TRY(graph_capture(c, key, tab.data(), (int)tab.size(), [&](const int* t, cudaStream_t cs) {
+        return encoder_kernels(c, p, Clips{t, batch}, audio, max_samples, stop_layer, stop_stage, out, cs);
+      }, &e));
+    }
+    if (e) return cuda_check(c, cudaGraphLaunch(e->exec, s), "graph launch");
+  }
   Clips clips;
   GAM_TRY(upload_table(c, p, s, &clips));
+  return encoder_kernels(c, p, clips, audio, max_samples, stop_layer, stop_stage, out, s);
+}
+
+// The encoder's kernel sequence for plan p (table already on the device).
+gam_status encoder_kernels(gam_ctx* c, const Plan& p, const Clips& clips, const float* audio, int64_t max_samples,
+                           int stop_layer, int stop_stage, float* out, cudaStream_t s) {
+  const gam_config& cfg = c->cfg;
   const int d = cfg.d_model, f = cfg.ffn_dim, H = cfg.n_heads, dh = c->d_head;
   const int ah = c->act_half;
   const float eps = cfg.ln_eps;
@@ -543,12 +671,13 @@ gam_status run_encoder(gam_ctx* c, const float* audio, const int32_t* lengths, i
       stopped = (l == stop_layer);
     }
   }
-  GAM_TRY(run_kernel(c, PK_MISC, s, [&] { return launch_scatter_out(c->x, clips, out, p.T2_max, d, s); }));
-  if (enc_len_out)
-    for (int i = 0; i < batch; ++i) enc_len_out[i] = p.len[i].L2;
-  return GAM_OK;
+  return run_kernel(c, PK_MISC, s, [&] { return launch_scatter_out(c->x, clips, out, p.T2_max, d, s); });
 }
 
+gam_status ctc_kernels(gam_ctx* c, const float* enc, const int* lo, int batch, int t_max, int M_valid, float* logp,
+                       int32_t* tokens, int32_t* counts, cudaStream_t s);
+
+// CTC decoding of encoder output; repeated identical calls replay a CUDA graph.
 gam_status run_ctc(gam_ctx* c, const float* enc, const int32_t* enc_len, int batch, int t_max, float* logp,
                    int32_t* tokens, int32_t* counts, cudaStream_t s) {
   const gam_config& cfg = c->cfg;
@@ -563,11 +692,30 @@ gam_status run_ctc(gam_ctx* c, const float* enc, const int32_t* enc_len, int bat
   for (int i = 0; i < batch; ++i) lo[i] = enc_len[i];
   lo[batch] = 0;
   for (int i = 0; i < batch; ++i) lo[batch + 1 + i] = lo[batch + i] + enc_len[i];
-  const int M_valid = lo[2 * batch];
+  if (graphs_usable(c)) {
+    std::vector<int64_t> key = {1, (int64_t)(uintptr_t)enc, batch, t_max, (int64_t)(uintptr_t)logp,
+                                (int64_t)(uintptr_t)tokens, (int64_t)(uintptr_t)counts};
+    key.insert(key.end(), enc_len, enc_len + batch);
+    GraphEntry* e = graph_find(c, key);
+    if (!e && graph_second_sighting(c, key)) {
+      GAM_TRY(graph_capture(c, key, lo.data(), (int)lo.size(), [&](const int* t, cudaStream_t cs) {
+        return ctc_kernels(c, enc, t, batch, t_max, lo[2 * batch], logp, tokens, counts, cs);
+      }, &e));
+    }
+    if (e) return cuda_check(c, cudaGraphLaunch(e->exec, s), "graph launch");
+  }
   const int* dev;
   GAM_TRY(upload_ints(c, lo.data(), 2 * batch + 1, s, &dev));
-  const int* lens = dev;
-  const int* off = dev + batch;
+  return ctc_kernels(c, enc, dev, batch, t_max, lo[2 * batch], logp, tokens, counts, s);
+}
+
+// CTC head, log-softmax / argmax and collapse; lo = [enc_len (batch) | offsets of the
+// compacted valid frames (batch + 1)] on the device, M_valid = total valid frames.
+gam_status ctc_kernels(gam_ctx* c, const float* enc, const int* lo, int batch, int t_max, int M_valid, float* logp,
+                       int32_t* tokens, int32_t* counts, cudaStream_t s) {
+  const gam_config& cfg = c->cfg;
+  const int* lens = lo;
+  const int* off = lo + batch;
   const int C = cfg.n_classes, M = batch * t_max;
   Clips none{nullptr, 0};
   if (c->head2.w) {
@@ -827,6 +975,8 @@ void destroy(gam_ctx* c) {
   }
   for (auto& e : c->prof.ev)
     if (e) cudaEventDestroy(e);
+  for (GraphEntry& e : c->graphs.entries) graph_free(e);
+  if (c->graphs.cap) cudaStreamDestroy(c->graphs.cap);
   delete c;
 }
 
@@ -895,6 +1045,7 @@ gam_status gam_create(const gam_config* cfg, const gam_tensor* tensors, int n_te
   c->act_half = cfg->precision == GAM_FP32 ? 0 : 1;
   c->wdtype = cfg->precision == GAM_FP32 ? 0 : (cfg->precision == GAM_FP16 ? 1 : 2);
   c->d_head = cfg->d_model / cfg->n_heads;
+  if (const char* v = std::getenv("GAM_CUDA_GRAPHS")) c->graphs.enabled = std::strcmp(v, "0") != 0;
   gam_status s = cuda_check(c, cudaSetDevice(device), "cudaSetDevice");
   if (s == GAM_OK) s = cuda_check(c, tc_init(&c->tc, device), "tensor-core init");
   if (s == GAM_OK) s = alloc_workspace(c);
@@ -994,6 +1145,13 @@ gam_status gam_transcribe(gam_ctx* c, const float* audio_host, const int32_t* le
   GAM_TRY(cuda_check(c, cudaMemcpyAsync(counts_host, c->counts_stage, (size_t)batch * 4, cudaMemcpyDeviceToHost, s),
                      "counts download"));
   return cuda_check(c, cudaStreamSynchronize(s), "transcribe sync");
+}
+
+gam_status gam_graphs_enable(gam_ctx* c, int on) {
+  GAM_TRY(enter(c));
+  c->graphs.enabled = on != 0;
+  c->graphs.seen.clear();
+  return GAM_OK;
 }
 
 gam_status gam_device_status(gam_ctx* c) {

@@ -28,8 +28,8 @@ STATUS = {0: "GAM_OK", 1: "GAM_ERR_INVALID_ARG", 2: "GAM_ERR_SHAPE", 3: "GAM_ERR
 EXPORTS = ("gam_status_string", "gam_last_error", "gam_plan_lengths", "gam_create", "gam_destroy", "gam_logmel",
            "gam_encode", "gam_encode_stage", "gam_ctc_greedy", "gam_ctc_collapse", "gam_transcribe",
            "gam_device_status", "gam_profile_enable", "gam_profile_reset", "gam_profile_kinds",
-           "gam_profile_kind_name", "gam_profile_read", "gam_ctc_collapse_noalloc", "gam_debug_gemm",
-           "gam_debug_inject_cuda_error")
+           "gam_profile_kind_name", "gam_profile_read", "gam_graphs_enable", "gam_ctc_collapse_noalloc",
+           "gam_debug_gemm", "gam_debug_inject_cuda_error")
 
 GAM_NOALLOC_MAX_FRAMES = 1 << 20
 
@@ -88,6 +88,7 @@ def lib() -> ctypes.CDLL:
         L.gam_profile_kind_name.restype = ctypes.c_char_p
         L.gam_profile_kind_name.argtypes = [ctypes.c_int]
         L.gam_profile_read.argtypes = [vp, ctypes.c_int, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_int64)]
+        L.gam_graphs_enable.argtypes = [vp, ctypes.c_int]
         L.gam_ctc_collapse_noalloc.argtypes = [vp, vp, ctypes.c_int, ctypes.c_int, ctypes.c_int, vp, vp, vp]
         L.gam_debug_gemm.argtypes = [vp, ctypes.c_int, vp, ctypes.c_int, vp, vp, ctypes.c_int, ctypes.c_int,
                                      ctypes.c_int, vp, ctypes.c_int, vp]
@@ -240,14 +241,20 @@ def gam_encode_stage(ctx: Context, audio, lengths, layer: int, stage: int, out=N
     return out
 
 
-def gam_ctc_greedy(ctx: Context, enc, enc_len, want_logp: bool = False, stream=None):
+def gam_ctc_greedy(ctx: Context, enc, enc_len, want_logp: bool = False, stream=None, tokens=None, counts=None,
+                   logp=None):
+    """Greedy CTC decoding of enc [B, T, d]; tokens / counts / logp may be passed in
+    (preallocated CUDA tensors, so repeated calls keep their pointers)."""
     import torch
     el = _i32(enc_len)
     B, tmax, _ = enc.shape
     C = ctx.cfg["n_classes"]
-    tokens = torch.empty((B, tmax), dtype=torch.int32, device=enc.device)
-    counts = torch.empty((B,), dtype=torch.int32, device=enc.device)
-    logp = torch.empty((B, tmax, C), dtype=torch.float32, device=enc.device) if want_logp else None
+    if tokens is None:
+        tokens = torch.empty((B, tmax), dtype=torch.int32, device=enc.device)
+    if counts is None:
+        counts = torch.empty((B,), dtype=torch.int32, device=enc.device)
+    if logp is None and want_logp:
+        logp = torch.empty((B, tmax, C), dtype=torch.float32, device=enc.device)
     _check(lib().gam_ctc_greedy(ctx.handle, enc.data_ptr(), _ptr_i32(el), B, tmax,
                                 logp.data_ptr() if logp is not None else None, tokens.data_ptr(), counts.data_ptr(),
                                 _stream(stream)), ctx)
@@ -329,6 +336,11 @@ def gam_ctc_collapse_noalloc(logits, lengths_dev, tokens, counts, stream=None):
     _check(lib().gam_ctc_collapse_noalloc(logits.data_ptr(), lengths_dev.data_ptr(), B, T, C, tokens.data_ptr(),
                                           counts.data_ptr(), _stream(stream)))
     return tokens, counts
+
+
+def gam_graphs_enable(ctx: Context, on: bool = True):
+    """Replay CUDA graphs for repeated identical calls (on by default)."""
+    _check(lib().gam_graphs_enable(ctx.handle, 1 if on else 0), ctx)
 
 
 def gam_debug_gemm(ctx: Context, impl: int, a, w, bias, out, stream=None):

@@ -235,6 +235,21 @@ gam_status gam_profile_read(gam_ctx* ctx, int kind, double* total_ms, int64_t* l
 gam_status gam_ctc_collapse_noalloc(const float* logits_dev, const int32_t* lengths_dev, int batch, int t_max,
                                     int n_classes, int32_t* tokens_dev, int32_t* counts_dev, void* stream);
 
+/* ---- CUDA graphs ---- */
+
+/* Repeated calls of gam_encode, gam_encode_stage and gam_ctc_greedy with the
+ * same clip lengths and the same buffer pointers replay a CUDA graph of the
+ * call's kernel sequence: the first such call runs eagerly, the second is
+ * captured (on a private stream, with a private device copy of the call's
+ * clip table) and launched on `stream`, later ones are one graph launch.
+ * Buffer contents may change between calls; pointers and lengths may not
+ * (a different pointer or length is a different graph, up to 16 are kept,
+ * least recently used first out).  No graph is used while profiling is
+ * enabled (gam_profile_enable) or an error is injected.  On by default; the
+ * environment variable GAM_CUDA_GRAPHS=0 (read by gam_create) or on = 0 here
+ * turns it off.  Outputs are bit-identical either way. */
+gam_status gam_graphs_enable(gam_ctx* ctx, int on);
+
 /* ---- kernel unit test (tests) ---- */
 
 /* One GEMM of the encoder's kind through the chosen implementation:
