@@ -198,8 +198,9 @@ __device__ __forceinline__ float swish_t(float v) {
 // 256 threads: thread (channel c, row half h) produces rows 32h .. 32h+31 of
 // channel c in 4 groups of 8, sliding over the staged input rows so each
 // shared-memory value feeds up to 8 outputs.  Weights (tap-major [K][d], BN
-// folded) live in registers.  Clip bounds are looked up once per row; rows
-// whose whole window lies inside their clip skip the per-tap checks.
+// folded) live in registers.  Clip bounds are looked up once per row; groups
+// whose whole window lies inside one clip take the plain path, the others
+// repeat it once per clip among their rows with out-of-clip inputs zeroed.
 template <typename T, int K>
 __global__ void __launch_bounds__(256)
 dwconv_kernel(const T* __restrict__ g, const float* __restrict__ w, const float* __restrict__ bias, Clips clips,
@@ -275,20 +276,34 @@ dwconv_kernel(const T* __restrict__ g, const float* __restrict__ w, const float*
 #pragma unroll
       for (int i = 0; i < 8; ++i) acc[i] = swish_t<T>(acc[i]);
     } else {
-#pragma unroll 1
-      for (int i = 0; i < 8; ++i) {
-        const int ri = r + i, li = s_lo[j0 + i], hiI = s_hi[j0 + i];
-        float a = 0.f;
-        if (ri >= li && ri < hiI) {
-          a = bv;
+      // near a clip edge: the group's rows fall into runs of the same clip (rows of
+      // a clip are contiguous); each run takes the interior computation over the
+      // window with the input rows outside its clip read as zero
 #pragma unroll
-          for (int k = 0; k < K; ++k) {
-            const int src = ri + k - PAD;
-            if (src >= li && src < hiI) a = fmaf(wk[k], tile[j0 + i + k][cc], a);
+      for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+      int i0 = 0;
+#pragma unroll 1
+      while (i0 < 8) {
+        const int li = s_lo[j0 + i0], hiI = s_hi[j0 + i0];
+        int i1 = i0 + 1;
+        while (i1 < 8 && s_lo[j0 + i1] == li) ++i1;
+        const unsigned span = (unsigned)(hiI - li);
+        float a[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) a[i] = bv;
+#pragma unroll
+        for (int t = 0; t < K + 7; ++t) {
+          const float xm = ((unsigned)(r - PAD + t - li) < span) ? tile[j0 + t][cc] : 0.f;  // input row r - PAD + t
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const int k = t - i;
+            if (k >= 0 && k < K) a[i] = fmaf(wk[k], xm, a[i]);
           }
-          a = swish_t<T>(a);
         }
-        acc[i] = a;
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+          if (i >= i0 && i < i1 && (unsigned)(r + i - li) < span) acc[i] = swish_t<T>(a[i]);
+        i0 = i1;
       }
     }
 #pragma unroll
