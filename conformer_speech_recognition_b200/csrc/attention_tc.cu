@@ -76,6 +76,8 @@ constexpr float kRescaleThreshold = 8.f;
 
 __global__ void __launch_bounds__(192, 2)
 attn_tc_kernel(const __grid_constant__ CUtensorMap mQK, const __grid_constant__ CUtensorMap mVT, const AttnArgs p) {
+  pdl_launch_dependents();
+  pdl_wait();  // Q, K, V^T from the previous kernel are complete
   const int b = blockIdx.z, h = blockIdx.y;
   const int L = p.clips.L2(b), e0 = p.clips.e(b);
   const int q0 = blockIdx.x * BQ;
@@ -384,8 +386,7 @@ cudaError_t launch_attention_tc(TcGemmCache* cache, const void* qk, const void* 
   e = cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
   if (e != cudaSuccess) return e;
   dim3 grid((t_max + BQ - 1) / BQ, n_heads, clips.B);
-  attn_tc_kernel<<<grid, 192, SMEM_BYTES, s>>>(mQK, mVT, a);
-  return cudaGetLastError();
+  return launch_pdl(attn_tc_kernel, grid, 192, SMEM_BYTES, s, mQK, mVT, a);
 }
 
 }  // namespace gam

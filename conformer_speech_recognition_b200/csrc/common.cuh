@@ -23,6 +23,34 @@
 
 namespace gam {
 
+// Programmatic dependent launch.  The encoder's kernels are launched with the
+// programmatic-serialisation attribute, so a kernel's CTAs may be scheduled
+// (and do their setup: barriers, TMEM, descriptor prefetch) while the previous
+// kernel in the stream is still finishing.  Each such kernel calls pdl_wait()
+// before its first global-memory access: it returns once the previous kernel
+// has completed and its writes are visible, so the stream order of the data is
+// unchanged.  pdl_launch_dependents() lets the next kernel be scheduled early.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+// Host side: launch with the programmatic-serialisation attribute (unless
+// GAM_PDL=0 in the environment), for kernels that call pdl_wait() first.
+bool pdl_enabled();
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s, Args... args) {
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl_enabled() ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
 // Device view of the per-call clip table: 5 arrays of B (+1) ints.
 struct Clips {
   const int* tab;  // [5][B+1]: e (B+1 entries), F, L1, L2, N

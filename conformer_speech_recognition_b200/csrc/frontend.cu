@@ -145,6 +145,8 @@ frontend_kernel(const float* __restrict__ audio, int64_t stride, Clips clips, in
 template <bool VEC>
 __global__ void __launch_bounds__(256)
 frames_kernel(const float* __restrict__ audio, int64_t stride, Clips clips, int rows, __half* __restrict__ frames) {
+  pdl_launch_dependents();
+  pdl_wait();
   const int r = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
   if (r >= rows) return;
   const int ci = clips.find(r, 4, 6);
@@ -172,6 +174,8 @@ constexpr size_t MEL_SMEM = (size_t)(FT * NBIN + NBIN * NMEL) * sizeof(float);
 __global__ void __launch_bounds__(256)
 mel_log_kernel(const float* __restrict__ power, int ld, const float* __restrict__ fb, Clips clips, int rows,
                void* __restrict__ mel, int out_half) {
+  pdl_launch_dependents();
+  pdl_wait();
   extern __shared__ float dyn[];
   float (*sp)[NBIN] = reinterpret_cast<float (*)[NBIN]>(dyn);  // [FT][NBIN]
   float* sfb = dyn + FT * NBIN;                                // [NBIN][NMEL]
@@ -214,9 +218,8 @@ cudaError_t launch_frames(const float* audio, int64_t audio_stride, Clips clips,
                           cudaStream_t s) {
   if (rows <= 0) return cudaSuccess;
   const bool vec = audio_stride % 4 == 0 && (reinterpret_cast<uintptr_t>(audio) & 15) == 0;
-  if (vec) frames_kernel<true><<<(rows + 7) / 8, 256, 0, s>>>(audio, audio_stride, clips, rows, frames);
-  else frames_kernel<false><<<(rows + 7) / 8, 256, 0, s>>>(audio, audio_stride, clips, rows, frames);
-  return cudaGetLastError();
+  if (vec) return launch_pdl(frames_kernel<true>, (rows + 7) / 8, 256, 0, s, audio, audio_stride, clips, rows, frames);
+  return launch_pdl(frames_kernel<false>, (rows + 7) / 8, 256, 0, s, audio, audio_stride, clips, rows, frames);
 }
 
 cudaError_t launch_mel_log(const float* power, int ld_power, const float* fb, Clips clips, int rows, void* mel,
@@ -224,8 +227,8 @@ cudaError_t launch_mel_log(const float* power, int ld_power, const float* fb, Cl
   if (rows <= 0) return cudaSuccess;
   cudaError_t e = cudaFuncSetAttribute(mel_log_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)MEL_SMEM);
   if (e != cudaSuccess) return e;
-  mel_log_kernel<<<(rows + FT - 1) / FT, 256, MEL_SMEM, s>>>(power, ld_power, fb, clips, rows, mel, out_half);
-  return cudaGetLastError();
+  return launch_pdl(mel_log_kernel, (rows + FT - 1) / FT, 256, MEL_SMEM, s, power, ld_power, fb, clips, rows, mel,
+                    out_half);
 }
 
 cudaError_t launch_frontend(const float* audio, int64_t audio_stride, Clips clips, int rows, int packed, int f_max,

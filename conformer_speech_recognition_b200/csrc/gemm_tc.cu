@@ -403,6 +403,8 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap mA, const __grid_constant__ C
   tc_fence_after();
   const uint32_t tmem = *tslot;
   const int KB = p.K / BK;
+  pdl_launch_dependents();
+  pdl_wait();  // the previous kernel's outputs (this GEMM's operands) are complete
 
   if (warp == 0) {
     if (lane == 0) {
@@ -669,6 +671,8 @@ gemm_tc_pair_kernel(const __grid_constant__ CUtensorMap mA, const __grid_constan
   tc_fence_after();
   const uint32_t tmem = *tslot;
   const int KB = p.K / BK;
+  pdl_launch_dependents();
+  pdl_wait();  // the previous kernel's outputs (this GEMM's operands) are complete
 
   if (warp == 0) {
     if (lane == 0) {
@@ -847,8 +851,7 @@ cudaError_t launch_epi(TcGemmCache* cache, const CUtensorMap& mA, const CUtensor
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::SMEM);
   if (e != cudaSuccess) return e;
   const int grid = args.tiles < cache->sm_count ? args.tiles : cache->sm_count;
-  kern<<<grid, threads_of<QB>(), C::SMEM, s>>>(mA, mA2, mB, mX, args);
-  return cudaGetLastError();
+  return launch_pdl(kern, grid, threads_of<QB>(), C::SMEM, s, mA, mA2, mB, mX, args);
 }
 
 template <int TN, int EPI>
@@ -859,11 +862,13 @@ cudaError_t launch_pair_epi(TcGemmCache* cache, const CUtensorMap& mA, const CUt
   static int max_clusters = 0;  // co-resident clusters of two (per process; one device model)
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::SMEM);
   if (e != cudaSuccess) return e;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = 2;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cudaLaunchConfig_t cfg = {};
   cfg.blockDim = dim3(threads_of<false>());
   cfg.dynamicSmemBytes = C::SMEM;
@@ -880,6 +885,7 @@ cudaError_t launch_pair_epi(TcGemmCache* cache, const CUtensorMap& mA, const CUt
   const int pairs = args.tiles < max_clusters ? args.tiles : max_clusters;
   cfg.gridDim = dim3(2 * pairs);
   cfg.stream = s;
+  cfg.numAttrs = pdl_enabled() ? 2 : 1;
   e = cudaLaunchKernelEx(&cfg, kern, mA, mA2, mB, mX, args);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();

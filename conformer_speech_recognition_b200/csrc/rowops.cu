@@ -85,6 +85,8 @@ template <typename T, int NV>
 __global__ void __launch_bounds__(256)
 ln_kernel(const float* __restrict__ x, const float* __restrict__ g, const float* __restrict__ b, float eps,
           T* __restrict__ u, int rows) {
+  pdl_launch_dependents();
+  pdl_wait();
   constexpr int d = NV * 128;
   const int lane = threadIdx.x & 31, nw = gridDim.x * 8;
   int row = blockIdx.x * 8 + (threadIdx.x >> 5);
@@ -107,6 +109,8 @@ template <typename T, int NV>
 __global__ void __launch_bounds__(256)
 ln_chain_kernel(float* __restrict__ x, const float* __restrict__ g1, const float* __restrict__ b1,
                 const float* __restrict__ g2, const float* __restrict__ b2, float eps, T* __restrict__ u, int rows) {
+  pdl_launch_dependents();
+  pdl_wait();
   constexpr int d = NV * 128;
   const int lane = threadIdx.x & 31, nw = gridDim.x * 8;
   int row = blockIdx.x * 8 + (threadIdx.x >> 5);
@@ -137,6 +141,8 @@ __global__ void __launch_bounds__(256)
 ln_rope_kernel(const float* __restrict__ x, const float* __restrict__ g, const float* __restrict__ b, float eps,
                const float* __restrict__ cos_tab, const float* __restrict__ sin_tab, Clips clips, T* __restrict__ u,
                T* __restrict__ urot, int rows) {
+  pdl_launch_dependents();
+  pdl_wait();
   constexpr int dh = DH, half = DH / 2, d = NV * 128;
   static_assert(half % 4 == 0, "a float4 of columns never straddles a half head");
   __shared__ __align__(16) float srow[8][d];
@@ -205,6 +211,8 @@ template <typename T, int K>
 __global__ void __launch_bounds__(256)
 dwconv_kernel(const T* __restrict__ g, const float* __restrict__ w, const float* __restrict__ bias, Clips clips,
               T* __restrict__ out, int rows, int d) {
+  pdl_launch_dependents();
+  pdl_wait();
   constexpr int PAD = (K - 1) / 2, R = 64, HALO = R + 2 * PAD;
   __shared__ __align__(16) float tile[HALO][128];
   __shared__ int s_lo[R], s_hi[R];
@@ -340,6 +348,8 @@ dwconv_generic_kernel(const T* __restrict__ g, const float* __restrict__ w, cons
 }
 
 __global__ void scatter_kernel(const float* __restrict__ x, Clips clips, float* __restrict__ out, int t_max, int d) {
+  pdl_launch_dependents();
+  pdl_wait();
   const int row = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
   if (row >= clips.B * t_max) return;
   const int b = row / t_max, t = row - b * t_max;
@@ -356,6 +366,8 @@ __global__ void scatter_kernel(const float* __restrict__ x, Clips clips, float* 
 __global__ void logsoftmax_argmax_kernel(const float* __restrict__ logits, int ld, const int* __restrict__ lens,
                                          int batch, int t_max, int C, float* __restrict__ logp,
                                          int* __restrict__ argmax, const int* __restrict__ off) {
+  pdl_launch_dependents();
+  pdl_wait();
   const int row = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
   if (row >= batch * t_max) return;
   const int b = row / t_max, t = row - b * t_max;
@@ -392,6 +404,8 @@ __global__ void logsoftmax_argmax_kernel(const float* __restrict__ logits, int l
 __global__ void __launch_bounds__(256)
 collapse_kernel(const int* __restrict__ argmax, const int* __restrict__ lens, int t_max, int blank,
                 int* __restrict__ tokens, int* __restrict__ counts) {
+  pdl_launch_dependents();
+  pdl_wait();
   __shared__ int warp_tot[8];
   __shared__ int s_total;
   const int b = blockIdx.x, tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
@@ -434,6 +448,8 @@ collapse_kernel(const int* __restrict__ argmax, const int* __restrict__ lens, in
 // read enc[b, v - off[b], :] and write the fp16 hi / lo split.
 __global__ void split_hi_lo_kernel(const float* __restrict__ enc, const int* __restrict__ off, int batch, int t_max,
                                    int d, int rows, __half* __restrict__ a) {
+  pdl_launch_dependents();
+  pdl_wait();
   const int v = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
   if (v >= rows) return;
   int lo = 0, hi = batch - 1;
@@ -488,8 +504,7 @@ int resident_grid(int rows) {
 
 template <typename T, int NV>
 cudaError_t ln_t(const float* x, const float* g, const float* b, float eps, void* u, int rows, cudaStream_t s) {
-  ln_kernel<T, NV><<<resident_grid<ln_kernel<T, NV>>(rows), 256, 0, s>>>(x, g, b, eps, (T*)u, rows);
-  return cudaGetLastError();
+  return launch_pdl(ln_kernel<T, NV>, resident_grid<ln_kernel<T, NV>>(rows), 256, 0, s, x, g, b, eps, (T*)u, rows);
 }
 
 cudaError_t launch_layernorm(const float* x, const float* g, const float* b, float eps, void* u, int u_half, int rows,
@@ -504,9 +519,8 @@ cudaError_t launch_layernorm(const float* x, const float* g, const float* b, flo
 template <typename T, int NV>
 cudaError_t ln_chain_t(float* x, const float* g1, const float* b1, const float* g2, const float* b2, float eps, void* u,
                        int rows, cudaStream_t s) {
-  ln_chain_kernel<T, NV><<<resident_grid<ln_chain_kernel<T, NV>>(rows), 256, 0, s>>>(x, g1, b1, g2, b2, eps, (T*)u,
-                                                                                        rows);
-  return cudaGetLastError();
+  return launch_pdl(ln_chain_kernel<T, NV>, resident_grid<ln_chain_kernel<T, NV>>(rows), 256, 0, s, x, g1, b1, g2, b2,
+                    eps, (T*)u, rows);
 }
 
 cudaError_t launch_layernorm_chain(float* x, const float* g1, const float* b1, const float* g2, const float* b2,
@@ -521,9 +535,8 @@ cudaError_t launch_layernorm_chain(float* x, const float* g1, const float* b1, c
 template <typename T, int DH, int NV>
 cudaError_t rope_nv(const float* x, const float* g, const float* b, float eps, const float* cos_tab,
                     const float* sin_tab, Clips clips, void* u, void* urot, int rows, cudaStream_t s) {
-  ln_rope_kernel<T, DH, NV><<<resident_grid<ln_rope_kernel<T, DH, NV>>(rows), 256, 0, s>>>(
-      x, g, b, eps, cos_tab, sin_tab, clips, (T*)u, (T*)urot, rows);
-  return cudaGetLastError();
+  return launch_pdl(ln_rope_kernel<T, DH, NV>, resident_grid<ln_rope_kernel<T, DH, NV>>(rows), 256, 0, s, x, g, b, eps,
+                    cos_tab, sin_tab, clips, (T*)u, (T*)urot, rows);
 }
 
 template <typename T, int DH>
@@ -553,13 +566,11 @@ cudaError_t dwconv_t(const void* g, const float* w, const float* bias, Clips cli
   dim3 grid((rows + 63) / 64, d / 128);
   const T* gi = (const T*)g;
   T* o = (T*)out;
-  if (K == 31) dwconv_kernel<T, 31><<<grid, 256, 0, s>>>(gi, w, bias, clips, o, rows, d);
-  else if (K == 5) dwconv_kernel<T, 5><<<grid, 256, 0, s>>>(gi, w, bias, clips, o, rows, d);
-  else if (K == 15) dwconv_kernel<T, 15><<<grid, 256, 0, s>>>(gi, w, bias, clips, o, rows, d);
-  else {
-    const size_t n = (size_t)rows * d;
-    dwconv_generic_kernel<T><<<(unsigned)((n + 255) / 256), 256, 0, s>>>(gi, w, bias, clips, o, rows, d, K);
-  }
+  if (K == 31) return launch_pdl(dwconv_kernel<T, 31>, grid, 256, 0, s, gi, w, bias, clips, o, rows, d);
+  if (K == 5) return launch_pdl(dwconv_kernel<T, 5>, grid, 256, 0, s, gi, w, bias, clips, o, rows, d);
+  if (K == 15) return launch_pdl(dwconv_kernel<T, 15>, grid, 256, 0, s, gi, w, bias, clips, o, rows, d);
+  const size_t n = (size_t)rows * d;
+  dwconv_generic_kernel<T><<<(unsigned)((n + 255) / 256), 256, 0, s>>>(gi, w, bias, clips, o, rows, d, K);
   return cudaGetLastError();
 }
 
@@ -572,29 +583,26 @@ cudaError_t launch_dwconv(const void* g, const float* w, const float* bias, Clip
 
 cudaError_t launch_scatter_out(const float* x, Clips clips, float* out, int t_max, int d, cudaStream_t s) {
   const int rows = clips.B * t_max;
-  scatter_kernel<<<(rows + 7) / 8, 256, 0, s>>>(x, clips, out, t_max, d);
-  return cudaGetLastError();
+  return launch_pdl(scatter_kernel, (rows + 7) / 8, 256, 0, s, x, clips, out, t_max, d);
 }
 
 cudaError_t launch_logsoftmax_argmax(const float* logits, int ld, const int* lens, int batch, int t_max, int C,
                                      float* logp, int* argmax, cudaStream_t s, const int* off) {
   const int rows = batch * t_max;
-  logsoftmax_argmax_kernel<<<(rows + 7) / 8, 256, 0, s>>>(logits, ld, lens, batch, t_max, C, logp, argmax, off);
-  return cudaGetLastError();
+  return launch_pdl(logsoftmax_argmax_kernel, (rows + 7) / 8, 256, 0, s, logits, ld, lens, batch, t_max, C, logp,
+                    argmax, off);
 }
 
 cudaError_t launch_split_hi_lo(const float* enc, const int* off, int batch, int t_max, int d, int rows, __half* a,
                                cudaStream_t s) {
   if (rows <= 0) return cudaSuccess;
   if (d % 128) return cudaErrorInvalidValue;
-  split_hi_lo_kernel<<<(rows + 7) / 8, 256, 0, s>>>(enc, off, batch, t_max, d, rows, a);
-  return cudaGetLastError();
+  return launch_pdl(split_hi_lo_kernel, (rows + 7) / 8, 256, 0, s, enc, off, batch, t_max, d, rows, a);
 }
 
 cudaError_t launch_collapse(const int* argmax, const int* lens, int batch, int t_max, int blank, int* tokens,
                             int* counts, cudaStream_t s) {
-  collapse_kernel<<<batch, 256, 0, s>>>(argmax, lens, t_max, blank, tokens, counts);
-  return cudaGetLastError();
+  return launch_pdl(collapse_kernel, batch, 256, 0, s, argmax, lens, t_max, blank, tokens, counts);
 }
 
 cudaError_t launch_f32_to_f16(const float* in, __half* out, int64_t n, cudaStream_t s) {

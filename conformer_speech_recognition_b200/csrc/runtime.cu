@@ -990,6 +990,14 @@ gam_status enter(gam_ctx* c) {
 
 void gam::set_context_free_error(const std::string& msg) { g_create_error = msg; }
 
+bool gam::pdl_enabled() {
+  static const bool on = [] {
+    const char* v = std::getenv("GAM_PDL");
+    return !(v && std::strcmp(v, "0") == 0);
+  }();
+  return on;
+}
+
 extern "C" {
 
 const char* gam_status_string(gam_status s) {

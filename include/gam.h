@@ -139,7 +139,10 @@ gam_status gam_plan_lengths(const gam_config* cfg, const int32_t* lengths_host, 
  * device memory until gam_destroy.  The environment variable GAM_GEMM_TILES
  * (read here) sets the tile policy of the fp16 tensor-core GEMMs: "single"
  * (single-CTA tiles only), "pair" (paired-CTA tiles wherever one applies) or,
- * by default, "auto" (the cheaper of the two by the library's cost model). */
+ * by default, "auto" (the cheaper of the two by the library's cost model).
+ * The encoder's kernels are launched with programmatic dependent launch (each
+ * kernel's setup overlaps the previous kernel's tail; data order unchanged);
+ * GAM_PDL=0 in the environment turns that off. */
 gam_status gam_create(const gam_config* cfg, const gam_tensor* tensors, int n_tensors, int device,
                       gam_ctx** out);
 
