@@ -136,8 +136,9 @@ cudaError_t launch_frontend(const float* audio, int64_t audio_stride, Clips clip
 // clipped log from the power spectrum power[rows, ld_power] (first 161 bins).
 cudaError_t launch_frames(const float* audio, int64_t audio_stride, Clips clips, int rows, __half* frames,
                           cudaStream_t s);
-cudaError_t launch_mel_log(const float* power, int ld_power, const float* fb, Clips clips, int rows, void* mel,
-                           int out_half, cudaStream_t s);
+// fb_range: int pairs (first, last) nonzero filterbank row per mel bin (last < first: none).
+cudaError_t launch_mel_log(const float* power, int ld_power, const float* fb, const int* fb_range, Clips clips,
+                           int rows, void* mel, int out_half, cudaStream_t s);
 
 cudaError_t launch_layernorm(const float* x, const float* g, const float* b, float eps, void* u, int u_half,
                              int rows, int d, cudaStream_t s);

@@ -169,16 +169,18 @@ frames_kernel(const float* __restrict__ audio, int64_t stride, Clips clips, int 
 }
 
 // mel = power[:, :161] . fb, then log(clip(mel, 1e-9, 1e9)); 32 rows per CTA.
-constexpr size_t MEL_SMEM = (size_t)(FT * NBIN + NBIN * NMEL) * sizeof(float);
+// fb_range[m] = (first, last) filterbank row with a nonzero weight in column m
+// (found when the context is built): the other rows add exact zeros, so the
+// sum runs over that range only.  The filterbank is read through L1.
+constexpr size_t MEL_SMEM = (size_t)(FT * NBIN) * sizeof(float);
 
 __global__ void __launch_bounds__(256)
-mel_log_kernel(const float* __restrict__ power, int ld, const float* __restrict__ fb, Clips clips, int rows,
-               void* __restrict__ mel, int out_half) {
+mel_log_kernel(const float* __restrict__ power, int ld, const float* __restrict__ fb, const int2* __restrict__ fb_range,
+               Clips clips, int rows, void* __restrict__ mel, int out_half) {
   pdl_launch_dependents();
   pdl_wait();
   extern __shared__ float dyn[];
   float (*sp)[NBIN] = reinterpret_cast<float (*)[NBIN]>(dyn);  // [FT][NBIN]
-  float* sfb = dyn + FT * NBIN;                                // [NBIN][NMEL]
   __shared__ int s_valid[FT];
   const int tid = threadIdx.x, row0 = blockIdx.x * FT;
   if (tid < FT) {
@@ -191,7 +193,6 @@ mel_log_kernel(const float* __restrict__ power, int ld, const float* __restrict_
     }
     s_valid[tid] = ok;
   }
-  for (int idx = tid; idx < NBIN * NMEL; idx += 256) sfb[idx] = __ldg(fb + idx);
   for (int idx = tid; idx < FT * NBIN; idx += 256) {
     const int j = idx / NBIN, k = idx - j * NBIN;
     const int r = row0 + j;
@@ -199,11 +200,12 @@ mel_log_kernel(const float* __restrict__ power, int ld, const float* __restrict_
   }
   __syncthreads();
   const int m = tid & 63;
+  const int2 kr = __ldg(fb_range + m);
 #pragma unroll
   for (int j = 0; j < FT / 4; ++j) {
     const int a = (tid >> 6) + 4 * j;
     float acc = 0.f;
-    for (int k = 0; k < NBIN; ++k) acc = fmaf(sp[a][k], sfb[k * NMEL + m], acc);
+    for (int k = kr.x; k <= kr.y; ++k) acc = fmaf(sp[a][k], __ldg(fb + k * NMEL + m), acc);
     const int r = row0 + a;
     if (r >= rows) continue;
     const float v = s_valid[a] ? logf(fminf(fmaxf(acc, 1e-9f), 1e9f)) : 0.f;
@@ -222,13 +224,11 @@ cudaError_t launch_frames(const float* audio, int64_t audio_stride, Clips clips,
   return launch_pdl(frames_kernel<false>, (rows + 7) / 8, 256, 0, s, audio, audio_stride, clips, rows, frames);
 }
 
-cudaError_t launch_mel_log(const float* power, int ld_power, const float* fb, Clips clips, int rows, void* mel,
-                           int out_half, cudaStream_t s) {
+cudaError_t launch_mel_log(const float* power, int ld_power, const float* fb, const int* fb_range, Clips clips,
+                           int rows, void* mel, int out_half, cudaStream_t s) {
   if (rows <= 0) return cudaSuccess;
-  cudaError_t e = cudaFuncSetAttribute(mel_log_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)MEL_SMEM);
-  if (e != cudaSuccess) return e;
-  return launch_pdl(mel_log_kernel, (rows + FT - 1) / FT, 256, MEL_SMEM, s, power, ld_power, fb, clips, rows, mel,
-                    out_half);
+  return launch_pdl(mel_log_kernel, (rows + FT - 1) / FT, 256, MEL_SMEM, s, power, ld_power, fb,
+                    reinterpret_cast<const int2*>(fb_range), clips, rows, mel, out_half);
 }
 
 cudaError_t launch_frontend(const float* audio, int64_t audio_stride, Clips clips, int rows, int packed, int f_max,

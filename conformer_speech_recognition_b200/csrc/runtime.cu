@@ -115,6 +115,7 @@ struct gam_ctx {
   // weights
   float* basis = nullptr;  // [320][320]
   float* fb = nullptr;     // [161][64]
+  int* fb_range = nullptr; // [64][2]: first and last nonzero filterbank row of each mel bin
   DevLinear dft;           // fp16 modes: windowed DFT basis as a [512, 320] GEMM weight,
                            // rows [cos 64 bins | sin 64 bins] per 128 (bins 0..255, zero past 160)
   __half* frames = nullptr;  // [R0_cap, 320] fp16 frames
@@ -605,7 +606,7 @@ gam_status encoder_kernels(gam_ctx* c, const Plan& p, const Clips& clips, const 
     GAM_TRY(gemm(c, PK_FRONTEND, s, c->frames, nullptr, 0, cfg.n_fft, c->dft, p.R0, EPI_POWER, 1.f, c->power, 256,
                  clips));
     GAM_TRY(run_kernel(c, PK_FRONTEND, s, [&] {
-      return launch_mel_log(c->power, 256, c->fb, clips, p.R0, c->mel, ah, s);
+      return launch_mel_log(c->power, 256, c->fb, c->fb_range, clips, p.R0, c->mel, ah, s);
     }));
   } else {
     GAM_TRY(run_kernel(c, PK_FRONTEND, s, [&] {
@@ -768,6 +769,21 @@ gam_status build_weights(gam_ctx* c, const gam_tensor* tensors, int n) {
       }
     GAM_TRY(upload_f32(c, &c->basis, basis));
     GAM_TRY(upload_f32(c, &c->fb, fbv));
+    {
+      const int nb = cfg.n_fft / 2 + 1, nm = cfg.n_mels;
+      std::vector<int> range(2 * (size_t)nm);
+      for (int m = 0; m < nm; ++m) {
+        int lo = nb, hi = -1;
+        for (int k = 0; k < nb; ++k)
+          if ((float)fbv[(size_t)k * nm + m] != 0.f) {
+            lo = std::min(lo, k);
+            hi = k;
+          }
+        range[2 * m] = hi < 0 ? 0 : lo;
+        range[2 * m + 1] = hi;
+      }
+      GAM_TRY(upload(c, &c->fb_range, range.data(), range.size() * sizeof(int)));
+    }
     if (cfg.precision != GAM_FP32) {
       HostLinear hd;
       hd.N = 512;

@@ -179,3 +179,24 @@ def test_fp32_subsampling_every_length_residue():
         assert out[i, :el[i]].shape == dump["x0"].shape
         assert max_abs(out[i, :el[i]], dump["x0"]) <= TOL_FP32_LAYER, i
     ctx.close()
+
+
+def test_fp16_subsampling_tensor_core_frontend():
+    """fp16 mode: tensor-core frontend (fp16 frames, DFT GEMM with the power
+    epilogue, mel over the filterbank's nonzero ranges, log) and the two
+    subsampling GEMMs, against the oracle's subsampling output."""
+    model = small_model(d=256, heads=4, ffn=512, layers=1, K=5)
+    cfg, W = config_and_weights(model, 34, "fp16")
+    lengths = [1280, 16000, 37123, 320 + 160 * 40]
+    audio, lens = synth.random_audio(lengths, seed=17)
+    ctx = gam.gam_create(cfg, W, len(lens), int(max(lens)))
+    out = gam.gam_encode_stage(ctx, to_torch(audio), lens, 0, gam.STAGE_SUBSAMPLING).cpu().numpy()
+    _, el, _, _ = gam.gam_plan_lengths(cfg, lens)
+    for i in range(len(lens)):
+        _, dump = oracle_clip(audio[i], lens[i], W, cfg, dump=True, n_layers=0)
+        got = out[i, :el[i]]
+        assert got.shape == dump["x0"].shape
+        assert rel_fro(got, dump["x0"]) <= TOL_REL_FRO, i
+        assert max_abs(got, dump["x0"]) <= TOL_MAX_ABS, i
+        assert np.all(out[i, el[i]:] == 0)
+    ctx.close()
