@@ -54,6 +54,31 @@ def load_peaks():
     return d
 
 
+def fp16_vs_bf16_matmul(device, n=8192, iters=10):
+    """Library (cuBLAS) dense matmul rate in fp16 and bf16 on this GPU, n^3 shape,
+    best of `iters` with CUDA events: a check that the fp16 tensor-core peak the
+    roofline uses equals the measured bf16 one.  Not part of the timed path."""
+    import torch
+    out = {}
+    for name, dt in (("fp16", torch.float16), ("bf16", torch.bfloat16)):
+        a = torch.randn(n, n, device=device, dtype=dt)
+        b = torch.randn(n, n, device=device, dtype=dt)
+        for _ in range(3):
+            torch.matmul(a, b)
+        best = float("inf")
+        for _ in range(iters):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            torch.matmul(a, b)
+            e1.record()
+            torch.cuda.synchronize(device)
+            best = min(best, e0.elapsed_time(e1))
+        out[name + "_tflops"] = 2.0 * n ** 3 / (best / 1e3) / 1e12
+        del a, b
+    out["fp16_over_bf16"] = out["fp16_tflops"] / out["bf16_tflops"]
+    return out
+
+
 def algorithmic_work(cfg, lens):
     """Per-kernel-family algorithmic FLOPs or bytes for ONE step, and the number of
     launches of each family per step.  Valid frames only (padding excluded)."""
@@ -405,6 +430,7 @@ def run_ours(args, rank, world, local_rank):
             roof = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
                     "traffic": measured_traffic(name, dominant), "kernel": dominant,
                     "peak_source": f"{peaks['source']} HBM copy"}
+        peak_check = fp16_vs_bf16_matmul(dev) if world == 1 else None
         gemm_flops = sum(v for k, v in fl.items() if k.startswith("gemm_"))
         # GEMM kernel time per step from the profiled steps (every family timed there)
         gemm_ms = sum(v[0] for k, v in warm.items() if k.startswith("gemm_")) / n_prof
@@ -437,6 +463,7 @@ def run_ours(args, rank, world, local_rank):
             "gemm_tflops_per_s_of_gemm_time": gemm_flops / (gemm_ms / 1e3) / 1e12 if gemm_ms > 0 else None,
             "gemm_frac_of_fp16_peak": (gemm_flops / (gemm_ms / 1e3) / 1e12) / peaks["bf16_tflops_sustained"]
             if gemm_ms > 0 else None,
+            "fp16_peak_check": peak_check,
             "cpu_baseline": cpu,
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
             "gpu_launches": int(launches),
