@@ -422,7 +422,8 @@ def run_ours(args, rank, world, local_rank):
             peak = peaks["bf16_tflops_sustained"]
             roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                     "frac": achieved / peak, "traffic": measured_traffic(name, dominant), "kernel": dominant,
-                    "peak_source": f"{peaks['source']} bf16 sustained (fp16 dense rate equal to bf16)"}
+                    "peak_source": f"{peaks['source']} bf16 sustained, used for the fp16 kernels "
+                                   "(fp16_peak_check: library fp16 / bf16 matmul rates in this run)"}
         else:
             per_launch = by.get(dominant, 0.0) / max(per_step_launches_dom, 1)
             achieved = per_launch / (avg_launch_ms / 1e3) / 1e9
