@@ -52,6 +52,13 @@ def test_plan_lengths_matches_oracle(L):
     assert list(fr) == [99, 1999] and list(el) == [24, 499] and tmax == 500
 
 
+def test_plan_rejects_empty_batch(L):
+    cfg = synth.workload_config("c1_1s_b1_d768")
+    with pytest.raises(gam.GamError) as e:
+        gam.gam_plan_lengths(cfg, [])
+    assert e.value.name == "GAM_ERR_INVALID_ARG"
+
+
 def test_plan_rejects_short_clip(L):
     cfg = synth.workload_config("c1_1s_b1_d768")
     with pytest.raises(gam.GamError) as e:
