@@ -10,7 +10,7 @@ import pytest
 
 import oracle
 from conformer_speech_recognition_b200 import synth
-from conftest import read_golden
+from conftest import read_golden, read_golden_rows
 
 
 def test_layer_norm_invariants():
@@ -43,6 +43,141 @@ def test_batch_norm_eval_identity_case():
     eps = 1e-5
     y = oracle.batch_norm_eval(x, np.ones(3), np.zeros(3), np.zeros(3), np.full(3, 1 - eps), eps)
     np.testing.assert_allclose(y, x, rtol=1e-12)
+
+
+def _silu_table():
+    """x -> (sigma(x), x sigma(x)) from the golden fixture."""
+    return {float(x): (float(s), float(y)) for x, s, y in read_golden_rows("activations.txt")}
+
+
+# Inference BatchNorm, hand-worked cases with var + eps a perfect square:
+# gamma (x - mean) / sqrt(var + eps) + beta, per channel.
+#   x = 3,  mean = 1,   var + eps = 4,    gamma = 2,  beta = 0.5 ->  2 / 2 * 2 + 0.5 = 2.5
+#   x = -1, mean = 0.5, var + eps = 0.25, gamma = 1,  beta = 0   -> -1.5 / 0.5      = -3
+#   x = 0,  mean = -2,  var + eps = 16,   gamma = -1, beta = 1   ->  2 / 4 * -1 + 1 = 0.5
+_BN_EPS = 1e-5
+_BN_CASE = dict(x=[3.0, -1.0, 0.0], mean=[1.0, 0.5, -2.0], var_eps=[4.0, 0.25, 16.0], gamma=[2.0, 1.0, -1.0],
+                beta=[0.5, 0.0, 1.0], expected=[2.5, -3.0, 0.5])
+
+
+def _bn_pin_holds():
+    import oracle.gigaam as og
+    c = _BN_CASE
+    y = og.batch_norm_eval(np.array([c["x"]]), np.array(c["gamma"]), np.array(c["beta"]), np.array(c["mean"]),
+                               np.array(c["var_eps"]) - _BN_EPS, _BN_EPS)
+    return bool(np.allclose(y[0], c["expected"], rtol=0, atol=1e-12))
+
+
+def test_batch_norm_eval_hand_cases():
+    assert _bn_pin_holds()
+
+
+def test_batch_norm_folded_equals_unfolded():
+    """BatchNorm after the depthwise conv folds into the conv's weight and bias:
+    w' = w g / sqrt(v + eps), b' = (b - mu) g / sqrt(v + eps) + beta."""
+    rng = np.random.default_rng(11)
+    T, d, K = 9, 5, 5
+    x = rng.normal(size=(T, d))
+    w, b = rng.normal(size=(d, 1, K)), rng.normal(size=d)
+    g, beta = rng.normal(1.0, 0.3, size=d), rng.normal(size=d)
+    mu, var = rng.normal(size=d), rng.uniform(0.2, 3.0, size=d)
+    unfolded = oracle.batch_norm_eval(oracle.depthwise_conv1d(x, w, b), g, beta, mu, var, _BN_EPS)
+    sc = g / np.sqrt(var + _BN_EPS)
+    folded = oracle.depthwise_conv1d(x, w * sc[:, None, None], (b - mu) * sc + beta)
+    np.testing.assert_allclose(unfolded, folded, rtol=0, atol=1e-12)
+
+
+def _ffn_pin_holds():
+    """linear1 = [I; 0], linear2 = [I | 0], zero biases: FFN(u) = SiLU(u), compared
+    with the fixture's SiLU values."""
+    tab = _silu_table()
+    d, f = 4, 8
+    u = np.array([[1.0, -1.0, 2.0, 0.5], [-2.0, 3.0, -0.5, 1.0]])
+    W = {"f.linear1.weight": np.vstack([np.eye(d), np.zeros((f - d, d))]), "f.linear1.bias": np.zeros(f),
+         "f.linear2.weight": np.hstack([np.eye(d), np.zeros((d, f - d))]), "f.linear2.bias": np.zeros(d)}
+    y = oracle.feed_forward(u, W, "f", np.float64)
+    expected = np.vectorize(lambda v: tab[float(v)][1])(u)
+    return bool(np.allclose(y, expected, rtol=0, atol=1e-15))
+
+
+def test_feed_forward_activation_is_silu():
+    assert _ffn_pin_holds()
+
+
+def _conv_module_pin_holds():
+    """Conv module with a non-identity BatchNorm.  pointwise1 = [I; 0] (GLU gate 0,
+    so sigma = 1/2), depthwise = centre tap 1 and bias 0, pointwise2 = I, and per
+    channel a BatchNorm chosen so that BN(u / 2) is 1, -1 and 2:
+      ch0: u = 4  -> 2   -> (2 - 1) / 2 * 2         = 1  -> SiLU(1)
+      ch1: u = -2 -> -1  -> (-1 - 0) / 1 * 1        = -1 -> SiLU(-1)
+      ch2: u = 1  -> 0.5 -> (0.5 - 0.5) / 0.5 + 2   = 2  -> SiLU(2)
+    BatchNorm after SiLU, or no BatchNorm, or another activation gives other values."""
+    tab = _silu_table()
+    d, K, T = 3, 5, 3
+    cfg, W = _zero_layer_weights(d, 8, K)
+    p = "layers.0.conv"
+    W[p + ".pointwise1.weight"] = np.concatenate([np.eye(d), np.zeros((d, d))])[:, :, None]
+    W[p + ".depthwise.weight"][:, 0, K // 2] = 1.0
+    W[p + ".pointwise2.weight"] = np.eye(d)[:, :, None]
+    W[p + ".bn.running_mean"] = np.array([1.0, 0.0, 0.5])
+    W[p + ".bn.running_var"] = np.array([4.0, 1.0, 0.25]) - cfg["bn_eps"]
+    W[p + ".bn.weight"] = np.array([2.0, 1.0, 1.0])
+    W[p + ".bn.bias"] = np.array([0.0, 0.0, 2.0])
+    u = np.tile(np.array([[4.0, -2.0, 1.0]]), (T, 1))
+    y = oracle.conv_module(u, W, p, cfg, np.float64)
+    expected = np.tile(np.array([[tab[1.0][1], tab[-1.0][1], tab[2.0][1]]]), (T, 1))
+    return bool(np.allclose(y, expected, rtol=0, atol=1e-14))
+
+
+def test_conv_module_batchnorm_before_silu():
+    assert _conv_module_pin_holds()
+
+
+def _relu(x):
+    return np.maximum(x, 0.0)
+
+
+def _identity(x):
+    return x
+
+
+def _gelu_tanh(x):
+    return 0.5 * x * (1.0 + np.tanh(np.sqrt(2.0 / np.pi) * (x + 0.044715 * x ** 3)))
+
+
+@pytest.mark.parametrize("mutant", [_relu, _identity, _gelu_tanh], ids=["relu", "identity", "gelu"])
+def test_activation_pins_catch_a_wrong_activation(monkeypatch, mutant):
+    """A mistake planted in the oracle (another activation in place of SiLU) is
+    caught by the FFN and conv-module pins."""
+    import oracle.gigaam as og
+    monkeypatch.setattr(og, "swish", mutant)
+    assert not _ffn_pin_holds()
+    assert not _conv_module_pin_holds()
+
+
+def _bn_x_plus_mean(x, gamma, beta, mean, var, eps):
+    return (x + mean) / np.sqrt(var + eps) * gamma + beta
+
+
+def _bn_times_root(x, gamma, beta, mean, var, eps):
+    return (x - mean) * np.sqrt(var + eps) * gamma + beta
+
+
+def _bn_eps_outside(x, gamma, beta, mean, var, eps):
+    return (x - mean) / (np.sqrt(var) + eps) * gamma + beta
+
+
+def _bn_missing(x, gamma, beta, mean, var, eps):
+    return x
+
+
+@pytest.mark.parametrize("mutant", [_bn_x_plus_mean, _bn_times_root, _bn_eps_outside, _bn_missing],
+                         ids=["x_plus_mean", "times_root", "eps_outside_root", "missing"])
+def test_batchnorm_pins_catch_a_wrong_formula(monkeypatch, mutant):
+    import oracle.gigaam as og
+    monkeypatch.setattr(og, "batch_norm_eval", mutant)
+    assert not _bn_pin_holds()
+    assert not _conv_module_pin_holds()
 
 
 def test_depthwise_conv_vs_numpy_correlate():
