@@ -12,10 +12,15 @@
 // library holds GAM_NOALLOC_MAX_FRAMES * 4 bytes (4 MiB) of it until the
 // process exits.  Host code cannot use the array's name as a device address;
 // on the first call on a device (with that device current) the address is
-// looked up once with cudaGetSymbolAddress and cached.  Every call on a device
+// looked up once with cudaGetSymbolAddress and cached together with the
+// device's current CUDA context: after a cudaDeviceReset the device gets a new
+// context (and the module a new load), so the lookup is done again there
+// instead of reusing an address that no longer exists.  Every call on a device
 // shares the one array: calls whose GPU work overlaps (two streams, or two
 // threads) race on it.  The argmax kernel writes every entry the collapse
 // kernel later reads, so nothing has to be cleared between calls.
+#include <cuda.h>
+
 #include <mutex>
 #include <string>
 
@@ -30,6 +35,23 @@ static __device__ __align__(256) int g_noalloc_argmax[GAM_NOALLOC_MAX_FRAMES];
 
 std::mutex g_mu;
 int* g_addr[kMaxDevices] = {};
+CUcontext g_addr_ctx[kMaxDevices] = {};  // the context each cached address belongs to
+
+// The calling thread's current CUDA context (driver entry point resolved through
+// the runtime, so the library links against cudart only).
+cudaError_t current_context(CUcontext* out) {
+  using Fn = CUresult (*)(CUcontext*);
+  static Fn fn = [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return (Fn) nullptr;
+    return reinterpret_cast<Fn>(f);
+  }();
+  if (!fn) return cudaErrorNotSupported;
+  return fn(out) == CUDA_SUCCESS ? cudaSuccess : cudaErrorDeviceUninitialized;
+}
 
 gam_status fail(gam_status s, const std::string& msg) {
   gam::set_context_free_error(msg);
@@ -56,12 +78,20 @@ extern "C" gam_status gam_ctc_collapse_noalloc(const float* logits_dev, const in
   int* scratch = nullptr;
   {
     std::lock_guard<std::mutex> lock(g_mu);
-    if (!g_addr[dev]) {
+    CUcontext ctx = nullptr;
+    if (g_addr[dev]) {
+      e = current_context(&ctx);
+      if (e != cudaSuccess) return fail(GAM_ERR_CUDA, std::string("cuCtxGetCurrent: ") + cudaGetErrorString(e));
+    }
+    if (!g_addr[dev] || ctx != g_addr_ctx[dev]) {
       void* p = nullptr;
-      e = cudaGetSymbolAddress(&p, g_noalloc_argmax);
+      e = cudaGetSymbolAddress(&p, g_noalloc_argmax);  // also makes the device's primary context current
       if (e != cudaSuccess)
         return fail(GAM_ERR_CUDA, std::string("cudaGetSymbolAddress: ") + cudaGetErrorString(e));
+      e = current_context(&ctx);
+      if (e != cudaSuccess) return fail(GAM_ERR_CUDA, std::string("cuCtxGetCurrent: ") + cudaGetErrorString(e));
       g_addr[dev] = static_cast<int*>(p);
+      g_addr_ctx[dev] = ctx;
     }
     scratch = g_addr[dev];
   }

@@ -49,6 +49,8 @@ struct TcArgs {
   EpiParams ep;
   const __half* scale_t;  // INT8 weights: fp16 scales transposed to [K/64][N]
   int* status;
+  uint64_t wait_ns;       // limit of every bounded wait
+  int debug_skip;         // test hook: k-block counter value whose loads are not issued (-1: none)
 };
 
 // Residual epilogue: per epilogue warp a 32 x 32 fp32 staging tile (4 KB, 128-byte
@@ -416,7 +418,11 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap mA, const __grid_constant__ C
         const CUtensorMap* ma = (n0 >= p.n_split) ? &mA2 : &mA;
         for (int kb = 0; kb < KB; ++kb) {
           const int s = it % STAGES;
-          if (!mbar_wait(&empty[s], ((it / STAGES) & 1) ^ 1, abort_flag)) {
+          if (it == p.debug_skip) {  // test hook: this stage never fills, its consumer's wait runs out
+            ++it;
+            continue;
+          }
+          if (!mbar_wait(&empty[s], ((it / STAGES) & 1) ^ 1, abort_flag, p.wait_ns)) {
             ok = false;
             break;
           }
@@ -437,14 +443,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap mA, const __grid_constant__ C
       }
       // every issued copy has landed before the CTA can exit (bounded)
       const int first = it > STAGES ? it - STAGES : 0;
-      for (int j = first; j < it; ++j) {
-        const uint64_t t0 = globaltimer_ns();
-        while (!mbar_try_wait(&full[j % STAGES], (j / STAGES) & 1))
-          if (globaltimer_ns() - t0 > kWaitLimitNs) {
-            *abort_flag = 1;
-            break;
-          }
-      }
+      for (int j = first; j < it; ++j) mbar_settle(&full[j % STAGES], (j / STAGES) & 1, abort_flag, p.wait_ns);
     }
   } else if (warp == 1) {
     if (lane == 0) {
@@ -454,12 +453,12 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap mA, const __grid_constant__ C
       for (int tile = blockIdx.x; tile < p.tiles && ok; tile += gridDim.x, ++local) {
         const int acc = local & 1;
         const uint32_t use = (uint32_t)(local >> 1);
-        if (!mbar_wait(&tempty[acc], (use & 1) ^ 1, abort_flag)) break;
+        if (!mbar_wait(&tempty[acc], (use & 1) ^ 1, abort_flag, p.wait_ns)) break;
         tc_fence_after();
         const uint32_t d = tmem + (uint32_t)(acc * BN);
         for (int kb = 0; kb < KB; ++kb) {
           const int s = it % STAGES;
-          if (!mbar_wait(QB ? &bready[s] : &full[s], (it / STAGES) & 1, abort_flag)) {
+          if (!mbar_wait(QB ? &bready[s] : &full[s], (it / STAGES) & 1, abort_flag, p.wait_ns)) {
             ok = false;
             break;
           }
@@ -475,12 +474,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap mA, const __grid_constant__ C
       }
       // drain: all MMAs issued by this thread complete before TMEM is freed (bounded)
       umma_commit(drain);
-      const uint64_t t0 = globaltimer_ns();
-      while (!mbar_try_wait(drain, 0))
-        if (globaltimer_ns() - t0 > kWaitLimitNs) {
-          *abort_flag = 1;
-          break;
-        }
+      mbar_settle(drain, 0, abort_flag, p.wait_ns);
     }
   } else if (QB && warp >= 2 + kEpiWarps) {
     // converter warps: INT8 tile (BN rows x 64 B) -> fp16 swizzled operand (BN rows x 128 B)
@@ -492,7 +486,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap mA, const __grid_constant__ C
       const int n0 = (tile % p.n_blocks) * BN;
       for (int kb = 0; kb < KB; ++kb) {
         const int s = it % STAGES;
-        if (!mbar_wait(&full[s], (it / STAGES) & 1, abort_flag)) {
+        if (!mbar_wait(&full[s], (it / STAGES) & 1, abort_flag, p.wait_ns)) {
           ok = false;
           break;
         }
@@ -525,7 +519,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap mA, const __grid_constant__ C
     for (int tile = blockIdx.x; tile < p.tiles; tile += gridDim.x, ++local) {
       const int acc = local & 1;
       const uint32_t use = (uint32_t)(local >> 1);
-      if (!mbar_wait(&tfull[acc], use & 1, abort_flag)) break;
+      if (!mbar_wait(&tfull[acc], use & 1, abort_flag, p.wait_ns)) break;
       tc_fence_after();
       const int nb = tile % p.n_blocks, mb = tile / p.n_blocks;
       const int r = mb * BM + q * 32 + lane;
@@ -684,7 +678,7 @@ gemm_tc_pair_kernel(const __grid_constant__ CUtensorMap mA, const __grid_constan
         const CUtensorMap* ma = (n0 >= p.n_split) ? &mA2 : &mA;
         for (int kb = 0; kb < KB; ++kb) {
           const int s = it % STAGES;
-          if (!mbar_wait(&empty[s], ((it / STAGES) & 1) ^ 1, abort_flag)) {
+          if (!mbar_wait(&empty[s], ((it / STAGES) & 1) ^ 1, abort_flag, p.wait_ns)) {
             ok = false;
             break;
           }
@@ -705,14 +699,7 @@ gemm_tc_pair_kernel(const __grid_constant__ CUtensorMap mA, const __grid_constan
       // the pair has landed before either CTA passes the final cluster barrier
       if (leader) {
         const int first = it > STAGES ? it - STAGES : 0;
-        for (int j = first; j < it; ++j) {
-          const uint64_t t0 = globaltimer_ns();
-          while (!mbar_try_wait(&full[j % STAGES], (j / STAGES) & 1))
-            if (globaltimer_ns() - t0 > kWaitLimitNs) {
-              *abort_flag = 1;
-              break;
-            }
-        }
+        for (int j = first; j < it; ++j) mbar_settle(&full[j % STAGES], (j / STAGES) & 1, abort_flag, p.wait_ns);
       }
     }
   } else if (warp == 1) {
@@ -723,12 +710,12 @@ gemm_tc_pair_kernel(const __grid_constant__ CUtensorMap mA, const __grid_constan
       for (int tile = pair; tile < p.tiles && ok; tile += npairs, ++local) {
         const int acc = local & 1;
         const uint32_t use = (uint32_t)(local >> 1);
-        if (!mbar_wait(&tempty[acc], (use & 1) ^ 1, abort_flag)) break;
+        if (!mbar_wait(&tempty[acc], (use & 1) ^ 1, abort_flag, p.wait_ns)) break;
         tc_fence_after();
         const uint32_t d = tmem + (uint32_t)(acc * BN);
         for (int kb = 0; kb < KB; ++kb) {
           const int s = it % STAGES;
-          if (!mbar_wait(&full[s], (it / STAGES) & 1, abort_flag)) {
+          if (!mbar_wait(&full[s], (it / STAGES) & 1, abort_flag, p.wait_ns)) {
             ok = false;
             break;
           }
@@ -744,12 +731,7 @@ gemm_tc_pair_kernel(const __grid_constant__ CUtensorMap mA, const __grid_constan
         if (ok) umma_commit_pair(&tfull[acc]);
       }
       umma_commit_pair_local(drain);
-      const uint64_t t0 = globaltimer_ns();
-      while (!mbar_try_wait(drain, 0))
-        if (globaltimer_ns() - t0 > kWaitLimitNs) {
-          *abort_flag = 1;
-          break;
-        }
+      mbar_settle(drain, 0, abort_flag, p.wait_ns);
     }
   } else {
     const int q = warp & 3, half = (warp - 2) / 4;
@@ -759,7 +741,7 @@ gemm_tc_pair_kernel(const __grid_constant__ CUtensorMap mA, const __grid_constan
     for (int tile = pair; tile < p.tiles; tile += npairs, ++local) {
       const int acc = local & 1;
       const uint32_t use = (uint32_t)(local >> 1);
-      if (!mbar_wait(&tfull[acc], use & 1, abort_flag)) break;
+      if (!mbar_wait(&tfull[acc], use & 1, abort_flag, p.wait_ns)) break;
       tc_fence_after();
       const int nb = tile % p.n_blocks, mb = tile / p.n_blocks;
       const int r = mb * 256 + (int)rank * 128 + q * 32 + lane;
@@ -1033,6 +1015,10 @@ cudaError_t launch_gemm_tc(TcGemmCache* cache, const void* A, const void* A2, in
   args.ep = ep;
   args.scale_t = B.scale_t;
   args.status = cache->status;
+  args.wait_ns = cache->debug_limit_ns ? cache->debug_limit_ns : kWaitLimitNs;
+  args.debug_skip = pair ? -1 : cache->debug_skip;
+  cache->debug_limit_ns = 0;  // the hook applies to one launch
+  cache->debug_skip = -1;
   // residual epilogue: fp32 map over x [M, N] (row stride ldo) for the TMA reduction
   CUtensorMap mX = mB;
   if (epi == EPI_RESID) {

@@ -13,6 +13,12 @@ struct TcGemmCache {
   // fp16 GEMM tiles: 0 single-CTA only, 1 single- or paired-CTA (cta_group::2)
   // tiles, whichever is cheaper, 2 paired-CTA tiles wherever one applies
   int pair_mode = 1;
+  // Test hook, consumed by the next tensor-core GEMM launch: its bounded waits
+  // give up after debug_limit_ns, and (single-CTA tiles) its producer never
+  // issues the loads of the debug_skip-th k-block it handles, so the wait for
+  // that stage runs out.  -1 / 0: off.
+  int debug_skip = -1;
+  uint64_t debug_limit_ns = 0;
 };
 
 // Resolves the driver's tensor-map encoder and allocates the status word.

@@ -363,6 +363,12 @@ __global__ void scatter_kernel(const float* __restrict__ x, Clips clips, float* 
   }
 }
 
+// a ranks strictly above b in argmax order (NaN above everything, as in numpy)
+__device__ __forceinline__ bool ranks_above(float a, float b) {
+  if (isnan(b)) return false;
+  return isnan(a) || a > b;
+}
+
 __global__ void logsoftmax_argmax_kernel(const float* __restrict__ logits, int ld, const int* __restrict__ lens,
                                          int batch, int t_max, int C, float* __restrict__ logp,
                                          int* __restrict__ argmax, const int* __restrict__ off) {
@@ -378,17 +384,22 @@ __global__ void logsoftmax_argmax_kernel(const float* __restrict__ logits, int l
     return;
   }
   const float* z = logits + (size_t)(off ? __ldg(off + b) + t : row) * ld;
+  // First index of the maximum in the order of numpy's argmax: a NaN ranks above
+  // every number (the first NaN wins) and a row of equal values, -inf included,
+  // gives its first index.  A lane's own scan runs in increasing c and takes its
+  // first element unconditionally; lanes without elements keep bi = INT_MAX.
   float best = -INFINITY;
   int bi = 0x7fffffff;
   for (int c = lane; c < C; c += 32) {
     const float v = z[c];
-    if (v > best) { best = v; bi = c; }  // lane-local scan is in increasing c: keeps the first maximum
+    if (bi == 0x7fffffff || ranks_above(v, best)) { best = v; bi = c; }
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) {
     const float ob = __shfl_xor_sync(0xffffffffu, best, o);
     const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
-    if (ob > best || (ob == best && oi < bi)) { best = ob; bi = oi; }
+    const bool same = (ob == best) || (isnan(ob) && isnan(best));
+    if (oi != 0x7fffffff && (bi == 0x7fffffff || ranks_above(ob, best) || (same && oi < bi))) { best = ob; bi = oi; }
   }
   float s = 0.f;
   for (int c = lane; c < C; c += 32) s += expf(z[c] - best);

@@ -85,12 +85,16 @@ constexpr int kRing = 8;
 // kernel sequence depends on besides buffer contents: the entry point, the
 // clip lengths (hence the plan and every launch shape) and the caller's
 // pointers.  The first call with a key runs eagerly; the second is captured
-// (on a private stream) into a graph together with a private device copy of
-// its clip table, and every later call replays it with one cudaGraphLaunch.
+// (on a private stream) into a graph that reads the call's clip table from one
+// of kGraphCap table slots preallocated with the context, and every later call
+// replays it with one cudaGraphLaunch.  A slot's table is uploaded with an
+// asynchronous copy on the caller's stream (from the pinned ring), after the
+// last replay of the slot's previous graph (an event recorded at each launch),
+// so capture and eviction neither allocate nor synchronise.
 struct GraphEntry {
   std::vector<int64_t> key;
   cudaGraphExec_t exec = nullptr;
-  int* table = nullptr;  // device: the call's table, read by the captured kernels
+  int slot = -1;         // table slot: the captured kernels read c->graph_tables + slot * stride
   uint64_t used = 0;
 };
 struct GraphCache {
@@ -151,6 +155,11 @@ struct gam_ctx {
   int* tab_dev[kRing] = {};
   cudaEvent_t tab_ev[kRing] = {};
   int ring = 0;
+  size_t tab_ints = 0;  // ints per table (ring entries and graph slots)
+  // graph table slots [kGraphCap][tab_ints] and, per slot, an event recorded after
+  // every launch of the graph that reads it
+  int* graph_tables = nullptr;
+  cudaEvent_t graph_ev[kGraphCap] = {};
   cudaStream_t last_stream = nullptr;
   // tcgen05 GEMM plans
   TcGemmCache tc;
@@ -480,29 +489,58 @@ bool graph_second_sighting(gam_ctx* c, const std::vector<int64_t>& key) {
   return false;
 }
 
+// An executable graph still in flight is freed by the driver when it completes.
 void graph_free(GraphEntry& e) {
   if (e.exec) cudaGraphExecDestroy(e.exec);
-  if (e.table) cudaFree(e.table);  // synchronises the device: no replay still reads it
   e.exec = nullptr;
-  e.table = nullptr;
 }
 
-// Capture body(device table, capture stream) into a graph for key, with a private
-// device copy of table_host (n ints).  On success *out is the new cache entry.
+// Replay a cached graph on stream s and mark its table slot as in use until then.
+gam_status graph_launch(gam_ctx* c, GraphEntry* e, cudaStream_t s) {
+  GAM_TRY(cuda_check(c, cudaGraphLaunch(e->exec, s), "graph launch"));
+  return cuda_check(c, cudaEventRecord(c->graph_ev[e->slot], s), "graph event");
+}
+
+// Capture body(device table, capture stream) into a graph for key.  The graph
+// reads the call's table (table_host, n ints) from a preallocated slot: a free
+// one, else the least recently used entry's (that entry is dropped).  The table
+// is copied into the slot on stream s once the slot's last replay is done, so the
+// graph's first launch on s sees it.  On success *out is the new cache entry.
 template <class F>
 gam_status graph_capture(gam_ctx* c, const std::vector<int64_t>& key, const int* table_host, int n, F&& body,
-                         GraphEntry** out) {
+                         cudaStream_t s, GraphEntry** out) {
   GraphCache& gc = c->graphs;
-  if (!gc.cap) GAM_TRY(cuda_check(c, cudaStreamCreateWithFlags(&gc.cap, cudaStreamNonBlocking), "capture stream"));
+  if ((size_t)n > c->tab_ints) return fail(c, GAM_ERR_CAPACITY, "clip table larger than its graph slot");
+  int slot = -1;
+  if (gc.entries.size() < kGraphCap) {
+    std::vector<bool> used(kGraphCap, false);
+    for (const GraphEntry& e : gc.entries) used[e.slot] = true;
+    for (size_t i = 0; i < kGraphCap && slot < 0; ++i)
+      if (!used[i]) slot = (int)i;
+  } else {
+    auto lru = std::min_element(gc.entries.begin(), gc.entries.end(),
+                                [](const GraphEntry& a, const GraphEntry& b) { return a.used < b.used; });
+    slot = lru->slot;
+    graph_free(*lru);
+    gc.entries.erase(lru);
+  }
+  int* table = c->graph_tables + (size_t)slot * c->tab_ints;
+  // the pinned ring entry holds the table until the copy has run
+  const int r = c->ring;
+  c->ring = (c->ring + 1) % kRing;
+  GAM_TRY(cuda_check(c, cudaEventSynchronize(c->tab_ev[r]), "ring event"));
+  std::memcpy(c->tab_host[r], table_host, (size_t)n * sizeof(int));
+  GAM_TRY(cuda_check(c, cudaStreamWaitEvent(s, c->graph_ev[slot], 0), "slot wait"));
+  GAM_TRY(cuda_check(c, cudaMemcpyAsync(table, c->tab_host[r], (size_t)n * sizeof(int), cudaMemcpyHostToDevice, s),
+                     "graph table upload"));
+  GAM_TRY(cuda_check(c, cudaEventRecord(c->tab_ev[r], s), "ring event record"));
   GraphEntry e;
   e.key = key;
-  GAM_TRY(cuda_check(c, cudaMalloc((void**)&e.table, (size_t)n * sizeof(int)), "graph table"));
-  gam_status st = cuda_check(c, cudaMemcpy(e.table, table_host, (size_t)n * sizeof(int), cudaMemcpyHostToDevice),
-                             "graph table upload");
+  e.slot = slot;
   cudaGraph_t g = nullptr;
-  if (st == GAM_OK) st = cuda_check(c, cudaStreamBeginCapture(gc.cap, cudaStreamCaptureModeThreadLocal), "capture");
+  gam_status st = cuda_check(c, cudaStreamBeginCapture(gc.cap, cudaStreamCaptureModeThreadLocal), "capture");
   if (st == GAM_OK) {
-    st = body(e.table, gc.cap);
+    st = body(table, gc.cap);
     const gam_status end = cuda_check(c, cudaStreamEndCapture(gc.cap, &g), "end capture");
     if (st == GAM_OK) st = end;
   }
@@ -511,12 +549,6 @@ gam_status graph_capture(gam_ctx* c, const std::vector<int64_t>& key, const int*
   if (st != GAM_OK) {
     graph_free(e);
     return st;
-  }
-  if (gc.entries.size() >= kGraphCap) {
-    auto lru = std::min_element(gc.entries.begin(), gc.entries.end(),
-                                [](const GraphEntry& a, const GraphEntry& b) { return a.used < b.used; });
-    graph_free(*lru);
-    gc.entries.erase(lru);
   }
   e.used = ++gc.tick;
   gc.entries.push_back(e);
@@ -582,9 +614,9 @@ gam_status run_encoder(gam_ctx* c, const float* audio, const int32_t* lengths, i
       fill_table(p, tab.data());
       GAM_TRY(graph_capture(c, key, tab.data(), (int)tab.size(), [&](const int* t, cudaStream_t cs) {
         return encoder_kernels(c, p, Clips{t, batch}, audio, max_samples, stop_layer, stop_stage, out, cs);
-      }, &e));
+      }, s, &e));
     }
-    if (e) return cuda_check(c, cudaGraphLaunch(e->exec, s), "graph launch");
+    if (e) return graph_launch(c, e, s);
   }
   Clips clips;
   GAM_TRY(upload_table(c, p, s, &clips));
@@ -701,9 +733,9 @@ gam_status run_ctc(gam_ctx* c, const float* enc, const int32_t* enc_len, int bat
     if (!e && graph_second_sighting(c, key)) {
       GAM_TRY(graph_capture(c, key, lo.data(), (int)lo.size(), [&](const int* t, cudaStream_t cs) {
         return ctc_kernels(c, enc, t, batch, t_max, lo[2 * batch], logp, tokens, counts, cs);
-      }, &e));
+      }, s, &e));
     }
-    if (e) return cuda_check(c, cudaGraphLaunch(e->exec, s), "graph launch");
+    if (e) return graph_launch(c, e, s);
   }
   const int* dev;
   GAM_TRY(upload_ints(c, lo.data(), 2 * batch + 1, s, &dev));
@@ -968,11 +1000,17 @@ gam_status alloc_workspace(gam_ctx* c) {
   GAM_TRY(cuda_check(c, cudaMemset(c->vt, 0, (size_t)H * 64 * E * es), "memset"));
   GAM_TRY(cuda_check(c, cudaMemset(c->dev_status, 0, 16), "memset"));
   const size_t tab_ints = 5 * (size_t)(cfg.max_batch + 1) + 16;  // also >= 2 * max_batch + 1
+  c->tab_ints = tab_ints;
   for (int i = 0; i < kRing; ++i) {
     GAM_TRY(cuda_check(c, cudaMallocHost((void**)&c->tab_host[i], tab_ints * 4), "cudaMallocHost"));
     GAM_TRY(dev_alloc(c, (void**)&c->tab_dev[i], tab_ints * 4));
     GAM_TRY(cuda_check(c, cudaEventCreateWithFlags(&c->tab_ev[i], cudaEventDisableTiming), "event"));
   }
+  // CUDA-graph table slots, their events and the private capture stream
+  GAM_TRY(dev_alloc(c, (void**)&c->graph_tables, kGraphCap * tab_ints * 4));
+  for (size_t i = 0; i < kGraphCap; ++i)
+    GAM_TRY(cuda_check(c, cudaEventCreateWithFlags(&c->graph_ev[i], cudaEventDisableTiming), "event"));
+  GAM_TRY(cuda_check(c, cudaStreamCreateWithFlags(&c->graphs.cap, cudaStreamNonBlocking), "capture stream"));
   c->prof.ev.resize(2 * 16384);
   c->prof.pair_kind.assign(16384, -1);
   for (auto& e : c->prof.ev) GAM_TRY(cuda_check(c, cudaEventCreate(&e), "event"));
@@ -992,6 +1030,8 @@ void destroy(gam_ctx* c) {
   for (auto& e : c->prof.ev)
     if (e) cudaEventDestroy(e);
   for (GraphEntry& e : c->graphs.entries) graph_free(e);
+  for (size_t i = 0; i < kGraphCap; ++i)
+    if (c->graph_ev[i]) cudaEventDestroy(c->graph_ev[i]);
   if (c->graphs.cap) cudaStreamDestroy(c->graphs.cap);
   delete c;
 }
@@ -1259,6 +1299,14 @@ gam_status gam_debug_gemm(gam_ctx* c, int impl, const void* a, int lda, const vo
   }
   if (k % 16 || n % 128) return fail(c, GAM_ERR_SHAPE, "CUDA-core GEMM needs N % 128 == 0, K % 16 == 0");
   return run_kernel(c, PK_MISC, s, [&] { return launch_gemm_simt(1, a, nullptr, 0, lda, W, m, n, k, EPI_RESID, 0, ep, s); });
+}
+
+gam_status gam_debug_wait_timeout(gam_ctx* c, int64_t limit_ns, int skip_k_block) {
+  GAM_TRY(enter(c));
+  if (limit_ns <= 0) return fail(c, GAM_ERR_INVALID_ARG, "limit_ns must be positive");
+  c->tc.debug_limit_ns = (uint64_t)limit_ns;
+  c->tc.debug_skip = skip_k_block >= 0 ? skip_k_block : -1;
+  return GAM_OK;
 }
 
 gam_status gam_debug_inject_cuda_error(gam_ctx* c, int cuda_error, int count) {

@@ -49,18 +49,31 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
   return t;
 }
 // Wait for the phase of parity `parity` to complete.  Returns false if the
-// CTA's abort flag is up or the wait ran past kWaitLimitNs (then raises it).
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
+// CTA's abort flag is up or the wait ran past limit_ns (then raises it).
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                          uint64_t limit_ns = kWaitLimitNs) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
     if (*abort_flag) return false;
-    if (globaltimer_ns() - t0 > kWaitLimitNs) {
+    if (globaltimer_ns() - t0 > limit_ns) {
       *abort_flag = 1;
       return false;
     }
   }
+}
+// Wait for a phase without watching the abort flag (draining copies or MMAs that
+// are already in flight before the CTA exits); gives up after limit_ns and then
+// raises the abort flag.
+__device__ __forceinline__ void mbar_settle(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                            uint64_t limit_ns) {
+  const uint64_t t0 = globaltimer_ns();
+  while (!mbar_try_wait(bar, parity))
+    if (globaltimer_ns() - t0 > limit_ns) {
+      *abort_flag = 1;
+      return;
+    }
 }
 
 // 2D tiled TMA load into shared memory, completion counted on `bar`.

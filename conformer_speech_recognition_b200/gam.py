@@ -29,7 +29,7 @@ EXPORTS = ("gam_status_string", "gam_last_error", "gam_plan_lengths", "gam_creat
            "gam_encode", "gam_encode_stage", "gam_ctc_greedy", "gam_ctc_collapse", "gam_transcribe",
            "gam_device_status", "gam_profile_enable", "gam_profile_reset", "gam_profile_kinds",
            "gam_profile_kind_name", "gam_profile_read", "gam_graphs_enable", "gam_ctc_collapse_noalloc",
-           "gam_debug_gemm", "gam_debug_inject_cuda_error")
+           "gam_debug_gemm", "gam_debug_wait_timeout", "gam_debug_inject_cuda_error")
 
 GAM_NOALLOC_MAX_FRAMES = 1 << 20
 
@@ -92,6 +92,7 @@ def lib() -> ctypes.CDLL:
         L.gam_ctc_collapse_noalloc.argtypes = [vp, vp, ctypes.c_int, ctypes.c_int, ctypes.c_int, vp, vp, vp]
         L.gam_debug_gemm.argtypes = [vp, ctypes.c_int, vp, ctypes.c_int, vp, vp, ctypes.c_int, ctypes.c_int,
                                      ctypes.c_int, vp, ctypes.c_int, vp]
+        L.gam_debug_wait_timeout.argtypes = [vp, ctypes.c_int64, ctypes.c_int]
         L.gam_debug_inject_cuda_error.argtypes = [vp, ctypes.c_int, ctypes.c_int]
         for name in EXPORTS:
             if name not in ("gam_status_string", "gam_last_error", "gam_profile_kind_name"):
@@ -112,6 +113,21 @@ def _i32(a) -> np.ndarray:
 
 def _ptr_i32(a: np.ndarray):
     return a.ctypes.data_as(ctypes.POINTER(ctypes.c_int32))
+
+
+def _dev_tensor(t, dtype, name: str, device=None):
+    """Check that t is a contiguous CUDA tensor of `dtype` (on `device` if given):
+    the C ABI reads it as a packed array through its data pointer."""
+    import torch
+    if not isinstance(t, torch.Tensor) or t.device.type != "cuda":
+        raise GamError(1, f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise GamError(1, f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise GamError(1, f"{name} must be contiguous")
+    if device is not None and t.device != device:
+        raise GamError(1, f"{name} is on {t.device}, expected {device}")
+    return t
 
 
 def _stream(stream) -> Optional[int]:
@@ -207,9 +223,11 @@ def gam_logmel(ctx: Context, audio, lengths, out=None, stream=None):
     import torch
     ln = _i32(lengths)
     _, _, fmax, _ = gam_plan_lengths(ctx.cfg, ln)
+    _dev_tensor(audio, torch.float32, "audio")
     B, nmax = audio.shape
     if out is None:
         out = torch.empty((B, fmax, ctx.cfg["n_mels"]), dtype=torch.float32, device=audio.device)
+    _dev_tensor(out, torch.float32, "out", audio.device)
     frames = np.zeros(B, np.int32)
     _check(lib().gam_logmel(ctx.handle, audio.data_ptr(), _ptr_i32(ln), B, nmax, out.data_ptr(), _ptr_i32(frames),
                             _stream(stream)), ctx)
@@ -220,9 +238,11 @@ def gam_encode(ctx: Context, audio, lengths, out=None, stream=None):
     import torch
     ln = _i32(lengths)
     _, _, _, tmax = gam_plan_lengths(ctx.cfg, ln)
+    _dev_tensor(audio, torch.float32, "audio")
     B, nmax = audio.shape
     if out is None:
         out = torch.empty((B, tmax, ctx.cfg["d_model"]), dtype=torch.float32, device=audio.device)
+    _dev_tensor(out, torch.float32, "out", audio.device)
     enc_len = np.zeros(B, np.int32)
     _check(lib().gam_encode(ctx.handle, audio.data_ptr(), _ptr_i32(ln), B, nmax, out.data_ptr(), _ptr_i32(enc_len),
                             _stream(stream)), ctx)
@@ -233,9 +253,11 @@ def gam_encode_stage(ctx: Context, audio, lengths, layer: int, stage: int, out=N
     import torch
     ln = _i32(lengths)
     _, _, _, tmax = gam_plan_lengths(ctx.cfg, ln)
+    _dev_tensor(audio, torch.float32, "audio")
     B, nmax = audio.shape
     if out is None:
         out = torch.empty((B, tmax, ctx.cfg["d_model"]), dtype=torch.float32, device=audio.device)
+    _dev_tensor(out, torch.float32, "out", audio.device)
     _check(lib().gam_encode_stage(ctx.handle, audio.data_ptr(), _ptr_i32(ln), B, nmax, layer, stage, out.data_ptr(),
                                   _stream(stream)), ctx)
     return out
@@ -247,6 +269,7 @@ def gam_ctc_greedy(ctx: Context, enc, enc_len, want_logp: bool = False, stream=N
     (preallocated CUDA tensors, so repeated calls keep their pointers)."""
     import torch
     el = _i32(enc_len)
+    _dev_tensor(enc, torch.float32, "enc")
     B, tmax, _ = enc.shape
     C = ctx.cfg["n_classes"]
     if tokens is None:
@@ -255,6 +278,10 @@ def gam_ctc_greedy(ctx: Context, enc, enc_len, want_logp: bool = False, stream=N
         counts = torch.empty((B,), dtype=torch.int32, device=enc.device)
     if logp is None and want_logp:
         logp = torch.empty((B, tmax, C), dtype=torch.float32, device=enc.device)
+    _dev_tensor(tokens, torch.int32, "tokens", enc.device)
+    _dev_tensor(counts, torch.int32, "counts", enc.device)
+    if logp is not None:
+        _dev_tensor(logp, torch.float32, "logp", enc.device)
     _check(lib().gam_ctc_greedy(ctx.handle, enc.data_ptr(), _ptr_i32(el), B, tmax,
                                 logp.data_ptr() if logp is not None else None, tokens.data_ptr(), counts.data_ptr(),
                                 _stream(stream)), ctx)
@@ -264,6 +291,7 @@ def gam_ctc_greedy(ctx: Context, enc, enc_len, want_logp: bool = False, stream=N
 def gam_ctc_collapse(ctx: Context, logits, lengths, stream=None):
     import torch
     ln = _i32(lengths)
+    _dev_tensor(logits, torch.float32, "logits")
     B, tmax, C = logits.shape
     tokens = torch.empty((B, tmax), dtype=torch.int32, device=logits.device)
     counts = torch.empty((B,), dtype=torch.int32, device=logits.device)
@@ -332,7 +360,14 @@ def gam_ctc_collapse_noalloc(logits, lengths_dev, tokens, counts, stream=None):
     logits: CUDA f32 [B, T, C]; lengths_dev: CUDA int32 [B]; tokens (CUDA int32
     [B, T]) and counts (CUDA int32 [B]) are written.  The caller allocates all
     four; the library keeps its per-frame scratch in a fixed device array."""
+    import torch
+    _dev_tensor(logits, torch.float32, "logits")
+    for t, dt, n in ((lengths_dev, torch.int32, "lengths_dev"), (tokens, torch.int32, "tokens"),
+                     (counts, torch.int32, "counts")):
+        _dev_tensor(t, dt, n, logits.device)
     B, T, C = logits.shape
+    if tuple(lengths_dev.shape) != (B,) or tuple(tokens.shape) != (B, T) or tuple(counts.shape) != (B,):
+        raise GamError(1, "lengths_dev [B], tokens [B, T] and counts [B] must match logits [B, T, C]")
     _check(lib().gam_ctc_collapse_noalloc(logits.data_ptr(), lengths_dev.data_ptr(), B, T, C, tokens.data_ptr(),
                                           counts.data_ptr(), _stream(stream)))
     return tokens, counts
@@ -350,6 +385,12 @@ def gam_debug_gemm(ctx: Context, impl: int, a, w, bias, out, stream=None):
     _check(lib().gam_debug_gemm(ctx.handle, impl, a.data_ptr(), a.stride(0), w.data_ptr(), bias.data_ptr(), M, N, K,
                                 out.data_ptr(), out.stride(0), _stream(stream)), ctx)
     return out
+
+
+def gam_debug_wait_timeout(ctx: Context, limit_ns: int, skip_k_block: int = -1):
+    """The next tensor-core GEMM's waits give up after limit_ns; with
+    skip_k_block >= 0 its producer leaves that k-block's stage empty."""
+    _check(lib().gam_debug_wait_timeout(ctx.handle, int(limit_ns), int(skip_k_block)), ctx)
 
 
 def gam_debug_inject_cuda_error(ctx: Context, cuda_error: int, count: int = 1):

@@ -21,10 +21,15 @@
  *   on the context's GPU (cudaMalloc, torch, ...); "host pointer" means CPU
  *   memory.  `stream` is a cudaStream_t passed as void* (NULL = legacy
  *   default stream).  All GPU work of a call is enqueued on that stream; no
- *   call synchronises it except gam_transcribe and gam_device_status.
+ *   call synchronises it except gam_transcribe, gam_device_status and the
+ *   profiling calls (gam_profile_reset / gam_profile_read).
  * - The caller owns every buffer it passes.  A context owns its weights and
- *   one workspace sized at creation for (max_batch, max_samples); calls do no
- *   device allocation.  One context serves one stream at a time.
+ *   one workspace sized at creation for (max_batch, max_samples); calls after
+ *   gam_create do no device allocation (CUDA-graph replay included, see
+ *   gam_graphs_enable).  Small per-call tables go to the device through a
+ *   ring of 8 pinned host buffers; a call waits on the host only if the copy
+ *   made 8 calls earlier has not run yet.  One context serves one stream at a
+ *   time.
  * - Errors are returned, never thrown and never abort the process.  Arguments
  *   are checked before any launch.  An asynchronous device error shows up as
  *   GAM_ERR_CUDA on a later call.  Device-side waits are bounded; a wait that
@@ -116,14 +121,22 @@ const char* gam_status_string(gam_status status);
  * (gam_create, gam_plan_lengths, gam_ctc_collapse_noalloc). */
 const char* gam_last_error(const gam_ctx* ctx);
 
-/* Host-only length planning for `batch` clips of `lengths_host[i]` samples.
+/* Lengths of the frontend and subsampling ("GigaAM v3 MLX", "Frontend
+ * configuration": window 320, hop 160, center false; "Validation" prints a
+ * 1 s clip as [64, 99] features and [1, 768, 25] encoder output).
+ * Host-only length planning for `batch` clips of `lengths_host[i]` samples.
  * Writes (each optional, may be NULL) frames_out[i] = F_i, enc_len_out[i] =
  * L'_i, and dims_out[0..1] = (F_max, T'_max), the padded sizes of the mel and
  * encoder outputs.  Fails with GAM_ERR_SHAPE for a clip shorter than 1280. */
 gam_status gam_plan_lengths(const gam_config* cfg, const int32_t* lengths_host, int batch,
                             int32_t* frames_out, int32_t* enc_len_out, int32_t* dims_out);
 
-/* Build a context on CUDA device `device`: checks the device (sm_100),
+/* Model setup ("GigaAM on MLX: the transcripts matched, but the model was
+ * broken", "Trap 3" (the stored window and filterbank are inputs) and "Trap 4"
+ * (PyTorch weight layouts, fp16 checkpoints); "GigaAM v3 MLX",
+ * "Architecture details"; "GigaAM MLX port for Mac", "How precision affects
+ * size and speed" (one scale per group of 64 weights).
+ * Build a context on CUDA device `device`: checks the device (sm_100),
  * validates every tensor the config needs by name/shape/dtype, repacks the
  * weights (fold the window into a DFT basis, fold BatchNorm into the depthwise
  * conv, reorder GLU halves, transpose conv weights, quantised layouts), and
@@ -157,7 +170,12 @@ gam_status gam_destroy(gam_ctx* ctx);
 gam_status gam_logmel(gam_ctx* ctx, const float* audio_dev, const int32_t* lengths_host, int batch,
                       int64_t max_samples, float* mel_dev, int32_t* frames_host_out, void* stream);
 
-/* Frontend + subsampling + all Conformer blocks.  enc_dev: device f32
+/* The encoder ("GigaAM v3 MLX", "Runtime pipeline" and "Architecture
+ * details"; the Russian original of "GigaAM MLX port for Mac", pipeline list
+ * under "What is inside the model": log-mel -> two Conv1d layers -> Conformer
+ * blocks of FFN, attention, convolution, FFN; RoPE per "GigaAM on MLX ...",
+ * "Trap 1" and "Trap 2").
+ * Frontend + subsampling + all Conformer blocks.  enc_dev: device f32
  * [batch, T'_max, d]; frames at or beyond L'_i are zero.  enc_len_host_out
  * (optional): L'_i. */
 gam_status gam_encode(gam_ctx* ctx, const float* audio_dev, const int32_t* lengths_host, int batch,
@@ -169,17 +187,26 @@ gam_status gam_encode(gam_ctx* ctx, const float* audio_dev, const int32_t* lengt
 gam_status gam_encode_stage(gam_ctx* ctx, const float* audio_dev, const int32_t* lengths_host, int batch,
                             int64_t max_samples, int layer, int stage, float* out_dev, void* stream);
 
-/* CTC head + greedy decoding.  enc_dev: device f32 [batch, t_max, d] with
+/* CTC head + greedy decoding (the Russian original of "GigaAM MLX port for
+ * Mac", pipeline list under "What is inside the model": a CTC layer gives each
+ * symbol's probability per step, decoding removes repeats and blanks; blank =
+ * len(vocabulary) per "GigaAM v3 RNNT -- MLX (Apple Silicon)", "Notes for
+ * other runtimes").
+ * enc_dev: device f32 [batch, t_max, d] with
  * clip i valid on its first enc_len_host[i] <= t_max frames.  logp_dev
  * (optional, device f32 [batch, t_max, n_classes]): log-softmax of the head's
  * logits, zero beyond a clip.  tokens_dev: device i32 [batch, t_max], the
  * collapsed ids (runs merged, then blanks dropped; argmax = lowest index of
- * the fp32 maximum), -1 after the last token.  counts_dev: device i32 [batch]. */
+ * the fp32 maximum), -1 after the last token.  counts_dev: device i32 [batch].
+ * The argmax follows numpy's order: a NaN logit ranks above every number (the
+ * first NaN wins) and a frame whose logits are all equal, all -inf included,
+ * gives index 0; such frames have NaN log-probabilities. */
 gam_status gam_ctc_greedy(gam_ctx* ctx, const float* enc_dev, const int32_t* enc_len_host, int batch,
                           int t_max, float* logp_dev, int32_t* tokens_dev, int32_t* counts_dev,
                           void* stream);
 
-/* Greedy decoding from given scores (test entry for the collapse kernel):
+/* Greedy decoding from given scores, the decoding step of gam_ctc_greedy on
+ * its own (same passages as gam_ctc_greedy):
  * logits_dev device f32 [batch, t_max, n_classes]; blank = n_classes - 1;
  * outputs as gam_ctc_greedy.  Uses the context's workspace for the per-frame
  * argmax, so batch * t_max must fit its capacity. */
@@ -230,8 +257,10 @@ gam_status gam_profile_read(gam_ctx* ctx, int kind, double* total_ms, int64_t* l
  *   tokens_dev  device i32 [batch, t_max]; counts_dev device i32 [batch]
  * batch * t_max above GAM_NOALLOC_MAX_FRAMES fails with GAM_ERR_CAPACITY
  * before any launch (text in gam_last_error(NULL)).  The first call on a
- * device (that device current) looks up the array's device address once;
- * make that first call before any stream capture.  All calls on a device
+ * device (that device current) looks up the array's device address once and
+ * keeps it with the device's current CUDA context; a call that finds another
+ * context current (after cudaDeviceReset) looks it up again.  Make the first
+ * call on a device before any stream capture.  All calls on a device
  * share the array and each fully rewrites the part it reads, so nothing needs
  * clearing, but calls whose GPU work overlaps (other streams or threads) race
  * on it.  Runs on the current device and on `stream`. */
@@ -243,14 +272,18 @@ gam_status gam_ctc_collapse_noalloc(const float* logits_dev, const int32_t* leng
 /* Repeated calls of gam_encode, gam_encode_stage and gam_ctc_greedy with the
  * same clip lengths and the same buffer pointers replay a CUDA graph of the
  * call's kernel sequence: the first such call runs eagerly, the second is
- * captured (on a private stream, with a private device copy of the call's
- * clip table) and launched on `stream`, later ones are one graph launch.
- * Buffer contents may change between calls; pointers and lengths may not
- * (a different pointer or length is a different graph, up to 16 are kept,
- * least recently used first out).  No graph is used while profiling is
- * enabled (gam_profile_enable) or an error is injected.  On by default; the
- * environment variable GAM_CUDA_GRAPHS=0 (read by gam_create) or on = 0 here
- * turns it off.  Outputs are bit-identical either way. */
+ * captured (on a private stream created with the context) and launched on
+ * `stream`, later ones are one graph launch.  Each graph reads its clip table
+ * from one of 16 device slots allocated by gam_create; the table is copied
+ * into its slot asynchronously on `stream` (after the slot's previous graph
+ * has finished its last replay), so capturing and evicting allocate no device
+ * memory and do not synchronise.  Buffer contents may change between calls;
+ * pointers and lengths may not (a different pointer or length is a different
+ * graph, up to 16 are kept, least recently used first out; the driver frees
+ * an evicted graph once its last replay is done).  No graph is used while
+ * profiling is enabled (gam_profile_enable) or an error is injected.  On by
+ * default; the environment variable GAM_CUDA_GRAPHS=0 (read by gam_create) or
+ * on = 0 here turns it off.  Outputs are bit-identical either way. */
 gam_status gam_graphs_enable(gam_ctx* ctx, int on);
 
 /* ---- kernel unit test (tests) ---- */
@@ -272,6 +305,19 @@ gam_status gam_graphs_enable(gam_ctx* ctx, int on);
  * residual-update epilogue of the encoder (alpha 1). */
 gam_status gam_debug_gemm(gam_ctx* ctx, int impl, const void* a_dev, int lda, const void* w_dev,
                           const float* bias_dev, int m, int n, int k, float* out_dev, int ldo, void* stream);
+
+/* ---- bounded device waits (tests) ---- */
+
+/* Test hook for the bounded waits of the tensor-core GEMM.  Applies to the
+ * next tensor-core GEMM this context launches (gam_debug_gemm with impl kind 2
+ * is the intended one), then switches itself off: that launch's waits give up
+ * after limit_ns nanoseconds (> 0) instead of 2 s, and, when skip_k_block >= 0,
+ * its producer does not issue the loads of its skip_k_block-th k-block, so the
+ * MMA issuer's wait for that stage runs out.  The kernel then drains what is in
+ * flight, frees its tensor memory and returns; gam_device_status reports
+ * GAM_ERR_DEVICE_TIMEOUT until gam_profile_reset, and the context stays usable.
+ * Nothing faults or hangs: every wait involved is bounded. */
+gam_status gam_debug_wait_timeout(gam_ctx* ctx, int64_t limit_ns, int skip_k_block);
 
 /* ---- host-side fault injection (tests) ---- */
 

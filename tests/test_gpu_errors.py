@@ -1,6 +1,8 @@
-"""Failure handling through the C ABI on a GPU context, all made on the host:
-bad arguments, capacity overflow, short clips, missing / misshaped weights and
-an injected CUDA error.  No test here faults, traps or hangs the GPU."""
+"""Failure handling through the C ABI on a GPU context: bad arguments, capacity
+overflow, short clips, missing / misshaped weights and an injected CUDA error
+(all made on the host), and a bounded device wait that runs out (a pipeline
+stage that is never filled; the kernel gives up after 1 ms and returns).  No
+test here faults, traps or hangs the GPU."""
 import numpy as np
 import pytest
 
@@ -62,4 +64,33 @@ def test_injected_cuda_error_then_recovery(ctx_small):
     assert e.value.name == "GAM_ERR_CUDA"
     again, _ = gam.gam_encode(ctx, a, lens)
     assert np.array_equal(again.cpu().numpy(), ref.cpu().numpy())
+    gam.gam_device_status(ctx)
+
+
+def test_bounded_wait_runs_out_and_context_recovers(ctx_small):
+    """One GEMM tile whose second k-block is never loaded: the MMA issuer's wait
+    gives up after 1 ms, the kernel drains and returns, the status word reports
+    the timeout, and the next GEMM on the same context is correct."""
+    import torch
+    cfg, W, ctx = ctx_small
+    gam.gam_device_status(ctx)
+    g = torch.Generator().manual_seed(5)
+    M, N, K = 128, 256, 128
+    a = (torch.randn(M, K, generator=g) * 0.5).half().cuda()
+    w = (torch.randn(N, K, generator=g) * 0.5).half().cuda()
+    bias = torch.randn(N, generator=g).float().cuda()
+    out = torch.zeros(M, N, dtype=torch.float32, device="cuda")
+    gam.gam_debug_wait_timeout(ctx, 1_000_000, 1)
+    gam.gam_debug_gemm(ctx, 2, a, w, bias, out)
+    torch.cuda.synchronize()
+    with pytest.raises(gam.GamError) as e:
+        gam.gam_device_status(ctx)
+    assert e.value.name == "GAM_ERR_DEVICE_TIMEOUT"
+    gam.gam_profile_reset(ctx)          # clears the status word
+    gam.gam_device_status(ctx)
+    out.zero_()
+    gam.gam_debug_gemm(ctx, 2, a, w, bias, out)
+    torch.cuda.synchronize()
+    ref = a.float() @ w.float().T + bias
+    assert torch.allclose(out, ref, rtol=1e-3, atol=1e-3)
     gam.gam_device_status(ctx)

@@ -50,6 +50,9 @@ def _crafted_logits(rng, B, T, C):
             m = z[b, t].max() + 1.0
             z[b, t, 1] = m
             z[b, t, 4] = m  # tie: lowest index (1) must win
+        z[b, 9::23, :] = -np.inf  # all -inf: numpy's argmax gives index 0
+        z[b, 10::29, 3] = np.nan  # a NaN ranks above every number, the first NaN wins
+        z[b, 10::29, 6] = np.nan
     return z
 
 

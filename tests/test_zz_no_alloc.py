@@ -2,10 +2,13 @@
 device memory (no context, scratch in a fixed device array).  Its tokens and
 counts must equal gam_ctc_collapse's on the same logits, exactly (the collapse
 is integer work), on two calls in a row, so that the second call sees the
-scratch the first one left behind.  This file is collected last."""
+scratch the first one left behind; and both must equal the oracle's collapse
+of numpy's argmax of the same logits.  One case runs without creating any
+context.  This file is collected last."""
 import numpy as np
 import pytest
 
+import oracle
 from conformer_speech_recognition_b200 import gam
 from gpu_common import config_and_weights, small_model
 
@@ -19,7 +22,43 @@ def _logits(rng, B, T, C):
     m = z[:, 2::11].max(axis=2) + 1.0
     z[:, 2::11, 1] = m                # exact ties: the lowest index wins
     z[:, 2::11, 2] = m
+    z[:, 4::17, :] = -np.inf          # frames of all -inf: index 0, as numpy's argmax
+    z[:, 6::19, 5 % C] = np.nan       # a NaN ranks above every number
+    z[:, 6::19, 7 % C] = np.nan       # (the first NaN wins)
     return z
+
+
+def _oracle_tokens(z, lens, C):
+    out = []
+    for b in range(z.shape[0]):
+        a = np.argmax(z[b, :lens[b]], axis=1) if lens[b] else np.zeros(0, np.int64)
+        out.append(oracle.greedy_collapse(a, C - 1))
+    return out
+
+
+def _check_against_oracle(tok, cnt, z, lens, C):
+    tok, cnt = tok.cpu().numpy(), cnt.cpu().numpy()
+    for b, ref in enumerate(_oracle_tokens(z, lens, C)):
+        assert cnt[b] == len(ref), b
+        assert tok[b, :cnt[b]].tolist() == ref, b
+        assert np.all(tok[b, cnt[b]:] == -1), b
+
+
+def test_noalloc_without_any_context():
+    """No gam_ctx is created in this test: the call needs none."""
+    import torch
+    rng = np.random.default_rng(7)
+    B, T, C = 4, 200, 34
+    lens = np.array([200, 1, 0, 123], np.int32)
+    z_np = _logits(rng, B, T, C)
+    z = torch.from_numpy(z_np).cuda()
+    lens_dev = torch.from_numpy(lens).cuda()
+    for _ in range(2):
+        tok = torch.full((B, T), 777, dtype=torch.int32, device="cuda")
+        cnt = torch.full((B,), 777, dtype=torch.int32, device="cuda")
+        gam.gam_ctc_collapse_noalloc(z, lens_dev, tok, cnt)
+        torch.cuda.synchronize()
+        _check_against_oracle(tok, cnt, z_np, lens, C)
 
 
 def test_noalloc_matches_collapse_two_calls():
@@ -29,9 +68,12 @@ def test_noalloc_matches_collapse_two_calls():
     rng = np.random.default_rng(2024)
     cases = [(6, 300, 34, [300, 0, 1, 299, 150, 17]), (3, 257, 257, [257, 200, 3])]
     for B, T, C, lens in cases:
-        z = torch.from_numpy(_logits(rng, B, T, C)).cuda()
+        z_np = _logits(rng, B, T, C)
+        z = torch.from_numpy(z_np).cuda()
         lens = np.array(lens, np.int32)
         ref_tok, ref_cnt = gam.gam_ctc_collapse(ctx, z, lens)
+        torch.cuda.synchronize()
+        _check_against_oracle(ref_tok, ref_cnt, z_np, lens, C)
         lens_dev = torch.from_numpy(lens).cuda()
         for _ in range(2):
             tok = torch.full((B, T), 12345, dtype=torch.int32, device="cuda")
@@ -40,6 +82,7 @@ def test_noalloc_matches_collapse_two_calls():
             torch.cuda.synchronize()
             assert torch.equal(cnt, ref_cnt)
             assert torch.equal(tok, ref_tok)
+            _check_against_oracle(tok, cnt, z_np, lens, C)
     ctx.close()
 
 
