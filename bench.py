@@ -34,7 +34,9 @@ from conformer_speech_recognition_b200 import synth  # noqa: E402
 
 METRIC = "audio-sec/sec (×realtime) encoder+CTC at 1 B200; GEMM TFLOP/s vs fp16 peak"
 UNIT = "audio-sec/sec"
-DEFAULT_WORKLOAD = "c2_varlen_b32_d768"
+# The largest configuration that runs on one GPU: 32 x 30 s clips on the 24-layer
+# d1024 encoder (about 30 TFLOP per step).
+DEFAULT_WORKLOAD = "c4_30s_b32_d1024"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
@@ -77,6 +79,54 @@ def fp16_vs_bf16_matmul(device, n=8192, iters=10):
         del a, b
     out["fp16_over_bf16"] = out["fp16_tflops"] / out["bf16_tflops"]
     return out
+
+
+def pick_peak(peaks, clocks):
+    """The measured tensor peak that applies to this run: the burst figure when
+    the SM clock sampled during the timed region sat within 3% of its maximum
+    (no power-cap throttling), else the sustained figure (measured under the
+    power cap).  Returns (peak TFLOP/s, "burst" | "sustained")."""
+    sm, smax = (clocks or {}).get("sm_mhz"), (clocks or {}).get("sm_max_mhz")
+    if sm and smax and sm >= 0.97 * smax:
+        return peaks["bf16_tflops"], "burst"
+    return peaks["bf16_tflops_sustained"], "sustained"
+
+
+# Dense fp16 tensor-core work per SM per clock on sm_100 (4096 FMA), for the
+# nominal peak at the sampled clock reported beside the measured one.
+FP16_FLOP_PER_SM_CLK = 8192
+
+
+def roofline_object(dominant, fl, by, dom_ms, dom_n, steps, peaks, clocks, workload, sms=148):
+    """Roofline of the dominant kernel family over the timed region: algorithmic
+    work per launch / mean launch time, against the measured peak that applies."""
+    avg_launch_ms = dom_ms / max(dom_n, 1)
+    launches_per_step = dom_n / steps
+    if dominant in fl and dominant != "frontend":
+        per_launch = fl[dominant] / launches_per_step
+        achieved = per_launch / (avg_launch_ms / 1e3) / 1e12
+        peak, kind = pick_peak(peaks, clocks)
+        roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
+                "traffic": measured_traffic(workload, dominant), "kernel": dominant,
+                "flop_per_launch": per_launch, "launches_per_step": launches_per_step,
+                "mean_launch_ms": avg_launch_ms,
+                "peak_source": f"{peaks['source']} bf16 dense {kind} (fp16 = bf16 rate on sm_100; "
+                               f"median SM clock {((clocks or {}).get('sm_mhz'))} of max "
+                               f"{((clocks or {}).get('sm_max_mhz'))} MHz)",
+                "frac_vs_burst": achieved / peaks["bf16_tflops"],
+                "frac_vs_sustained": achieved / peaks["bf16_tflops_sustained"]}
+        sm = (clocks or {}).get("sm_mhz")
+        if sm:
+            nominal = FP16_FLOP_PER_SM_CLK * sms * sm * 1e6 / 1e12
+            roof["nominal_fp16_at_sampled_clock_tflops"] = nominal
+            roof["frac_vs_nominal_at_sampled_clock"] = achieved / nominal
+        return roof
+    per_launch = by.get(dominant, 0.0) / max(launches_per_step, 1)
+    achieved = per_launch / (avg_launch_ms / 1e3) / 1e9
+    peak = peaks["hbm_gbs"]
+    return {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+            "traffic": measured_traffic(workload, dominant), "kernel": dominant, "bytes_per_launch": per_launch,
+            "mean_launch_ms": avg_launch_ms, "peak_source": f"{peaks['source']} HBM copy"}
 
 
 def algorithmic_work(cfg, lens):
@@ -133,9 +183,11 @@ def measured_traffic(workload, family):
         return None
 
 
-def time_workload(name, steps=5, warmup=3, weights=None, device=0):
+def time_workload(name, steps=5, warmup=3, weights=None, device=0, peaks=None, clocks=None):
     """×realtime of one workload on this GPU: gam_encode + gam_ctc_greedy with the
-    audio resident, CUDA events over `steps` steps after `warmup` steps."""
+    audio resident, CUDA events over `steps` steps after `warmup` steps (CUDA
+    graphs on).  Then `steps` more steps with the dominant kernel family timed by
+    events around each launch give its roofline object."""
     import torch
     from conformer_speech_recognition_b200 import gam
     cfg = synth.workload_config(name)
@@ -167,8 +219,25 @@ def time_workload(name, steps=5, warmup=3, weights=None, device=0):
         torch.cuda.synchronize(dev)
         ms = t0.elapsed_time(t1) / steps
         audio_s = float(np.sum(lens)) / synth.SAMPLE_RATE
-        return {"value": audio_s / (ms / 1e3), "unit": UNIT, "ms_per_step": ms, "steps": steps, "warmup": warmup,
-                "batch": int(B), "audio_seconds_per_step": audio_s, "precision": cfg["precision"]}
+        out = {"value": audio_s / (ms / 1e3), "unit": UNIT, "ms_per_step": ms, "steps": steps, "warmup": warmup,
+               "batch": int(B), "audio_seconds_per_step": audio_s, "precision": cfg["precision"]}
+        if peaks is not None:
+            gam.gam_profile_enable(ctx, -1)
+            step()
+            torch.cuda.synchronize(dev)
+            warm = gam.gam_profile_all(ctx)
+            dominant = max(warm, key=lambda n: warm[n][0])
+            kinds = {gam.gam_profile_kind_name(k): k for k in range(gam.gam_profile_kinds())}
+            gam.gam_profile_enable(ctx, 1 << kinds[dominant])
+            for _ in range(steps):
+                step()
+            torch.cuda.synchronize(dev)
+            dom_ms, dom_n = gam.gam_profile_read(ctx, kinds[dominant])
+            fl, by, _ = algorithmic_work(cfg, lens)
+            out["roofline"] = roofline_object(dominant, fl, by, dom_ms, dom_n, steps, peaks, clocks, name)
+            out["profile_ms_per_step"] = {k: round(v[0], 4) for k, v in warm.items() if v[1]}
+            gam.gam_profile_enable(ctx, 0)
+        return out
     finally:
         ctx.close()
 
@@ -285,13 +354,15 @@ def run_reference(args, rank, world):
     W = synth.random_weights(cfg, seed=0)
     audio, lens = synth.workload_audio(name)
     order = list(np.argsort(lens))  # shortest clips first keeps every step bounded
+    cap = int(args.ref_seconds * synth.SAMPLE_RATE)
     per_step = []
     audio_s = []
 
     def one(i):
+        n = int(min(lens[i], cap))
         t0 = time.perf_counter()
-        oracle.transcribe_clip(audio[i, :lens[i]], W, cfg, np.float32)
-        return time.perf_counter() - t0, lens[i] / synth.SAMPLE_RATE
+        oracle.transcribe_clip(audio[i, :n], W, cfg, np.float32)
+        return time.perf_counter() - t0, n / synth.SAMPLE_RATE
 
     k = 0
     for _ in range(args.warmup):
@@ -309,7 +380,8 @@ def run_reference(args, rank, world):
         threads = max((p.get("num_threads", 1) for p in threadpool_info()), default=os.cpu_count())
     except Exception:
         threads = os.cpu_count()
-    sample = f"one clip per step (shortest first) of {name}: {total_a:.1f} audio-s over {args.steps} steps"
+    sample = (f"one clip per step (shortest first, cut to at most {args.ref_seconds:g} s) of {name}: "
+              f"{total_a:.1f} audio-s over {args.steps} steps")
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000 * total_t / args.steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
@@ -414,27 +486,13 @@ def run_ours(args, rank, world, local_rank):
         fl, by, _ = algorithmic_work(cfg, lens)
         value = job_throughput(world, audio_seconds, args.steps, elapsed_ms)
         e2e_value = job_throughput(world, audio_seconds, args.steps, e2e_ms)
-        avg_launch_ms = dom_ms / max(dom_n, 1)
-        per_step_launches_dom = dom_n / args.steps
-        if dominant in fl and dominant != "frontend":
-            per_launch = fl[dominant] / per_step_launches_dom
-            achieved = per_launch / (avg_launch_ms / 1e3) / 1e12
-            peak = peaks["bf16_tflops_sustained"]
-            roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                    "frac": achieved / peak, "traffic": measured_traffic(name, dominant), "kernel": dominant,
-                    "peak_source": f"{peaks['source']} bf16 sustained, used for the fp16 kernels "
-                                   "(fp16_peak_check: library fp16 / bf16 matmul rates in this run)"}
-        else:
-            per_launch = by.get(dominant, 0.0) / max(per_step_launches_dom, 1)
-            achieved = per_launch / (avg_launch_ms / 1e3) / 1e9
-            peak = peaks["hbm_gbs"]
-            roof = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
-                    "traffic": measured_traffic(name, dominant), "kernel": dominant,
-                    "peak_source": f"{peaks['source']} HBM copy"}
+        roof = roofline_object(dominant, fl, by, dom_ms, dom_n, args.steps, peaks, clock_info, name)
         peak_check = fp16_vs_bf16_matmul(dev) if world == 1 else None
         gemm_flops = sum(v for k, v in fl.items() if k.startswith("gemm_"))
         # GEMM kernel time per step from the profiled steps (every family timed there)
         gemm_ms = sum(v[0] for k, v in warm.items() if k.startswith("gemm_")) / n_prof
+        gemm_rate = gemm_flops / (gemm_ms / 1e3) / 1e12 if gemm_ms > 0 else None
+        tensor_peak, peak_kind = pick_peak(peaks, clock_info)
         cpu = None
         if not args.no_cpu_baseline and world == 1:
             v, desc, threads = oracle_throughput(name, args.cpu_budget)
@@ -446,7 +504,8 @@ def run_ours(args, rank, world, local_rank):
                 if other == name:
                     continue
                 same_model = synth.workload_config(other) == cfg
-                per_workload[other] = time_workload(other, weights=W if same_model else None, device=local_rank)
+                per_workload[other] = time_workload(other, weights=W if same_model else None, device=local_rank,
+                                                    peaks=peaks, clocks=clock_info)
         h2d = int(B * nmax * 4 + 5 * (B + 1) * 4 + B * 4)
         d2h = int(B * tmax * 4 + B * 4)
         line = {
@@ -456,14 +515,16 @@ def run_ours(args, rank, world, local_rank):
             "config": {"workload": name, "batch": B, "audio_seconds_per_step": audio_seconds,
                        "valid_encoder_frames": int(np.sum(el)), "precision": cfg["precision"],
                        "layers": cfg["n_layers"], "d_model": cfg["d_model"],
-                       "l2": "not flushed: the fp16 weights (442 MB) and activations stream through the 126 MB L2 "
-                             "every step",
+                       "l2": "not flushed: the weights and activations of a step are larger than the 126 MB L2 "
+                             "(fp16 weights alone 442 MB at d768, 1.17 GB at d1024)",
                        "parallelism": f"replicas x{world} (independent batches, no collective on the data path)"},
             "roofline": roof,
             "gemm_tflops_per_step_algorithmic": gemm_flops / 1e12,
-            "gemm_tflops_per_s_of_gemm_time": gemm_flops / (gemm_ms / 1e3) / 1e12 if gemm_ms > 0 else None,
-            "gemm_frac_of_fp16_peak": (gemm_flops / (gemm_ms / 1e3) / 1e12) / peaks["bf16_tflops_sustained"]
-            if gemm_ms > 0 else None,
+            "gemm_tflops_per_s_of_gemm_time": gemm_rate,
+            "gemm_frac_of_fp16_peak": gemm_rate / tensor_peak if gemm_rate else None,
+            "gemm_frac_peak_kind": f"measured bf16 dense {peak_kind} (median SM clock vs max decides)",
+            "gemm_frac_of_library_fp16_this_run": gemm_rate / peak_check["fp16_tflops"]
+            if gemm_rate and peak_check else None,
             "fp16_peak_check": peak_check,
             "cpu_baseline": cpu,
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
@@ -480,13 +541,15 @@ def run_ours(args, rank, world, local_rank):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=30)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(synth.WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-per-workload", action="store_true", help="skip the ×realtime of the other workloads")
     ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle CPU time for cpu_baseline")
+    ap.add_argument("--ref-seconds", type=float, default=6.0,
+                    help="reference arm: each step runs the oracle on one clip cut to at most this many seconds")
     args = ap.parse_args()
     if args.warmup < 3:
         print("warning: at least 3 warm-up steps are required for a valid number", file=sys.stderr)

@@ -83,9 +83,7 @@ enum EpiKind {
   EPI_QKV = 3,       // scatter to Q/K head-major (padded to 64) and V^T
   EPI_CONV1 = 4,     // out_t = relu(acc + b), zero outside conv1 clip rows
   EPI_CONV2 = 5,     // x (fp32) = relu(acc + b), zero outside encoder clip rows
-  EPI_F32 = 6,       // out_f32[r, n] = acc + b[n] (n < n_valid, or N when n_valid == 0)
-  EPI_POWER = 7      // DFT basis rows interleaved in blocks of 64 (cos, sin):
-                     //   out_f32[r, 64j + c] = acc_cos^2 + acc_sin^2 (power spectrum)
+  EPI_F32 = 6        // out_f32[r, n] = acc + b[n] (n < n_valid, or N when n_valid == 0)
 };
 
 struct EpiParams {
@@ -131,14 +129,11 @@ cudaError_t launch_frontend(const float* audio, int64_t audio_stride, Clips clip
                             int f_max, const float* basis, const float* fb, void* out, int out_half,
                             cudaStream_t s);
 
-// Tensor-core frontend of the fp16 modes: fp16 frames of the packed mel rows
-// (zero rows outside clips), then (after the DFT GEMM with EPI_POWER) mel +
-// clipped log from the power spectrum power[rows, ld_power] (first 161 bins).
-cudaError_t launch_frames(const float* audio, int64_t audio_stride, Clips clips, int rows, __half* frames,
-                          cudaStream_t s);
-// fb_range: int pairs (first, last) nonzero filterbank row per mel bin (last < first: none).
-cudaError_t launch_mel_log(const float* power, int ld_power, const float* fb, const int* fb_range, Clips clips,
-                           int rows, void* mel, int out_half, cudaStream_t s);
+// Tensor-core frontend of the fp16 / INT8 modes (frontend_tc.cu), step 1: the
+// clips' samples as packed rows of 160 (row 4 e_i + 6 + g = samples 160 g ..
+// of clip i, g <= F_i), split into tf32 hi and lo parts; zero rows elsewhere.
+cudaError_t launch_audio_split(const float* audio, int64_t audio_stride, Clips clips, int rows, float* hi, float* lo,
+                               cudaStream_t s);
 
 cudaError_t launch_layernorm(const float* x, const float* g, const float* b, float eps, void* u, int u_half,
                              int rows, int d, cudaStream_t s);

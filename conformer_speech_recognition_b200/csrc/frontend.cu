@@ -1,5 +1,7 @@
-// Log-mel frontend ("GigaAM v3 MLX", "Frontend configuration"; "GigaAM v3
-// RNNT -- MLX (Apple Silicon)", "Notes for other runtimes").
+// Log-mel frontend of the fp32 build mode, on CUDA cores ("GigaAM v3 MLX",
+// "Frontend configuration"; "GigaAM v3 RNNT -- MLX (Apple Silicon)", "Notes for
+// other runtimes").  The fp16 / INT8 product modes use the tensor-core frontend
+// of frontend_tc.cu.
 //
 // Per frame f of clip i: x = audio[i, 160 f .. 160 f + 319] (center=false).
 // The stored Hann window is folded into a real-DFT basis built at context
@@ -140,96 +142,7 @@ frontend_kernel(const float* __restrict__ audio, int64_t stride, Clips clips, in
   }
 }
 
-// fp16 frames for the tensor-core DFT: row r of the packed mel rows holds
-// audio[clip, 160 f .. 160 f + 319] (zeros for rows outside every clip).
-template <bool VEC>
-__global__ void __launch_bounds__(256)
-frames_kernel(const float* __restrict__ audio, int64_t stride, Clips clips, int rows, __half* __restrict__ frames) {
-  pdl_launch_dependents();
-  pdl_wait();
-  const int r = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
-  if (r >= rows) return;
-  const int ci = clips.find(r, 4, 6);
-  const int f = r - (4 * clips.e(ci) + 6);
-  const bool valid = f >= 0 && f < clips.F(ci);
-  __half* dst = frames + (size_t)r * NFFT;
-  const float* src = audio + (int64_t)ci * stride + (int64_t)f * HOP;
-  for (int c = lane * 4; c < NFFT; c += 128) {  // 80 float4 per frame
-    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (valid) {
-      if (VEC) v = __ldg(reinterpret_cast<const float4*>(src + c));
-      else v = make_float4(__ldg(src + c), __ldg(src + c + 1), __ldg(src + c + 2), __ldg(src + c + 3));
-    }
-    const __half2 a = __floats2half2_rn(v.x, v.y), b = __floats2half2_rn(v.z, v.w);
-    uint2 w;
-    w.x = *reinterpret_cast<const uint32_t*>(&a);
-    w.y = *reinterpret_cast<const uint32_t*>(&b);
-    *reinterpret_cast<uint2*>(dst + c) = w;
-  }
-}
-
-// mel = power[:, :161] . fb, then log(clip(mel, 1e-9, 1e9)); 32 rows per CTA.
-// fb_range[m] = (first, last) filterbank row with a nonzero weight in column m
-// (found when the context is built): the other rows add exact zeros, so the
-// sum runs over that range only.  The filterbank is read through L1.
-constexpr size_t MEL_SMEM = (size_t)(FT * NBIN) * sizeof(float);
-
-__global__ void __launch_bounds__(256)
-mel_log_kernel(const float* __restrict__ power, int ld, const float* __restrict__ fb, const int2* __restrict__ fb_range,
-               Clips clips, int rows, void* __restrict__ mel, int out_half) {
-  pdl_launch_dependents();
-  pdl_wait();
-  extern __shared__ float dyn[];
-  float (*sp)[NBIN] = reinterpret_cast<float (*)[NBIN]>(dyn);  // [FT][NBIN]
-  __shared__ int s_valid[FT];
-  const int tid = threadIdx.x, row0 = blockIdx.x * FT;
-  if (tid < FT) {
-    const int r = row0 + tid;
-    int ok = 0;
-    if (r < rows) {
-      const int ci = clips.find(r, 4, 6);
-      const int f = r - (4 * clips.e(ci) + 6);
-      ok = f >= 0 && f < clips.F(ci);
-    }
-    s_valid[tid] = ok;
-  }
-  for (int idx = tid; idx < FT * NBIN; idx += 256) {
-    const int j = idx / NBIN, k = idx - j * NBIN;
-    const int r = row0 + j;
-    sp[j][k] = r < rows ? __ldg(power + (size_t)r * ld + k) : 0.f;
-  }
-  __syncthreads();
-  const int m = tid & 63;
-  const int2 kr = __ldg(fb_range + m);
-#pragma unroll
-  for (int j = 0; j < FT / 4; ++j) {
-    const int a = (tid >> 6) + 4 * j;
-    float acc = 0.f;
-    for (int k = kr.x; k <= kr.y; ++k) acc = fmaf(sp[a][k], __ldg(fb + k * NMEL + m), acc);
-    const int r = row0 + a;
-    if (r >= rows) continue;
-    const float v = s_valid[a] ? logf(fminf(fmaxf(acc, 1e-9f), 1e9f)) : 0.f;
-    if (out_half) reinterpret_cast<__half*>(mel)[(size_t)r * NMEL + m] = __float2half_rn(v);
-    else reinterpret_cast<float*>(mel)[(size_t)r * NMEL + m] = v;
-  }
-}
-
 }  // namespace
-
-cudaError_t launch_frames(const float* audio, int64_t audio_stride, Clips clips, int rows, __half* frames,
-                          cudaStream_t s) {
-  if (rows <= 0) return cudaSuccess;
-  const bool vec = audio_stride % 4 == 0 && (reinterpret_cast<uintptr_t>(audio) & 15) == 0;
-  if (vec) return launch_pdl(frames_kernel<true>, (rows + 7) / 8, 256, 0, s, audio, audio_stride, clips, rows, frames);
-  return launch_pdl(frames_kernel<false>, (rows + 7) / 8, 256, 0, s, audio, audio_stride, clips, rows, frames);
-}
-
-cudaError_t launch_mel_log(const float* power, int ld_power, const float* fb, const int* fb_range, Clips clips,
-                           int rows, void* mel, int out_half, cudaStream_t s) {
-  if (rows <= 0) return cudaSuccess;
-  return launch_pdl(mel_log_kernel, (rows + FT - 1) / FT, 256, MEL_SMEM, s, power, ld_power, fb,
-                    reinterpret_cast<const int2*>(fb_range), clips, rows, mel, out_half);
-}
 
 cudaError_t launch_frontend(const float* audio, int64_t audio_stride, Clips clips, int rows, int packed, int f_max,
                             const float* basis, const float* fb, void* out, int out_half, cudaStream_t s) {

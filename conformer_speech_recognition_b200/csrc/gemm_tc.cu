@@ -61,8 +61,8 @@ template <int EPI>
 __host__ __device__ constexpr int epi_smem() { return EPI == EPI_RESID ? kEpiWarps * kStageTile : 0; }
 // Bias of the tile's columns, one 128-float copy per epilogue warp, loaded one
 // tile ahead so the epilogue never waits on it.  Used by the fp16-weight kernels
-// (the INT8 mainloop is bound by its converters, the power epilogue has no bias),
-// and by the residual epilogue only where it costs no pipeline stage.
+// (the INT8 mainloop is bound by its converters), and by the residual epilogue
+// only where it costs no pipeline stage.
 constexpr int kBiasStage = 128 * 4;
 constexpr int kBiasSmem = kEpiWarps * kBiasStage;
 __host__ __device__ constexpr int min8(int n) { return n < 8 ? n : 8; }
@@ -70,19 +70,22 @@ __host__ __device__ constexpr int min8(int n) { return n < 8 ? n : 8; }
 // 1.25 KB of alignment slack and barriers; at most 8 stages.
 template <int EPI>
 __host__ __device__ constexpr int ring_budget() { return 227 * 1024 - 1280 - epi_smem<EPI>(); }
-template <int EPI, bool QB, int STAGE>
+template <int EPI, int QBITS, int STAGE>
 __host__ __device__ constexpr bool staged_bias() {
-  return !QB && EPI != EPI_POWER &&
+  return QBITS == 0 &&
          (EPI != EPI_RESID || min8((ring_budget<EPI>() - kBiasSmem) / STAGE) == min8(ring_budget<EPI>() / STAGE));
 }
 
-template <int BN, bool QB, int EPI>
+// QBITS: 0 for fp16 weights, else the bits per quantised weight (8, 6 or 4).
+template <int BN, int QBITS, int EPI>
 struct Cfg {
+  static constexpr bool QB = QBITS != 0;
+  static constexpr int RAW_ROW = BK * QBITS / 8;             // bytes of one weight row per k-block as stored
   static constexpr int B_TILE = BN * BK * 2;                 // fp16 B operand (128-byte swizzle)
-  static constexpr int RAW_TILE = QB ? BN * BK : 0;          // INT8 weights as loaded (64-byte rows)
+  static constexpr int RAW_TILE = BN * RAW_ROW;              // quantised weights as loaded (unswizzled rows)
   static constexpr int TX = A_TILE + (QB ? RAW_TILE : B_TILE);  // bytes landed by TMA per stage
   static constexpr int STAGE = A_TILE + B_TILE + RAW_TILE;
-  static constexpr bool SB = staged_bias<EPI, QB, STAGE>();
+  static constexpr bool SB = staged_bias<EPI, QBITS, STAGE>();
   static constexpr int BIAS_SMEM = SB ? kBiasSmem : 0;
   static constexpr int STAGES = min8((ring_budget<EPI>() - BIAS_SMEM) / STAGE);
   static constexpr int TMEM_COLS = BN == 128 ? 256 : 512;  // two accumulators, rounded to a power of two
@@ -194,7 +197,7 @@ __device__ __forceinline__ void epi_chunk(const TcArgs& p, int r, int n, bool va
 }
 
 // Epilogue of this warp's half of a tile for row r: columns [half BN/2, (half+1) BN/2),
-// or for the paired epilogues (GLU, power: 128-column blocks [first 64 | second 64])
+// or for the paired epilogue (GLU: 128-column blocks [value 64 | gate 64])
 // the (first, second) pairs of 32-column chunks number half * BN/128 .. (half+1) * BN/128 - 1.
 // bt: bias of the tile's columns (bt[c] = bias[n0 + c]), in shared memory if SB.
 template <int BN, int EPI, bool SB>
@@ -212,30 +215,7 @@ __device__ __forceinline__ void epilogue_tile(const TcArgs& p, int r, int n0, ui
       valid = t >= 0 && t < (EPI == EPI_CONV1 ? ep.clips.L1(ci) : ep.clips.L2(ci));
     }
   }
-  if constexpr (EPI == EPI_POWER) {
-    // DFT basis rows interleaved in blocks of 64: [cos 64 bins | sin 64 bins] per 128 columns
-#pragma unroll 1
-    for (int pr = half * (BN / 128); pr < (half + 1) * (BN / 128); ++pr) {
-      const int blk = (pr >> 1) * 128, hh = (pr & 1) * 32;
-      {
-        uint32_t a[32], g[32];
-        tmem_ld32(tbase + blk + hh, a);
-        tmem_ld32(tbase + blk + 64 + hh, g);
-        tmem_ld_wait();
-        if (!in_m) continue;
-        float4* o = reinterpret_cast<float4*>(reinterpret_cast<float*>(ep.out) + (size_t)r * ep.ldo + (n0 + blk) / 2 + hh);
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          float4 w;
-          w.x = __uint_as_float(a[4 * j]) * __uint_as_float(a[4 * j]) + __uint_as_float(g[4 * j]) * __uint_as_float(g[4 * j]);
-          w.y = __uint_as_float(a[4 * j + 1]) * __uint_as_float(a[4 * j + 1]) + __uint_as_float(g[4 * j + 1]) * __uint_as_float(g[4 * j + 1]);
-          w.z = __uint_as_float(a[4 * j + 2]) * __uint_as_float(a[4 * j + 2]) + __uint_as_float(g[4 * j + 2]) * __uint_as_float(g[4 * j + 2]);
-          w.w = __uint_as_float(a[4 * j + 3]) * __uint_as_float(a[4 * j + 3]) + __uint_as_float(g[4 * j + 3]) * __uint_as_float(g[4 * j + 3]);
-          o[j] = w;
-        }
-      }
-    }
-  } else if constexpr (EPI == EPI_GLU) {
+  if constexpr (EPI == EPI_GLU) {
     // weight rows interleaved in blocks of 64: [value 64 | gate 64] per 128 columns
 #pragma unroll 1
     for (int pr = half * (BN / 128); pr < (half + 1) * (BN / 128); ++pr) {
@@ -335,6 +315,44 @@ constexpr int kCvtWarps = 4;  // INT8 variant: warps that dequantise the weight 
 template <bool QB>
 constexpr int threads_of() { return 64 + 32 * kEpiWarps + (QB ? 32 * kCvtWarps : 0); }
 
+// 4- and 6-bit weights are stored as u = q + 8 (resp. q + 32), in 1 .. 15 (1 .. 63),
+// and laid out per 16 consecutive weights v0 .. v15 of a row so that each fp16
+// pair (v_2p, v_2p+1) comes out of one shift and one mask: 32-bit word w0 holds
+// the low nibbles of v0 .. v7 with v_2i in nibble i and v_2i+1 in nibble 4 + i
+// (i < 4), word w1 the same for v8 .. v15; 6-bit weights add word w2 with the
+// top two bits of v_2p in bits 2p .. 2p+1 and of v_2p+1 in bits 16 + 2p ..
+// Writing a value u < 1024 into the mantissa of 1024.0 (fp16 0x6400) gives
+// exactly 1024 + u; subtracting 1024 + the offset gives q exactly, and the
+// product with the group scale is rounded once to fp16, as for INT8.
+__device__ __forceinline__ uint32_t scale_pair(uint32_t u2, __half2 off, __half2 s2) {
+  __half2 h = __hmul2(__hsub2(*reinterpret_cast<__half2*>(&u2), off), s2);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+__device__ __forceinline__ void dequant16_i4(uint32_t w0, uint32_t w1, __half2 s2, uint4& out0, uint4& out1) {
+  const __half2 off = __floats2half2_rn(1032.f, 1032.f);
+  uint32_t o[8];
+#pragma unroll
+  for (int p = 0; p < 4; ++p) {
+    o[p] = scale_pair(((w0 >> (4 * p)) & 0x000f000fu) | 0x64006400u, off, s2);
+    o[4 + p] = scale_pair(((w1 >> (4 * p)) & 0x000f000fu) | 0x64006400u, off, s2);
+  }
+  out0 = make_uint4(o[0], o[1], o[2], o[3]);
+  out1 = make_uint4(o[4], o[5], o[6], o[7]);
+}
+__device__ __forceinline__ void dequant16_i6(uint32_t w0, uint32_t w1, uint32_t w2, __half2 s2, uint4& out0,
+                                             uint4& out1) {
+  const __half2 off = __floats2half2_rn(1056.f, 1056.f);
+  uint32_t o[8];
+#pragma unroll
+  for (int p = 0; p < 8; ++p) {
+    const uint32_t lo = (((p < 4 ? w0 : w1) >> (4 * (p & 3))) & 0x000f000fu);
+    const uint32_t hi = ((w2 >> (2 * p)) & 0x00030003u) << 4;
+    o[p] = scale_pair(lo | hi | 0x64006400u, off, s2);
+  }
+  out0 = make_uint4(o[0], o[1], o[2], o[3]);
+  out1 = make_uint4(o[4], o[5], o[6], o[7]);
+}
+
 // INT8 -> fp16 dequantisation of one 16-byte chunk (16 weights of one row)
 // into two 16-byte chunks of the swizzled fp16 operand.  An int8 x becomes
 // exactly x in fp16 by writing the byte x + 128 into the low mantissa bits of
@@ -357,11 +375,12 @@ __device__ __forceinline__ void dequant16(uint4 raw, __half2 s2, uint4& out0, ui
   out1 = make_uint4(o[4], o[5], o[6], o[7]);
 }
 
-template <int BN, int EPI, bool QB>
-__global__ void __launch_bounds__(threads_of<QB>(), 1)
+template <int BN, int EPI, int QBITS>
+__global__ void __launch_bounds__(threads_of<QBITS != 0>(), 1)
 gemm_tc_kernel(const __grid_constant__ CUtensorMap mA, const __grid_constant__ CUtensorMap mA2,
                const __grid_constant__ CUtensorMap mB, const __grid_constant__ CUtensorMap mX, const TcArgs p) {
-  using C = Cfg<BN, QB, EPI>;
+  using C = Cfg<BN, QBITS, EPI>;
+  constexpr bool QB = C::QB;
   constexpr int STAGES = C::STAGES;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
@@ -436,7 +455,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap mA, const __grid_constant__ C
           }
           mbar_arrive_expect_tx(&full[s], C::TX);
           tma_load_2d(sA + s * A_TILE, ma, &full[s], ax, ay);
-          if (QB) tma_load_2d(sRaw + s * C::RAW_TILE, &mB, &full[s], kb * BK, n0);
+          if (QB) tma_load_2d(sRaw + s * C::RAW_TILE, &mB, &full[s], kb * C::RAW_ROW, n0);
           else tma_load_2d(sB + s * C::B_TILE, &mB, &full[s], kb * BK, n0);
           ++it;
         }
@@ -477,9 +496,10 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap mA, const __grid_constant__ C
       mbar_settle(drain, 0, abort_flag, p.wait_ns);
     }
   } else if (QB && warp >= 2 + kEpiWarps) {
-    // converter warps: INT8 tile (BN rows x 64 B) -> fp16 swizzled operand (BN rows x 128 B)
+    // converter warps: quantised tile (BN rows x RAW_ROW bytes) -> fp16 swizzled operand
+    // (BN rows x 128 B); each thread converts 16 weights of a row per pass
     const int t = threadIdx.x - 32 * (2 + kEpiWarps);  // 0 .. 127
-    const int ch = t & 3;                              // 16-byte chunk of a 64-byte INT8 row
+    const int ch = t & 3;                              // 16-weight chunk of the row's 64
     int it = 0;
     bool ok = true;
     for (int tile = blockIdx.x; tile < p.tiles && ok; tile += gridDim.x) {
@@ -496,10 +516,18 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap mA, const __grid_constant__ C
 #pragma unroll 4
         for (int pass = 0; pass < BN / 32; ++pass) {
           const int row = pass * 32 + (t >> 2);
-          const uint4 q = *reinterpret_cast<const uint4*>(raw + row * 64 + ch * 16);
+          const uint8_t* src = raw + row * C::RAW_ROW + ch * (C::RAW_ROW / 4);
           const __half sv = __ldg(sc + row);
           uint4 o0, o1;
-          dequant16(q, __half2(sv, sv), o0, o1);
+          if constexpr (QBITS == 8) {
+            dequant16(*reinterpret_cast<const uint4*>(src), __half2(sv, sv), o0, o1);
+          } else if constexpr (QBITS == 6) {
+            const uint32_t* w = reinterpret_cast<const uint32_t*>(src);
+            dequant16_i6(w[0], w[1], w[2], __half2(sv, sv), o0, o1);
+          } else {
+            const uint2 w = *reinterpret_cast<const uint2*>(src);
+            dequant16_i4(w.x, w.y, __half2(sv, sv), o0, o1);
+          }
           uint8_t* drow = dst + (row >> 3) * 1024 + (row & 7) * 128;
           *reinterpret_cast<uint4*>(drow + (((2 * ch) ^ (row & 7)) << 4)) = o0;
           *reinterpret_cast<uint4*>(drow + (((2 * ch + 1) ^ (row & 7)) << 4)) = o1;
@@ -605,7 +633,7 @@ struct PairCfg {
   static constexpr int BH = TN / 2;                      // B rows per CTA
   static constexpr int B_TILE = BH * BK * 2;
   static constexpr int STAGE = A_TILE + B_TILE;
-  static constexpr bool SB = staged_bias<EPI, false, STAGE>();
+  static constexpr bool SB = staged_bias<EPI, 0, STAGE>();
   static constexpr int BIAS_SMEM = SB ? kBiasSmem : 0;
   static constexpr int STAGES = min8((ring_budget<EPI>() - BIAS_SMEM) / STAGE);
   static constexpr int TMEM_COLS = TN == 128 ? 256 : 512;
@@ -825,11 +853,12 @@ cudaError_t make_map_i8(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_
   return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
-template <int BN, int EPI, bool QB>
+template <int BN, int EPI, int QBITS>
 cudaError_t launch_epi(TcGemmCache* cache, const CUtensorMap& mA, const CUtensorMap& mA2, const CUtensorMap& mB,
                        const CUtensorMap& mX, const TcArgs& args, cudaStream_t s) {
-  using C = Cfg<BN, QB, EPI>;
-  auto kern = gemm_tc_kernel<BN, EPI, QB>;
+  using C = Cfg<BN, QBITS, EPI>;
+  constexpr bool QB = C::QB;
+  auto kern = gemm_tc_kernel<BN, EPI, QBITS>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::SMEM);
   if (e != cudaSuccess) return e;
   const int grid = args.tiles < cache->sm_count ? args.tiles : cache->sm_count;
@@ -884,33 +913,43 @@ cudaError_t launch_pair(TcGemmCache* cache, const CUtensorMap& mA, const CUtenso
     case EPI_CONV1: return launch_pair_epi<TN, EPI_CONV1>(cache, mA, mA2, mB, mX, args, s);
     case EPI_CONV2: return launch_pair_epi<TN, EPI_CONV2>(cache, mA, mA2, mB, mX, args, s);
     case EPI_F32: return launch_pair_epi<TN, EPI_F32>(cache, mA, mA2, mB, mX, args, s);
-    case EPI_POWER: return launch_pair_epi<TN, EPI_POWER>(cache, mA, mA2, mB, mX, args, s);
     default: return cudaErrorInvalidValue;
   }
 }
 
-template <int BN, bool QB>
+template <int BN, int QBITS>
 cudaError_t launch_bn(TcGemmCache* cache, const CUtensorMap& mA, const CUtensorMap& mA2, const CUtensorMap& mB,
                       const CUtensorMap& mX, const TcArgs& args, cudaStream_t s) {
   switch (args.epi) {
-    case EPI_SWISH: return launch_epi<BN, EPI_SWISH, QB>(cache, mA, mA2, mB, mX, args, s);
-    case EPI_GLU: return launch_epi<BN, EPI_GLU, QB>(cache, mA, mA2, mB, mX, args, s);
-    case EPI_RESID: return launch_epi<BN, EPI_RESID, QB>(cache, mA, mA2, mB, mX, args, s);
-    case EPI_QKV: return launch_epi<BN, EPI_QKV, QB>(cache, mA, mA2, mB, mX, args, s);
-    case EPI_CONV1: return launch_epi<BN, EPI_CONV1, QB>(cache, mA, mA2, mB, mX, args, s);
-    case EPI_CONV2: return launch_epi<BN, EPI_CONV2, QB>(cache, mA, mA2, mB, mX, args, s);
-    case EPI_F32: return launch_epi<BN, EPI_F32, QB>(cache, mA, mA2, mB, mX, args, s);
-    case EPI_POWER: return launch_epi<BN, EPI_POWER, QB>(cache, mA, mA2, mB, mX, args, s);
+    case EPI_SWISH: return launch_epi<BN, EPI_SWISH, QBITS>(cache, mA, mA2, mB, mX, args, s);
+    case EPI_GLU: return launch_epi<BN, EPI_GLU, QBITS>(cache, mA, mA2, mB, mX, args, s);
+    case EPI_RESID: return launch_epi<BN, EPI_RESID, QBITS>(cache, mA, mA2, mB, mX, args, s);
+    case EPI_QKV: return launch_epi<BN, EPI_QKV, QBITS>(cache, mA, mA2, mB, mX, args, s);
+    case EPI_F32: return launch_epi<BN, EPI_F32, QBITS>(cache, mA, mA2, mB, mX, args, s);
+    case EPI_CONV1:
+      if constexpr (QBITS == 0) return launch_epi<BN, EPI_CONV1, 0>(cache, mA, mA2, mB, mX, args, s);
+      return cudaErrorInvalidValue;  // the subsampling convs keep fp16 weights
+    case EPI_CONV2:
+      if constexpr (QBITS == 0) return launch_epi<BN, EPI_CONV2, 0>(cache, mA, mA2, mB, mX, args, s);
+      return cudaErrorInvalidValue;
     default: return cudaErrorInvalidValue;
   }
+}
+
+template <int QBITS>
+cudaError_t launch_width(int BN, TcGemmCache* cache, const CUtensorMap& mA, const CUtensorMap& mA2,
+                         const CUtensorMap& mB, const CUtensorMap& mX, const TcArgs& args, cudaStream_t s) {
+  if (BN == 256) return launch_bn<256, QBITS>(cache, mA, mA2, mB, mX, args, s);
+  if (BN == 192) return launch_bn<192, QBITS>(cache, mA, mA2, mB, mX, args, s);
+  return launch_bn<128, QBITS>(cache, mA, mA2, mB, mX, args, s);
 }
 
 }  // namespace
 
 bool tc_supported(int a_dtype, int b_dtype, int N, int K, int epi) {
-  return a_dtype == 1 && (b_dtype == 1 || b_dtype == 2) && N % 256 == 0 && K % 64 == 0 && K >= 64 &&
+  return a_dtype == 1 && b_dtype >= 1 && b_dtype <= 4 && N % 256 == 0 && K % 64 == 0 && K >= 64 &&
          (epi == EPI_SWISH || epi == EPI_GLU || epi == EPI_RESID || epi == EPI_QKV || epi == EPI_CONV1 ||
-          epi == EPI_CONV2 || epi == EPI_F32 || epi == EPI_POWER);
+          epi == EPI_CONV2 || epi == EPI_F32);
 }
 
 cudaError_t tc_init(TcGemmCache* cache, int device) {
@@ -941,7 +980,7 @@ constexpr double kPairCost = 0.7;
 constexpr double kWaveRoundUp = 0.25;
 
 // Tile shape: over single-CTA tiles (128 rows) and paired-CTA tiles (256 rows
-// on two SMs) of width 256, 192 or 128 dividing N (GLU / power epilogues need
+// on two SMs) of width 256, 192 or 128 dividing N (the GLU epilogue needs
 // 128-column blocks), the one that minimises (waves of tiles over the SMs) x
 // (per-SM tile cost), counting a fixed per-tile overhead of 32 columns.  The
 // constants were fitted to measured times of the encoder's GEMM shapes on B200.
@@ -959,7 +998,7 @@ TileShape choose_tile(const TcGemmCache* cache, int M, int N, int epi, bool qb, 
     const int mt = pair ? (M + 255) / 256 : (M + BM - 1) / BM;
     for (int bn : {256, 192, 128}) {
       if (N % bn || (width && bn != width) || (n_split > 0 && n_split % bn)) continue;
-      if ((epi == EPI_GLU || epi == EPI_POWER) && bn % 128) continue;
+      if (epi == EPI_GLU && bn % 128) continue;
       const int tiles = mt * (N / bn);
       const double round_up = qb ? 1.0 : kWaveRoundUp;
       const double waves = round_up * (double)((tiles + units - 1) / units) + (1.0 - round_up) * (double)tiles / units;
@@ -983,7 +1022,8 @@ cudaError_t launch_gemm_tc(TcGemmCache* cache, const void* A, const void* A2, in
       ((reinterpret_cast<uintptr_t>(ep.out) & 31) || ep.ldo % 16))
     return cudaErrorInvalidValue;
   if (epi == EPI_QKV && ((reinterpret_cast<uintptr_t>(ep.qk) & 31) || ep.d_head % 16)) return cudaErrorInvalidValue;
-  const bool qb = B.dtype == 2;
+  const bool qb = B.dtype >= 2;  // INT8 / INT6 / INT4 g64 weights: dequantised in the mainloop
+  const int qbits = B.dtype == 2 ? 8 : B.dtype == 3 ? 6 : 4;
   if (qb && !B.scale_t) return cudaErrorInvalidValue;
   const TileShape t = choose_tile(cache, M, N, epi, qb, variant, width, A2 ? n_split : 0);
   if (!t.width) return cudaErrorInvalidValue;
@@ -999,7 +1039,7 @@ cudaError_t launch_gemm_tc(TcGemmCache* cache, const void* A, const void* A2, in
   if (e == cudaSuccess && !conv) e = make_map_f16(&mA2, A2 ? A2 : A, K, M, (uint64_t)lda * 2, BK, BM);
   if (conv) mA2 = mA;
   if (e == cudaSuccess)
-    e = qb ? make_map_i8(&mB, B.w, K, N, BK, BN)
+    e = qb ? make_map_i8(&mB, B.w, (uint64_t)K * qbits / 8, N, BK * qbits / 8, BN)
            : make_map_f16(&mB, B.w, K, N, (uint64_t)K * 2, BK, pair ? (uint32_t)(BN / 2) : (uint32_t)BN);
   if (e != cudaSuccess) return e;
   TcArgs args;
@@ -1030,14 +1070,10 @@ cudaError_t launch_gemm_tc(TcGemmCache* cache, const void* A, const void* A2, in
     if (BN == 192) return launch_pair<192>(cache, mA, mA2, mB, mX, args, s);
     return launch_pair<128>(cache, mA, mA2, mB, mX, args, s);
   }
-  if (qb) {
-    if (BN == 256) return launch_bn<256, true>(cache, mA, mA2, mB, mX, args, s);
-    if (BN == 192) return launch_bn<192, true>(cache, mA, mA2, mB, mX, args, s);
-    return launch_bn<128, true>(cache, mA, mA2, mB, mX, args, s);
-  }
-  if (BN == 256) return launch_bn<256, false>(cache, mA, mA2, mB, mX, args, s);
-  if (BN == 192) return launch_bn<192, false>(cache, mA, mA2, mB, mX, args, s);
-  return launch_bn<128, false>(cache, mA, mA2, mB, mX, args, s);
+  if (B.dtype == 2) return launch_width<8>(BN, cache, mA, mA2, mB, mX, args, s);
+  if (B.dtype == 3) return launch_width<6>(BN, cache, mA, mA2, mB, mX, args, s);
+  if (B.dtype == 4) return launch_width<4>(BN, cache, mA, mA2, mB, mX, args, s);
+  return launch_width<0>(BN, cache, mA, mA2, mB, mX, args, s);
 }
 
 cudaError_t launch_attention(TcGemmCache* cache, const void* qk, const void* vt, Clips clips, void* o, int t_half,

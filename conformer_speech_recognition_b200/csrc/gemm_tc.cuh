@@ -51,6 +51,16 @@ cudaError_t launch_attention_tc(TcGemmCache* cache, const void* qk, const void* 
 cudaError_t launch_attention(TcGemmCache* cache, const void* qk, const void* vt, Clips clips, void* o, int t_half,
                              int rows_pad, int n_heads, int d_head, int t_max, cudaStream_t s);
 
+// Tensor-core frontend (frontend_tc.cu), step 2: 3xTF32 windowed DFT of the
+// frames (pairs of split rows, split_rows >= rows + 1) against the basis
+// [384][320] (hi and lo parts), power, filterbank fb [161][64] over the nonzero
+// rows fb_range (int pairs per mel bin) and log(clip(., 1e-9, 1e9)).  mode 0:
+// out = fp16 packed mel rows [rows][64], zero outside clips; mode 1: out = fp32
+// [B][f_max][64], written for valid frames only.
+cudaError_t launch_dft_mel(TcGemmCache* cache, const float* hi, const float* lo, int split_rows,
+                           const float* basis_hi, const float* basis_lo, const float* fb, const int* fb_range,
+                           Clips clips, int rows, int mode, int f_max, void* out, cudaStream_t s);
+
 cudaError_t tc_read_status(TcGemmCache* cache, int* status);
 cudaError_t tc_reset_status(TcGemmCache* cache);
 void tc_release(TcGemmCache* cache);

@@ -52,11 +52,11 @@ int seg_rows(const ClipLen& l) {
 }
 
 struct DevLinear {
-  void* w = nullptr;          // [N, K] f32 / f16 / int8
+  void* w = nullptr;          // [N, K] f32 / f16 / int8, or packed 6- / 4-bit rows (see upload_linear)
   __half* scale = nullptr;    // int8: [N, K/64]
   __half* scale_t = nullptr;  // int8: [K/64, N]
   float* b = nullptr;         // [N]
-  int N = 0, K = 0, dtype = 0;
+  int N = 0, K = 0, dtype = 0;  // dtype: 0 f32, 1 f16, 2 int8, 3 int6, 4 int4 (g64 scales)
   WeightOp op() const { return WeightOp{w, scale, dtype, scale_t}; }
 };
 struct DevLN {
@@ -112,7 +112,7 @@ struct gam_ctx {
   gam_config cfg{};
   int device = 0;
   int act_half = 0;  // activations between GEMMs in fp16 (1) or fp32 (0)
-  int wdtype = 0;    // GEMM weight dtype: 0 f32, 1 f16, 2 int8-g64
+  int wdtype = 0;    // GEMM weight dtype: 0 f32, 1 f16, 2 int8-g64, 3 int6-g64, 4 int4-g64
   int d_head = 0;
   std::string err;
   std::vector<void*> allocs;
@@ -120,10 +120,12 @@ struct gam_ctx {
   float* basis = nullptr;  // [320][320]
   float* fb = nullptr;     // [161][64]
   int* fb_range = nullptr; // [64][2]: first and last nonzero filterbank row of each mel bin
-  DevLinear dft;           // fp16 modes: windowed DFT basis as a [512, 320] GEMM weight,
-                           // rows [cos 64 bins | sin 64 bins] per 128 (bins 0..255, zero past 160)
-  __half* frames = nullptr;  // [R0_cap, 320] fp16 frames
-  float* power = nullptr;    // [R0_cap, 256] power spectrum
+  // fp16 / INT8 modes: windowed DFT basis [384][320] as tf32 hi and lo parts, rows
+  // [cos 64 bins | sin 64 bins] per 128 (bins 0 .. 191, zero past 160)
+  float* dft_hi = nullptr;
+  float* dft_lo = nullptr;
+  float* split_hi = nullptr;  // [R0_cap + 2][160] packed samples, tf32 hi / lo parts
+  float* split_lo = nullptr;
   DevLinear conv1, conv2, head;
   DevLinear head2;         // tensor-core CTC head: [W | W] padded to a multiple of 256 rows, K = 2d
   __half* ctc_a = nullptr; // [rows, 2d] fp16 hi / lo split of the valid encoder frames
@@ -281,8 +283,8 @@ gam_status load_ln(gam_ctx* c, const WeightTable& t, const std::string& name, in
 struct HostLinear {
   int N = 0, K = 0, dtype = 0;
   std::vector<double> w;        // f32 / f16 modes: [N, K] values
-  std::vector<int8_t> q;        // int8 mode
-  std::vector<__half> s;        // int8 mode [N, K/64]
+  std::vector<int8_t> q;        // quantised modes: [N, K] integer values
+  std::vector<__half> s;        // quantised modes: [N, K/64] group scales
   std::vector<double> b;
 };
 
@@ -297,8 +299,13 @@ gam_status read_linear(gam_ctx* c, const WeightTable& t, const std::string& name
     GAM_TRY(find(c, t, name + ".weight_scale", {N, K / 64}, &gs));
     if (gq->dtype != GAM_DTYPE_I8 || gs->dtype != GAM_DTYPE_F16)
       return fail(c, GAM_ERR_WEIGHTS, name + ": weight_q must be int8 and weight_scale f16");
-    out.dtype = 2;
+    out.dtype = c->wdtype;
     out.q.assign((const int8_t*)gq->data, (const int8_t*)gq->data + (size_t)N * K);
+    const int qmax = c->wdtype == 2 ? 127 : c->wdtype == 3 ? 31 : 7;
+    for (int8_t v : out.q)
+      if (v < -qmax || v > qmax)
+        return fail(c, GAM_ERR_WEIGHTS, name + ".weight_q holds " + std::to_string((int)v) + ", outside +-" +
+                                            std::to_string(qmax) + " of this precision");
     out.s.assign((const __half*)gs->data, (const __half*)gs->data + (size_t)N * (K / 64));
     return GAM_OK;
   }
@@ -314,7 +321,7 @@ void permute_rows(HostLinear& l, const std::vector<int>& perm) {
   for (int i = 0; i < l.N; ++i) {
     const int j = perm[i];
     o.b[i] = l.b[j];
-    if (l.dtype == 2) {
+    if (l.dtype >= 2) {
       std::memcpy(&o.q[(size_t)i * l.K], &l.q[(size_t)j * l.K], l.K);
       std::memcpy(&o.s[(size_t)i * (l.K / 64)], &l.s[(size_t)j * (l.K / 64)], (l.K / 64) * sizeof(__half));
     } else {
@@ -324,13 +331,44 @@ void permute_rows(HostLinear& l, const std::vector<int>& perm) {
   l = std::move(o);
 }
 
+// 6- and 4-bit weights, stored as u = q + 32 (q + 8), packed per 16 consecutive
+// weights v0 .. v15 of a row into the layout the GEMM's converter warps read
+// (gemm_tc.cu): word w0 = low nibbles of v0 .. v7 with v_2i in nibble i and
+// v_2i+1 in nibble 4 + i, word w1 the same for v8 .. v15, and for 6 bits a word
+// w2 with the top two bits of v_2p in bits 2p .. 2p+1 and of v_2p+1 in bits
+// 16 + 2p ..  Rows of K * bits / 8 bytes, chunks in K order.
+void pack_subbyte(const HostLinear& l, std::vector<uint8_t>& out) {
+  const bool six = l.dtype == 3;
+  const int off = six ? 32 : 8, words = six ? 3 : 2;
+  const size_t row_bytes = (size_t)l.K * (six ? 6 : 4) / 8;
+  out.assign((size_t)l.N * row_bytes, 0);
+  for (int n = 0; n < l.N; ++n)
+    for (int c0 = 0; c0 < l.K; c0 += 16) {
+      uint32_t w[3] = {0, 0, 0};
+      for (int j = 0; j < 16; ++j) {
+        const uint32_t u = (uint32_t)(l.q[(size_t)n * l.K + c0 + j] + off);
+        const int jj = j & 7, p = j >> 1;
+        const int nib = (jj & 1) ? 4 + (jj >> 1) : (jj >> 1);
+        w[j >> 3] |= (u & 15u) << (4 * nib);
+        if (six) w[2] |= (u >> 4) << ((j & 1) ? 16 + 2 * p : 2 * p);
+      }
+      std::memcpy(&out[(size_t)n * row_bytes + (size_t)(c0 / 16) * 4 * words], w, 4 * words);
+    }
+}
+
 gam_status upload_linear(gam_ctx* c, const HostLinear& l, DevLinear& d) {
   d.N = l.N;
   d.K = l.K;
   d.dtype = l.dtype;
   GAM_TRY(upload_f32(c, &d.b, l.b));
-  if (l.dtype == 2) {
-    GAM_TRY(upload(c, (int8_t**)&d.w, l.q.data(), l.q.size()));
+  if (l.dtype >= 2) {
+    if (l.dtype == 2) {
+      GAM_TRY(upload(c, (int8_t**)&d.w, l.q.data(), l.q.size()));
+    } else {
+      std::vector<uint8_t> packed;
+      pack_subbyte(l, packed);
+      GAM_TRY(upload(c, (uint8_t**)&d.w, packed.data(), packed.size()));
+    }
     const int G = l.K / 64;
     std::vector<__half> st((size_t)G * l.N);
     for (int n = 0; n < l.N; ++n)
@@ -367,6 +405,18 @@ gam_status load_conv(gam_ctx* c, const WeightTable& t, const std::string& name, 
   return upload_linear(c, l, d);
 }
 
+// Nearest tf32 value of x (10 explicit mantissa bits; ties away from zero), as fp32.
+float tf32_round(float x) {
+  uint32_t u;
+  std::memcpy(&u, &x, 4);
+  if ((u & 0x7f800000u) != 0x7f800000u) {  // finite: round the magnitude at bit 13
+    u += 0x1000u;
+    u &= 0xffffe000u;
+  }
+  std::memcpy(&x, &u, 4);
+  return x;
+}
+
 gam_status validate_config(const gam_config* cfg) {
   if (!cfg) return fail(nullptr, GAM_ERR_INVALID_ARG, "null config");
   const gam_config& c = *cfg;
@@ -382,7 +432,7 @@ gam_status validate_config(const gam_config* cfg) {
   if (c.conv_kernel < 1 || c.conv_kernel > 63 || c.conv_kernel % 2 == 0)
     return fail(nullptr, GAM_ERR_INVALID_ARG, "conv_kernel must be odd and <= 63");
   if (c.n_classes < 2 || c.n_classes > 1024) return fail(nullptr, GAM_ERR_INVALID_ARG, "n_classes must be 2..1024");
-  if (c.precision < GAM_FP32 || c.precision > GAM_INT8_G64) return fail(nullptr, GAM_ERR_INVALID_ARG, "bad precision");
+  if (c.precision < GAM_FP32 || c.precision > GAM_INT4_G64) return fail(nullptr, GAM_ERR_INVALID_ARG, "bad precision");
   if (!(c.rope_base > 0) || !(c.ln_eps > 0) || !(c.bn_eps > 0))
     return fail(nullptr, GAM_ERR_INVALID_ARG, "rope_base / eps must be positive");
   if (c.max_batch < 1 || c.max_batch > 4096) return fail(nullptr, GAM_ERR_INVALID_ARG, "max_batch must be 1..4096");
@@ -632,13 +682,15 @@ gam_status encoder_kernels(gam_ctx* c, const Plan& p, const Clips& clips, const 
   const float eps = cfg.ln_eps;
   const int M = p.E_pad;
 
-  if (c->dft.w) {
-    // tensor-core frontend: fp16 frames -> DFT GEMM with the power epilogue -> mel + log
-    GAM_TRY(run_kernel(c, PK_FRONTEND, s, [&] { return launch_frames(audio, max_samples, clips, p.R0, c->frames, s); }));
-    GAM_TRY(gemm(c, PK_FRONTEND, s, c->frames, nullptr, 0, cfg.n_fft, c->dft, p.R0, EPI_POWER, 1.f, c->power, 256,
-                 clips));
+  if (c->dft_hi) {
+    // tensor-core frontend: samples split into tf32 hi / lo rows, then the 3xTF32 DFT
+    // with power, filterbank and log in its epilogue (fp16 packed mel rows)
     GAM_TRY(run_kernel(c, PK_FRONTEND, s, [&] {
-      return launch_mel_log(c->power, 256, c->fb, c->fb_range, clips, p.R0, c->mel, ah, s);
+      return launch_audio_split(audio, max_samples, clips, p.R0 + 1, c->split_hi, c->split_lo, s);
+    }));
+    GAM_TRY(run_kernel(c, PK_FRONTEND, s, [&] {
+      return launch_dft_mel(&c->tc, c->split_hi, c->split_lo, p.R0 + 1, c->dft_hi, c->dft_lo, c->fb, c->fb_range,
+                            clips, p.R0, 0, 0, c->mel, s);
     }));
   } else {
     GAM_TRY(run_kernel(c, PK_FRONTEND, s, [&] {
@@ -782,7 +834,7 @@ gam_status build_weights(gam_ctx* c, const gam_tensor* tensors, int n) {
     t.by_name[tensors[i].name] = &tensors[i];
   }
   const int d = cfg.d_model, f = cfg.ffn_dim, K = cfg.conv_kernel;
-  const bool q8 = cfg.precision == GAM_INT8_G64;
+  const bool q8 = cfg.precision >= GAM_INT8_G64;  // quantised linear weights (8, 6 or 4 bits)
   // frontend: window folded into the DFT basis
   {
     std::vector<double> win, fbv;
@@ -817,23 +869,25 @@ gam_status build_weights(gam_ctx* c, const gam_tensor* tensors, int n) {
       GAM_TRY(upload(c, &c->fb_range, range.data(), range.size() * sizeof(int)));
     }
     if (cfg.precision != GAM_FP32) {
-      HostLinear hd;
-      hd.N = 512;
-      hd.K = N;
-      hd.dtype = 1;
-      hd.b.assign(512, 0.0);
-      hd.w.assign((size_t)512 * N, 0.0);
-      for (int row = 0; row < 512; ++row) {
-        const int tile = row / 256, blk = (row % 256) / 128, within = row % 128;
+      // tensor-core DFT basis: row n = [cos | sin] block n / 128, bin 64 (n / 128) + n % 64,
+      // each value as tf32 hi + lo (lo = the remainder, itself rounded to tf32)
+      const int rows = 384;
+      std::vector<float> bh((size_t)rows * N, 0.f), bl((size_t)rows * N, 0.f);
+      for (int row = 0; row < rows; ++row) {
+        const int within = row % 128;
         const bool is_sin = within >= 64;
-        const int bin = tile * 128 + blk * 64 + (within % 64);
+        const int bin = (row / 128) * 64 + (within % 64);
         if (bin > N / 2 || (is_sin && (bin == 0 || bin == N / 2))) continue;
         for (int nn = 0; nn < N; ++nn) {
           const double a = two_pi * (double)((int64_t)bin * nn % N) / N;
-          hd.w[(size_t)row * N + nn] = win[nn] * (is_sin ? std::sin(a) : std::cos(a));
+          const double v = win[nn] * (is_sin ? std::sin(a) : std::cos(a));
+          const float hi = tf32_round((float)v);
+          bh[(size_t)row * N + nn] = hi;
+          bl[(size_t)row * N + nn] = tf32_round((float)(v - (double)hi));
         }
       }
-      GAM_TRY(upload_linear(c, hd, c->dft));
+      GAM_TRY(upload(c, &c->dft_hi, bh.data(), bh.size() * sizeof(float)));
+      GAM_TRY(upload(c, &c->dft_lo, bl.data(), bl.size() * sizeof(float)));
     }
   }
   GAM_TRY(load_conv(c, t, "subsampling.conv1", d, cfg.n_mels, cfg.sub_kernel, c->conv1));
@@ -927,7 +981,7 @@ gam_status build_weights(gam_ctx* c, const gam_tensor* tensors, int n) {
       h2.dtype = hl.dtype;
       h2.b.assign(Cp, 0.0);
       for (int n = 0; n < cfg.n_classes; ++n) h2.b[n] = hl.b[n];
-      if (hl.dtype == 2) {
+      if (hl.dtype >= 2) {
         h2.q.assign((size_t)Cp * 2 * d, 0);
         h2.s.assign((size_t)Cp * (2 * d / 64), __float2half(1.f));
         const int G = d / 64;
@@ -975,8 +1029,8 @@ gam_status alloc_workspace(gam_ctx* c) {
   const int64_t E = c->E_cap;
   GAM_TRY(dev_alloc(c, &c->mel, (size_t)c->R0_cap * cfg.n_mels * es));
   if (cfg.precision != GAM_FP32) {
-    GAM_TRY(dev_alloc(c, (void**)&c->frames, (size_t)c->R0_cap * cfg.n_fft * 2));
-    GAM_TRY(dev_alloc(c, (void**)&c->power, (size_t)c->R0_cap * 256 * 4));
+    GAM_TRY(dev_alloc(c, (void**)&c->split_hi, (size_t)(c->R0_cap + 2) * cfg.hop * 4));
+    GAM_TRY(dev_alloc(c, (void**)&c->split_lo, (size_t)(c->R0_cap + 2) * cfg.hop * 4));
   }
   GAM_TRY(dev_alloc(c, &c->c1, (size_t)c->R1_cap * d * es));
   GAM_TRY(dev_alloc(c, (void**)&c->x, (size_t)E * d * 4));
@@ -1107,7 +1161,7 @@ gam_status gam_create(const gam_config* cfg, const gam_tensor* tensors, int n_te
   c->cfg = *cfg;
   c->device = device;
   c->act_half = cfg->precision == GAM_FP32 ? 0 : 1;
-  c->wdtype = cfg->precision == GAM_FP32 ? 0 : (cfg->precision == GAM_FP16 ? 1 : 2);
+  c->wdtype = cfg->precision == GAM_FP32 ? 0 : (cfg->precision == GAM_FP16 ? 1 : cfg->precision);
   c->d_head = cfg->d_model / cfg->n_heads;
   if (const char* v = std::getenv("GAM_CUDA_GRAPHS")) c->graphs.enabled = std::strcmp(v, "0") != 0;
   gam_status s = cuda_check(c, cudaSetDevice(device), "cudaSetDevice");
@@ -1139,10 +1193,24 @@ gam_status gam_logmel(gam_ctx* c, const float* audio, const int32_t* lengths, in
   cudaStream_t s = (cudaStream_t)stream;
   c->last_stream = s;
   Clips clips;
-  GAM_TRY(upload_table(c, p, s, &clips));
-  GAM_TRY(run_kernel(c, PK_FRONTEND, s, [&] {
-    return launch_frontend(audio, max_samples, clips, batch * p.F_max, 0, p.F_max, c->basis, c->fb, mel, 0, s);
-  }));
+  if (c->dft_hi) {
+    // the tensor-core frontend gam_encode runs, writing the padded fp32 output
+    if (p.R0 > c->R0_cap) return fail(c, GAM_ERR_CAPACITY, "clips longer than the context's workspace");
+    GAM_TRY(upload_table(c, p, s, &clips));
+    GAM_TRY(cuda_check(c, cudaMemsetAsync(mel, 0, (size_t)batch * p.F_max * c->cfg.n_mels * 4, s), "memset"));
+    GAM_TRY(run_kernel(c, PK_FRONTEND, s, [&] {
+      return launch_audio_split(audio, max_samples, clips, p.R0 + 1, c->split_hi, c->split_lo, s);
+    }));
+    GAM_TRY(run_kernel(c, PK_FRONTEND, s, [&] {
+      return launch_dft_mel(&c->tc, c->split_hi, c->split_lo, p.R0 + 1, c->dft_hi, c->dft_lo, c->fb, c->fb_range,
+                            clips, p.R0, 1, p.F_max, mel, s);
+    }));
+  } else {
+    GAM_TRY(upload_table(c, p, s, &clips));
+    GAM_TRY(run_kernel(c, PK_FRONTEND, s, [&] {
+      return launch_frontend(audio, max_samples, clips, batch * p.F_max, 0, p.F_max, c->basis, c->fb, mel, 0, s);
+    }));
+  }
   if (frames_out)
     for (int i = 0; i < batch; ++i) frames_out[i] = p.len[i].F;
   return GAM_OK;

@@ -16,8 +16,9 @@ import numpy as np
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libgam.so")
 
-GAM_FP32, GAM_FP16, GAM_INT8_G64 = 0, 1, 2
-PRECISION = {"fp32": GAM_FP32, "fp16": GAM_FP16, "int8_g64": GAM_INT8_G64}
+GAM_FP32, GAM_FP16, GAM_INT8_G64, GAM_INT6_G64, GAM_INT4_G64 = 0, 1, 2, 3, 4
+PRECISION = {"fp32": GAM_FP32, "fp16": GAM_FP16, "int8_g64": GAM_INT8_G64, "int6_g64": GAM_INT6_G64,
+             "int4_g64": GAM_INT4_G64}
 DTYPE_F32, DTYPE_F16, DTYPE_I8 = 0, 1, 2
 (STAGE_SUBSAMPLING, STAGE_FFN1, STAGE_MHSA, STAGE_CONV, STAGE_FFN2, STAGE_LAYER) = range(6)
 

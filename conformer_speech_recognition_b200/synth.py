@@ -17,10 +17,11 @@ as stored inputs rather than computing them:
   a periodic Hann window and triangular HTK filters with f_min = 0 Hz and
   f_max = 8000 Hz (both limits are not printed on the pages; they are the
   plainest reading for 16 kHz audio).
-* INT8 group-64 weights.  "GigaAM MLX port for Mac", section "How precision
-  affects size and speed", says that each group of 64 weights shares one scale.
-  Quantisation is an offline conversion step, so it lives with the inputs: the
-  GPU path consumes (q, scale) and the oracle consumes q * scale.
+* INT8 / INT6 / INT4 group-64 weights.  "GigaAM MLX port for Mac", section "How
+  precision affects size and speed", says that each group of 64 weights shares
+  one scale and measures 8, 6 and 4 bits.  Quantisation is an offline conversion
+  step, so it lives with the inputs: the GPU path consumes (q, scale) and the
+  oracle consumes q * scale.
 
 Recipes (seeded with numpy PCG64):
   audio  C1-C4: sum of 3 sinusoids, f ~ U[200, 3000] Hz, amplitude 0.1 each,
@@ -53,7 +54,8 @@ _FRONT = dict(n_mels=64, n_fft=320, win=320, hop=160, sub_kernel=5,
 V3 = dict(n_layers=16, d_model=768, n_heads=16, ffn_dim=3072, conv_kernel=31, **_FRONT)
 LARGE = dict(n_layers=24, d_model=1024, n_heads=16, ffn_dim=4096, conv_kernel=31, **_FRONT)
 
-PRECISIONS = {"fp32": 0, "fp16": 1, "int8_g64": 2}
+PRECISIONS = {"fp32": 0, "fp16": 1, "int8_g64": 2, "int6_g64": 3, "int4_g64": 4}
+QUANT_BITS = {"int8_g64": 8, "int6_g64": 6, "int4_g64": 4}
 
 # The five benchmark / parity workloads.
 WORKLOADS = {
@@ -66,6 +68,12 @@ WORKLOADS = {
     "c4_30s_b32_d1024": dict(model=LARGE, n_classes=257, precision="fp16", kind="fixed",
                              batch=32, seconds=30.0, audio_seed=103),
     "c5_300s_chunks15_d1024_int8": dict(model=LARGE, n_classes=257, precision="int8_g64",
+                                        kind="chirp", batch=15, seconds=20.0, audio_seed=104),
+    # the same long-form input with 6- and 4-bit g64 weights ("GigaAM MLX port for
+    # Mac", "How precision affects size and speed")
+    "c5_300s_chunks15_d1024_int6": dict(model=LARGE, n_classes=257, precision="int6_g64",
+                                        kind="chirp", batch=15, seconds=20.0, audio_seed=104),
+    "c5_300s_chunks15_d1024_int4": dict(model=LARGE, n_classes=257, precision="int4_g64",
                                         kind="chirp", batch=15, seconds=20.0, audio_seed=104),
 }
 
@@ -188,14 +196,19 @@ def htk_mel_filterbank(n_fft: int = 320, n_mels: int = 64, sample_rate: int = SA
 # Weights
 # ---------------------------------------------------------------------------
 
-def quantize_g64(w: np.ndarray) -> Tuple[np.ndarray, np.ndarray]:
-    """Symmetric INT8 weight-only quantisation, groups of 64 along the input dim.
+def quantize_g64(w: np.ndarray, bits: int = 8) -> Tuple[np.ndarray, np.ndarray]:
+    """Symmetric weight-only quantisation to `bits` (8, 6 or 4), groups of 64 along
+    the input dim.
 
     w: [out, in] (or [out, in, 1]).  Returns q int8 of w's shape and scale fp16
-    [out, in/64] with w ~= q * scale.  scale = fp16(max|w| / 127) per group
-    (1 when the group is all zero); q = clamp(round_half_even(w / scale), -127, 127)
-    computed in fp64 with the fp16-rounded scale.
+    [out, in/64] with w ~= q * scale.  With qmax = 2^(bits-1) - 1: scale =
+    fp16(max|w| / qmax) per group (1 when the group is all zero); q =
+    clamp(round_half_even(w / scale), -qmax, qmax) computed in fp64 with the
+    fp16-rounded scale.
     """
+    if bits not in (8, 6, 4):
+        raise ValueError("bits must be 8, 6 or 4")
+    qmax = 2 ** (bits - 1) - 1
     shape = w.shape
     w2 = np.asarray(w, dtype=np.float64).reshape(shape[0], -1)
     out_f, in_f = w2.shape
@@ -203,14 +216,14 @@ def quantize_g64(w: np.ndarray) -> Tuple[np.ndarray, np.ndarray]:
         raise ValueError("input dimension must be a multiple of 64")
     g = w2.reshape(out_f, in_f // 64, 64)
     amax = np.abs(g).max(axis=2)
-    scale = np.where(amax > 0, amax / 127.0, 1.0).astype(np.float16)
+    scale = np.where(amax > 0, amax / qmax, 1.0).astype(np.float16)
     s64 = scale.astype(np.float64)[:, :, None]
-    q = np.clip(np.rint(g / s64), -127, 127).astype(np.int8)
+    q = np.clip(np.rint(g / s64), -qmax, qmax).astype(np.int8)
     return q.reshape(shape), scale
 
 
 def quantized_linear_names(cfg: dict):
-    """Names of the linear weights stored as INT8 g64 in the int8_g64 precision."""
+    """Names of the linear weights stored quantised (g64) in the int*_g64 precisions."""
     names = []
     for l in range(cfg["n_layers"]):
         p = f"layers.{l}."
@@ -270,8 +283,9 @@ def _is_gamma(name: str) -> bool:
 def random_weights(cfg: dict, seed: int = 0) -> Dict[str, np.ndarray]:
     """Seeded weights for ``cfg``.  fp16 tensors (fp32 window / filterbank).
 
-    For precision "int8_g64" each quantised linear ``X.weight`` is replaced by
-    ``X.weight_q`` (int8) and ``X.weight_scale`` (fp16 [out, in/64]).
+    For the precisions "int8_g64", "int6_g64" and "int4_g64" each quantised
+    linear ``X.weight`` is replaced by ``X.weight_q`` (int8 array holding q) and
+    ``X.weight_scale`` (fp16 [out, in/64]).
     """
     rng = np.random.Generator(np.random.PCG64(seed))
     out: Dict[str, np.ndarray] = {}
@@ -289,10 +303,11 @@ def random_weights(cfg: dict, seed: int = 0) -> Dict[str, np.ndarray]:
         else:
             v = rng.normal(0.0, 0.02, size=shape)
         out[name] = v.astype(np.float16)
-    if cfg.get("precision") == "int8_g64":
+    if cfg.get("precision") in QUANT_BITS:
+        bits = QUANT_BITS[cfg["precision"]]
         for base in quantized_linear_names(cfg):
             w = out.pop(base + ".weight")
-            q, s = quantize_g64(w)
+            q, s = quantize_g64(w, bits)
             out[base + ".weight_q"] = q
             out[base + ".weight_scale"] = s
     return out

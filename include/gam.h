@@ -64,8 +64,13 @@ typedef enum {
   GAM_ERR_DEVICE_TIMEOUT = 7      /* a bounded device-side wait gave up           */
 } gam_status;
 
-/* gam_config.precision */
-enum { GAM_FP32 = 0, GAM_FP16 = 1, GAM_INT8_G64 = 2 };
+/* gam_config.precision.  The quantised modes store the linear weights of the
+ * encoder blocks and the CTC head as integers q with one fp16 scale s per group
+ * of 64 consecutive input weights (w = q s): INT8 q in [-127, 127], INT6 in
+ * [-31, 31], INT4 in [-7, 7] ("GigaAM MLX port for Mac", "How precision affects
+ * size and speed": INT8, INT6 and INT4 with group 64).  The weights are
+ * dequantised to fp16 inside the tensor-core GEMM's mainloop. */
+enum { GAM_FP32 = 0, GAM_FP16 = 1, GAM_INT8_G64 = 2, GAM_INT6_G64 = 3, GAM_INT4_G64 = 4 };
 
 /* gam_tensor.dtype */
 enum { GAM_DTYPE_F32 = 0, GAM_DTYPE_F16 = 1, GAM_DTYPE_I8 = 2 };
@@ -96,7 +101,7 @@ typedef struct {
   float rope_base;   /* 5000 (pos_emb_max_len), not 10000                     */
   float ln_eps;      /* LayerNorm eps (1e-5)                                  */
   float bn_eps;      /* BatchNorm eps (1e-5)                                  */
-  int precision;     /* GAM_FP32, GAM_FP16 or GAM_INT8_G64                    */
+  int precision;     /* GAM_FP32, GAM_FP16, GAM_INT8_G64, GAM_INT6_G64, GAM_INT4_G64 */
   int max_batch;     /* capacity: clips per call                              */
   int64_t max_samples; /* capacity: samples per clip                          */
 } gam_config;
@@ -146,9 +151,11 @@ gam_status gam_plan_lengths(const gam_config* cfg, const int32_t* lengths_host, 
  * "layers.l.attn.{norm,linear_q,linear_k,linear_v,linear_out}.*",
  * "layers.l.conv.{norm,pointwise1,depthwise,bn,pointwise2}.*",
  * "layers.l.norm_out.*", "head.{weight,bias}" ([C, d] or [C, d, 1]).  In
- * GAM_INT8_G64 precision the eleven linear weights of a block and the head's
- * are given as "<name>.weight_q" (int8, same shape) and "<name>.weight_scale"
- * (f16 [out, in/64]); all other tensors f16 or f32.  On success *out owns
+ * the quantised precisions the eleven linear weights of a block and the head's
+ * are given as "<name>.weight_q" (int8 array of the weight's shape holding q,
+ * within the precision's range, else GAM_ERR_WEIGHTS) and "<name>.weight_scale"
+ * (f16 [out, in/64]); all other tensors f16 or f32.  6- and 4-bit weights are
+ * packed on the device at 6 and 4 bits per weight.  On success *out owns
  * device memory until gam_destroy.  The environment variable GAM_GEMM_TILES
  * (read here) sets the tile policy of the fp16 tensor-core GEMMs: "single"
  * (single-CTA tiles only), "pair" (paired-CTA tiles wherever one applies) or,

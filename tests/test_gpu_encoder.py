@@ -51,8 +51,21 @@ def test_fp32_every_stage_every_layer(model):
     print(f"fp32 worst per-stage max|delta| = {worst:.3e}")
 
 
-def _product_check(name, cfg, W, ctx, audio, lens, sample):
-    """Run the whole batch on the GPU; compare sampled clips with the oracle."""
+def _batch_invariance(ctx, audio, lens, enc, el):
+    """Every clip run alone gives the frames it has inside the full batch, so the
+    oracle comparison of sampled clips carries over to the clips in between."""
+    worst = 0.0
+    for i in range(len(lens)):
+        alone, el1 = gam.gam_encode(ctx, to_torch(audio[i:i + 1, :lens[i]]), lens[i:i + 1])
+        assert el1[0] == el[i]
+        worst = max(worst, max_abs(alone.cpu().numpy()[0, :el1[0]], enc[i, :el[i]]))
+    assert worst <= 1e-5, worst
+    return worst
+
+
+def _product_check(name, cfg, W, ctx, audio, lens, sample, every_clip_alone=False):
+    """Run the whole batch on the GPU; compare sampled clips with the oracle and,
+    optionally, every clip of the batch with the same clip run alone."""
     a = to_torch(audio)
     enc, el = gam.gam_encode(ctx, a, lens)
     tok, cnt, logp = gam.gam_ctc_greedy(ctx, enc, el, want_logp=True)
@@ -75,6 +88,8 @@ def _product_check(name, cfg, W, ctx, audio, lens, sample):
     frac = agree / total
     print(name, "per-clip (clip, rel_fro, max_abs):", report, "argmax agreement", frac)
     assert frac >= MIN_ARGMAX_AGREE, (name, frac)
+    if every_clip_alone:
+        print(name, "batch invariance worst max|delta|", _batch_invariance(ctx, audio, lens, enc, el))
     return enc, el, tok, cnt
 
 
@@ -111,7 +126,7 @@ def test_c3_fp16_full_batch_sampled():
     _, W = config_and_weights(synth.V3, 257, "fp16")
     audio, lens = synth.workload_audio(name)
     ctx = gam.gam_create(cfg, W, 64, 320000)
-    _product_check(name, cfg, W, ctx, audio, lens, [0, 63])
+    _product_check(name, cfg, W, ctx, audio, lens, [0, 31, 63], every_clip_alone=True)
     ctx.close()
 
 
@@ -121,23 +136,27 @@ def test_c4_fp16_full_batch_sampled():
     _, W = config_and_weights(synth.LARGE, 257, "fp16")
     audio, lens = synth.workload_audio(name)
     ctx = gam.gam_create(cfg, W, 32, 480000)
-    _product_check(name, cfg, W, ctx, audio, lens, [31])
+    _product_check(name, cfg, W, ctx, audio, lens, [0, 16, 31], every_clip_alone=True)
     ctx.close()
 
 
-def test_c5_int8_full_batch_sampled():
-    name = "c5_300s_chunks15_d1024_int8"
+@pytest.mark.parametrize("name", ["c5_300s_chunks15_d1024_int8", "c5_300s_chunks15_d1024_int6",
+                                  "c5_300s_chunks15_d1024_int4"])
+def test_c5_quantized_full_batch_sampled(name):
+    """Long-form chunks on the d1024 encoder with 8-, 6- and 4-bit g64 weights
+    dequantised in the GEMM mainloop; the oracle uses the same q * s in fp64."""
     cfg = synth.workload_config(name)
-    _, W = config_and_weights(synth.LARGE, 257, "int8_g64")
+    _, W = config_and_weights(synth.LARGE, 257, cfg["precision"])
     audio, lens = synth.workload_audio(name)
     ctx = gam.gam_create(cfg, W, 15, 320000)
-    _product_check(name, cfg, W, ctx, audio, lens, [7])
+    _product_check(name, cfg, W, ctx, audio, lens, [0, 7, 14], every_clip_alone=True)
     ctx.close()
 
 
-def test_int8_small_every_layer():
+@pytest.mark.parametrize("precision", ["int8_g64", "int6_g64", "int4_g64"])
+def test_quantized_small_model(precision):
     model = small_model(d=256, heads=4, ffn=512, layers=2, K=31)
-    cfg, W = config_and_weights(model, 257, "int8_g64")
+    cfg, W = config_and_weights(model, 257, precision)
     audio, lens = synth.random_audio([20000, 9000], seed=5)
     ctx = gam.gam_create(cfg, W, 2, 20000)
     enc, el = gam.gam_encode(ctx, to_torch(audio), lens)

@@ -30,6 +30,34 @@ def test_logmel_parity_ragged(small_ctx):
         assert np.all(mel[i, frames[i]:] == 0)
 
 
+@pytest.mark.parametrize("precision", ["fp16", "int8_g64"])
+def test_logmel_product_context_parity(precision):
+    """fp16 / INT8 contexts: gam_logmel runs the tensor-core frontend that
+    gam_encode uses (3xTF32 DFT, power, filterbank and log in one kernel).  Its
+    log-mel must match the oracle element by element at the fp32 frontend's
+    tolerance on a ragged batch with a quiet clip (tones at 1e-4, noise 1e-5),
+    a loud one (tones at 0.9) and clips of 1280 samples and of a ragged number
+    of frames, with the padded frames zero."""
+    cfg, W = config_and_weights(small_model(layers=1), 34, precision)
+    lengths = [16000, 1280, 37123, 48000, 4321, 160001]
+    audio, lens = synth.random_audio(lengths, seed=19)
+    audio[0] *= 1e-3   # quiet: tones at 1e-4, noise sigma 1e-5
+    audio[3] *= 9.0    # loud: tones at 0.9
+    ctx = gam.gam_create(cfg, W, len(lens), int(max(lens)))
+    mel, frames = gam.gam_logmel(ctx, to_torch(audio), lens)
+    mel = mel.cpu().numpy()
+    worst = 0.0
+    for i, n in enumerate(lens):
+        ref = oracle.log_mel(audio[i, :n].astype(np.float64), W["frontend.window"], W["frontend.mel_fb"], cfg)
+        assert frames[i] == ref.shape[0]
+        err = max_abs(mel[i, :frames[i]], ref)
+        worst = max(worst, err)
+        assert err <= TOL_LOGMEL, (i, err)
+        assert np.all(mel[i, frames[i]:] == 0)
+    print(precision, "worst log-mel max|delta|", worst)
+    ctx.close()
+
+
 def test_logmel_shape_printed_on_pages(small_ctx):
     cfg, W, ctx = small_ctx
     audio, lens = synth.random_audio([16000], seed=8)
@@ -92,7 +120,8 @@ def test_ctc_greedy_head_parity(small_ctx):
             assert tok[b, :cnt[b]].tolist() == ref
 
 
-@pytest.mark.parametrize("precision,C", [("fp16", 34), ("fp16", 257), ("int8_g64", 257)])
+@pytest.mark.parametrize("precision,C", [("fp16", 34), ("fp16", 257), ("int8_g64", 257), ("int6_g64", 257),
+                                         ("int4_g64", 34)])
 def test_ctc_greedy_tensor_core_head(precision, C):
     """fp16 / INT8 contexts run the head on tensor cores with the fp32 frames
     split into fp16 hi + lo parts, so the activations keep ~22 bits.  fp16
@@ -100,7 +129,8 @@ def test_ctc_greedy_tensor_core_head(precision, C):
     dequantised in the mainloop and q*s is rounded once to fp16 (rms relative
     error 2^-11/sqrt(3) ~ 2.8e-4 per weight): here |z| ~ sqrt(256) * 0.02 = 0.32,
     so the logit error has sigma ~ 9e-5 and its maximum over the 38k values of
-    this test stays below ~5 sigma: bound 1e-3 for INT8."""
+    this test stays below ~5 sigma: bound 1e-3 for INT8.  The 6- and 4-bit weights
+    are dequantised the same way (one fp16 rounding of q*s), so the same bound holds."""
     cfg, W = config_and_weights(small_model(layers=1), C, precision)
     ctx = gam.gam_create(cfg, W, 6, 100000)
     rng = np.random.default_rng(C)
@@ -111,7 +141,7 @@ def test_ctc_greedy_tensor_core_head(precision, C):
     tok, cnt, logp = tok.cpu().numpy(), cnt.cpu().numpy(), logp.cpu().numpy()
     for b in range(B):
         z, lp, a = oracle.ctc_head(enc[b, :lens[b]].astype(np.float64), W)
-        assert max_abs(logp[b, :lens[b]], lp) < (1e-3 if precision == "int8_g64" else 1e-4)
+        assert max_abs(logp[b, :lens[b]], lp) < (1e-3 if precision.startswith("int") else 1e-4)
         assert np.all(logp[b, lens[b]:] == 0)
         zs = np.sort(z, axis=1) if lens[b] else np.zeros((0, 2))
         if np.all(zs[:, -1] - zs[:, -2] > 2e-3):

@@ -59,6 +59,29 @@ def test_int8_g64_round_trip_bound():
     assert np.all((g >= 126) | (s == 1.0))
 
 
+@pytest.mark.parametrize("bits,qmax", [(8, 127), (6, 31), (4, 7)])
+def test_g64_round_trip_bound_every_width(bits, qmax):
+    """q * s reproduces w within s / 2 per element at 8, 6 and 4 bits; each
+    group's largest magnitude maps to +-qmax; hand case: a group of 64 values
+    -7 .. 7 (times 0.01) at 4 bits has scale 0.01 in fp16 and q = the integers."""
+    rng = np.random.default_rng(bits)
+    w = rng.normal(0, 0.02, size=(8, 192)).astype(np.float16)
+    w[2, :64] = 0
+    q, s = synth.quantize_g64(w, bits)
+    assert q.dtype == np.int8 and np.abs(q).max() <= qmax
+    back = oracle.dequant_g64(q, s)
+    bound = np.repeat(s.astype(np.float64), 64, axis=1) / 2
+    assert np.all(np.abs(back - w.astype(np.float64)) <= bound * (1 + 1e-9) + 1e-12)
+    g = np.abs(q.reshape(8, 3, 64)).max(axis=2)
+    assert np.all((g >= qmax - 1) | (s == 1.0))
+    assert s[2, 0] == 1.0 and np.all(q[2, :64] == 0)
+    if bits == 4:
+        ints = np.tile(np.arange(-7, 8), 5)[:64].astype(np.float64)
+        q4, s4 = synth.quantize_g64((ints * 0.01)[None, :], 4)
+        assert s4[0, 0] == np.float16(0.01)
+        assert np.array_equal(q4[0], ints.astype(np.int8))
+
+
 def test_int8_weights_replace_every_linear():
     cfg = synth.model_config(dict(synth.LARGE, n_layers=1, d_model=128, n_heads=2, ffn_dim=256), 257, "int8_g64")
     W = synth.random_weights(cfg)
