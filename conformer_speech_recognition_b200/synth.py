@@ -311,3 +311,48 @@ def random_weights(cfg: dict, seed: int = 0) -> Dict[str, np.ndarray]:
             out[base + ".weight_q"] = q
             out[base + ".weight_scale"] = s
     return out
+
+
+# ---------------------------------------------------------------------------
+# RNNT head (predictor LSTM + joint network)
+# ---------------------------------------------------------------------------
+
+RNNT = dict(pred_dim=320, joint_dim=320, max_symbols=10, joint_act="relu")
+
+
+def rnnt_weight_shapes(d_model: int, n_classes: int, pred_dim: int = 320, joint_dim: int = 320) -> Dict[str, tuple]:
+    """Named tensors of the RNNT head, PyTorch layout (embedding [C, P], LSTM
+    weight_ih_l0 / weight_hh_l0 [4P, P] with two biases, Linear [out, in])."""
+    P, J, C = pred_dim, joint_dim, n_classes
+    return {"rnnt.embed.weight": (C, P),
+            "rnnt.lstm.weight_ih_l0": (4 * P, P), "rnnt.lstm.weight_hh_l0": (4 * P, P),
+            "rnnt.lstm.bias_ih_l0": (4 * P,), "rnnt.lstm.bias_hh_l0": (4 * P,),
+            "rnnt.joint.enc.weight": (J, d_model), "rnnt.joint.enc.bias": (J,),
+            "rnnt.joint.pred.weight": (J, P), "rnnt.joint.pred.bias": (J,),
+            "rnnt.joint.out.weight": (C, J), "rnnt.joint.out.bias": (C,)}
+
+
+def random_rnnt_weights(d_model: int, n_classes: int, seed: int = 7, pred_dim: int = 320, joint_dim: int = 320,
+                        blank_bias: float = 7.0) -> Dict[str, np.ndarray]:
+    """Seeded RNNT head weights, fp16.  Recipe: embedding N(0, 0.5); LSTM
+    weights and both biases N(0, 0.05); joint enc / pred weights N(0, 0.05) and
+    biases N(0, 0.02); joint out weights N(0, 0.1) and bias N(0, 0.1), plus
+    `blank_bias` on the blank row (last class).  Random weights alone would
+    rarely pick blank among 34 or 1025 classes, and the weak predictor path lets
+    a frame that picks a symbol repeat it up to the per-frame cap; with the
+    default offset, unit-variance encoder frames give about 0.7 (34 classes) to
+    1.7 (1025 classes) symbols per frame on average, the order of a character
+    or piece rate of speech at 40 ms frames."""
+    rng = np.random.Generator(np.random.PCG64(seed))
+    sd = {"rnnt.embed.weight": 0.5, "rnnt.lstm.weight_ih_l0": 0.05, "rnnt.lstm.weight_hh_l0": 0.05,
+          "rnnt.lstm.bias_ih_l0": 0.05, "rnnt.lstm.bias_hh_l0": 0.05, "rnnt.joint.enc.weight": 0.05,
+          "rnnt.joint.enc.bias": 0.02, "rnnt.joint.pred.weight": 0.05, "rnnt.joint.pred.bias": 0.02,
+          "rnnt.joint.out.weight": 0.1, "rnnt.joint.out.bias": 0.1}
+    out = {}
+    for name, shape in rnnt_weight_shapes(d_model, n_classes, pred_dim, joint_dim).items():
+        v = rng.normal(0.0, sd[name], size=shape)
+        if name == "rnnt.joint.out.bias":
+            v[-1] += blank_bias
+        out[name] = v.astype(np.float16)
+    return out
+
