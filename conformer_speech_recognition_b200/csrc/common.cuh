@@ -105,7 +105,8 @@ enum ProfKind {
   PK_FRONTEND = 0, PK_GEMM_SUB = 1, PK_GEMM_FFN_UP = 2, PK_GEMM_FFN_DOWN = 3, PK_GEMM_QKV = 4,
   PK_GEMM_OUT = 5, PK_GEMM_PW1 = 6, PK_GEMM_PW2 = 7, PK_ATTENTION = 8, PK_LAYERNORM = 9,
   PK_DWCONV = 10, PK_CTC_GEMM = 11, PK_CTC_SOFTMAX = 12, PK_CTC_COLLAPSE = 13, PK_MISC = 14,
-  PK_COUNT = 15
+  PK_RNNT_ENC_PROJ = 15, PK_RNNT_DECODE = 16,
+  PK_COUNT = 17
 };
 
 // Weight operand of a GEMM: [N, K] row-major (PyTorch Linear layout).
@@ -159,6 +160,18 @@ cudaError_t launch_split_hi_lo(const float* enc, const int* off, int batch, int 
 cudaError_t launch_collapse(const int* argmax, const int* lens, int batch, int t_max, int blank,
                             int* tokens, int* counts, cudaStream_t s);
 cudaError_t launch_f32_to_f16(const float* in, __half* out, int64_t n, cudaStream_t s);
+
+// Greedy RNNT decoding (rnnt.cu), one CTA per clip.  eproj [rows][J]: the joint's
+// encoder projection per valid frame (row off[b] + t, or b * t_max + t when off
+// is NULL); gtab [(C + 1)][4P]: LSTM input gates per symbol (row C: zero start
+// input); whhT [P][4P], wpT [P][J], woT [J][C] fp16 (transposed weights); act
+// 0 ReLU, 1 tanh.  Writes tokens / frames ([B][max_tokens], -1 after the last
+// symbol; frames may be NULL) and counts [B].
+size_t rnnt_smem_bytes(int C, int P, int J);
+cudaError_t launch_rnnt_greedy(const float* eproj, const int* lens, const int* off, int batch, int t_max,
+                               const float* gtab, const __half* whhT, const __half* wpT, const float* bp,
+                               const __half* woT, const float* bo, int C, int P, int J, int max_symbols, int act,
+                               int max_tokens, int* tokens, int* frames, int* counts, cudaStream_t s);
 
 }  // namespace gam
 

@@ -25,7 +25,8 @@ thread_local std::string g_create_error;
 const char* kKindNames[PK_COUNT] = {"frontend",  "gemm_subsampling", "gemm_ffn_up",  "gemm_ffn_down",
                                     "gemm_qkv",  "gemm_attn_out",    "gemm_pw1_glu", "gemm_pw2",
                                     "attention", "layernorm",        "dwconv",       "ctc_gemm",
-                                    "ctc_softmax_argmax", "ctc_collapse", "misc"};
+                                    "ctc_softmax_argmax", "ctc_collapse", "misc", "rnnt_enc_proj",
+                                    "rnnt_decode"};
 
 inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 inline int64_t round_up(int64_t a, int64_t b) { return ceil_div(a, b) * b; }
@@ -68,6 +69,21 @@ struct DevLayer {
   DevLinear ffn1_up, ffn1_down, qkv, out, pw1, pw2, ffn2_up, ffn2_down;
   float* dw_w = nullptr;  // [K][d], BatchNorm folded
   float* dw_b = nullptr;  // [d]
+};
+
+// RNNT head (gam_rnnt_attach): the joint's encoder projection as a GEMM weight,
+// the LSTM input-gate table per symbol and transposed fp16 weights of the
+// sequential part.
+struct RnntHead {
+  int C = 0, P = 0, E = 0, J = 0, max_symbols = 0, act = 0;
+  DevLinear enc;            // fp16 modes: [W_enc | W_enc] rows padded to 256, K = 2d; fp32 mode: W_enc
+  float* gtab = nullptr;    // [(C + 1)][4P]
+  __half* whhT = nullptr;   // [P][4P]
+  __half* wpT = nullptr;    // [P][J]
+  float* bp = nullptr;      // [J]
+  __half* woT = nullptr;    // [J][C]
+  float* bo = nullptr;      // [C]
+  float* eproj = nullptr;   // [max_batch * T2_cap][J]
 };
 
 struct Prof {
@@ -165,6 +181,7 @@ struct gam_ctx {
   cudaStream_t last_stream = nullptr;
   // tcgen05 GEMM plans
   TcGemmCache tc;
+  RnntHead rnnt;
   Prof prof;
   GraphCache graphs;
   int inject_err = 0, inject_count = 0;
@@ -225,14 +242,21 @@ struct WeightTable {
   std::map<std::string, const gam_tensor*> by_name;
 };
 
+// shape entries of -1 accept any positive extent of at most max_free (when max_free > 0)
 gam_status find(gam_ctx* c, const WeightTable& t, const std::string& name, std::vector<int64_t> shape,
-                const gam_tensor** out, bool allow_trailing_one = false) {
+                const gam_tensor** out, bool allow_trailing_one = false, int64_t max_free = 0) {
   auto it = t.by_name.find(name);
   if (it == t.by_name.end()) return fail(c, GAM_ERR_WEIGHTS, "missing tensor " + name);
   const gam_tensor* g = it->second;
   std::vector<int64_t> got(g->shape, g->shape + std::max(0, std::min(g->ndim, 4)));
   if (allow_trailing_one && got.size() == shape.size() + 1 && got.back() == 1) got.pop_back();
-  if (got != shape || g->data == nullptr) {
+  bool free_ok = got.size() == shape.size();
+  for (size_t i = 0; free_ok && i < shape.size(); ++i)
+    if (shape[i] == -1) {
+      free_ok = got[i] >= 1 && (max_free <= 0 || got[i] <= max_free);
+      shape[i] = got[i];
+    }
+  if (!free_ok || got != shape || g->data == nullptr) {
     std::string s = "tensor " + name + " has shape [";
     for (auto v : got) s += std::to_string(v) + ",";
     s += "], expected [";
@@ -1090,6 +1114,136 @@ void destroy(gam_ctx* c) {
   delete c;
 }
 
+gam_status rnnt_attach(gam_ctx* c, const gam_rnnt_config& rc, const gam_tensor* tensors, int n) {
+  const int d = c->cfg.d_model;
+  const int C = rc.n_classes, P = rc.pred_dim, J = rc.joint_dim;
+  if (C < 2 || C > 4096 || P < 2 || P > 1024 || (P & 1) || J < 2 || J > 1024 || (J & 1) || rc.max_symbols < 1 ||
+      rc.max_symbols > 64 || (rc.joint_act != 0 && rc.joint_act != 1))
+    return fail(c, GAM_ERR_INVALID_ARG, "rnnt config: n_classes 2..4096, even pred_dim / joint_dim <= 1024, "
+                                        "max_symbols 1..64, joint_act 0 or 1");
+  if (rnnt_smem_bytes(C, P, J) > 200 * 1024) return fail(c, GAM_ERR_INVALID_ARG, "rnnt head too large");
+  WeightTable t;
+  for (int i = 0; i < n; ++i) {
+    if (!tensors[i].name) return fail(c, GAM_ERR_WEIGHTS, "tensor without a name");
+    t.by_name[tensors[i].name] = &tensors[i];
+  }
+  const gam_tensor* ge;
+  GAM_TRY(find(c, t, "rnnt.embed.weight", {C, -1}, &ge, false, 4096));
+  const int E = (int)ge->shape[1];
+  std::vector<double> emb, wih, whh, bih, bhh, we, be, wp, bp, wo, bo;
+  GAM_TRY(read_f(c, ge, emb));
+  const gam_tensor* g;
+  GAM_TRY(find(c, t, "rnnt.lstm.weight_ih_l0", {4 * P, E}, &g));
+  GAM_TRY(read_f(c, g, wih));
+  GAM_TRY(find(c, t, "rnnt.lstm.weight_hh_l0", {4 * P, P}, &g));
+  GAM_TRY(read_f(c, g, whh));
+  GAM_TRY(get_vec(c, t, "rnnt.lstm.bias_ih_l0", 4 * P, bih));
+  GAM_TRY(get_vec(c, t, "rnnt.lstm.bias_hh_l0", 4 * P, bhh));
+  GAM_TRY(find(c, t, "rnnt.joint.enc.weight", {J, d}, &g));
+  GAM_TRY(read_f(c, g, we));
+  GAM_TRY(get_vec(c, t, "rnnt.joint.enc.bias", J, be));
+  GAM_TRY(find(c, t, "rnnt.joint.pred.weight", {J, P}, &g));
+  GAM_TRY(read_f(c, g, wp));
+  GAM_TRY(get_vec(c, t, "rnnt.joint.pred.bias", J, bp));
+  GAM_TRY(find(c, t, "rnnt.joint.out.weight", {C, J}, &g));
+  GAM_TRY(read_f(c, g, wo));
+  GAM_TRY(get_vec(c, t, "rnnt.joint.out.bias", C, bo));
+  RnntHead& r = c->rnnt;
+  if (r.gtab) return fail(c, GAM_ERR_INVALID_ARG, "an RNNT head is attached already");
+  // input gates per symbol, emb[k] W_ih^T + b_ih + b_hh (both biases), and the start row (zero input)
+  std::vector<double> gt((size_t)(C + 1) * 4 * P);
+  for (int k = 0; k <= C; ++k)
+    for (int row = 0; row < 4 * P; ++row) {
+      double v = bih[row] + bhh[row];
+      if (k < C)
+        for (int e = 0; e < E; ++e) v += emb[(size_t)k * E + e] * wih[(size_t)row * E + e];
+      gt[(size_t)k * 4 * P + row] = v;
+    }
+  auto transpose_h = [](const std::vector<double>& w, int rows, int cols) {  // [rows][cols] -> [cols][rows] fp16
+    std::vector<__half> o((size_t)rows * cols);
+    for (int i = 0; i < rows; ++i)
+      for (int j = 0; j < cols; ++j) o[(size_t)j * rows + i] = __float2half_rn((float)w[(size_t)i * cols + j]);
+    return o;
+  };
+  std::vector<__half> whhT = transpose_h(whh, 4 * P, P), wpT = transpose_h(wp, J, P), woT = transpose_h(wo, C, J);
+  GAM_TRY(upload_f32(c, &r.gtab, gt));
+  GAM_TRY(upload(c, &r.whhT, whhT.data(), whhT.size() * sizeof(__half)));
+  GAM_TRY(upload(c, &r.wpT, wpT.data(), wpT.size() * sizeof(__half)));
+  GAM_TRY(upload_f32(c, &r.bp, bp));
+  GAM_TRY(upload(c, &r.woT, woT.data(), woT.size() * sizeof(__half)));
+  GAM_TRY(upload_f32(c, &r.bo, bo));
+  HostLinear hl;
+  if (c->cfg.precision == GAM_FP32) {
+    hl.N = J;
+    hl.K = d;
+    hl.dtype = 0;
+    hl.w = we;
+    hl.b = be;
+  } else {
+    // [W | W] against the fp16 hi / lo split of the frames (as the CTC head): fp32-grade projection
+    const int Np = (int)round_up(J, 256);
+    hl.N = Np;
+    hl.K = 2 * d;
+    hl.dtype = 1;
+    hl.b.assign(Np, 0.0);
+    hl.w.assign((size_t)Np * 2 * d, 0.0);
+    for (int j = 0; j < J; ++j) {
+      hl.b[j] = be[j];
+      for (int h = 0; h < 2; ++h)
+        std::memcpy(&hl.w[(size_t)j * 2 * d + h * d], &we[(size_t)j * d], d * sizeof(double));
+    }
+  }
+  GAM_TRY(upload_linear(c, hl, r.enc));
+  GAM_TRY(dev_alloc(c, (void**)&r.eproj, (size_t)c->cfg.max_batch * c->T2_cap * J * 4));
+  r.C = C;
+  r.P = P;
+  r.E = E;
+  r.J = J;
+  r.max_symbols = rc.max_symbols;
+  r.act = rc.joint_act;
+  return cuda_check(c, cudaDeviceSynchronize(), "rnnt attach sync");
+}
+
+gam_status rnnt_greedy(gam_ctx* c, const float* enc, const int32_t* enc_len, int batch, int t_max, int max_tokens,
+                       int32_t* tokens, int32_t* frames, int32_t* counts, cudaStream_t s) {
+  const gam_config& cfg = c->cfg;
+  RnntHead& r = c->rnnt;
+  if (!r.gtab) return fail(c, GAM_ERR_INVALID_ARG, "no RNNT head attached (gam_rnnt_attach)");
+  if (!enc || !enc_len || !tokens || !counts) return fail(c, GAM_ERR_INVALID_ARG, "null pointer");
+  if (batch < 1 || t_max < 1 || max_tokens < 1) return fail(c, GAM_ERR_INVALID_ARG, "batch, t_max, max_tokens >= 1");
+  if (batch > cfg.max_batch || t_max > c->T2_cap) return fail(c, GAM_ERR_CAPACITY, "batch or t_max above capacity");
+  for (int i = 0; i < batch; ++i)
+    if (enc_len[i] < 0 || enc_len[i] > t_max) return fail(c, GAM_ERR_SHAPE, "enc_len outside [0, t_max]");
+  c->last_stream = s;
+  std::vector<int32_t> lo(2 * batch + 1);
+  for (int i = 0; i < batch; ++i) lo[i] = enc_len[i];
+  lo[batch] = 0;
+  for (int i = 0; i < batch; ++i) lo[batch + 1 + i] = lo[batch + i] + enc_len[i];
+  const int M_valid = lo[2 * batch];
+  const int* dev;
+  GAM_TRY(upload_ints(c, lo.data(), 2 * batch + 1, s, &dev));
+  const int* lens = dev;
+  const int* off = dev + batch;
+  Clips none{nullptr, 0};
+  if (cfg.precision != GAM_FP32) {
+    if (M_valid > 0) {
+      GAM_TRY(run_kernel(c, PK_RNNT_ENC_PROJ, s, [&] {
+        return launch_split_hi_lo(enc, off, batch, t_max, cfg.d_model, M_valid, c->ctc_a, s);
+      }));
+      GAM_TRY(gemm(c, PK_RNNT_ENC_PROJ, s, c->ctc_a, nullptr, 0, 2 * cfg.d_model, r.enc, M_valid, EPI_F32, 1.f,
+                   r.eproj, r.J, none, 0, r.J));
+    }
+  } else {
+    GAM_TRY(gemm(c, PK_RNNT_ENC_PROJ, s, enc, nullptr, 0, cfg.d_model, r.enc, batch * t_max, EPI_F32, 1.f, r.eproj,
+                 r.J, none, 1));
+    off = nullptr;  // rows b * t_max + t
+  }
+  return run_kernel(c, PK_RNNT_DECODE, s, [&] {
+    return launch_rnnt_greedy(r.eproj, lens, off, batch, t_max, r.gtab, r.whhT, r.wpT, r.bp, r.woT, r.bo, r.C, r.P,
+                              r.J, r.max_symbols, r.act, max_tokens, tokens, frames, counts, s);
+  });
+}
+
 gam_status enter(gam_ctx* c) {
   if (!c) return GAM_ERR_INVALID_ARG;
   c->err.clear();
@@ -1367,6 +1521,18 @@ gam_status gam_debug_gemm(gam_ctx* c, int impl, const void* a, int lda, const vo
   }
   if (k % 16 || n % 128) return fail(c, GAM_ERR_SHAPE, "CUDA-core GEMM needs N % 128 == 0, K % 16 == 0");
   return run_kernel(c, PK_MISC, s, [&] { return launch_gemm_simt(1, a, nullptr, 0, lda, W, m, n, k, EPI_RESID, 0, ep, s); });
+}
+
+gam_status gam_rnnt_attach(gam_ctx* c, const gam_rnnt_config* cfg, const gam_tensor* tensors, int n_tensors) {
+  GAM_TRY(enter(c));
+  if (!cfg || !tensors || n_tensors <= 0) return fail(c, GAM_ERR_INVALID_ARG, "null config or no tensors");
+  return rnnt_attach(c, *cfg, tensors, n_tensors);
+}
+
+gam_status gam_rnnt_greedy(gam_ctx* c, const float* enc, const int32_t* enc_len, int batch, int t_max,
+                           int max_tokens, int32_t* tokens, int32_t* frames, int32_t* counts, void* stream) {
+  GAM_TRY(enter(c));
+  return rnnt_greedy(c, enc, enc_len, batch, t_max, max_tokens, tokens, frames, counts, (cudaStream_t)stream);
 }
 
 gam_status gam_debug_wait_timeout(gam_ctx* c, int64_t limit_ns, int skip_k_block) {

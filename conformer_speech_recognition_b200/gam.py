@@ -30,6 +30,7 @@ EXPORTS = ("gam_status_string", "gam_last_error", "gam_plan_lengths", "gam_creat
            "gam_encode", "gam_encode_stage", "gam_ctc_greedy", "gam_ctc_collapse", "gam_transcribe",
            "gam_device_status", "gam_profile_enable", "gam_profile_reset", "gam_profile_kinds",
            "gam_profile_kind_name", "gam_profile_read", "gam_graphs_enable", "gam_ctc_collapse_noalloc",
+           "gam_rnnt_attach", "gam_rnnt_greedy",
            "gam_debug_gemm", "gam_debug_wait_timeout", "gam_debug_inject_cuda_error")
 
 GAM_NOALLOC_MAX_FRAMES = 1 << 20
@@ -42,6 +43,11 @@ class GamConfig(ctypes.Structure):
                 ("sub_kernel", ctypes.c_int), ("n_classes", ctypes.c_int), ("rope_base", ctypes.c_float),
                 ("ln_eps", ctypes.c_float), ("bn_eps", ctypes.c_float), ("precision", ctypes.c_int),
                 ("max_batch", ctypes.c_int), ("max_samples", ctypes.c_int64)]
+
+
+class GamRnntConfig(ctypes.Structure):
+    _fields_ = [("n_classes", ctypes.c_int), ("pred_dim", ctypes.c_int), ("joint_dim", ctypes.c_int),
+                ("max_symbols", ctypes.c_int), ("joint_act", ctypes.c_int)]
 
 
 class GamTensor(ctypes.Structure):
@@ -91,6 +97,8 @@ def lib() -> ctypes.CDLL:
         L.gam_profile_read.argtypes = [vp, ctypes.c_int, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_int64)]
         L.gam_graphs_enable.argtypes = [vp, ctypes.c_int]
         L.gam_ctc_collapse_noalloc.argtypes = [vp, vp, ctypes.c_int, ctypes.c_int, ctypes.c_int, vp, vp, vp]
+        L.gam_rnnt_attach.argtypes = [vp, ctypes.POINTER(GamRnntConfig), ctypes.POINTER(GamTensor), ctypes.c_int]
+        L.gam_rnnt_greedy.argtypes = [vp, vp, i32p, ctypes.c_int, ctypes.c_int, ctypes.c_int, vp, vp, vp, vp]
         L.gam_debug_gemm.argtypes = [vp, ctypes.c_int, vp, ctypes.c_int, vp, vp, ctypes.c_int, ctypes.c_int,
                                      ctypes.c_int, vp, ctypes.c_int, vp]
         L.gam_debug_wait_timeout.argtypes = [vp, ctypes.c_int64, ctypes.c_int]
@@ -372,6 +380,42 @@ def gam_ctc_collapse_noalloc(logits, lengths_dev, tokens, counts, stream=None):
     _check(lib().gam_ctc_collapse_noalloc(logits.data_ptr(), lengths_dev.data_ptr(), B, T, C, tokens.data_ptr(),
                                           counts.data_ptr(), _stream(stream)))
     return tokens, counts
+
+
+def gam_rnnt_attach(ctx: Context, rnnt_cfg: dict, weights: Dict[str, np.ndarray]):
+    """Attach the RNNT head: rnnt_cfg has n_classes, pred_dim, joint_dim,
+    max_symbols and joint_act ("relu" or "tanh"); weights named as in gam.h."""
+    act = rnnt_cfg.get("joint_act", "relu")
+    c = GamRnntConfig(int(rnnt_cfg["n_classes"]), int(rnnt_cfg.get("pred_dim", 320)),
+                      int(rnnt_cfg.get("joint_dim", 320)), int(rnnt_cfg.get("max_symbols", 10)),
+                      0 if act in ("relu", 0) else 1)
+    arr, keep = _tensor_table(weights)
+    _check(lib().gam_rnnt_attach(ctx.handle, ctypes.byref(c), arr, len(weights)), ctx)
+    del keep
+    ctx.rnnt_cfg = dict(rnnt_cfg)
+
+
+def gam_rnnt_greedy(ctx: Context, enc, enc_len, max_tokens: Optional[int] = None, stream=None, tokens=None,
+                    frames=None, counts=None):
+    """Greedy RNNT decoding of enc [B, T, d]: (tokens [B, max_tokens], frames
+    [B, max_tokens], counts [B]) as CUDA int32 tensors."""
+    import torch
+    el = _i32(enc_len)
+    _dev_tensor(enc, torch.float32, "enc")
+    B, tmax, _ = enc.shape
+    if max_tokens is None:
+        max_tokens = tmax * int(ctx.rnnt_cfg.get("max_symbols", 10))
+    if tokens is None:
+        tokens = torch.empty((B, max_tokens), dtype=torch.int32, device=enc.device)
+    if frames is None:
+        frames = torch.empty((B, max_tokens), dtype=torch.int32, device=enc.device)
+    if counts is None:
+        counts = torch.empty((B,), dtype=torch.int32, device=enc.device)
+    for t, n in ((tokens, "tokens"), (frames, "frames"), (counts, "counts")):
+        _dev_tensor(t, torch.int32, n, enc.device)
+    _check(lib().gam_rnnt_greedy(ctx.handle, enc.data_ptr(), _ptr_i32(el), B, tmax, int(max_tokens),
+                                 tokens.data_ptr(), frames.data_ptr(), counts.data_ptr(), _stream(stream)), ctx)
+    return tokens, frames, counts
 
 
 def gam_graphs_enable(ctx: Context, on: bool = True):

@@ -245,6 +245,50 @@ const char* gam_profile_kind_name(int kind);
  * events).  Launch counts are kept even when timing is off. */
 gam_status gam_profile_read(gam_ctx* ctx, int kind, double* total_ms, int64_t* launches);
 
+/* ---- RNNT head ---- */
+
+/* RNNT head of the v3 RNNT and E2E RNNT models ("GigaAM on MLX: the
+ * transcripts matched, but the model was broken", "What we're porting": a
+ * single-layer LSTM of size 320 plus a joint network; "Trap 4" and "GigaAM v3
+ * RNNT -- MLX (Apple Silicon)", "Notes for other runtimes": PyTorch LSTM
+ * weights, bias = bias_ih + bias_hh, blank = len(vocabulary); "GigaAM v3 MLX",
+ * "Architecture details": greedy RNNT decoding, 1025 classes with blank 1024). */
+typedef struct {
+  int n_classes;    /* vocabulary + 1; blank = n_classes - 1 (34 or 1025); <= 4096        */
+  int pred_dim;     /* LSTM hidden size P (320), even                                      */
+  int joint_dim;    /* joint hidden width J (320), even                                    */
+  int max_symbols;  /* symbols emitted per encoder frame at most (10), 1..64               */
+  int joint_act;    /* 0: ReLU, 1: tanh, applied to W_enc f + b_enc + W_pred g + b_pred     */
+} gam_rnnt_config;
+
+/* Attach an RNNT head to a context (once).  Tensors, HOST memory, f16 or f32,
+ * PyTorch layout: "rnnt.embed.weight" [C, E], "rnnt.lstm.weight_ih_l0"
+ * [4P, E], "rnnt.lstm.weight_hh_l0" [4P, P], "rnnt.lstm.bias_ih_l0" and
+ * "rnnt.lstm.bias_hh_l0" [4P] (gate order i, f, g, o), "rnnt.joint.enc.weight"
+ * [J, d_model], "rnnt.joint.enc.bias" [J], "rnnt.joint.pred.weight" [J, P],
+ * "rnnt.joint.pred.bias" [J], "rnnt.joint.out.weight" [C, J],
+ * "rnnt.joint.out.bias" [C].  The head's weights stay fp16 / fp32 in every
+ * precision.  Allocates device memory (weights, a per-symbol table of the
+ * LSTM's input gates and a projection buffer for max_batch clips) and
+ * synchronises the device once. */
+gam_status gam_rnnt_attach(gam_ctx* ctx, const gam_rnnt_config* cfg, const gam_tensor* tensors, int n_tensors);
+
+/* Greedy RNNT decoding of encoder output.  enc_dev: device f32 [batch, t_max,
+ * d] (gam_encode's output), clip i valid on its first enc_len_host[i] frames.
+ * The predictor starts from a zero input and zero state and takes the
+ * embedding of each emitted symbol; at frame t the decoder repeats {joint
+ * logits = W_out act(W_enc f_t + b_enc + W_pred g + b_pred) + b_out; argmax,
+ * lowest index on ties; blank -> next frame, else emit} with at most
+ * max_symbols symbols per frame.  tokens_dev device i32 [batch, max_tokens]:
+ * the symbols, -1 after the last; frames_dev (optional, device i32 [batch,
+ * max_tokens]): the encoder frame of each symbol, -1 after the last;
+ * counts_dev device i32 [batch]: symbols stored (at most max_tokens; symbols
+ * past max_tokens are decoded but not stored, and t_max * max_symbols never
+ * loses any). */
+gam_status gam_rnnt_greedy(gam_ctx* ctx, const float* enc_dev, const int32_t* enc_len_host, int batch, int t_max,
+                           int max_tokens, int32_t* tokens_dev, int32_t* frames_dev, int32_t* counts_dev,
+                           void* stream);
+
 /* ---- greedy decoding without any allocation ---- */
 
 /* Frames of the fixed scratch array behind gam_ctc_collapse_noalloc. */

@@ -1,0 +1,100 @@
+"""GPU parity of the RNNT head (gam_rnnt_attach / gam_rnnt_greedy) against the
+oracle's greedy decoding, through the C ABI.
+
+The decoder takes a discrete decision at every step, so symbols and frames are
+compared exactly on every clip whose oracle path never came within GAP of a
+tie between its two best logits (the GPU computes in fp32 from the same fp16
+weights; its logits differ from the fp64 oracle's by ~1e-6 here, far below
+GAP).  Clips closer to a tie are reported, and nearly all clips must qualify."""
+import numpy as np
+import pytest
+
+import oracle
+from conformer_speech_recognition_b200 import gam, synth
+from gpu_common import config_and_weights, small_model, to_torch
+
+pytestmark = pytest.mark.gpu
+
+GAP = 1e-3
+
+
+def _compare(enc, lens, Wr, C, tok, fr, cnt, max_symbols=10, act="relu", min_checked=0.75):
+    tok, fr, cnt = tok.cpu().numpy(), fr.cpu().numpy(), cnt.cpu().numpy()
+    checked = 0
+    for b in range(len(lens)):
+        sym, frames, gap = oracle.rnnt_greedy_clip(enc[b, :lens[b]].astype(np.float64), Wr, C, max_symbols, act)
+        assert np.all(tok[b, cnt[b]:] == -1) and np.all(fr[b, cnt[b]:] == -1)
+        if gap <= GAP:
+            print("clip", b, "skipped: oracle path within", gap, "of a tie")
+            continue
+        checked += 1
+        assert cnt[b] == len(sym), (b, cnt[b], len(sym))
+        assert tok[b, :cnt[b]].tolist() == sym, b
+        assert fr[b, :cnt[b]].tolist() == frames, b
+    assert checked >= min_checked * len(lens), (checked, len(lens))
+    return checked
+
+
+@pytest.mark.parametrize("precision,C,act", [("fp16", 34, "relu"), ("fp16", 1025, "relu"), ("int8_g64", 257, "relu"),
+                                             ("fp32", 34, "relu"), ("fp16", 34, "tanh")])
+def test_rnnt_greedy_matches_oracle(precision, C, act):
+    cfg, W = config_and_weights(small_model(layers=1), 34, precision)
+    d = cfg["d_model"]
+    B, T = 6, 60
+    ctx = gam.gam_create(cfg, W, B, 40000)
+    Wr = synth.random_rnnt_weights(d, C, seed=C)
+    gam.gam_rnnt_attach(ctx, dict(n_classes=C, pred_dim=320, joint_dim=320, max_symbols=10, joint_act=act), Wr)
+    rng = np.random.default_rng(C + 1)
+    enc = rng.normal(size=(B, T, d)).astype(np.float32)
+    lens = np.array([60, 1, 0, 37, 59, 12], np.int32)
+    tok, fr, cnt = gam.gam_rnnt_greedy(ctx, to_torch(enc), lens)
+    n = _compare(enc, lens, Wr, C, tok, fr, cnt, act=act)
+    print(precision, C, act, "clips compared", n, "symbols", cnt.cpu().numpy().tolist())
+    ctx.close()
+
+
+def test_rnnt_max_tokens_truncates_and_max_symbols_caps():
+    cfg, W = config_and_weights(small_model(layers=1), 34, "fp16")
+    d = cfg["d_model"]
+    ctx = gam.gam_create(cfg, W, 2, 40000)
+    C = 34
+    Wr = synth.random_rnnt_weights(d, C, seed=3, blank_bias=2.0)  # frequent symbols: runs reach the cap
+    gam.gam_rnnt_attach(ctx, dict(n_classes=C, max_symbols=3), Wr)
+    enc = np.random.default_rng(4).normal(size=(2, 40, d)).astype(np.float32)
+    lens = np.array([40, 25], np.int32)
+    tok, fr, cnt = gam.gam_rnnt_greedy(ctx, to_torch(enc), lens)
+    _compare(enc, lens, Wr, C, tok, fr, cnt, max_symbols=3, min_checked=0.5)
+    f = fr.cpu().numpy()
+    for b in range(2):
+        counts = np.bincount(f[b, :cnt[b].item()], minlength=40)
+        assert counts.max() <= 3
+    full_tok, full_cnt = tok.cpu().numpy(), cnt.cpu().numpy()
+    tok5, fr5, cnt5 = gam.gam_rnnt_greedy(ctx, to_torch(enc), lens, max_tokens=5)
+    cnt5 = cnt5.cpu().numpy()
+    assert np.array_equal(cnt5, np.minimum(full_cnt, 5))
+    for b in range(2):
+        assert tok5.cpu().numpy()[b, :cnt5[b]].tolist() == full_tok[b, :cnt5[b]].tolist()
+    ctx.close()
+
+
+def test_rnnt_on_c2_encoder_output():
+    """Full-size batch: the 32 variable-length clips of the C2 workload through the
+    16-layer d768 encoder, then the 34-class RNNT head of the v3 RNNT model
+    shape; the oracle decodes sampled clips from the same encoder output."""
+    name = "c2_varlen_b32_d768"
+    cfg = synth.workload_config(name)
+    _, W = config_and_weights(synth.V3, 34, "fp16")
+    audio, lens = synth.workload_audio(name)
+    ctx = gam.gam_create(cfg, W, 32, int(lens.max()))
+    Wr = synth.random_rnnt_weights(cfg["d_model"], 34)
+    gam.gam_rnnt_attach(ctx, dict(n_classes=34), Wr)
+    enc, el = gam.gam_encode(ctx, to_torch(audio), lens)
+    tok, fr, cnt = gam.gam_rnnt_greedy(ctx, enc, el)
+    enc_h = enc.cpu().numpy()
+    order = np.argsort(lens)
+    sample = [order[0], order[len(order) // 2], order[-1]]
+    sub = lambda x: x[sample]  # noqa: E731
+    n = _compare(enc_h[sample], el[sample], Wr, 34, sub(tok), sub(fr), sub(cnt), min_checked=0.6)
+    print("C2 RNNT clips compared", n, "symbols per clip", cnt.cpu().numpy().tolist())
+    gam.gam_device_status(ctx)
+    ctx.close()
