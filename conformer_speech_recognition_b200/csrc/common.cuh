@@ -157,8 +157,9 @@ cudaError_t launch_logsoftmax_argmax(const float* logits, int ld, const int* len
 // split into fp16 hi and lo parts: a[v, c] = hi, a[v, d + c] = lo (x ~= hi + lo).
 cudaError_t launch_split_hi_lo(const float* enc, const int* off, int batch, int t_max, int d, int rows,
                                __half* a, cudaStream_t s);
+// frames (optional): the first frame of each token's run, -1 after the last token.
 cudaError_t launch_collapse(const int* argmax, const int* lens, int batch, int t_max, int blank,
-                            int* tokens, int* counts, cudaStream_t s);
+                            int* tokens, int* counts, cudaStream_t s, int* frames = nullptr);
 cudaError_t launch_f32_to_f16(const float* in, __half* out, int64_t n, cudaStream_t s);
 
 // Greedy RNNT decoding (rnnt.cu), one CTA per clip.  eproj [rows][J]: the joint's

@@ -414,7 +414,7 @@ __global__ void logsoftmax_argmax_kernel(const float* __restrict__ logits, int l
 // exclusive scan of keep flags over contiguous per-thread chunks, compaction.
 __global__ void __launch_bounds__(256)
 collapse_kernel(const int* __restrict__ argmax, const int* __restrict__ lens, int t_max, int blank,
-                int* __restrict__ tokens, int* __restrict__ counts) {
+                int* __restrict__ tokens, int* __restrict__ counts, int* __restrict__ frames) {
   pdl_launch_dependents();
   pdl_wait();
   __shared__ int warp_tot[8];
@@ -446,12 +446,19 @@ collapse_kernel(const int* __restrict__ argmax, const int* __restrict__ lens, in
   __syncthreads();
   int pos = warp_tot[w] + inc - cnt;
   int* tok = tokens + (size_t)b * t_max;
+  int* frm = frames ? frames + (size_t)b * t_max : nullptr;
   for (int t = t0; t < t1; ++t) {
     const int v = a[t];
-    if (v != blank && (t == 0 || v != a[t - 1])) tok[pos++] = v;
+    if (v != blank && (t == 0 || v != a[t - 1])) {
+      if (frm) frm[pos] = t;  // the first frame of the symbol's run
+      tok[pos++] = v;
+    }
   }
   const int total = s_total;
-  for (int t = total + tid; t < t_max; t += 256) tok[t] = -1;
+  for (int t = total + tid; t < t_max; t += 256) {
+    tok[t] = -1;
+    if (frm) frm[t] = -1;
+  }
   if (tid == 0) counts[b] = total;
 }
 
@@ -612,8 +619,8 @@ cudaError_t launch_split_hi_lo(const float* enc, const int* off, int batch, int 
 }
 
 cudaError_t launch_collapse(const int* argmax, const int* lens, int batch, int t_max, int blank, int* tokens,
-                            int* counts, cudaStream_t s) {
-  return launch_pdl(collapse_kernel, batch, 256, 0, s, argmax, lens, t_max, blank, tokens, counts);
+                            int* counts, cudaStream_t s, int* frames) {
+  return launch_pdl(collapse_kernel, batch, 256, 0, s, argmax, lens, t_max, blank, tokens, counts, frames);
 }
 
 cudaError_t launch_f32_to_f16(const float* in, __half* out, int64_t n, cudaStream_t s) {

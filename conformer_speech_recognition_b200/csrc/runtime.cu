@@ -187,6 +187,25 @@ struct gam_ctx {
   int inject_err = 0, inject_count = 0;
 };
 
+// Pseudo-streaming state (gam_stream_*): the last `window` samples of the audio
+// pushed so far, in one of two device buffers (each push writes the new window
+// into the other one, so in steady state the encoder sees two alternating
+// pointers and its CUDA graphs replay), plus the per-step outputs.
+struct gam_stream {
+  gam_ctx* ctx = nullptr;
+  int64_t window = 0;   // samples kept (at most 30 s at 16 kHz by default)
+  int64_t len = 0;      // samples in the current window
+  int64_t total = 0;    // samples pushed since the last reset
+  int cur = 0;          // buffer holding the window
+  float* buf[2] = {nullptr, nullptr};
+  float* enc = nullptr;    // [1][T'(window)][d]
+  int32_t* tok = nullptr;  // [T'(window)]
+  int32_t* cnt = nullptr;  // [1]
+  int t_cap = 0;
+  int32_t* tok_host = nullptr;  // pinned [T'(window) + 1]
+  std::vector<void*> allocs;
+};
+
 namespace {
 
 gam_status fail(gam_ctx* c, gam_status s, const std::string& msg) {
@@ -784,11 +803,11 @@ gam_status encoder_kernels(gam_ctx* c, const Plan& p, const Clips& clips, const 
 }
 
 gam_status ctc_kernels(gam_ctx* c, const float* enc, const int* lo, int batch, int t_max, int M_valid, float* logp,
-                       int32_t* tokens, int32_t* counts, cudaStream_t s);
+                       int32_t* tokens, int32_t* counts, int32_t* frames, cudaStream_t s);
 
 // CTC decoding of encoder output; repeated identical calls replay a CUDA graph.
 gam_status run_ctc(gam_ctx* c, const float* enc, const int32_t* enc_len, int batch, int t_max, float* logp,
-                   int32_t* tokens, int32_t* counts, cudaStream_t s) {
+                   int32_t* tokens, int32_t* counts, cudaStream_t s, int32_t* frames = nullptr) {
   const gam_config& cfg = c->cfg;
   if (!enc || !enc_len || !tokens || !counts) return fail(c, GAM_ERR_INVALID_ARG, "null pointer");
   if (batch < 1 || t_max < 1) return fail(c, GAM_ERR_INVALID_ARG, "batch and t_max must be >= 1");
@@ -803,25 +822,25 @@ gam_status run_ctc(gam_ctx* c, const float* enc, const int32_t* enc_len, int bat
   for (int i = 0; i < batch; ++i) lo[batch + 1 + i] = lo[batch + i] + enc_len[i];
   if (graphs_usable(c)) {
     std::vector<int64_t> key = {1, (int64_t)(uintptr_t)enc, batch, t_max, (int64_t)(uintptr_t)logp,
-                                (int64_t)(uintptr_t)tokens, (int64_t)(uintptr_t)counts};
+                                (int64_t)(uintptr_t)tokens, (int64_t)(uintptr_t)counts, (int64_t)(uintptr_t)frames};
     key.insert(key.end(), enc_len, enc_len + batch);
     GraphEntry* e = graph_find(c, key);
     if (!e && graph_second_sighting(c, key)) {
       GAM_TRY(graph_capture(c, key, lo.data(), (int)lo.size(), [&](const int* t, cudaStream_t cs) {
-        return ctc_kernels(c, enc, t, batch, t_max, lo[2 * batch], logp, tokens, counts, cs);
+        return ctc_kernels(c, enc, t, batch, t_max, lo[2 * batch], logp, tokens, counts, frames, cs);
       }, s, &e));
     }
     if (e) return graph_launch(c, e, s);
   }
   const int* dev;
   GAM_TRY(upload_ints(c, lo.data(), 2 * batch + 1, s, &dev));
-  return ctc_kernels(c, enc, dev, batch, t_max, lo[2 * batch], logp, tokens, counts, s);
+  return ctc_kernels(c, enc, dev, batch, t_max, lo[2 * batch], logp, tokens, counts, frames, s);
 }
 
 // CTC head, log-softmax / argmax and collapse; lo = [enc_len (batch) | offsets of the
 // compacted valid frames (batch + 1)] on the device, M_valid = total valid frames.
 gam_status ctc_kernels(gam_ctx* c, const float* enc, const int* lo, int batch, int t_max, int M_valid, float* logp,
-                       int32_t* tokens, int32_t* counts, cudaStream_t s) {
+                       int32_t* tokens, int32_t* counts, int32_t* frames, cudaStream_t s) {
   const gam_config& cfg = c->cfg;
   const int* lens = lo;
   const int* off = lo + batch;
@@ -846,7 +865,7 @@ gam_status ctc_kernels(gam_ctx* c, const float* enc, const int* lo, int batch, i
     }));
   }
   return run_kernel(c, PK_CTC_COLLAPSE, s, [&] {
-    return launch_collapse(c->argmax, lens, batch, t_max, C - 1, tokens, counts, s);
+    return launch_collapse(c->argmax, lens, batch, t_max, C - 1, tokens, counts, s, frames);
   });
 }
 
@@ -1391,6 +1410,13 @@ gam_status gam_ctc_greedy(gam_ctx* c, const float* enc, const int32_t* enc_len, 
   return run_ctc(c, enc, enc_len, batch, t_max, logp, tokens, counts, (cudaStream_t)stream);
 }
 
+gam_status gam_ctc_greedy_frames(gam_ctx* c, const float* enc, const int32_t* enc_len, int batch, int t_max,
+                                 int32_t* tokens, int32_t* frames, int32_t* counts, void* stream) {
+  GAM_TRY(enter(c));
+  if (!frames) return fail(c, GAM_ERR_INVALID_ARG, "null frames pointer");
+  return run_ctc(c, enc, enc_len, batch, t_max, nullptr, tokens, counts, (cudaStream_t)stream, frames);
+}
+
 gam_status gam_ctc_collapse(gam_ctx* c, const float* logits, const int32_t* lengths, int batch, int t_max,
                             int n_classes, int32_t* tokens, int32_t* counts, void* stream) {
   GAM_TRY(enter(c));
@@ -1533,6 +1559,93 @@ gam_status gam_rnnt_greedy(gam_ctx* c, const float* enc, const int32_t* enc_len,
                            int max_tokens, int32_t* tokens, int32_t* frames, int32_t* counts, void* stream) {
   GAM_TRY(enter(c));
   return rnnt_greedy(c, enc, enc_len, batch, t_max, max_tokens, tokens, frames, counts, (cudaStream_t)stream);
+}
+
+gam_status gam_stream_create(gam_ctx* c, int64_t window_samples, gam_stream** out) {
+  GAM_TRY(enter(c));
+  if (!out) return fail(c, GAM_ERR_INVALID_ARG, "null output pointer");
+  *out = nullptr;
+  if (window_samples < 1280 || window_samples > c->cfg.max_samples)
+    return fail(c, GAM_ERR_CAPACITY, "window must be 1280 samples .. the context's max_samples");
+  gam_stream* st = new gam_stream();
+  st->ctx = c;
+  st->window = window_samples;
+  ClipLen l = clip_len(window_samples, c->cfg);
+  st->t_cap = l.T2;
+  auto alloc = [&](void** p, size_t bytes) {
+    cudaError_t e = cudaMalloc(p, bytes);
+    if (e == cudaSuccess) st->allocs.push_back(*p);
+    return cuda_check(c, e, "cudaMalloc");
+  };
+  gam_status s = alloc((void**)&st->buf[0], (size_t)window_samples * 4);
+  if (s == GAM_OK) s = alloc((void**)&st->buf[1], (size_t)window_samples * 4);
+  if (s == GAM_OK) s = alloc((void**)&st->enc, (size_t)st->t_cap * c->cfg.d_model * 4);
+  if (s == GAM_OK) s = alloc((void**)&st->tok, (size_t)st->t_cap * 4);
+  if (s == GAM_OK) s = alloc((void**)&st->cnt, 16);
+  if (s == GAM_OK)
+    s = cuda_check(c, cudaMallocHost((void**)&st->tok_host, ((size_t)st->t_cap + 1) * 4), "cudaMallocHost");
+  if (s != GAM_OK) {
+    gam_stream_destroy(st);
+    return s;
+  }
+  *out = st;
+  return GAM_OK;
+}
+
+gam_status gam_stream_destroy(gam_stream* st) {
+  if (!st) return GAM_OK;
+  if (st->ctx) cudaSetDevice(st->ctx->device);
+  cudaDeviceSynchronize();
+  for (void* p : st->allocs) cudaFree(p);
+  if (st->tok_host) cudaFreeHost(st->tok_host);
+  delete st;
+  return GAM_OK;
+}
+
+gam_status gam_stream_reset(gam_stream* st) {
+  if (!st) return GAM_ERR_INVALID_ARG;
+  st->len = 0;
+  st->total = 0;
+  return GAM_OK;
+}
+
+gam_status gam_stream_push(gam_stream* st, const float* samples_host, int64_t n, int32_t* tokens_host,
+                           int max_tokens, int32_t* count_out, int64_t* window_start_out, void* stream) {
+  if (!st) return GAM_ERR_INVALID_ARG;
+  gam_ctx* c = st->ctx;
+  GAM_TRY(enter(c));
+  if (n < 0 || (n > 0 && !samples_host) || !tokens_host || !count_out || max_tokens < 0)
+    return fail(c, GAM_ERR_INVALID_ARG, "bad push arguments");
+  cudaStream_t s = (cudaStream_t)stream;
+  c->last_stream = s;
+  // new window = the last `window` samples of (old window + new samples), written to the other buffer
+  const int64_t keep_new = std::min(n, st->window);
+  const int64_t keep_old = std::min(st->len, st->window - keep_new);
+  float* dst = st->buf[st->cur ^ 1];
+  if (keep_old > 0)
+    GAM_TRY(cuda_check(c, cudaMemcpyAsync(dst, st->buf[st->cur] + (st->len - keep_old), (size_t)keep_old * 4,
+                                          cudaMemcpyDeviceToDevice, s), "window copy"));
+  if (keep_new > 0)
+    GAM_TRY(cuda_check(c, cudaMemcpyAsync(dst + keep_old, samples_host + (n - keep_new), (size_t)keep_new * 4,
+                                          cudaMemcpyHostToDevice, s), "samples upload"));
+  st->cur ^= 1;
+  st->len = keep_old + keep_new;
+  st->total += n;
+  if (window_start_out) *window_start_out = st->total - st->len;
+  *count_out = 0;
+  if (st->len < 1280) return cuda_check(c, cudaStreamSynchronize(s), "stream sync");  // no encoder frame yet
+  const int32_t len32 = (int32_t)st->len;
+  int32_t el = 0;
+  GAM_TRY(run_encoder(c, st->buf[st->cur], &len32, 1, st->len, -1, -1, st->enc, &el, s));
+  GAM_TRY(run_ctc(c, st->enc, &el, 1, el, nullptr, st->tok, st->cnt, s));
+  GAM_TRY(cuda_check(c, cudaMemcpyAsync(st->tok_host, st->cnt, 4, cudaMemcpyDeviceToHost, s), "count download"));
+  GAM_TRY(cuda_check(c, cudaMemcpyAsync(st->tok_host + 1, st->tok, (size_t)el * 4, cudaMemcpyDeviceToHost, s),
+                     "tokens download"));
+  GAM_TRY(cuda_check(c, cudaStreamSynchronize(s), "stream sync"));
+  const int cnt = st->tok_host[0];
+  *count_out = cnt;
+  std::memcpy(tokens_host, st->tok_host + 1, (size_t)std::min(cnt, max_tokens) * 4);
+  return GAM_OK;
 }
 
 gam_status gam_debug_wait_timeout(gam_ctx* c, int64_t limit_ns, int skip_k_block) {

@@ -27,10 +27,12 @@ STATUS = {0: "GAM_OK", 1: "GAM_ERR_INVALID_ARG", 2: "GAM_ERR_SHAPE", 3: "GAM_ERR
 
 # Every entry point declared in include/gam.h.
 EXPORTS = ("gam_status_string", "gam_last_error", "gam_plan_lengths", "gam_create", "gam_destroy", "gam_logmel",
-           "gam_encode", "gam_encode_stage", "gam_ctc_greedy", "gam_ctc_collapse", "gam_transcribe",
+           "gam_encode", "gam_encode_stage", "gam_ctc_greedy", "gam_ctc_greedy_frames", "gam_ctc_collapse",
+           "gam_transcribe",
            "gam_device_status", "gam_profile_enable", "gam_profile_reset", "gam_profile_kinds",
            "gam_profile_kind_name", "gam_profile_read", "gam_graphs_enable", "gam_ctc_collapse_noalloc",
-           "gam_rnnt_attach", "gam_rnnt_greedy",
+           "gam_rnnt_attach", "gam_rnnt_greedy", "gam_stream_create", "gam_stream_destroy", "gam_stream_reset",
+           "gam_stream_push",
            "gam_debug_gemm", "gam_debug_wait_timeout", "gam_debug_inject_cuda_error")
 
 GAM_NOALLOC_MAX_FRAMES = 1 << 20
@@ -86,6 +88,7 @@ def lib() -> ctypes.CDLL:
         L.gam_encode.argtypes = [vp, vp, i32p, ctypes.c_int, i64, vp, i32p, vp]
         L.gam_encode_stage.argtypes = [vp, vp, i32p, ctypes.c_int, i64, ctypes.c_int, ctypes.c_int, vp, vp]
         L.gam_ctc_greedy.argtypes = [vp, vp, i32p, ctypes.c_int, ctypes.c_int, vp, vp, vp, vp]
+        L.gam_ctc_greedy_frames.argtypes = [vp, vp, i32p, ctypes.c_int, ctypes.c_int, vp, vp, vp, vp]
         L.gam_ctc_collapse.argtypes = [vp, vp, i32p, ctypes.c_int, ctypes.c_int, ctypes.c_int, vp, vp, vp]
         L.gam_transcribe.argtypes = [vp, vp, i32p, ctypes.c_int, i64, vp, vp, vp]
         L.gam_device_status.argtypes = [vp]
@@ -99,6 +102,11 @@ def lib() -> ctypes.CDLL:
         L.gam_ctc_collapse_noalloc.argtypes = [vp, vp, ctypes.c_int, ctypes.c_int, ctypes.c_int, vp, vp, vp]
         L.gam_rnnt_attach.argtypes = [vp, ctypes.POINTER(GamRnntConfig), ctypes.POINTER(GamTensor), ctypes.c_int]
         L.gam_rnnt_greedy.argtypes = [vp, vp, i32p, ctypes.c_int, ctypes.c_int, ctypes.c_int, vp, vp, vp, vp]
+        L.gam_stream_create.argtypes = [vp, ctypes.c_int64, ctypes.POINTER(vp)]
+        L.gam_stream_destroy.argtypes = [vp]
+        L.gam_stream_reset.argtypes = [vp]
+        L.gam_stream_push.argtypes = [vp, vp, ctypes.c_int64, i32p, ctypes.c_int, i32p,
+                                      ctypes.POINTER(ctypes.c_int64), vp]
         L.gam_debug_gemm.argtypes = [vp, ctypes.c_int, vp, ctypes.c_int, vp, vp, ctypes.c_int, ctypes.c_int,
                                      ctypes.c_int, vp, ctypes.c_int, vp]
         L.gam_debug_wait_timeout.argtypes = [vp, ctypes.c_int64, ctypes.c_int]
@@ -297,6 +305,26 @@ def gam_ctc_greedy(ctx: Context, enc, enc_len, want_logp: bool = False, stream=N
     return tokens, counts, logp
 
 
+def gam_ctc_greedy_frames(ctx: Context, enc, enc_len, stream=None, tokens=None, frames=None, counts=None):
+    """Greedy CTC decoding with the first frame of each token: (tokens, frames,
+    counts) as CUDA int32 tensors [B, T], [B, T], [B]."""
+    import torch
+    el = _i32(enc_len)
+    _dev_tensor(enc, torch.float32, "enc")
+    B, tmax, _ = enc.shape
+    if tokens is None:
+        tokens = torch.empty((B, tmax), dtype=torch.int32, device=enc.device)
+    if frames is None:
+        frames = torch.empty((B, tmax), dtype=torch.int32, device=enc.device)
+    if counts is None:
+        counts = torch.empty((B,), dtype=torch.int32, device=enc.device)
+    for t, n in ((tokens, "tokens"), (frames, "frames"), (counts, "counts")):
+        _dev_tensor(t, torch.int32, n, enc.device)
+    _check(lib().gam_ctc_greedy_frames(ctx.handle, enc.data_ptr(), _ptr_i32(el), B, tmax, tokens.data_ptr(),
+                                       frames.data_ptr(), counts.data_ptr(), _stream(stream)), ctx)
+    return tokens, frames, counts
+
+
 def gam_ctc_collapse(ctx: Context, logits, lengths, stream=None):
     import torch
     ln = _i32(lengths)
@@ -416,6 +444,45 @@ def gam_rnnt_greedy(ctx: Context, enc, enc_len, max_tokens: Optional[int] = None
     _check(lib().gam_rnnt_greedy(ctx.handle, enc.data_ptr(), _ptr_i32(el), B, tmax, int(max_tokens),
                                  tokens.data_ptr(), frames.data_ptr(), counts.data_ptr(), _stream(stream)), ctx)
     return tokens, frames, counts
+
+
+class Stream:
+    """Pseudo-streaming recogniser over a context (gam_stream_*)."""
+
+    def __init__(self, ctx: Context, window_samples: int = 30 * 16000):
+        h = ctypes.c_void_p()
+        _check(lib().gam_stream_create(ctx.handle, int(window_samples), ctypes.byref(h)), ctx)
+        self.handle, self.ctx, self.window = h, ctx, int(window_samples)
+        _, _, _, self.t_cap = gam_plan_lengths(ctx.cfg, [max(1280, self.window)])
+        self._tok = np.zeros(self.t_cap, np.int32)
+
+    def push(self, samples, stream=None):
+        """Append host float32 samples; returns (tokens of the current window, index
+        of the window's first sample in the stream)."""
+        x = np.ascontiguousarray(np.asarray(samples, dtype=np.float32))
+        cnt = np.zeros(1, np.int32)
+        start = ctypes.c_int64()
+        _check(lib().gam_stream_push(self.handle, x.ctypes.data if x.size else None, x.size, _ptr_i32(self._tok),
+                                     self.t_cap, _ptr_i32(cnt), ctypes.byref(start), _stream(stream)), self.ctx)
+        return self._tok[:min(int(cnt[0]), self.t_cap)].copy(), int(start.value)
+
+    def reset(self):
+        _check(lib().gam_stream_reset(self.handle), self.ctx)
+
+    def close(self):
+        if self.handle:
+            lib().gam_stream_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+def gam_stream_create(ctx: Context, window_samples: int = 30 * 16000) -> Stream:
+    return Stream(ctx, window_samples)
 
 
 def gam_graphs_enable(ctx: Context, on: bool = True):

@@ -212,6 +212,15 @@ gam_status gam_ctc_greedy(gam_ctx* ctx, const float* enc_dev, const int32_t* enc
                           int t_max, float* logp_dev, int32_t* tokens_dev, int32_t* counts_dev,
                           void* stream);
 
+/* gam_ctc_greedy with each token's position: frames_dev device i32 [batch,
+ * t_max] receives the encoder frame where the token's run of equal argmax
+ * values starts (-1 after the last token), which places the token in time for
+ * joining the transcripts of overlapping long-form chunks ("GigaAM v3 MLX",
+ * "Long-form transcription": 20 s chunks, 0-2 s overlap).  No log-probs. */
+gam_status gam_ctc_greedy_frames(gam_ctx* ctx, const float* enc_dev, const int32_t* enc_len_host, int batch,
+                                 int t_max, int32_t* tokens_dev, int32_t* frames_dev, int32_t* counts_dev,
+                                 void* stream);
+
 /* Greedy decoding from given scores, the decoding step of gam_ctc_greedy on
  * its own (same passages as gam_ctc_greedy):
  * logits_dev device f32 [batch, t_max, n_classes]; blank = n_classes - 1;
@@ -288,6 +297,37 @@ gam_status gam_rnnt_attach(gam_ctx* ctx, const gam_rnnt_config* cfg, const gam_t
 gam_status gam_rnnt_greedy(gam_ctx* ctx, const float* enc_dev, const int32_t* enc_len_host, int batch, int t_max,
                            int max_tokens, int32_t* tokens_dev, int32_t* frames_dev, int32_t* counts_dev,
                            void* stream);
+
+/* ---- pseudo-streaming ---- */
+
+/* Pseudo-streaming as "GigaAM on MLX: the transcripts matched, but the model
+ * was broken", "Streaming" describes it: the model is not a streaming model, so
+ * every step re-recognises the audio received so far, but no more than the
+ * last window_samples (30 s = 480000 samples there).  A gam_stream belongs to
+ * one context and allocates its buffers at creation (two window buffers, the
+ * encoder output and tokens of one window); pushes allocate nothing.  Once the
+ * window is full, every push encodes the same length from one of two buffers,
+ * so the context's CUDA graphs replay from the fourth push on. */
+typedef struct gam_stream gam_stream;
+
+/* window_samples: 1280 .. the context's max_samples (GAM_ERR_CAPACITY). */
+gam_status gam_stream_create(gam_ctx* ctx, int64_t window_samples, gam_stream** out);
+gam_status gam_stream_destroy(gam_stream* st);
+/* Forget the audio pushed so far. */
+gam_status gam_stream_reset(gam_stream* st);
+
+/* Append n samples (HOST f32, 16 kHz mono) and recognise the window, i.e. the
+ * last min(total, window_samples) samples: gam_encode + gam_ctc_greedy of that
+ * window as one clip, on `stream`, synchronised before returning.
+ * tokens_host receives the window's CTC tokens (at most max_tokens of them),
+ * *count_out the window's token count (possibly above max_tokens), and
+ * *window_start_out (optional) the index of the window's first sample in the
+ * pushed stream.  A window shorter than 1280 samples has no encoder frame and
+ * gives 0 tokens.  The tokens of a step are the whole window's transcript, not
+ * only the new part: as the page notes, the cost of a step grows with the
+ * window, and text at its start can change from step to step. */
+gam_status gam_stream_push(gam_stream* st, const float* samples_host, int64_t n, int32_t* tokens_host,
+                           int max_tokens, int32_t* count_out, int64_t* window_start_out, void* stream);
 
 /* ---- greedy decoding without any allocation ---- */
 

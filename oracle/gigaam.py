@@ -47,7 +47,7 @@ __all__ = [
     "rope_tables", "rotate_half", "apply_rope", "masked_attention",
     "feed_forward", "rotary_mhsa", "conv_module", "conformer_layer",
     "dequant_g64", "get_linear",
-    "encode_clip", "ctc_head", "greedy_collapse", "transcribe_clip",
+    "encode_clip", "ctc_head", "greedy_collapse", "greedy_collapse_frames", "transcribe_clip",
     "oracle_weight_inventory",
 ]
 
@@ -393,6 +393,23 @@ def greedy_collapse(a, blank: int) -> List[int]:
             out.append(s)
         prev = s
     return out
+
+
+def greedy_collapse_frames(a, blank: int):
+    """greedy_collapse with the frame where each kept symbol's run starts:
+    (symbols, frames).  The frame places a symbol in time, which is what joins
+    the transcripts of overlapping long-form chunks ([v3-MLX] "Long-form
+    transcription": 20 s chunks with 0-2 s of overlap)."""
+    out: List[int] = []
+    frames: List[int] = []
+    prev = None
+    for t, s in enumerate(a):
+        s = int(s)
+        if s != prev and s != blank:
+            out.append(s)
+            frames.append(t)
+        prev = s
+    return out, frames
 
 
 def transcribe_clip(audio: np.ndarray, W, cfg: dict, dtype=np.float64) -> dict:

@@ -27,6 +27,21 @@ def test_collapse_vs_groupby_bruteforce():
         assert oracle.greedy_collapse(seq, blank) == ref
 
 
+def test_collapse_frames_hand_cases():
+    """Each kept symbol carries the first frame of its run."""
+    assert oracle.greedy_collapse_frames([5, 5, 7, 7], 33) == ([5, 7], [0, 2])
+    assert oracle.greedy_collapse_frames([33, 5, 33, 5, 5], 33) == ([5, 5], [1, 3])
+    assert oracle.greedy_collapse_frames([33, 33], 33) == ([], [])
+    rng = np.random.default_rng(3)
+    for _ in range(200):
+        blank = int(rng.integers(1, 4))
+        seq = rng.integers(0, blank + 1, size=int(rng.integers(0, 15))).tolist()
+        sym, fr = oracle.greedy_collapse_frames(seq, blank)
+        assert sym == oracle.greedy_collapse(seq, blank)
+        assert all(seq[f] == k and (f == 0 or seq[f - 1] != k) for k, f in zip(sym, fr))
+        assert fr == sorted(fr) and len(set(fr)) == len(fr)
+
+
 def test_ctc_head_logsoftmax_and_first_argmax():
     rng = np.random.default_rng(1)
     d, C, T = 6, 5, 4
