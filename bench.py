@@ -242,6 +242,152 @@ def time_workload(name, steps=5, warmup=3, weights=None, device=0, peaks=None, c
         ctx.close()
 
 
+def time_rnnt(name, n_classes, steps=5, warmup=3, weights=None, device=0):
+    """Encoder + greedy RNNT decoding of a workload's batch (audio resident): the
+    whole step, and the decoder part (joint encoder projection + sequential
+    decode) alone, with CUDA events."""
+    import torch
+    from conformer_speech_recognition_b200 import gam
+    cfg = synth.workload_config(name)
+    W = weights if weights is not None else synth.random_weights(cfg, seed=0)
+    audio_np, lens = synth.workload_audio(name)
+    B, nmax = audio_np.shape
+    ctx = gam.gam_create(cfg, W, B, nmax, device=device)
+    try:
+        dev = torch.device("cuda", device)
+        gam.gam_rnnt_attach(ctx, dict(synth.RNNT, n_classes=n_classes),
+                            synth.random_rnnt_weights(cfg["d_model"], n_classes))
+        audio = torch.from_numpy(audio_np).to(dev)
+        _, el, _, tmax = gam.gam_plan_lengths(cfg, lens)
+        enc = torch.empty((B, tmax, cfg["d_model"]), dtype=torch.float32, device=dev)
+        mt = tmax * synth.RNNT["max_symbols"]
+        tok = torch.empty((B, mt), dtype=torch.int32, device=dev)
+        frm = torch.empty((B, mt), dtype=torch.int32, device=dev)
+        cnt = torch.empty((B,), dtype=torch.int32, device=dev)
+        stream = torch.cuda.current_stream(dev)
+
+        def dec():
+            gam.gam_rnnt_greedy(ctx, enc, el, max_tokens=mt, stream=stream, tokens=tok, frames=frm, counts=cnt)
+
+        def step():
+            gam.gam_encode(ctx, audio, lens, out=enc, stream=stream)
+            dec()
+
+        for _ in range(warmup):
+            step()
+        torch.cuda.synchronize(dev)
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+        ev[0].record(stream)
+        for _ in range(steps):
+            step()
+        ev[1].record(stream)
+        for _ in range(steps):
+            dec()
+        ev[2].record(stream)
+        torch.cuda.synchronize(dev)
+        ms = ev[0].elapsed_time(ev[1]) / steps
+        dec_ms = ev[1].elapsed_time(ev[2]) / steps
+        gam.gam_profile_enable(ctx, -1)
+        dec()
+        torch.cuda.synchronize(dev)
+        prof = gam.gam_profile_all(ctx)
+        gam.gam_profile_enable(ctx, 0)
+        audio_s = float(np.sum(lens)) / synth.SAMPLE_RATE
+        symbols = cnt.cpu().numpy()
+        return {"value": audio_s / (ms / 1e3), "unit": UNIT, "ms_per_step": ms, "decode_ms": dec_ms,
+                "decode_share": dec_ms / ms, "n_classes": n_classes, "steps": steps, "batch": int(B),
+                "symbols_per_clip_mean": float(symbols.mean()), "valid_frames": int(np.sum(el)),
+                "rnnt_enc_proj_ms": prof["rnnt_enc_proj"][0], "rnnt_decode_kernel_ms": prof["rnnt_decode"][0],
+                "audio_seconds_per_step": audio_s}
+    finally:
+        ctx.close()
+
+
+def time_streaming(window_s=30.0, push_s=1.0, total_s=60.0, weights=None, device=0):
+    """Pseudo-streaming on the v3 d768 model: pushes of push_s seconds of audio
+    for total_s seconds, every push re-recognising the last window_s seconds.
+    Reports audio pushed per second of wall time and the per-push latency once
+    the window is full (host-timed: each push synchronises)."""
+    import torch
+    from conformer_speech_recognition_b200 import gam
+    cfg = synth.workload_config("c1_1s_b1_d768")
+    W = weights if weights is not None else synth.random_weights(cfg, seed=0)
+    win = int(window_s * synth.SAMPLE_RATE)
+    ctx = gam.gam_create(cfg, W, 1, win, device=device)
+    try:
+        st = gam.Stream(ctx, win)
+        x, _ = synth.random_audio([int(total_s * synth.SAMPLE_RATE)], seed=55)
+        x = x[0]
+        n = int(push_s * synth.SAMPLE_RATE)
+        for k in range(3):  # warm-up pushes (graphs are captured on the window's second sighting)
+            st.push(x[k * n:(k + 1) * n])
+        st.reset()
+        torch.cuda.synchronize(device)
+        lat = []
+        t_all = time.perf_counter()
+        for k in range(0, len(x) // n):
+            t0 = time.perf_counter()
+            st.push(x[k * n:(k + 1) * n])
+            lat.append(time.perf_counter() - t0)
+        wall = time.perf_counter() - t_all
+        full = lat[int(window_s / push_s) + 2:]
+        st.close()
+        return {"value": total_s / wall, "unit": UNIT, "window_s": window_s, "push_s": push_s,
+                "pushes": len(lat), "latency_ms_full_window_median": 1e3 * statistics.median(full) if full else None,
+                "latency_ms_first_push": 1e3 * lat[0]}
+    finally:
+        ctx.close()
+
+
+def chunk_sweep(device=0, steps=3):
+    """The pages' long-form shape question ("GigaAM MLX port for Mac",
+    "Which optimizations actually made the model faster": 20 s vs 40 s chunks,
+    groups of 8): the 300 s chirp on the d1024 model as 15 x 20 s or 8 x 40 s
+    chunks, all in one batch or in groups of 8, with fp16 and INT8 weights."""
+    import torch
+    from conformer_speech_recognition_b200 import gam
+    full, _ = synth.workload_audio("c5_300s_chunks15_d1024_int8")
+    x = full.reshape(-1)
+    out = {}
+    for prec in ("fp16", "int8_g64"):
+        cfg = synth.model_config(synth.LARGE, 257, prec)
+        W = synth.random_weights(cfg, seed=0)
+        ctx = gam.gam_create(cfg, W, 15, 40 * synth.SAMPLE_RATE, device=device)
+        try:
+            for chunk_s in (20, 40):
+                c = chunk_s * synth.SAMPLE_RATE
+                n = (len(x) + c - 1) // c
+                audio = np.zeros((n, c), np.float32)
+                lens = np.zeros(n, np.int32)
+                for k in range(n):
+                    seg = x[k * c:(k + 1) * c]
+                    audio[k, :len(seg)] = seg
+                    lens[k] = len(seg)
+                a = torch.from_numpy(audio).cuda(device)
+                for group in (n, 8):
+                    calls = [(i, min(i + group, n)) for i in range(0, n, group)]
+
+                    def step():
+                        for i0, i1 in calls:
+                            enc, el = gam.gam_encode(ctx, a[i0:i1], lens[i0:i1])
+                            gam.gam_ctc_greedy(ctx, enc, el)
+                    for _ in range(2):
+                        step()
+                    torch.cuda.synchronize(device)
+                    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                    e0.record()
+                    for _ in range(steps):
+                        step()
+                    e1.record()
+                    torch.cuda.synchronize(device)
+                    ms = e0.elapsed_time(e1) / steps
+                    out[f"{prec}_{chunk_s}s_x{n}_groups_of_{group}"] = {"value": (len(x) / synth.SAMPLE_RATE) / (ms / 1e3),
+                                                                       "unit": UNIT, "ms": ms}
+        finally:
+            ctx.close()
+    return out
+
+
 def reduce_max_over_ranks(values, device=None):
     """Element-wise max over all ranks (torch.distributed all_reduce MAX)."""
     import torch
@@ -506,6 +652,16 @@ def run_ours(args, rank, world, local_rank):
                 same_model = synth.workload_config(other) == cfg
                 per_workload[other] = time_workload(other, weights=W if same_model else None, device=local_rank,
                                                     peaks=peaks, clocks=clock_info)
+        rnnt = stream_res = sweep = None
+        if world == 1 and not args.no_per_workload:
+            v3 = synth.workload_config("c2_varlen_b32_d768")
+            W3 = W if v3 == cfg else None
+            rnnt = {"c2_varlen_b32_d768_rnnt34": time_rnnt("c2_varlen_b32_d768", 34, weights=W3, device=local_rank),
+                    "c2_varlen_b32_d768_rnnt1025": time_rnnt("c2_varlen_b32_d768", 1025, weights=W3,
+                                                             device=local_rank)}
+            stream_res = time_streaming(device=local_rank)
+        if world == 1 and args.sweep:
+            sweep = chunk_sweep(device=local_rank)
         h2d = int(B * nmax * 4 + 5 * (B + 1) * 4 + B * 4)
         d2h = int(B * tmax * 4 + B * 4)
         line = {
@@ -532,6 +688,9 @@ def run_ours(args, rank, world, local_rank):
             "clocks": clock_info,
             "profile_ms_per_step": {k: round(v[0] / n_prof, 4) for k, v in warm.items() if v[1]},
             "per_workload": per_workload,
+            "rnnt": rnnt,
+            "streaming": stream_res,
+            "chunk_sweep": sweep,
         }
         print(json.dumps(line), flush=True)
     ctx.close()
@@ -548,6 +707,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-per-workload", action="store_true", help="skip the ×realtime of the other workloads")
     ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle CPU time for cpu_baseline")
+    ap.add_argument("--sweep", action="store_true",
+                    help="also time the long-form chunk / batch shapes (20 s vs 40 s chunks, groups of 8)")
     ap.add_argument("--ref-seconds", type=float, default=6.0,
                     help="reference arm: each step runs the oracle on one clip cut to at most this many seconds")
     args = ap.parse_args()

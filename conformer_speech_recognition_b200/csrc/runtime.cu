@@ -9,8 +9,11 @@
 #include <cstdlib>
 #include <cstring>
 #include <map>
+#include <optional>
 #include <string>
 #include <vector>
+
+#include <nvtx3/nvToolsExt.h>
 
 #include "../../include/gam.h"
 #include "common.cuh"
@@ -19,6 +22,16 @@
 using namespace gam;
 
 namespace {
+
+// An NVTX range for the lifetime of the object (one per stage of the path), so a
+// timeline tool shows frontend / subsampling / each block / the heads by name.
+// Header-only NVTX: without an attached tool each call is a no-op.
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+  NvtxRange(const NvtxRange&) = delete;
+  NvtxRange& operator=(const NvtxRange&) = delete;
+};
 
 thread_local std::string g_create_error;
 
@@ -725,6 +738,8 @@ gam_status encoder_kernels(gam_ctx* c, const Plan& p, const Clips& clips, const 
   const float eps = cfg.ln_eps;
   const int M = p.E_pad;
 
+  std::optional<NvtxRange> stage_range;
+  stage_range.emplace("gam.frontend");
   if (c->dft_hi) {
     // tensor-core frontend: samples split into tf32 hi / lo rows, then the 3xTF32 DFT
     // with power, filterbank and log in its epilogue (fp16 packed mel rows)
@@ -740,13 +755,22 @@ gam_status encoder_kernels(gam_ctx* c, const Plan& p, const Clips& clips, const 
       return launch_frontend(audio, max_samples, clips, p.R0, 1, 0, c->basis, c->fb, c->mel, ah, s);
     }));
   }
+  stage_range.reset();
+  stage_range.emplace("gam.subsampling");
   GAM_TRY(gemm(c, PK_GEMM_SUB, s, c->mel, nullptr, 0, 2 * cfg.n_mels, c->conv1, p.R1, EPI_CONV1, 1.f, c->c1, d,
                clips));
   GAM_TRY(gemm(c, PK_GEMM_SUB, s, c->c1, nullptr, 0, 2 * d, c->conv2, M, EPI_CONV2, 1.f, c->x, d, clips));
 
   const int L = cfg.n_layers;
   bool stopped = stop_stage == GAM_STAGE_SUBSAMPLING;
+  stage_range.reset();
+  static const char* const kLayerNames[] = {
+      "gam.layer.0",  "gam.layer.1",  "gam.layer.2",  "gam.layer.3",  "gam.layer.4",  "gam.layer.5",
+      "gam.layer.6",  "gam.layer.7",  "gam.layer.8",  "gam.layer.9",  "gam.layer.10", "gam.layer.11",
+      "gam.layer.12", "gam.layer.13", "gam.layer.14", "gam.layer.15", "gam.layer.16", "gam.layer.17",
+      "gam.layer.18", "gam.layer.19", "gam.layer.20", "gam.layer.21", "gam.layer.22", "gam.layer.23"};
   for (int l = 0; l < L && !stopped; ++l) {
+    NvtxRange layer_range(l < 24 ? kLayerNames[l] : "gam.layer");
     DevLayer& w = c->layers[l];
     if (l == 0)
       GAM_TRY(run_kernel(c, PK_LAYERNORM, s, [&] {
@@ -841,6 +865,7 @@ gam_status run_ctc(gam_ctx* c, const float* enc, const int32_t* enc_len, int bat
 // compacted valid frames (batch + 1)] on the device, M_valid = total valid frames.
 gam_status ctc_kernels(gam_ctx* c, const float* enc, const int* lo, int batch, int t_max, int M_valid, float* logp,
                        int32_t* tokens, int32_t* counts, int32_t* frames, cudaStream_t s) {
+  NvtxRange range("gam.ctc");
   const gam_config& cfg = c->cfg;
   const int* lens = lo;
   const int* off = lo + batch;
@@ -1234,6 +1259,7 @@ gam_status rnnt_greedy(gam_ctx* c, const float* enc, const int32_t* enc_len, int
   for (int i = 0; i < batch; ++i)
     if (enc_len[i] < 0 || enc_len[i] > t_max) return fail(c, GAM_ERR_SHAPE, "enc_len outside [0, t_max]");
   c->last_stream = s;
+  NvtxRange range("gam.rnnt");
   std::vector<int32_t> lo(2 * batch + 1);
   for (int i = 0; i < batch; ++i) lo[i] = enc_len[i];
   lo[batch] = 0;
