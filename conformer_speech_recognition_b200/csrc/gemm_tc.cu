@@ -88,7 +88,8 @@ struct Cfg {
   static constexpr bool SB = staged_bias<EPI, QBITS, STAGE>();
   static constexpr int BIAS_SMEM = SB ? kBiasSmem : 0;
   static constexpr int STAGES = min8((ring_budget<EPI>() - BIAS_SMEM) / STAGE);
-  static constexpr int TMEM_COLS = BN == 128 ? 256 : 512;  // two accumulators, rounded to a power of two
+  // two accumulators, rounded to a power of two
+  static constexpr int TMEM_COLS = BN == 64 ? 128 : BN == 128 ? 256 : 512;
   static constexpr size_t SMEM = (size_t)STAGES * STAGE + epi_smem<EPI>() + BIAS_SMEM + 1024 + 256;
 };
 
@@ -939,6 +940,10 @@ cudaError_t launch_bn(TcGemmCache* cache, const CUtensorMap& mA, const CUtensorM
 template <int QBITS>
 cudaError_t launch_width(int BN, TcGemmCache* cache, const CUtensorMap& mA, const CUtensorMap& mA2,
                          const CUtensorMap& mB, const CUtensorMap& mX, const TcArgs& args, cudaStream_t s) {
+  if (BN == 64) {  // narrow tiles: fp16 weights and few rows only
+    if constexpr (QBITS == 0) return launch_bn<64, 0>(cache, mA, mA2, mB, mX, args, s);
+    return cudaErrorInvalidValue;
+  }
   if (BN == 256) return launch_bn<256, QBITS>(cache, mA, mA2, mB, mX, args, s);
   if (BN == 192) return launch_bn<192, QBITS>(cache, mA, mA2, mB, mX, args, s);
   return launch_bn<128, QBITS>(cache, mA, mA2, mB, mX, args, s);
@@ -996,8 +1001,11 @@ TileShape choose_tile(const TcGemmCache* cache, int M, int N, int epi, bool qb, 
     if (variant < 0 && ((pair && cache->pair_mode == 0) || (!pair && cache->pair_mode == 2))) continue;
     const int units = pair ? sms / 2 : sms;
     const int mt = pair ? (M + 255) / 256 : (M + BM - 1) / BM;
-    for (int bn : {256, 192, 128}) {
+    for (int bn : {256, 192, 128, 64}) {
       if (N % bn || (width && bn != width) || (n_split > 0 && n_split % bn)) continue;
+      // 64-column tiles spread a weight matrix over more SMs when the rows are few
+      // (batch-1 latency); single-CTA, fp16 weights, at most 256 rows
+      if (bn == 64 && (pair || qb || epi == EPI_GLU || M > 256)) continue;
       if (epi == EPI_GLU && bn % 128) continue;
       const int tiles = mt * (N / bn);
       const double round_up = qb ? 1.0 : kWaveRoundUp;

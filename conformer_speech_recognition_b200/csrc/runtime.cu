@@ -1560,8 +1560,9 @@ gam_status gam_debug_gemm(gam_ctx* c, int impl, const void* a, int lda, const vo
   ep.ldo = ldo;
   WeightOp W{w, nullptr, 1, nullptr};
   const int kind = impl & 0xff, width = impl >> 8;
-  if (impl < 0 || kind > 3 || (kind == 1 && width) || (width && width != 128 && width != 192 && width != 256))
-    return fail(c, GAM_ERR_INVALID_ARG, "impl: kind 0 .. 3 plus (tile width 128, 192 or 256) << 8");
+  if (impl < 0 || kind > 3 || (kind == 1 && width) ||
+      (width && width != 64 && width != 128 && width != 192 && width != 256) || (width == 64 && kind == 3))
+    return fail(c, GAM_ERR_INVALID_ARG, "impl: kind 0 .. 3 plus (tile width 64 (single-CTA), 128, 192 or 256) << 8");
   if (kind != 1) {
     if (!tc_supported(1, 1, n, k, EPI_RESID)) return fail(c, GAM_ERR_SHAPE, "tensor-core GEMM needs N % 256 == 0, K % 64 == 0");
     const int variant = kind == 0 ? -1 : kind == 2 ? 0 : 1;

@@ -386,7 +386,9 @@ gam_status gam_graphs_enable(gam_ctx* ctx, int on);
  * shape the encoder would choose, 1 = CUDA cores, 2 = tensor cores with
  * single-CTA tiles (128 rows), 3 = tensor cores with paired-CTA tiles (256
  * rows on two SMs, cta_group::2); width 0 lets the library choose the tile
- * width, else 128, 192 or 256 output columns (tensor-core kinds only).
+ * width, else 128, 192 or 256 output columns, or 64 with single-CTA tiles of at
+ * most 256 rows (tensor-core kinds only; the library picks 64 for such few rows
+ * so that more SMs share the weight stream).
  * N % 256 == 0 and K % 64 == 0 for the tensor-core kinds, N % 128 == 0 and
  * K % 16 == 0 for CUDA cores; a width that does not divide N fails with
  * GAM_ERR_SHAPE, an impl outside these values with GAM_ERR_INVALID_ARG.

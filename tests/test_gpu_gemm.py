@@ -71,6 +71,15 @@ def test_gemm_tile_shapes(ctx, M, N, K, lda, kind, width):
     test_gemm_parity(ctx, kind | (width << 8), M, N, K, lda)
 
 
+@pytest.mark.parametrize("M,N,K", [(24, 768, 768), (128, 3072, 768), (200, 768, 3072), (256, 2304, 768)],
+                         ids=["batch1_rows", "one_m_block", "deep_k", "two_m_blocks"])
+def test_gemm_narrow_tiles_few_rows(ctx, M, N, K):
+    """64-column single-CTA tiles, which the library picks for GEMMs of at most
+    256 rows; forced and chosen."""
+    test_gemm_parity(ctx, 2 | (64 << 8), M, N, K, K)
+    test_gemm_parity(ctx, 0, M, N, K, K)
+
+
 def test_gemm_width_must_divide_n(ctx):
     import torch
     a = torch.zeros(256, 64, dtype=torch.float16, device="cuda")
