@@ -165,13 +165,14 @@ cudaError_t launch_f32_to_f16(const float* in, __half* out, int64_t n, cudaStrea
 // Greedy RNNT decoding (rnnt.cu), one CTA per clip.  eproj [rows][J]: the joint's
 // encoder projection per valid frame (row off[b] + t, or b * t_max + t when off
 // is NULL); gtab [(C + 1)][4P]: LSTM input gates per symbol (row C: zero start
-// input); whhT [P][4P], wpT [P][J], woT [J][C] fp16 (transposed weights); act
-// 0 ReLU, 1 tanh.  Writes tokens / frames ([B][max_tokens], -1 after the last
-// symbol; frames may be NULL) and counts [B].
+// input); whh [4P][P], wp [J][P], wo [C][J] fp16, row-major (PyTorch layout),
+// 16-byte aligned, P and J multiples of 8; act 0 ReLU, 1 tanh.  Writes tokens /
+// frames ([B][max_tokens], -1 after the last symbol; frames may be NULL) and
+// counts [B].
 size_t rnnt_smem_bytes(int C, int P, int J);
 cudaError_t launch_rnnt_greedy(const float* eproj, const int* lens, const int* off, int batch, int t_max,
-                               const float* gtab, const __half* whhT, const __half* wpT, const float* bp,
-                               const __half* woT, const float* bo, int C, int P, int J, int max_symbols, int act,
+                               const float* gtab, const __half* whh, const __half* wp, const float* bp,
+                               const __half* wo, const float* bo, int C, int P, int J, int max_symbols, int act,
                                int max_tokens, int* tokens, int* frames, int* counts, cudaStream_t s);
 
 }  // namespace gam

@@ -91,10 +91,10 @@ struct RnntHead {
   int C = 0, P = 0, E = 0, J = 0, max_symbols = 0, act = 0;
   DevLinear enc;            // fp16 modes: [W_enc | W_enc] rows padded to 256, K = 2d; fp32 mode: W_enc
   float* gtab = nullptr;    // [(C + 1)][4P]
-  __half* whhT = nullptr;   // [P][4P]
-  __half* wpT = nullptr;    // [P][J]
+  __half* whh = nullptr;    // [4P][P]
+  __half* wp = nullptr;     // [J][P]
   float* bp = nullptr;      // [J]
-  __half* woT = nullptr;    // [J][C]
+  __half* wo = nullptr;     // [C][J]
   float* bo = nullptr;      // [C]
   float* eproj = nullptr;   // [max_batch * T2_cap][J]
 };
@@ -1161,10 +1161,10 @@ void destroy(gam_ctx* c) {
 gam_status rnnt_attach(gam_ctx* c, const gam_rnnt_config& rc, const gam_tensor* tensors, int n) {
   const int d = c->cfg.d_model;
   const int C = rc.n_classes, P = rc.pred_dim, J = rc.joint_dim;
-  if (C < 2 || C > 4096 || P < 2 || P > 1024 || (P & 1) || J < 2 || J > 1024 || (J & 1) || rc.max_symbols < 1 ||
+  if (C < 2 || C > 4096 || P < 8 || P > 1024 || P % 8 || J < 8 || J > 1024 || J % 8 || rc.max_symbols < 1 ||
       rc.max_symbols > 64 || (rc.joint_act != 0 && rc.joint_act != 1))
-    return fail(c, GAM_ERR_INVALID_ARG, "rnnt config: n_classes 2..4096, even pred_dim / joint_dim <= 1024, "
-                                        "max_symbols 1..64, joint_act 0 or 1");
+    return fail(c, GAM_ERR_INVALID_ARG, "rnnt config: n_classes 2..4096, pred_dim / joint_dim multiples of 8 up to "
+                                        "1024, max_symbols 1..64, joint_act 0 or 1");
   if (rnnt_smem_bytes(C, P, J) > 200 * 1024) return fail(c, GAM_ERR_INVALID_ARG, "rnnt head too large");
   WeightTable t;
   for (int i = 0; i < n; ++i) {
@@ -1203,18 +1203,17 @@ gam_status rnnt_attach(gam_ctx* c, const gam_rnnt_config& rc, const gam_tensor* 
         for (int e = 0; e < E; ++e) v += emb[(size_t)k * E + e] * wih[(size_t)row * E + e];
       gt[(size_t)k * 4 * P + row] = v;
     }
-  auto transpose_h = [](const std::vector<double>& w, int rows, int cols) {  // [rows][cols] -> [cols][rows] fp16
-    std::vector<__half> o((size_t)rows * cols);
-    for (int i = 0; i < rows; ++i)
-      for (int j = 0; j < cols; ++j) o[(size_t)j * rows + i] = __float2half_rn((float)w[(size_t)i * cols + j]);
+  auto to_half = [](const std::vector<double>& w) {  // row-major, as given
+    std::vector<__half> o(w.size());
+    for (size_t i = 0; i < w.size(); ++i) o[i] = __float2half_rn((float)w[i]);
     return o;
   };
-  std::vector<__half> whhT = transpose_h(whh, 4 * P, P), wpT = transpose_h(wp, J, P), woT = transpose_h(wo, C, J);
+  std::vector<__half> whh_h = to_half(whh), wp_h = to_half(wp), wo_h = to_half(wo);
   GAM_TRY(upload_f32(c, &r.gtab, gt));
-  GAM_TRY(upload(c, &r.whhT, whhT.data(), whhT.size() * sizeof(__half)));
-  GAM_TRY(upload(c, &r.wpT, wpT.data(), wpT.size() * sizeof(__half)));
+  GAM_TRY(upload(c, &r.whh, whh_h.data(), whh_h.size() * sizeof(__half)));
+  GAM_TRY(upload(c, &r.wp, wp_h.data(), wp_h.size() * sizeof(__half)));
   GAM_TRY(upload_f32(c, &r.bp, bp));
-  GAM_TRY(upload(c, &r.woT, woT.data(), woT.size() * sizeof(__half)));
+  GAM_TRY(upload(c, &r.wo, wo_h.data(), wo_h.size() * sizeof(__half)));
   GAM_TRY(upload_f32(c, &r.bo, bo));
   HostLinear hl;
   if (c->cfg.precision == GAM_FP32) {
@@ -1284,7 +1283,7 @@ gam_status rnnt_greedy(gam_ctx* c, const float* enc, const int32_t* enc_len, int
     off = nullptr;  // rows b * t_max + t
   }
   return run_kernel(c, PK_RNNT_DECODE, s, [&] {
-    return launch_rnnt_greedy(r.eproj, lens, off, batch, t_max, r.gtab, r.whhT, r.wpT, r.bp, r.woT, r.bo, r.C, r.P,
+    return launch_rnnt_greedy(r.eproj, lens, off, batch, t_max, r.gtab, r.whh, r.wp, r.bp, r.wo, r.bo, r.C, r.P,
                               r.J, r.max_symbols, r.act, max_tokens, tokens, frames, counts, s);
   });
 }

@@ -264,8 +264,8 @@ gam_status gam_profile_read(gam_ctx* ctx, int kind, double* total_ms, int64_t* l
  * "Architecture details": greedy RNNT decoding, 1025 classes with blank 1024). */
 typedef struct {
   int n_classes;    /* vocabulary + 1; blank = n_classes - 1 (34 or 1025); <= 4096        */
-  int pred_dim;     /* LSTM hidden size P (320), even                                      */
-  int joint_dim;    /* joint hidden width J (320), even                                    */
+  int pred_dim;     /* LSTM hidden size P (320), a multiple of 8                           */
+  int joint_dim;    /* joint hidden width J (320), a multiple of 8                         */
   int max_symbols;  /* symbols emitted per encoder frame at most (10), 1..64               */
   int joint_act;    /* 0: ReLU, 1: tanh, applied to W_enc f + b_enc + W_pred g + b_pred     */
 } gam_rnnt_config;

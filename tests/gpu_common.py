@@ -16,6 +16,49 @@ TOL_FP32_LAYER = 1e-4
 # synthetic tones + noise floor): 2 * 42 * 6e-8 * 40 = 2.0e-4 on the log scale.
 # (The pages' own frontend ports report 3e-5 and 4.2e-4 against PyTorch fp32.)
 TOL_LOGMEL = 2e-4
+
+
+def logmel_bound_tensor_core(x, window, fb, win=320, hop=160):
+    """Per-element bound on |log-mel error| of the tensor-core frontend (3xTF32
+    DFT with fp32 accumulation), derived from its arithmetic on the clip x:
+
+      DFT:   each product term x w cos is formed from tf32 parts as
+             hi*hi + lo*hi + hi*lo; the tf32 roundings of the lo parts and the
+             dropped lo*lo leave <= 3 * 2^-22 of |x w cos|.  The accumulator
+             takes 120 steps (3 products x 40 instructions of 8 samples), each
+             allowed 2^-22 of the running sum's bound (one rounding of the
+             8-product group and one of the add), so
+             |dRe_k| <= eps * S^c_k,  eps = 3 * 2^-22 + 120 * 2^-22,
+             S^c_k = sum_n |x_n w_n cos(2 pi k n / 320)|  (sin likewise).
+      power: |dP_k| <= 2 |Re| dRe + dRe^2 + 2 |Im| dIm + dIm^2 + 2^-22 P_k.
+      mel:   |dmel| <= sum_k fb[k, m] |dP_k| + 2^-24 * (rows in the sum) * mel.
+      log:   |dlog| <= dmel / (mel - dmel) + 2^-22 |log mel|.
+    Returns the bound [F, n_mels] and the exact log-mel in fp64."""
+    import numpy as np
+    x = np.asarray(x, np.float64)
+    F = 1 + (len(x) - win) // hop
+    idx = np.arange(F)[:, None] * hop + np.arange(win)[None, :]
+    fr = x[idx] * np.asarray(window, np.float64)[None, :]
+    k = np.arange(win // 2 + 1)[:, None]
+    n = np.arange(win)[None, :]
+    ang = 2 * np.pi * ((k * n) % win) / win
+    c, s = np.cos(ang), np.sin(ang)
+    re, im = fr @ c.T, fr @ s.T
+    sc, ss = np.abs(fr) @ np.abs(c).T, np.abs(fr) @ np.abs(s).T
+    eps = 3 * 2.0 ** -22 + 120 * 2.0 ** -22
+    dre, dim_ = eps * sc, eps * ss
+    P = re ** 2 + im ** 2
+    dP = 2 * np.abs(re) * dre + dre ** 2 + 2 * np.abs(im) * dim_ + dim_ ** 2 + 2.0 ** -22 * P
+    fb = np.asarray(fb, np.float64)
+    mel = P @ fb
+    rows = (fb != 0).sum(axis=0)[None, :]
+    dmel = dP @ fb + 2.0 ** -24 * rows * mel
+    mel_c = np.clip(mel, 1e-9, 1e9)
+    lo = np.maximum(mel - dmel, 1e-9)
+    bound = np.where(mel - dmel > 1e-9, dmel / lo, np.log(np.maximum(mel + dmel, 1e-9) / 1e-9))
+    return bound + 2.0 ** -22 * np.abs(np.log(mel_c)), np.log(mel_c)
+
+
 # fp16 / INT8 product modes: relative Frobenius error, max |delta|, argmax agreement.
 TOL_REL_FRO = 1e-2
 TOL_MAX_ABS = 5e-2

@@ -27,9 +27,10 @@ def test_stream_matches_direct_window():
     window = 3 * 16000
     ctx = gam.gam_create(cfg, W, 1, window)
     st = gam.Stream(ctx, window)
-    audio, _ = synth.random_audio([200000], seed=31)
+    audio, _ = synth.random_audio([220000], seed=31)
     x = audio[0]
     sizes = [100, 1000, 0, 5920, 8000, 16000, 1, 37123, 70000, 4000, 0] + [8000] * 8
+    assert sum(sizes) <= len(x)
     pos = 0
     direct_ctx = gam.gam_create(cfg, W, 1, window)  # a second context: its graphs never see the stream's pointers
     for n in sizes:
