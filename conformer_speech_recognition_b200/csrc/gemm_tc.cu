@@ -501,24 +501,36 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap mA, const __grid_constant__ C
     // (BN rows x 128 B); each thread converts 16 weights of a row per pass
     const int t = threadIdx.x - 32 * (2 + kEpiWarps);  // 0 .. 127
     const int ch = t & 3;                              // 16-weight chunk of the row's 64
+    // A thread converts rows pass * 32 + t / 4 of every tile, so the group scales of
+    // its rows for the next k-block are loaded into registers one k-block ahead,
+    // off the conversion's critical path.
+    constexpr int NP = BN / 32;
+    __half scur[NP], snext[NP];
+    auto load_scales = [&](int tile, int kb, __half (&dst)[NP]) {
+      if (tile >= p.tiles) return;
+      const __half* sc = p.scale_t + (size_t)kb * p.N + (tile % p.n_blocks) * BN + (t >> 2);
+#pragma unroll
+      for (int pass = 0; pass < NP; ++pass) dst[pass] = __ldg(sc + pass * 32);
+    };
+    load_scales(blockIdx.x, 0, scur);
     int it = 0;
     bool ok = true;
     for (int tile = blockIdx.x; tile < p.tiles && ok; tile += gridDim.x) {
-      const int n0 = (tile % p.n_blocks) * BN;
       for (int kb = 0; kb < KB; ++kb) {
         const int s = it % STAGES;
+        if (kb + 1 < KB) load_scales(tile, kb + 1, snext);
+        else load_scales(tile + gridDim.x, 0, snext);
         if (!mbar_wait(&full[s], (it / STAGES) & 1, abort_flag, p.wait_ns)) {
           ok = false;
           break;
         }
         const uint8_t* raw = sRaw + s * C::RAW_TILE;
         uint8_t* dst = sB + s * C::B_TILE;
-        const __half* sc = p.scale_t + (size_t)kb * p.N + n0;
-#pragma unroll 4
-        for (int pass = 0; pass < BN / 32; ++pass) {
+#pragma unroll
+        for (int pass = 0; pass < NP; ++pass) {
           const int row = pass * 32 + (t >> 2);
           const uint8_t* src = raw + row * C::RAW_ROW + ch * (C::RAW_ROW / 4);
-          const __half sv = __ldg(sc + row);
+          const __half sv = scur[pass];
           uint4 o0, o1;
           if constexpr (QBITS == 8) {
             dequant16(*reinterpret_cast<const uint4*>(src), __half2(sv, sv), o0, o1);
@@ -536,6 +548,8 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap mA, const __grid_constant__ C
         fence_async_smem();
         __syncwarp();
         if (lane == 0) mbar_arrive(&bready[s]);
+#pragma unroll
+        for (int pass = 0; pass < NP; ++pass) scur[pass] = snext[pass];
         ++it;
       }
     }
@@ -1086,6 +1100,11 @@ cudaError_t launch_gemm_tc(TcGemmCache* cache, const void* A, const void* A2, in
 
 cudaError_t launch_attention(TcGemmCache* cache, const void* qk, const void* vt, Clips clips, void* o, int t_half,
                              int rows_pad, int n_heads, int d_head, int t_max, cudaStream_t s) {
+  static const bool first_form = [] {
+    const char* v = std::getenv("GAM_ATTN");
+    return v && std::strcmp(v, "1") == 0;
+  }();
+  if (t_half && !first_form) return launch_attention_tc2(cache, qk, vt, clips, o, rows_pad, n_heads, d_head, t_max, s);
   if (t_half) return launch_attention_tc(cache, qk, vt, clips, o, rows_pad, n_heads, d_head, t_max, s);
   return launch_attention_simt(qk, vt, clips, o, t_half, rows_pad, n_heads, d_head, t_max, s);
 }

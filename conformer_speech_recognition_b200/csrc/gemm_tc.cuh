@@ -47,7 +47,13 @@ cudaError_t launch_gemm_tc(TcGemmCache* cache, const void* A, const void* A2, in
 cudaError_t launch_attention_tc(TcGemmCache* cache, const void* qk, const void* vt, Clips clips, void* o,
                                 int rows_pad, int n_heads, int d_head, int t_max, cudaStream_t s);
 
-// Masked multi-head attention: tensor cores for fp16 activations, CUDA cores for fp32.
+// The same with 64-key blocks, the score tile double-buffered in TMEM and P kept
+// in TMEM for the P.V product (attention_tc2.cu).
+cudaError_t launch_attention_tc2(TcGemmCache* cache, const void* qk, const void* vt, Clips clips, void* o,
+                                 int rows_pad, int n_heads, int d_head, int t_max, cudaStream_t s);
+
+// Masked multi-head attention: tensor cores for fp16 activations (the double-buffered
+// form unless GAM_ATTN=1 in the environment), CUDA cores for fp32.
 cudaError_t launch_attention(TcGemmCache* cache, const void* qk, const void* vt, Clips clips, void* o, int t_half,
                              int rows_pad, int n_heads, int d_head, int t_max, cudaStream_t s);
 
