@@ -297,7 +297,13 @@ def time_rnnt(name, n_classes, steps=5, warmup=3, weights=None, device=0):
         gam.gam_profile_enable(ctx, 0)
         audio_s = float(np.sum(lens)) / synth.SAMPLE_RATE
         symbols = cnt.cpu().numpy()
+        # the clips decode in parallel, one CTA each: the clip with the most decisions
+        # (frames + emitted symbols) sets the kernel's time
+        decisions = np.asarray(el, np.int64) + symbols.astype(np.int64)
+        worst = int(np.argmax(decisions))
         return {"value": audio_s / (ms / 1e3), "unit": UNIT, "ms_per_step": ms, "decode_ms": dec_ms,
+                "slowest_clip": {"frames": int(el[worst]), "symbols": int(symbols[worst]),
+                                 "us_per_decision": prof["rnnt_decode"][0] * 1e3 / max(int(decisions[worst]), 1)},
                 "decode_share": dec_ms / ms, "n_classes": n_classes, "steps": steps, "batch": int(B),
                 "symbols_per_clip_mean": float(symbols.mean()), "valid_frames": int(np.sum(el)),
                 "symbols_per_frame": float(symbols.sum()) / max(int(np.sum(el)), 1), "blank_bias": blank_bias,

@@ -21,7 +21,8 @@
 //               only rises when a score exceeds it by 2^8 (then O, after the
 //               previous P.V has finished, and the row sum are rescaled);
 //               exp2 of the scaled scores, fp16 pairs stored over the scores
-//               (32 TMEM columns), row sum in fp32; finally O / sum.
+//               (32 TMEM columns), row sum in fp32; finally O / sum, read once
+//               the MMA thread's closing commit (all MMAs done) has landed.
 // Q, K come from the head-major buffer [2][H][rows][64] (head dim padded to
 // 64) and V from V^T [H][64][rows]; clip starts are multiples of 8 rows, so
 // every TMA x coordinate is 16-byte aligned.  All waits are bounded.
@@ -279,8 +280,11 @@ attn_tc2_kernel(const __grid_constant__ CUtensorMap mQK, const __grid_constant__
       __syncwarp();
       if (lane == 0) mbar_arrive(&p_full[buf]);
     }
-    // epilogue: O / l after the last P.V (its completion is phase nblk - 1 of o_full)
-    if (ok && !__all_sync(0xffffffffu, mbar_wait(o_full, (nblk - 1) & 1, abort_flag))) ok = false;
+    // epilogue: O / l once every MMA has finished.  Here P.V(nblk - 2) may still be
+    // in flight as well as P.V(nblk - 1) (S(nblk - 1) was issued before it), so a
+    // parity wait on o_full could see the phase of P.V(nblk - 3) and pass early;
+    // `drain` completes once, after the MMA thread's last commit.
+    if (ok && !__all_sync(0xffffffffu, mbar_wait(drain, 0, abort_flag))) ok = false;
     tc_fence_after();
     uint32_t o0[32], o1[32];
     tmem_ld32(tO + lane_off, o0);

@@ -51,7 +51,8 @@ constexpr int A_STAGE = 2 * OP_TILE;            // hi + lo
 constexpr int B_STAGE = 2 * OP_TILE;
 constexpr int RING = SA * A_STAGE + SB * B_STAGE;  // 192 KB
 constexpr int PROW = NBIN;  // floats per power row: odd, so a warp's rows fall in distinct banks
-static_assert(FBM * PROW * 4 <= RING, "the power rows reuse the operand ring");
+constexpr int FB_OFF = (FBM * PROW * 4 + 15) / 16 * 16;  // filterbank copy after the power rows
+static_assert(FB_OFF + NBIN * NMEL * 4 <= RING, "the power rows and the filterbank reuse the operand ring");
 constexpr size_t SMEM_BYTES = RING + 1024 + 256;
 constexpr uint32_t TMEM_COLS = 512;  // 3 x 128 accumulator columns, rounded to a power of two
 
@@ -239,9 +240,16 @@ dft_mel_tf32_kernel(const __grid_constant__ CUtensorMap mAh, const __grid_consta
     const uint32_t lane_off = (uint32_t)(q * 32) << 16;
     const bool ok = __all_sync(0xffffffffu, mbar_wait(acc_full, 0, abort_flag));
     tc_fence_after();
+    // the operand ring is idle now (every MMA has completed): power rows and a copy
+    // of the filterbank go there; the four epilogue warps share the copy, and all of
+    // them pass the barrier below whether or not their wait succeeded
+    float* P = reinterpret_cast<float*>(base) + rl * PROW;
+    float* fbs = reinterpret_cast<float*>(base + FB_OFF);
+    if (ok)
+      for (int i = rl; i < NBIN * NMEL / 4; i += FBM)
+        reinterpret_cast<float4*>(fbs)[i] = __ldg(reinterpret_cast<const float4*>(p.fb) + i);
+    asm volatile("bar.sync 1, 128;" ::: "memory");  // the filterbank copy is complete
     if (ok) {
-      // the operand ring is idle now (every MMA has completed): power rows go there
-      float* P = reinterpret_cast<float*>(base) + rl * PROW;
 #pragma unroll 1
       for (int j = 0; j < NJ; ++j) {
 #pragma unroll 1
@@ -269,7 +277,8 @@ dft_mel_tf32_kernel(const __grid_constant__ CUtensorMap mAh, const __grid_consta
       for (int m = 0; m < NMEL; ++m) {
         const int2 kr = __ldg(p.fb_range + m);
         float acc = 0.f;
-        for (int k = kr.x; k <= kr.y; ++k) acc = fmaf(P[k], __ldg(p.fb + k * NMEL + m), acc);
+#pragma unroll 4
+        for (int k = kr.x; k <= kr.y; ++k) acc = fmaf(P[k], fbs[k * NMEL + m], acc);
         v[m] = ci >= 0 ? logf(fminf(fmaxf(acc, 1e-9f), 1e9f)) : 0.f;
       }
       if (p.mode == 0) {

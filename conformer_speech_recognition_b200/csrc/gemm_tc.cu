@@ -53,12 +53,19 @@ struct TcArgs {
   int debug_skip;         // test hook: k-block counter value whose loads are not issued (-1: none)
 };
 
-// Residual epilogue: per epilogue warp a 32 x 32 fp32 staging tile (4 KB, 128-byte
-// swizzle) that a TMA reduction adds into x.
+// Residual epilogue: per epilogue warp two 32 x 32 fp32 staging tiles (4 KB each,
+// 128-byte swizzle), used in turn, that TMA reductions add into x: a warp fills
+// one while the reduction of the other is still reading it.
 constexpr int kEpiWarps = 8;
 constexpr int kStageTile = 32 * 32 * 4;
-template <int EPI>
-__host__ __device__ constexpr int epi_smem() { return EPI == EPI_RESID ? kEpiWarps * kStageTile : 0; }
+// Quantised-weight kernels keep one tile per warp: their shared memory goes to the
+// pipeline, which their converter warps need more.
+template <bool QB>
+__host__ __device__ constexpr int stage_bufs() { return QB ? 1 : 2; }
+template <int EPI, bool QB = false>
+__host__ __device__ constexpr int epi_smem() {
+  return EPI == EPI_RESID ? kEpiWarps * stage_bufs<QB>() * kStageTile : 0;
+}
 // Bias of the tile's columns, one 128-float copy per epilogue warp, loaded one
 // tile ahead so the epilogue never waits on it.  Used by the fp16-weight kernels
 // (the INT8 mainloop is bound by its converters), and by the residual epilogue
@@ -68,8 +75,8 @@ constexpr int kBiasSmem = kEpiWarps * kBiasStage;
 __host__ __device__ constexpr int min8(int n) { return n < 8 ? n : 8; }
 // Shared memory for the operand ring: 227 KB less the epilogue staging and
 // 1.25 KB of alignment slack and barriers; at most 8 stages.
-template <int EPI>
-__host__ __device__ constexpr int ring_budget() { return 227 * 1024 - 1280 - epi_smem<EPI>(); }
+template <int EPI, bool QB = false>
+__host__ __device__ constexpr int ring_budget() { return 227 * 1024 - 1280 - epi_smem<EPI, QB>(); }
 template <int EPI, int QBITS, int STAGE>
 __host__ __device__ constexpr bool staged_bias() {
   return QBITS == 0 &&
@@ -87,10 +94,10 @@ struct Cfg {
   static constexpr int STAGE = A_TILE + B_TILE + RAW_TILE;
   static constexpr bool SB = staged_bias<EPI, QBITS, STAGE>();
   static constexpr int BIAS_SMEM = SB ? kBiasSmem : 0;
-  static constexpr int STAGES = min8((ring_budget<EPI>() - BIAS_SMEM) / STAGE);
+  static constexpr int STAGES = min8((ring_budget<EPI, QB>() - BIAS_SMEM) / STAGE);
   // two accumulators, rounded to a power of two
   static constexpr int TMEM_COLS = BN == 64 ? 128 : BN == 128 ? 256 : 512;
-  static constexpr size_t SMEM = (size_t)STAGES * STAGE + epi_smem<EPI>() + BIAS_SMEM + 1024 + 256;
+  static constexpr size_t SMEM = (size_t)STAGES * STAGE + epi_smem<EPI, QB>() + BIAS_SMEM + 1024 + 256;
 };
 
 // Hardware tanh (tanh.approx, one special-function op, relative error about
@@ -201,9 +208,10 @@ __device__ __forceinline__ void epi_chunk(const TcArgs& p, int r, int n, bool va
 // or for the paired epilogue (GLU: 128-column blocks [value 64 | gate 64])
 // the (first, second) pairs of 32-column chunks number half * BN/128 .. (half+1) * BN/128 - 1.
 // bt: bias of the tile's columns (bt[c] = bias[n0 + c]), in shared memory if SB.
-template <int BN, int EPI, bool SB>
+template <int BN, int EPI, bool SB, int NBUF>
 __device__ __forceinline__ void epilogue_tile(const TcArgs& p, int r, int n0, uint32_t tbase, int half,
-                                              const CUtensorMap* mX, uint8_t* stage, const float* bt) {
+                                              const CUtensorMap* mX, uint8_t* stage, const float* bt,
+                                              uint32_t& stage_seq) {
   const int c_lo = half * (BN / 2), c_hi = (half + 1) * (BN / 2);
   const EpiParams& ep = p.ep;
   const bool in_m = r < p.M;
@@ -259,9 +267,15 @@ __device__ __forceinline__ void epilogue_tile(const TcArgs& p, int r, int n0, ui
         bcur[j] = bnext[j];
       }
       if (row0 >= p.M) continue;
-      if (lane == 0) bulk_wait_read0();  // the previous reduction has read the staging tile
+      // with two tiles, this chunk's tile was last used two chunks ago: the reductions are
+      // committed in order, so waiting until at most one is still reading frees it
+      if (lane == 0) {
+        if (NBUF == 2) bulk_wait_read1();
+        else bulk_wait_read0();
+      }
       __syncwarp();
-      uint8_t* row = stage + lane * 128;
+      uint8_t* buf = stage + (NBUF == 2 ? (stage_seq++ & 1) * kStageTile : 0);  // alternating across tiles too
+      uint8_t* row = buf + lane * 128;
 #pragma unroll
       for (int j = 0; j < 8; ++j)
         *reinterpret_cast<float4*>(row + ((j ^ (lane & 7)) << 4)) =
@@ -269,7 +283,7 @@ __device__ __forceinline__ void epilogue_tile(const TcArgs& p, int r, int n0, ui
       fence_async_smem();
       __syncwarp();
       if (lane == 0) {
-        tma_reduce_add_2d(mX, stage, n0 + c, row0);
+        tma_reduce_add_2d(mX, buf, n0 + c, row0);
         bulk_commit();
       }
     }
@@ -388,8 +402,8 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap mA, const __grid_constant__ C
   uint8_t* sA = base;
   uint8_t* sB = base + STAGES * A_TILE;
   uint8_t* sRaw = sB + STAGES * C::B_TILE;  // INT8 variant only
-  uint8_t* sEpi = base + STAGES * C::STAGE;  // residual epilogue staging, kStageTile per warp
-  uint8_t* sBias = sEpi + epi_smem<EPI>();    // per-warp bias copies, kBiasStage each
+  uint8_t* sEpi = base + STAGES * C::STAGE;  // residual epilogue staging, kStageBufs tiles per warp
+  uint8_t* sBias = sEpi + epi_smem<EPI, QB>();  // per-warp bias copies, kBiasStage each
   uint64_t* full = reinterpret_cast<uint64_t*>(sBias + C::BIAS_SMEM);
   uint64_t* empty = full + STAGES;
   uint64_t* tfull = empty + STAGES;
@@ -558,6 +572,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap mA, const __grid_constant__ C
     const int half = (warp - 2) / 4;              // which half of the tile's columns
     constexpr bool SB = C::SB;
     BiasPrefetch<BN, SB> bias(p, half, reinterpret_cast<float*>(sBias + (warp - 2) * kBiasStage), blockIdx.x);
+    uint32_t stage_seq = 0;
     int local = 0;
     for (int tile = blockIdx.x; tile < p.tiles; tile += gridDim.x, ++local) {
       const int acc = local & 1;
@@ -568,7 +583,9 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap mA, const __grid_constant__ C
       const int r = mb * BM + q * 32 + lane;
       const uint32_t tbase = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN);
       const float* bt = bias.tile(p, nb * BN, tile + gridDim.x);
-      epilogue_tile<BN, EPI, SB>(p, r, nb * BN, tbase, half, &mX, sEpi + (warp - 2) * kStageTile, bt);
+      constexpr int NBUF = stage_bufs<QB>();
+      epilogue_tile<BN, EPI, SB, NBUF>(p, r, nb * BN, tbase, half, &mX, sEpi + (warp - 2) * NBUF * kStageTile, bt,
+                                       stage_seq);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&tempty[acc]);
@@ -665,7 +682,7 @@ gemm_tc_pair_kernel(const __grid_constant__ CUtensorMap mA, const __grid_constan
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
   uint8_t* sA = base;
   uint8_t* sB = base + STAGES * A_TILE;
-  uint8_t* sEpi = base + STAGES * C::STAGE;  // residual epilogue staging, kStageTile per warp
+  uint8_t* sEpi = base + STAGES * C::STAGE;  // residual epilogue staging, kStageBufs tiles per warp
   uint8_t* sBias = sEpi + epi_smem<EPI>();    // per-warp bias copies, kBiasStage each
   uint64_t* full = reinterpret_cast<uint64_t*>(sBias + C::BIAS_SMEM);
   uint64_t* empty = full + STAGES;
@@ -780,6 +797,7 @@ gemm_tc_pair_kernel(const __grid_constant__ CUtensorMap mA, const __grid_constan
     const int q = warp & 3, half = (warp - 2) / 4;
     constexpr bool SB = C::SB;
     BiasPrefetch<BN, SB> bias(p, half, reinterpret_cast<float*>(sBias + (warp - 2) * kBiasStage), pair);
+    uint32_t stage_seq = 0;
     int local = 0;
     for (int tile = pair; tile < p.tiles; tile += npairs, ++local) {
       const int acc = local & 1;
@@ -790,7 +808,8 @@ gemm_tc_pair_kernel(const __grid_constant__ CUtensorMap mA, const __grid_constan
       const int r = mb * 256 + (int)rank * 128 + q * 32 + lane;
       const uint32_t tbase = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN);
       const float* bt = bias.tile(p, nb * BN, tile + npairs);
-      epilogue_tile<BN, EPI, SB>(p, r, nb * BN, tbase, half, &mX, sEpi + (warp - 2) * kStageTile, bt);
+      epilogue_tile<BN, EPI, SB, 2>(p, r, nb * BN, tbase, half, &mX, sEpi + (warp - 2) * 2 * kStageTile, bt,
+                                    stage_seq);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_remote(map_to_cta(&tempty[acc], 0));

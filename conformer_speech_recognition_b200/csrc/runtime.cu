@@ -1284,7 +1284,7 @@ gam_status rnnt_greedy(gam_ctx* c, const float* enc, const int32_t* enc_len, int
   }
   return run_kernel(c, PK_RNNT_DECODE, s, [&] {
     return launch_rnnt_greedy(r.eproj, lens, off, batch, t_max, r.gtab, r.whh, r.wp, r.bp, r.wo, r.bo, r.C, r.P,
-                              r.J, r.max_symbols, r.act, max_tokens, tokens, frames, counts, s);
+                              r.J, r.max_symbols, r.act, max_tokens, tokens, frames, counts, c->tc.status, s);
   });
 }
 
