@@ -82,7 +82,7 @@ def fp16_vs_bf16_matmul(device, n=8192, iters=10):
 
 
 def pick_peak(peaks, clocks):
-    """The measured tensor peak that applies to this run: the burst figure when
+    """The tensor peak (measured, else the fallback) that applies to this run: the burst figure when
     the SM clock sampled during the timed region sat within 3% of its maximum
     (no power-cap throttling), else the sustained figure (measured under the
     power cap).  Returns (peak TFLOP/s, "burst" | "sustained")."""
@@ -688,7 +688,7 @@ def run_ours(args, rank, world, local_rank):
             "gemm_tflops_per_step_algorithmic": gemm_flops / 1e12,
             "gemm_tflops_per_s_of_gemm_time": gemm_rate,
             "gemm_frac_of_fp16_peak": gemm_rate / tensor_peak if gemm_rate else None,
-            "gemm_frac_peak_kind": f"measured bf16 dense {peak_kind} (median SM clock vs max decides)",
+            "gemm_frac_peak_kind": f"{peaks['source']} bf16 dense {peak_kind} (median SM clock vs max decides)",
             "gemm_frac_of_library_fp16_this_run": gemm_rate / peak_check["fp16_tflops"]
             if gemm_rate and peak_check else None,
             "fp16_peak_check": peak_check,

@@ -76,6 +76,28 @@ __device__ __forceinline__ void umma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, ui
       "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(0), "r"(0), "r"(0), "r"(0));
 }
 
+// Packed fp32 pairs (sm_100 .f32x2 arithmetic): a 64-bit register holds two floats.
+__device__ __forceinline__ uint64_t pack_f32x2(float a, float b) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+  return r;
+}
+__device__ __forceinline__ float2 unpack_f32x2(uint64_t v) {
+  float2 r;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(r.x), "=f"(r.y) : "l"(v));
+  return r;
+}
+__device__ __forceinline__ uint64_t fma_f32x2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t add_f32x2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+
 __device__ __forceinline__ float fast_exp2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
@@ -224,15 +246,19 @@ attn_tc2_kernel(const __grid_constant__ CUtensorMap mQK, const __grid_constant__
       tmem_ld32(tS + 32, u[1]);
       tmem_ld_wait();
       const int kvalid = L - j * BK2;  // keys [0, kvalid) of this block are valid
-      float mx = -INFINITY;
+      // row maximum as 8 independent partial maxima (short dependency chains)
+      float pm[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) pm[e] = -INFINITY;
       if (kvalid >= BK2) {
 #pragma unroll
-        for (int t = 0; t < BK2; ++t) mx = fmaxf(mx, __uint_as_float(u[t >> 5][t & 31]));
+        for (int t = 0; t < BK2; ++t) pm[t & 7] = fmaxf(pm[t & 7], __uint_as_float(u[t >> 5][t & 31]));
       } else {
 #pragma unroll
         for (int t = 0; t < BK2; ++t)
-          if (t < kvalid) mx = fmaxf(mx, __uint_as_float(u[t >> 5][t & 31]));
+          if (t < kvalid) pm[t & 7] = fmaxf(pm[t & 7], __uint_as_float(u[t >> 5][t & 31]));
       }
+      float mx = fmaxf(fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])), fmaxf(fmaxf(pm[4], pm[5]), fmaxf(pm[6], pm[7])));
       mx *= p.scale_log2;
       if (__any_sync(0xffffffffu, mx > m_used + kRescaleThreshold)) {
         // the previous P.V must have finished before O is rescaled (its phase j - 1)
@@ -260,20 +286,40 @@ attn_tc2_kernel(const __grid_constant__ CUtensorMap mQK, const __grid_constant__
           m_used = mx;
         }
       }
-      // exponentials, row sum, fp16 pairs of P over the scores (32 columns)
-      float sum = 0.f;
+      // exponentials, row sum, fp16 pairs of P over the scores (32 columns).  Scores go
+      // in pairs through packed fp32 ops (one fma.rn.f32x2 for both exponent arguments,
+      // one add.rn.f32x2 into 4 partial pair sums); each lane of a pair is still one
+      // fp32 fma / add.
+      const uint64_t sc2 = pack_f32x2(p.scale_log2, p.scale_log2), nm2 = pack_f32x2(-m_used, -m_used);
+      uint64_t ps2[4] = {0ull, 0ull, 0ull, 0ull};
       uint32_t pw[32];
+      if (kvalid >= BK2) {
 #pragma unroll
-      for (int t = 0; t < BK2; t += 2) {
-        const float a0 = (t < kvalid) ? fast_exp2(fmaf(__uint_as_float(u[t >> 5][t & 31]), p.scale_log2, -m_used)) : 0.f;
-        const float a1 = (t + 1 < kvalid)
-                             ? fast_exp2(fmaf(__uint_as_float(u[(t + 1) >> 5][(t + 1) & 31]), p.scale_log2, -m_used))
-                             : 0.f;
-        sum += a0 + a1;
-        __half2 hv = __floats2half2_rn(a0, a1);
-        pw[t >> 1] = *reinterpret_cast<uint32_t*>(&hv);
+        for (int t = 0; t < BK2; t += 2) {
+          const float2 z = unpack_f32x2(fma_f32x2(pack_f32x2(__uint_as_float(u[t >> 5][t & 31]),
+                                                             __uint_as_float(u[t >> 5][(t & 31) + 1])),
+                                                  sc2, nm2));
+          const float a0 = fast_exp2(z.x), a1 = fast_exp2(z.y);
+          ps2[(t >> 1) & 3] = add_f32x2(ps2[(t >> 1) & 3], pack_f32x2(a0, a1));
+          __half2 hv = __floats2half2_rn(a0, a1);
+          pw[t >> 1] = *reinterpret_cast<uint32_t*>(&hv);
+        }
+      } else {
+#pragma unroll
+        for (int t = 0; t < BK2; t += 2) {
+          const float2 z = unpack_f32x2(fma_f32x2(pack_f32x2(__uint_as_float(u[t >> 5][t & 31]),
+                                                             __uint_as_float(u[t >> 5][(t & 31) + 1])),
+                                                  sc2, nm2));
+          const float a0 = t < kvalid ? fast_exp2(z.x) : 0.f, a1 = t + 1 < kvalid ? fast_exp2(z.y) : 0.f;
+          ps2[(t >> 1) & 3] = add_f32x2(ps2[(t >> 1) & 3], pack_f32x2(a0, a1));
+          __half2 hv = __floats2half2_rn(a0, a1);
+          pw[t >> 1] = *reinterpret_cast<uint32_t*>(&hv);
+        }
       }
-      l += sum;
+      {
+        const float2 q = unpack_f32x2(add_f32x2(add_f32x2(ps2[0], ps2[1]), add_f32x2(ps2[2], ps2[3])));
+        l += q.x + q.y;
+      }
       tmem_st32(tS, pw);
       tmem_st_wait();
       tc_fence_before();
