@@ -162,17 +162,20 @@ cudaError_t launch_collapse(const int* argmax, const int* lens, int batch, int t
                             int* tokens, int* counts, cudaStream_t s, int* frames = nullptr);
 cudaError_t launch_f32_to_f16(const float* in, __half* out, int64_t n, cudaStream_t s);
 
-// Greedy RNNT decoding (rnnt.cu), one CTA per clip.  eproj [rows][J]: the joint's
-// encoder projection per valid frame (row off[b] + t, or b * t_max + t when off
-// is NULL); gtab [(C + 1)][4P]: LSTM input gates per symbol (row C: zero start
-// input); whh [4P][P], wp [J][P], wo [C][J] fp16, row-major (PyTorch layout),
-// 16-byte aligned, P and J multiples of 8 up to 1024; act 0 ReLU, 1 tanh.  status:
-// the device word a bounded wait that gave up sets.  Writes tokens /
-// frames ([B][max_tokens], -1 after the last symbol; frames may be NULL) and
-// counts [B].
+// Greedy RNNT decoding (rnnt.cu).  eproj [rows][J]: the joint's encoder
+// projection per valid frame (row off[b] + t, or b * t_max + t when off is NULL);
+// gtab [(C + 1)][4P]: LSTM input gates per symbol (row C: zero start input);
+// whh [4P][P], wp [J][P], wo [C][J] fp16, row-major (PyTorch layout), 16-byte
+// aligned, P and J multiples of 8 up to 1024; act 0 ReLU, 1 tanh.  order [B]: the
+// clips by decreasing length; with it, a head whose slices fit in the shared
+// memory of an 8-CTA cluster is decoded by one cluster per clip with resident
+// weights, otherwise (or with order NULL, or GAM_RNNT=ring in the environment)
+// by one CTA per clip that streams the weights.  status: the device word a
+// bounded wait that gave up sets.  Writes tokens / frames ([B][max_tokens], -1
+// after the last symbol; frames may be NULL) and counts [B].
 size_t rnnt_smem_bytes(int C, int P, int J);
-cudaError_t launch_rnnt_greedy(const float* eproj, const int* lens, const int* off, int batch, int t_max,
-                               const float* gtab, const __half* whh, const __half* wp, const float* bp,
+cudaError_t launch_rnnt_greedy(const float* eproj, const int* lens, const int* off, const int* order, int batch,
+                               int t_max, const float* gtab, const __half* whh, const __half* wp, const float* bp,
                                const __half* wo, const float* bo, int C, int P, int J, int max_symbols, int act,
                                int max_tokens, int* tokens, int* frames, int* counts, int* status, cudaStream_t s);
 

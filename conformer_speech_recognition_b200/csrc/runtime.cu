@@ -559,6 +559,7 @@ gam_status upload_table(gam_ctx* c, const Plan& p, cudaStream_t s, Clips* out) {
 }
 
 gam_status upload_ints(gam_ctx* c, const int32_t* src, int n, cudaStream_t s, const int** out) {
+  if (n < 0 || (size_t)n > c->tab_ints) return fail(c, GAM_ERR_CAPACITY, "table larger than a ring entry");
   const int slot = c->ring;
   c->ring = (c->ring + 1) % kRing;
   GAM_TRY(cuda_check(c, cudaEventSynchronize(c->tab_ev[slot]), "ring event"));
@@ -1121,7 +1122,7 @@ gam_status alloc_workspace(gam_ctx* c) {
   GAM_TRY(cuda_check(c, cudaMemset(c->qk, 0, (size_t)2 * H * E * 64 * es), "memset"));
   GAM_TRY(cuda_check(c, cudaMemset(c->vt, 0, (size_t)H * 64 * E * es), "memset"));
   GAM_TRY(cuda_check(c, cudaMemset(c->dev_status, 0, 16), "memset"));
-  const size_t tab_ints = 5 * (size_t)(cfg.max_batch + 1) + 16;  // also >= 2 * max_batch + 1
+  const size_t tab_ints = 5 * (size_t)(cfg.max_batch + 1) + 16;  // also >= 3 * max_batch + 1
   c->tab_ints = tab_ints;
   for (int i = 0; i < kRing; ++i) {
     GAM_TRY(cuda_check(c, cudaMallocHost((void**)&c->tab_host[i], tab_ints * 4), "cudaMallocHost"));
@@ -1259,15 +1260,20 @@ gam_status rnnt_greedy(gam_ctx* c, const float* enc, const int32_t* enc_len, int
     if (enc_len[i] < 0 || enc_len[i] > t_max) return fail(c, GAM_ERR_SHAPE, "enc_len outside [0, t_max]");
   c->last_stream = s;
   NvtxRange range("gam.rnnt");
-  std::vector<int32_t> lo(2 * batch + 1);
+  // lengths [B], first eproj rows [B + 1], clips by decreasing length [B]
+  std::vector<int32_t> lo(3 * batch + 1);
   for (int i = 0; i < batch; ++i) lo[i] = enc_len[i];
   lo[batch] = 0;
   for (int i = 0; i < batch; ++i) lo[batch + 1 + i] = lo[batch + i] + enc_len[i];
   const int M_valid = lo[2 * batch];
+  int32_t* order = lo.data() + 2 * batch + 1;
+  for (int i = 0; i < batch; ++i) order[i] = i;
+  std::stable_sort(order, order + batch, [&](int32_t x, int32_t y) { return enc_len[x] > enc_len[y]; });
   const int* dev;
-  GAM_TRY(upload_ints(c, lo.data(), 2 * batch + 1, s, &dev));
+  GAM_TRY(upload_ints(c, lo.data(), 3 * batch + 1, s, &dev));
   const int* lens = dev;
   const int* off = dev + batch;
+  const int* ord = dev + 2 * batch + 1;
   Clips none{nullptr, 0};
   if (cfg.precision != GAM_FP32) {
     if (M_valid > 0) {
@@ -1283,7 +1289,7 @@ gam_status rnnt_greedy(gam_ctx* c, const float* enc, const int32_t* enc_len, int
     off = nullptr;  // rows b * t_max + t
   }
   return run_kernel(c, PK_RNNT_DECODE, s, [&] {
-    return launch_rnnt_greedy(r.eproj, lens, off, batch, t_max, r.gtab, r.whh, r.wp, r.bp, r.wo, r.bo, r.C, r.P,
+    return launch_rnnt_greedy(r.eproj, lens, off, ord, batch, t_max, r.gtab, r.whh, r.wp, r.bp, r.wo, r.bo, r.C, r.P,
                               r.J, r.max_symbols, r.act, max_tokens, tokens, frames, counts, c->tc.status, s);
   });
 }

@@ -17,9 +17,18 @@ pytestmark = pytest.mark.gpu
 
 GAP = 1e-3
 
+# Blank-row offsets that make each head emit a real mix of symbols and blanks on
+# unit-variance encoder frames (oracle: about 1 to 5 symbols per frame, some
+# frames at the per-frame cap); the default offset of the weight recipe would
+# decode these short random inputs to blanks only.
+BLANK_BIAS = {(34, 320, 320): 3.0, (1025, 320, 320): 4.0, (257, 320, 320): 4.0, (4096, 320, 320): 4.0,
+              (34, 64, 128): 2.0, (257, 1024, 512): 4.0}
 
-def _compare(enc, lens, Wr, C, tok, fr, cnt, max_symbols=10, act="relu", min_checked=0.75):
+
+def _compare(enc, lens, Wr, C, tok, fr, cnt, max_symbols=10, act="relu", min_checked=0.75, min_rate=0.2):
     tok, fr, cnt = tok.cpu().numpy(), fr.cpu().numpy(), cnt.cpu().numpy()
+    # the decode must exercise the emission path, not only blanks
+    assert cnt.sum() >= min_rate * max(int(np.sum(lens)), 1), (cnt.tolist(), int(np.sum(lens)))
     checked = 0
     for b in range(len(lens)):
         sym, frames, gap = oracle.rnnt_greedy_clip(enc[b, :lens[b]].astype(np.float64), Wr, C, max_symbols, act)
@@ -42,7 +51,7 @@ def test_rnnt_greedy_matches_oracle(precision, C, act):
     d = cfg["d_model"]
     B, T = 6, 60
     ctx = gam.gam_create(cfg, W, B, 40000)
-    Wr = synth.random_rnnt_weights(d, C, seed=C)
+    Wr = synth.random_rnnt_weights(d, C, seed=C, blank_bias=BLANK_BIAS[(C, 320, 320)])
     gam.gam_rnnt_attach(ctx, dict(n_classes=C, pred_dim=320, joint_dim=320, max_symbols=10, joint_act=act), Wr)
     rng = np.random.default_rng(C + 1)
     enc = rng.normal(size=(B, T, d)).astype(np.float32)
@@ -50,6 +59,30 @@ def test_rnnt_greedy_matches_oracle(precision, C, act):
     tok, fr, cnt = gam.gam_rnnt_greedy(ctx, to_torch(enc), lens)
     n = _compare(enc, lens, Wr, C, tok, fr, cnt, act=act)
     print(precision, C, act, "clips compared", n, "symbols", cnt.cpu().numpy().tolist())
+    ctx.close()
+
+
+@pytest.mark.parametrize("C,P,J,ring", [(34, 320, 320, True), (1025, 320, 320, True), (34, 64, 128, False),
+                                        (4096, 320, 320, False), (257, 1024, 512, False)])
+def test_rnnt_decoder_forms(C, P, J, ring, monkeypatch):
+    """Both decoder forms against the oracle: the cluster form with resident weight
+    slices (the default where they fit: 34 / 1025 classes at 320, and 64 / 128
+    widths) and the streaming form (forced by GAM_RNNT=ring, and taken by heads
+    whose slices do not fit: 4096 classes, or a 1024-wide predictor)."""
+    if ring:
+        monkeypatch.setenv("GAM_RNNT", "ring")
+    cfg, W = config_and_weights(small_model(layers=1), 34, "fp16")
+    d = cfg["d_model"]
+    B, T = 4, 30
+    ctx = gam.gam_create(cfg, W, B, 40000)
+    Wr = synth.random_rnnt_weights(d, C, seed=C + P, pred_dim=P, joint_dim=J, blank_bias=BLANK_BIAS[(C, P, J)])
+    gam.gam_rnnt_attach(ctx, dict(n_classes=C, pred_dim=P, joint_dim=J, max_symbols=10, joint_act="relu"), Wr)
+    enc = np.random.default_rng(C + J).normal(size=(B, T, d)).astype(np.float32)
+    lens = np.array([30, 17, 1, 29], np.int32)
+    tok, fr, cnt = gam.gam_rnnt_greedy(ctx, to_torch(enc), lens)
+    n = _compare(enc, lens, Wr, C, tok, fr, cnt)
+    print("C", C, "P", P, "J", J, "ring" if ring else "default", "clips compared", n, cnt.cpu().numpy().tolist())
+    gam.gam_device_status(ctx)
     ctx.close()
 
 
@@ -86,7 +119,7 @@ def test_rnnt_on_c2_encoder_output():
     _, W = config_and_weights(synth.V3, 34, "fp16")
     audio, lens = synth.workload_audio(name)
     ctx = gam.gam_create(cfg, W, 32, int(lens.max()))
-    Wr = synth.random_rnnt_weights(cfg["d_model"], 34)
+    Wr = synth.random_rnnt_weights(cfg["d_model"], 34, blank_bias=3.0)  # about 1 symbol per frame here
     gam.gam_rnnt_attach(ctx, dict(n_classes=34), Wr)
     enc, el = gam.gam_encode(ctx, to_torch(audio), lens)
     tok, fr, cnt = gam.gam_rnnt_greedy(ctx, enc, el)
@@ -94,7 +127,8 @@ def test_rnnt_on_c2_encoder_output():
     order = np.argsort(lens)
     sample = [order[0], order[len(order) // 2], order[-1]]
     sub = lambda x: x[sample]  # noqa: E731
-    n = _compare(enc_h[sample], el[sample], Wr, 34, sub(tok), sub(fr), sub(cnt), min_checked=0.6)
+    assert cnt.cpu().numpy().sum() >= 0.2 * int(np.sum(el))  # the batch as a whole emits symbols
+    n = _compare(enc_h[sample], el[sample], Wr, 34, sub(tok), sub(fr), sub(cnt), min_checked=0.6, min_rate=0.0)
     print("C2 RNNT clips compared", n, "symbols per clip", cnt.cpu().numpy().tolist())
     gam.gam_device_status(ctx)
     ctx.close()
