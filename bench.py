@@ -353,13 +353,14 @@ def chunk_sweep(device=0, steps=3):
     """The pages' long-form shape question ("GigaAM MLX port for Mac",
     "Which optimizations actually made the model faster": 20 s vs 40 s chunks,
     groups of 8): the 300 s chirp on the d1024 model as 15 x 20 s or 8 x 40 s
-    chunks, all in one batch or in groups of 8, with fp16 and INT8 weights."""
+    chunks, all in one batch or in groups of 8, with fp16, INT8, INT6 and INT4
+    weights; then the batch size (1 to 64 clips of 20 s) on the d1024 model."""
     import torch
     from conformer_speech_recognition_b200 import gam
     full, _ = synth.workload_audio("c5_300s_chunks15_d1024_int8")
     x = full.reshape(-1)
     out = {}
-    for prec in ("fp16", "int8_g64"):
+    for prec in ("fp16", "int8_g64", "int6_g64", "int4_g64"):
         cfg = synth.model_config(synth.LARGE, 257, prec)
         W = synth.random_weights(cfg, seed=0)
         ctx = gam.gam_create(cfg, W, 15, 40 * synth.SAMPLE_RATE, device=device)
@@ -395,6 +396,33 @@ def chunk_sweep(device=0, steps=3):
                                                                        "unit": UNIT, "ms": ms}
         finally:
             ctx.close()
+    # batch size for throughput: B clips of 20 s (the C3 clip recipe) on the d1024 model, fp16
+    cfg = synth.model_config(synth.LARGE, 257, "fp16")
+    W = synth.random_weights(cfg, seed=0)
+    audio64, lens64 = synth.workload_audio("c3_20s_b64_d768")
+    ctx = gam.gam_create(cfg, W, 64, int(lens64.max()), device=device)
+    try:
+        for B in (1, 4, 8, 16, 32, 64):
+            a = torch.from_numpy(np.ascontiguousarray(audio64[:B])).cuda(device)
+            ln = lens64[:B]
+
+            def step():
+                enc, el = gam.gam_encode(ctx, a, ln)
+                gam.gam_ctc_greedy(ctx, enc, el)
+            for _ in range(2):
+                step()
+            torch.cuda.synchronize(device)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            for _ in range(steps):
+                step()
+            e1.record()
+            torch.cuda.synchronize(device)
+            ms = e0.elapsed_time(e1) / steps
+            out[f"fp16_d1024_20s_batch_{B}"] = {"value": float(np.sum(ln)) / synth.SAMPLE_RATE / (ms / 1e3),
+                                                "unit": UNIT, "ms": ms}
+    finally:
+        ctx.close()
     return out
 
 

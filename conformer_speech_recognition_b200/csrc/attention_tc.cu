@@ -23,7 +23,7 @@
 // Q, K come from the head-major buffer [2][H][rows][64] (head dim padded to
 // 64) and V from V^T [H][64][rows]; clip starts are multiples of 8 rows so
 // every TMA x coordinate is 16-byte aligned.  All waits are bounded.
-#include <cudaTypedefs.h>
+#include <cstdint>
 
 #include "gemm_tc.cuh"
 #include "tc_common.cuh"
@@ -340,30 +340,11 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap mQK, const __grid_constant__ 
   }
 }
 
-PFN_cuTensorMapEncodeTiled_v12000 encoder() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  if (!fn) {
-    cudaDriverEntryPointQueryResult q;
-    void* f = nullptr;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
-  }
-  return fn;
-}
-
+// fp16 rows of `inner` elements, 128-byte swizzle.
 cudaError_t map2d(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t outer, uint32_t box_inner,
                   uint32_t box_outer) {
-  auto fn = encoder();
-  if (!fn) return cudaErrorNotSupported;
-  cuuint64_t dims[2] = {inner, outer};
-  cuuint64_t strides[1] = {inner * 2};
-  cuuint32_t box[2] = {box_inner, box_outer};
-  cuuint32_t es[2] = {1, 1};
-  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void*>(ptr), dims, strides, box, es,
-                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+  return tma_map_2d(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, ptr, inner, outer, inner * 2, box_inner, box_outer,
+                    CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
 }  // namespace

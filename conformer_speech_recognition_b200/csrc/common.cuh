@@ -144,8 +144,11 @@ cudaError_t launch_layernorm_rope(const float* x, const float* g, const float* b
 cudaError_t launch_layernorm_chain(float* x, const float* g1, const float* b1, const float* g2,
                                    const float* b2, float eps, void* u, int u_half, int rows, int d,
                                    cudaStream_t s);
+// Depthwise conv + folded BN + Swish.  fp16 activations with K 31 / 15 / 5 run the
+// persistent TMA-fed form (needs status, the device word a bounded wait that gave
+// up sets, and sm_count for its grid); other sizes and fp32 run the tiled forms.
 cudaError_t launch_dwconv(const void* g, const float* w, const float* bias, Clips clips, void* out, int t_half,
-                          int rows, int d, int K, cudaStream_t s);
+                          int rows, int d, int K, int sm_count, int* status, cudaStream_t s);
 cudaError_t launch_scatter_out(const float* x, Clips clips, float* out, int t_max, int d, cudaStream_t s);
 cudaError_t launch_attention_simt(const void* qk, const void* vt, Clips clips, void* o, int t_half,
                                   int rows_pad, int n_heads, int d_head, int t_max, cudaStream_t s);

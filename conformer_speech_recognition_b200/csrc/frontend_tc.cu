@@ -29,7 +29,7 @@
 // 128-column block per stage), warp 1 allocates TMEM and one thread issues the
 // MMAs, warps 2..5 run the epilogue (warp w reads TMEM lanes 32 (w % 4) ..).
 // Every wait is bounded (tc_common.cuh).
-#include <cudaTypedefs.h>
+#include <cstdint>
 
 #include "gemm_tc.cuh"
 #include "tc_common.cuh"
@@ -313,31 +313,10 @@ dft_mel_tf32_kernel(const __grid_constant__ CUtensorMap mAh, const __grid_consta
   }
 }
 
-PFN_cuTensorMapEncodeTiled_v12000 encoder() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  if (!fn) {
-    cudaDriverEntryPointQueryResult q;
-    void* f = nullptr;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
-  }
-  return fn;
-}
-
 // 2D fp32 map, rows of `inner` floats, box 32 x 128 (128-byte swizzle), zero fill.
 cudaError_t map_f32(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t outer) {
-  auto fn = encoder();
-  if (!fn) return cudaErrorNotSupported;
-  if (reinterpret_cast<uintptr_t>(ptr) & 15) return cudaErrorInvalidValue;
-  cuuint64_t dims[2] = {inner, outer};
-  cuuint64_t strides[1] = {inner * 4};
-  cuuint32_t box[2] = {KCH, 128};
-  cuuint32_t es[2] = {1, 1};
-  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<void*>(ptr), dims, strides, box, es,
-                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+  return tma_map_2d(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, ptr, inner, outer, inner * 4, KCH, 128,
+                    CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
 }  // namespace

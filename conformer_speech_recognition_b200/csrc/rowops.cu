@@ -13,7 +13,10 @@
 //  * Encoder output scatter to the padded [B, T', d] layout.
 //  * CTC: log-softmax + first-index argmax per frame, then greedy collapse
 //    (runs merged, blanks dropped) with a block-wide scan.
+#include <algorithm>
+
 #include "common.cuh"
+#include "tc_common.cuh"
 
 namespace gam {
 namespace {
@@ -459,6 +462,162 @@ dwconv_pair_kernel(const __half* __restrict__ g, const float* __restrict__ w, co
   }
 }
 
+// fp16 activations, persistent and TMA-fed.  Work items are (64 rows, 128
+// channels) tiles; each CTA walks its items with a ring of kDwStages tiles in
+// shared memory that one thread fills by TMA (halo rows included: a negative or
+// past-the-end row coordinate reads zeros), so the load of the next tiles needs
+// no registers and overlaps this tile's arithmetic.  The arithmetic is that of
+// dwconv_pair_kernel, read straight from the fp16 tile: each thread owns two
+// adjacent channels and 16 rows in 2 groups of 8, one packed fma.rn.f32x2 per tap
+// for both channels (one fp32 fma per channel, in tap order), BN folded, clip
+// edges zeroed per row.  Waits are bounded; a wait that gives up sets `status`.
+constexpr int kDwStages = 2;
+
+template <int K>
+__global__ void __launch_bounds__(256, 2)
+dwconv_tma_kernel(const __grid_constant__ CUtensorMap mG, const float* __restrict__ w, const float* __restrict__ bias,
+                  Clips clips, __half* __restrict__ out, int rows, int d, int n_items, int* status) {
+  using namespace tc;
+  constexpr int PAD = (K - 1) / 2, R = 64, HALO = R + 2 * PAD;
+  constexpr uint32_t TILE_BYTES = HALO * 128 * 2;
+  extern __shared__ __align__(128) uint8_t dw_smem[];
+  // [kDwStages][HALO][128]; rows of 256 B keep every stage 128-byte aligned
+  __half* tiles = reinterpret_cast<__half*>((reinterpret_cast<uintptr_t>(dw_smem) + 127) & ~(uintptr_t)127);
+  __shared__ uint64_t full[kDwStages];
+  __shared__ int s_lo[R], s_hi[R];
+  __shared__ int s_abort;
+  const int n_cb = d / 128;
+  if (threadIdx.x == 0) {
+    prefetch_tmap(&mG);
+    for (int i = 0; i < kDwStages; ++i) mbar_init(&full[i], 1);
+    s_abort = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  pdl_launch_dependents();
+  pdl_wait();
+  volatile int* abort_flag = &s_abort;
+  auto issue = [&](int it) {  // item number it of this CTA into stage it % kDwStages
+    const int item = blockIdx.x + it * gridDim.x;
+    if (item >= n_items) return;
+    const int st = it % kDwStages;
+    mbar_arrive_expect_tx(&full[st], TILE_BYTES);
+    tma_load_2d(tiles + (size_t)st * HALO * 128, &mG, &full[st], (item % n_cb) * 128, (item / n_cb) * R - PAD);
+  };
+  if (threadIdx.x == 0)
+    for (int it = 0; it < kDwStages; ++it) issue(it);
+  const int cc = 2 * (threadIdx.x & 63);
+  const int rbase = (threadIdx.x >> 6) * 16;
+  int cur_cb = -1;
+  unsigned long long wk[K], bv = 0;
+  int it = 0;
+  for (int item = blockIdx.x; item < n_items; item += gridDim.x, ++it) {
+    const int cb = item % n_cb, r0 = (item / n_cb) * R, c = cb * 128 + cc;
+    const int st = it % kDwStages;
+    if (threadIdx.x < R) {
+      const int r = r0 + threadIdx.x;
+      int lo = 0, hi = 0;
+      if (r < rows) {
+        const int ci = clips.find(r, 1, 0);
+        lo = clips.e(ci);
+        hi = lo + clips.L2(ci);
+      }
+      s_lo[threadIdx.x] = lo;
+      s_hi[threadIdx.x] = hi;
+    }
+    if (cb != cur_cb) {
+#pragma unroll
+      for (int k = 0; k < K; ++k) wk[k] = __ldg(reinterpret_cast<const unsigned long long*>(w + (size_t)k * d + c));
+      bv = __ldg(reinterpret_cast<const unsigned long long*>(bias + c));
+      cur_cb = cb;
+    }
+    const bool ok = mbar_wait(&full[st], (it / kDwStages) & 1, abort_flag);
+    __syncthreads();  // s_lo / s_hi written; every thread's wait has returned
+    if (__syncthreads_or(!ok)) break;
+    const __half* tile = tiles + (size_t)st * HALO * 128;
+#pragma unroll 1
+    for (int grp = 0; grp < 2; ++grp) {
+      const int j0 = rbase + grp * 8;
+      const int lo = s_lo[j0], hi = s_hi[j0];
+      const bool same = s_lo[j0 + 7] == lo;
+      const int r = r0 + j0;
+      float2 res[8];
+      if (same && r - PAD >= lo && r + 7 + PAD < hi) {
+        unsigned long long acc[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) acc[i] = bv;
+#pragma unroll
+        for (int t = 0; t < K + 7; ++t) {
+          const float2 xf = __half22float2(*reinterpret_cast<const __half2*>(tile + (j0 + t) * 128 + cc));
+          const unsigned long long x = pk2(xf.x, xf.y);
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const int k = t - i;
+            if (k >= 0 && k < K) acc[i] = fma2(wk[k], x, acc[i]);
+          }
+        }
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const float2 a = upk2(acc[i]);
+          res[i] = make_float2(swish_t<__half>(a.x), swish_t<__half>(a.y));
+        }
+      } else {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) res[i] = make_float2(0.f, 0.f);
+        int i0 = 0;
+#pragma unroll 1
+        while (i0 < 8) {
+          const int li = s_lo[j0 + i0], hiI = s_hi[j0 + i0];
+          int i1 = i0 + 1;
+          while (i1 < 8 && s_lo[j0 + i1] == li) ++i1;
+          const unsigned span = (unsigned)(hiI - li);
+          unsigned long long a[8];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) a[i] = bv;
+#pragma unroll
+          for (int t = 0; t < K + 7; ++t) {
+            unsigned long long x = 0ull;
+            if ((unsigned)(r - PAD + t - li) < span) {
+              const float2 xf = __half22float2(*reinterpret_cast<const __half2*>(tile + (j0 + t) * 128 + cc));
+              x = pk2(xf.x, xf.y);
+            }
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              const int k = t - i;
+              if (k >= 0 && k < K) a[i] = fma2(wk[k], x, a[i]);
+            }
+          }
+#pragma unroll
+          for (int i = 0; i < 8; ++i)
+            if (i >= i0 && i < i1 && (unsigned)(r + i - li) < span) {
+              const float2 q = upk2(a[i]);
+              res[i] = make_float2(swish_t<__half>(q.x), swish_t<__half>(q.y));
+            }
+          i0 = i1;
+        }
+      }
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        if (r + i >= rows) break;
+        *reinterpret_cast<__half2*>(out + (size_t)(r + i) * d + c) = __floats2half2_rn(res[i].x, res[i].y);
+      }
+    }
+    __syncthreads();  // stage st and s_lo / s_hi are free again
+    if (threadIdx.x == 0) {
+      fence_async_smem();
+      issue(it + kDwStages);
+    }
+  }
+  // loads still in flight (an early exit) land before the CTA leaves (bounded)
+  if (threadIdx.x == 0) {
+    for (int k = 0; k < kDwStages; ++k) {
+      const int item = blockIdx.x + (it + k) * gridDim.x;
+      if (item < n_items) mbar_settle(&full[(it + k) % kDwStages], ((it + k) / kDwStages) & 1, abort_flag, kWaitLimitNs);
+    }
+    if (s_abort) atomicExch(status, 1);
+  }
+}
+
 // Any other odd kernel size (<= 63): one output per thread and tap loop.
 template <typename T>
 __global__ void __launch_bounds__(256)
@@ -714,13 +873,36 @@ cudaError_t launch_layernorm_rope(const float* x, const float* g, const float* b
   return rope_t<float, 64>(x, g, b, eps, cos_tab, sin_tab, clips, u, urot, rows, d, s);
 }
 
+template <int K>
+cudaError_t dwconv_tma(const __half* g, const float* w, const float* bias, Clips clips, __half* out, int rows, int d,
+                       int sm_count, int* status, cudaStream_t s) {
+  constexpr int HALO = 64 + K - 1;
+  CUtensorMap m;
+  cudaError_t e = tma_map_2d(&m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, g, (uint64_t)d, (uint64_t)rows, (uint64_t)d * 2, 128,
+                             HALO, CU_TENSOR_MAP_SWIZZLE_NONE);
+  if (e != cudaSuccess) return e;
+  const int n_cb = d / 128, n_items = ((rows + 63) / 64) * n_cb;
+  // two resident CTAs per SM; a multiple of n_cb, so that a CTA keeps one channel block
+  int grid = std::min(n_items, 2 * sm_count);
+  if (grid >= n_cb) grid -= grid % n_cb;
+  const size_t smem = (size_t)kDwStages * HALO * 128 * 2 + 128;
+  e = cudaFuncSetAttribute(dwconv_tma_kernel<K>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  return launch_pdl(dwconv_tma_kernel<K>, grid, 256, smem, s, m, w, bias, clips, out, rows, d, n_items, status);
+}
+
 template <typename T>
 cudaError_t dwconv_t(const void* g, const float* w, const float* bias, Clips clips, void* out, int rows, int d, int K,
-                     cudaStream_t s) {
+                     int sm_count, int* status, cudaStream_t s) {
   dim3 grid((rows + 63) / 64, d / 128);
   const T* gi = (const T*)g;
   T* o = (T*)out;
-  if constexpr (sizeof(T) == 2) {  // fp16 activations: packed fp32 pairs of channels
+  if constexpr (sizeof(T) == 2) {  // fp16 activations: TMA-fed persistent form
+    if (status && !(reinterpret_cast<uintptr_t>(g) & 15)) {
+      if (K == 31) return dwconv_tma<31>(gi, w, bias, clips, o, rows, d, sm_count, status, s);
+      if (K == 5) return dwconv_tma<5>(gi, w, bias, clips, o, rows, d, sm_count, status, s);
+      if (K == 15) return dwconv_tma<15>(gi, w, bias, clips, o, rows, d, sm_count, status, s);
+    }
     if (K == 31) return launch_pdl(dwconv_pair_kernel<31>, grid, 256, 0, s, gi, w, bias, clips, o, rows, d);
     if (K == 5) return launch_pdl(dwconv_pair_kernel<5>, grid, 256, 0, s, gi, w, bias, clips, o, rows, d);
     if (K == 15) return launch_pdl(dwconv_pair_kernel<15>, grid, 256, 0, s, gi, w, bias, clips, o, rows, d);
@@ -734,10 +916,10 @@ cudaError_t dwconv_t(const void* g, const float* w, const float* bias, Clips cli
 }
 
 cudaError_t launch_dwconv(const void* g, const float* w, const float* bias, Clips clips, void* out, int t_half,
-                          int rows, int d, int K, cudaStream_t s) {
+                          int rows, int d, int K, int sm_count, int* status, cudaStream_t s) {
   if (d % 128 || K > 63 || (K & 1) == 0) return cudaErrorInvalidValue;
-  if (t_half) return dwconv_t<__half>(g, w, bias, clips, out, rows, d, K, s);
-  return dwconv_t<float>(g, w, bias, clips, out, rows, d, K, s);
+  if (t_half) return dwconv_t<__half>(g, w, bias, clips, out, rows, d, K, sm_count, status, s);
+  return dwconv_t<float>(g, w, bias, clips, out, rows, d, K, sm_count, status, s);
 }
 
 cudaError_t launch_scatter_out(const float* x, Clips clips, float* out, int t_max, int d, cudaStream_t s) {

@@ -798,7 +798,8 @@ gam_status encoder_kernels(gam_ctx* c, const Plan& p, const Clips& clips, const 
     }));
     GAM_TRY(gemm(c, PK_GEMM_PW1, s, c->u, nullptr, 0, d, w.pw1, M, EPI_GLU, 1.f, c->g, d, clips));
     GAM_TRY(run_kernel(c, PK_DWCONV, s, [&] {
-      return launch_dwconv(c->g, w.dw_w, w.dw_b, clips, c->u, ah, M, d, cfg.conv_kernel, s);
+      return launch_dwconv(c->g, w.dw_w, w.dw_b, clips, c->u, ah, M, d, cfg.conv_kernel, c->tc.sm_count,
+                           c->tc.status, s);
     }));
     GAM_TRY(gemm(c, PK_GEMM_PW2, s, c->u, nullptr, 0, d, w.pw2, M, EPI_RESID, 1.f, c->x, d, clips));
     if (l == stop_layer && stop_stage == GAM_STAGE_CONV) { stopped = true; break; }

@@ -9,6 +9,13 @@
 #include "common.cuh"
 
 namespace gam {
+
+// A 2D tensor map (tma_host.cu): `outer` rows of `inner` elements of `dtype`, rows
+// stride_bytes apart (a multiple of 16; base 16-byte aligned), box box_inner x
+// box_outer, the given swizzle, zero fill outside the tensor.
+cudaError_t tma_map_2d(CUtensorMap* m, CUtensorMapDataType dtype, const void* ptr, uint64_t inner, uint64_t outer,
+                       uint64_t stride_bytes, uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle swizzle);
+
 namespace tc {
 
 // A bounded wait gives up after this many nanoseconds (%globaltimer).  Every
