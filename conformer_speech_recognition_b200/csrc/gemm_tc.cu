@@ -84,20 +84,25 @@ __host__ __device__ constexpr bool staged_bias() {
 }
 
 // QBITS: 0 for fp16 weights, else the bits per quantised weight (8, 6 or 4).
-template <int BN, int QBITS, int EPI>
+// MT: 128-row A tiles per CTA tile (1, or 2 for quantised weights: one converted
+// B stage then feeds two accumulators, which halves the dequantisation per FLOP).
+template <int BN, int QBITS, int EPI, int MT = 1>
 struct Cfg {
   static constexpr bool QB = QBITS != 0;
   static constexpr int RAW_ROW = BK * QBITS / 8;             // bytes of one weight row per k-block as stored
+  static constexpr int A_BYTES = MT * A_TILE;                // A tiles of one stage
   static constexpr int B_TILE = BN * BK * 2;                 // fp16 B operand (128-byte swizzle)
   static constexpr int RAW_TILE = BN * RAW_ROW;              // quantised weights as loaded (unswizzled rows)
-  static constexpr int TX = A_TILE + (QB ? RAW_TILE : B_TILE);  // bytes landed by TMA per stage
-  static constexpr int STAGE = A_TILE + B_TILE + RAW_TILE;
+  static constexpr int TX = A_BYTES + (QB ? RAW_TILE : B_TILE);  // bytes landed by TMA per stage
+  static constexpr int STAGE = A_BYTES + B_TILE + RAW_TILE;
   static constexpr bool SB = staged_bias<EPI, QBITS, STAGE>();
   static constexpr int BIAS_SMEM = SB ? kBiasSmem : 0;
   static constexpr int STAGES = min8((ring_budget<EPI, QB>() - BIAS_SMEM) / STAGE);
-  // two accumulators, rounded to a power of two
-  static constexpr int TMEM_COLS = BN == 64 ? 128 : BN == 128 ? 256 : 512;
+  // two accumulators of MT x BN columns, rounded to a power of two
+  static constexpr int ACC_COLS = MT * BN;
+  static constexpr int TMEM_COLS = 2 * ACC_COLS <= 128 ? 128 : 2 * ACC_COLS <= 256 ? 256 : 512;
   static constexpr size_t SMEM = (size_t)STAGES * STAGE + epi_smem<EPI, QB>() + BIAS_SMEM + 1024 + 256;
+  static_assert(MT == 1 || (QB && BN == 128), "two M tiles per CTA tile: quantised weights, 128 columns");
 };
 
 // Hardware tanh (tanh.approx, one special-function op, relative error about
@@ -390,17 +395,17 @@ __device__ __forceinline__ void dequant16(uint4 raw, __half2 s2, uint4& out0, ui
   out1 = make_uint4(o[4], o[5], o[6], o[7]);
 }
 
-template <int BN, int EPI, int QBITS>
+template <int BN, int EPI, int QBITS, int MT>
 __global__ void __launch_bounds__(threads_of<QBITS != 0>(), 1)
 gemm_tc_kernel(const __grid_constant__ CUtensorMap mA, const __grid_constant__ CUtensorMap mA2,
                const __grid_constant__ CUtensorMap mB, const __grid_constant__ CUtensorMap mX, const TcArgs p) {
-  using C = Cfg<BN, QBITS, EPI>;
+  using C = Cfg<BN, QBITS, EPI, MT>;
   constexpr bool QB = C::QB;
   constexpr int STAGES = C::STAGES;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
-  uint8_t* sA = base;
-  uint8_t* sB = base + STAGES * A_TILE;
+  uint8_t* sA = base;                        // [STAGES][MT][A_TILE]
+  uint8_t* sB = base + STAGES * C::A_BYTES;
   uint8_t* sRaw = sB + STAGES * C::B_TILE;  // INT8 variant only
   uint8_t* sEpi = base + STAGES * C::STAGE;  // residual epilogue staging, kStageBufs tiles per warp
   uint8_t* sBias = sEpi + epi_smem<EPI, QB>();  // per-warp bias copies, kBiasStage each
@@ -448,7 +453,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap mA, const __grid_constant__ C
       bool ok = true;
       for (int tile = blockIdx.x; tile < p.tiles && ok; tile += gridDim.x) {
         const int nb = tile % p.n_blocks, mb = tile / p.n_blocks;
-        const int m0 = mb * BM, n0 = nb * BN;
+        const int m0 = mb * BM * MT, n0 = nb * BN;
         const CUtensorMap* ma = (n0 >= p.n_split) ? &mA2 : &mA;
         for (int kb = 0; kb < KB; ++kb) {
           const int s = it % STAGES;
@@ -469,7 +474,8 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap mA, const __grid_constant__ C
             ay = m0 + (t >> 1);
           }
           mbar_arrive_expect_tx(&full[s], C::TX);
-          tma_load_2d(sA + s * A_TILE, ma, &full[s], ax, ay);
+#pragma unroll
+          for (int i = 0; i < MT; ++i) tma_load_2d(sA + s * C::A_BYTES + i * A_TILE, ma, &full[s], ax, ay + i * BM);
           if (QB) tma_load_2d(sRaw + s * C::RAW_TILE, &mB, &full[s], kb * C::RAW_ROW, n0);
           else tma_load_2d(sB + s * C::B_TILE, &mB, &full[s], kb * BK, n0);
           ++it;
@@ -489,7 +495,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap mA, const __grid_constant__ C
         const uint32_t use = (uint32_t)(local >> 1);
         if (!mbar_wait(&tempty[acc], (use & 1) ^ 1, abort_flag, p.wait_ns)) break;
         tc_fence_after();
-        const uint32_t d = tmem + (uint32_t)(acc * BN);
+        const uint32_t d = tmem + (uint32_t)(acc * C::ACC_COLS);
         for (int kb = 0; kb < KB; ++kb) {
           const int s = it % STAGES;
           if (!mbar_wait(QB ? &bready[s] : &full[s], (it / STAGES) & 1, abort_flag, p.wait_ns)) {
@@ -497,10 +503,14 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap mA, const __grid_constant__ C
             break;
           }
           tc_fence_after();
-          const uint64_t da = sdesc_k_sw128(smem_u32(sA + s * A_TILE));
           const uint64_t db = sdesc_k_sw128(smem_u32(sB + s * C::B_TILE));
 #pragma unroll
-          for (int k = 0; k < BK / 16; ++k) umma_f16(d, da + 2 * k, db + 2 * k, idesc, (kb | k) != 0 ? 1u : 0u);
+          for (int i = 0; i < MT; ++i) {  // M tile i into accumulator columns [i BN, (i + 1) BN)
+            const uint64_t da = sdesc_k_sw128(smem_u32(sA + s * C::A_BYTES + i * A_TILE));
+#pragma unroll
+            for (int k = 0; k < BK / 16; ++k)
+              umma_f16(d + (uint32_t)(i * BN), da + 2 * k, db + 2 * k, idesc, (kb | k) != 0 ? 1u : 0u);
+          }
           umma_commit(&empty[s]);
           ++it;
         }
@@ -569,7 +579,8 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap mA, const __grid_constant__ C
     }
   } else {
     const int q = warp & 3;                       // TMEM lane quarter of this warp
-    const int half = (warp - 2) / 4;              // which half of the tile's columns
+    // MT 1: which half of the tile's columns; MT 2: which M tile (all its columns)
+    const int half = (warp - 2) / 4;
     constexpr bool SB = C::SB;
     BiasPrefetch<BN, SB> bias(p, half, reinterpret_cast<float*>(sBias + (warp - 2) * kBiasStage), blockIdx.x);
     uint32_t stage_seq = 0;
@@ -580,12 +591,21 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap mA, const __grid_constant__ C
       if (!mbar_wait(&tfull[acc], use & 1, abort_flag, p.wait_ns)) break;
       tc_fence_after();
       const int nb = tile % p.n_blocks, mb = tile / p.n_blocks;
-      const int r = mb * BM + q * 32 + lane;
-      const uint32_t tbase = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN);
-      const float* bt = bias.tile(p, nb * BN, tile + gridDim.x);
       constexpr int NBUF = stage_bufs<QB>();
-      epilogue_tile<BN, EPI, SB, NBUF>(p, r, nb * BN, tbase, half, &mX, sEpi + (warp - 2) * NBUF * kStageTile, bt,
-                                       stage_seq);
+      uint8_t* stage = sEpi + (warp - 2) * NBUF * kStageTile;
+      if constexpr (MT == 1) {
+        const int r = mb * BM + q * 32 + lane;
+        const uint32_t tbase = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN);
+        const float* bt = bias.tile(p, nb * BN, tile + gridDim.x);
+        epilogue_tile<BN, EPI, SB, NBUF>(p, r, nb * BN, tbase, half, &mX, stage, bt, stage_seq);
+      } else {
+        const int r = mb * BM * MT + half * BM + q * 32 + lane;
+        const uint32_t tbase =
+            tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * C::ACC_COLS) + (uint32_t)(half * BN);
+        const float* bt = bias.tile(p, nb * BN, tile + gridDim.x);
+        epilogue_tile<BN, EPI, SB, NBUF>(p, r, nb * BN, tbase, 0, &mX, stage, bt, stage_seq);
+        epilogue_tile<BN, EPI, SB, NBUF>(p, r, nb * BN, tbase, 1, &mX, stage, bt, stage_seq);
+      }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&tempty[acc]);
@@ -887,12 +907,12 @@ cudaError_t make_map_i8(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_
   return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
-template <int BN, int EPI, int QBITS>
+template <int BN, int EPI, int QBITS, int MT = 1>
 cudaError_t launch_epi(TcGemmCache* cache, const CUtensorMap& mA, const CUtensorMap& mA2, const CUtensorMap& mB,
                        const CUtensorMap& mX, const TcArgs& args, cudaStream_t s) {
-  using C = Cfg<BN, QBITS, EPI>;
+  using C = Cfg<BN, QBITS, EPI, MT>;
   constexpr bool QB = C::QB;
-  auto kern = gemm_tc_kernel<BN, EPI, QBITS>;
+  auto kern = gemm_tc_kernel<BN, EPI, QBITS, MT>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::SMEM);
   if (e != cudaSuccess) return e;
   const int grid = args.tiles < cache->sm_count ? args.tiles : cache->sm_count;
@@ -951,15 +971,15 @@ cudaError_t launch_pair(TcGemmCache* cache, const CUtensorMap& mA, const CUtenso
   }
 }
 
-template <int BN, int QBITS>
+template <int BN, int QBITS, int MT = 1>
 cudaError_t launch_bn(TcGemmCache* cache, const CUtensorMap& mA, const CUtensorMap& mA2, const CUtensorMap& mB,
                       const CUtensorMap& mX, const TcArgs& args, cudaStream_t s) {
   switch (args.epi) {
-    case EPI_SWISH: return launch_epi<BN, EPI_SWISH, QBITS>(cache, mA, mA2, mB, mX, args, s);
-    case EPI_GLU: return launch_epi<BN, EPI_GLU, QBITS>(cache, mA, mA2, mB, mX, args, s);
-    case EPI_RESID: return launch_epi<BN, EPI_RESID, QBITS>(cache, mA, mA2, mB, mX, args, s);
-    case EPI_QKV: return launch_epi<BN, EPI_QKV, QBITS>(cache, mA, mA2, mB, mX, args, s);
-    case EPI_F32: return launch_epi<BN, EPI_F32, QBITS>(cache, mA, mA2, mB, mX, args, s);
+    case EPI_SWISH: return launch_epi<BN, EPI_SWISH, QBITS, MT>(cache, mA, mA2, mB, mX, args, s);
+    case EPI_GLU: return launch_epi<BN, EPI_GLU, QBITS, MT>(cache, mA, mA2, mB, mX, args, s);
+    case EPI_RESID: return launch_epi<BN, EPI_RESID, QBITS, MT>(cache, mA, mA2, mB, mX, args, s);
+    case EPI_QKV: return launch_epi<BN, EPI_QKV, QBITS, MT>(cache, mA, mA2, mB, mX, args, s);
+    case EPI_F32: return launch_epi<BN, EPI_F32, QBITS, MT>(cache, mA, mA2, mB, mX, args, s);
     case EPI_CONV1:
       if constexpr (QBITS == 0) return launch_epi<BN, EPI_CONV1, 0>(cache, mA, mA2, mB, mX, args, s);
       return cudaErrorInvalidValue;  // the subsampling convs keep fp16 weights
@@ -971,10 +991,16 @@ cudaError_t launch_bn(TcGemmCache* cache, const CUtensorMap& mA, const CUtensorM
 }
 
 template <int QBITS>
-cudaError_t launch_width(int BN, TcGemmCache* cache, const CUtensorMap& mA, const CUtensorMap& mA2,
+cudaError_t launch_width(int BN, int mt, TcGemmCache* cache, const CUtensorMap& mA, const CUtensorMap& mA2,
                          const CUtensorMap& mB, const CUtensorMap& mX, const TcArgs& args, cudaStream_t s) {
   if (BN == 64) {  // narrow tiles: fp16 weights and few rows only
     if constexpr (QBITS == 0) return launch_bn<64, 0>(cache, mA, mA2, mB, mX, args, s);
+    return cudaErrorInvalidValue;
+  }
+  if (mt == 2) {  // two M tiles per converted B stage: quantised weights, 128 columns
+    if constexpr (QBITS != 0) {
+      if (BN == 128) return launch_bn<128, QBITS, 2>(cache, mA, mA2, mB, mX, args, s);
+    }
     return cudaErrorInvalidValue;
   }
   if (BN == 256) return launch_bn<256, QBITS>(cache, mA, mA2, mB, mX, args, s);
@@ -1001,6 +1027,8 @@ cudaError_t tc_init(TcGemmCache* cache, int device) {
     else if (!std::strcmp(v, "pair")) cache->pair_mode = 2;
     else cache->pair_mode = 1;
   }
+  // GAM_QB_TILES=m1|m2 (default m2): M tiles per CTA tile of the quantised-weight GEMMs
+  if (const char* v = std::getenv("GAM_QB_TILES")) cache->qb_mt = std::strcmp(v, "m1") ? 2 : 1;
   e = cudaMalloc(&cache->status, sizeof(int));
   if (e != cudaSuccess) return e;
   return cudaMemset(cache->status, 0, sizeof(int));
@@ -1052,6 +1080,14 @@ TileShape choose_tile(const TcGemmCache* cache, int M, int N, int epi, bool qb, 
   }
   // the "pair" policy falls back to single-CTA tiles where no paired tile applies
   if (!best.width && variant < 0 && cache->pair_mode == 2) return choose_tile(cache, M, N, epi, qb, 0, width, n_split);
+  // Quantised weights: 256 x 128 tiles whose converted B stage feeds two 128-row
+  // accumulators, unless a width other than 128 was asked for or the context
+  // selected one M tile per CTA tile (GAM_QB_TILES=m1).  Their converter warps, not
+  // the tensor core, bound these GEMMs, so halving the dequantisation per FLOP
+  // outweighs the coarser tiles.
+  if (qb && cache->qb_mt == 2 && variant <= 0 && (width == 0 || width == 128) && N % 128 == 0 &&
+      (n_split <= 0 || n_split % 128 == 0))
+    return TileShape{false, 128, 2};
   return best;
 }
 
@@ -1069,7 +1105,7 @@ cudaError_t launch_gemm_tc(TcGemmCache* cache, const void* A, const void* A2, in
   const TileShape t = choose_tile(cache, M, N, epi, qb, variant, width, A2 ? n_split : 0);
   if (!t.width) return cudaErrorInvalidValue;
   const bool pair = t.pair;
-  const int BN = t.width;
+  const int BN = t.width, mt = t.mt;
   // lda < K: stride-2 convolution view (lda = 2C, K = taps * C, C % 64 == 0); the
   // buffer behind it holds (M + 2) * lda elements, mapped as M + 2 rows of 2C.
   const bool conv = lda < K;
@@ -1087,7 +1123,7 @@ cudaError_t launch_gemm_tc(TcGemmCache* cache, const void* A, const void* A2, in
   args.M = M;
   args.N = N;
   args.K = K;
-  args.m_blocks = pair ? (M + 255) / 256 : (M + BM - 1) / BM;
+  args.m_blocks = (pair || mt == 2) ? (M + 255) / 256 : (M + BM - 1) / BM;
   args.n_blocks = N / BN;
   args.tiles = args.m_blocks * args.n_blocks;
   args.n_split = A2 ? n_split : INT_MAX;
@@ -1111,10 +1147,10 @@ cudaError_t launch_gemm_tc(TcGemmCache* cache, const void* A, const void* A2, in
     if (BN == 192) return launch_pair<192>(cache, mA, mA2, mB, mX, args, s);
     return launch_pair<128>(cache, mA, mA2, mB, mX, args, s);
   }
-  if (B.dtype == 2) return launch_width<8>(BN, cache, mA, mA2, mB, mX, args, s);
-  if (B.dtype == 3) return launch_width<6>(BN, cache, mA, mA2, mB, mX, args, s);
-  if (B.dtype == 4) return launch_width<4>(BN, cache, mA, mA2, mB, mX, args, s);
-  return launch_width<0>(BN, cache, mA, mA2, mB, mX, args, s);
+  if (B.dtype == 2) return launch_width<8>(BN, mt, cache, mA, mA2, mB, mX, args, s);
+  if (B.dtype == 3) return launch_width<6>(BN, mt, cache, mA, mA2, mB, mX, args, s);
+  if (B.dtype == 4) return launch_width<4>(BN, mt, cache, mA, mA2, mB, mX, args, s);
+  return launch_width<0>(BN, 1, cache, mA, mA2, mB, mX, args, s);
 }
 
 cudaError_t launch_attention(TcGemmCache* cache, const void* qk, const void* vt, Clips clips, void* o, int t_half,

@@ -19,6 +19,9 @@ struct TcGemmCache {
   // that stage runs out.  -1 / 0: off.
   int debug_skip = -1;
   uint64_t debug_limit_ns = 0;
+  // quantised-weight GEMMs: 128-row A tiles per CTA tile (2: one converted B stage
+  // feeds two accumulators; 1: one), GAM_QB_TILES=m1|m2
+  int qb_mt = 2;
 };
 
 // Resolves the driver's tensor-map encoder and allocates the status word.
@@ -28,8 +31,9 @@ cudaError_t tc_init(TcGemmCache* cache, int device);
 bool tc_supported(int a_dtype, int b_dtype, int N, int K, int epi);
 
 struct TileShape {
-  bool pair;  // paired-CTA (cta_group::2) tile of 256 rows, else 128 rows on one SM
-  int width;  // output columns per tile (256, 192 or 128); 0: no shape applies
+  bool pair;   // paired-CTA (cta_group::2) tile of 256 rows, else 128 rows on one SM
+  int width;   // output columns per tile (256, 192 or 128); 0: no shape applies
+  int mt = 1;  // single-CTA tiles: 128-row A tiles per tile (2: quantised weights, 256 x 128)
 };
 
 // The tile shape launch_gemm_tc uses.  variant: -1 any, 0 single-CTA only,

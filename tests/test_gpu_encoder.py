@@ -153,8 +153,12 @@ def test_c5_quantized_full_batch_sampled(name):
     ctx.close()
 
 
+@pytest.mark.parametrize("tiles", ["m1", "m2"])
 @pytest.mark.parametrize("precision", ["int8_g64", "int6_g64", "int4_g64"])
-def test_quantized_small_model(precision):
+def test_quantized_small_model(precision, tiles, monkeypatch):
+    """Both tile forms of the quantised mainloop: one 128-row A tile per converted
+    B stage (GAM_QB_TILES=m1) and two (m2, the default)."""
+    monkeypatch.setenv("GAM_QB_TILES", tiles)
     model = small_model(d=256, heads=4, ffn=512, layers=2, K=31)
     cfg, W = config_and_weights(model, 257, precision)
     audio, lens = synth.random_audio([20000, 9000], seed=5)
