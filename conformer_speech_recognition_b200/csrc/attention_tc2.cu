@@ -98,6 +98,13 @@ __device__ __forceinline__ uint64_t add_f32x2(uint64_t a, uint64_t b) {
   return d;
 }
 
+// max of three floats in one instruction (sm_100); a NaN operand is ignored, as by fmaxf
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
 __device__ __forceinline__ float fast_exp2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
@@ -250,15 +257,22 @@ attn_tc2_kernel(const __grid_constant__ CUtensorMap mQK, const __grid_constant__
       float pm[8];
 #pragma unroll
       for (int e = 0; e < 8; ++e) pm[e] = -INFINITY;
-      if (kvalid >= BK2) {
+      if (kvalid >= BK2) {  // three-input maxima: 4 per 8 scores
 #pragma unroll
-        for (int t = 0; t < BK2; ++t) pm[t & 7] = fmaxf(pm[t & 7], __uint_as_float(u[t >> 5][t & 31]));
+        for (int e = 0; e < 8; ++e) {
+          const int t = 8 * e;
+          float m = fmax3(__uint_as_float(u[t >> 5][t & 31]), __uint_as_float(u[t >> 5][(t & 31) + 1]),
+                          __uint_as_float(u[t >> 5][(t & 31) + 2]));
+          m = fmax3(m, __uint_as_float(u[t >> 5][(t & 31) + 3]), __uint_as_float(u[t >> 5][(t & 31) + 4]));
+          m = fmax3(m, __uint_as_float(u[t >> 5][(t & 31) + 5]), __uint_as_float(u[t >> 5][(t & 31) + 6]));
+          pm[e] = fmaxf(m, __uint_as_float(u[t >> 5][(t & 31) + 7]));
+        }
       } else {
 #pragma unroll
         for (int t = 0; t < BK2; ++t)
           if (t < kvalid) pm[t & 7] = fmaxf(pm[t & 7], __uint_as_float(u[t >> 5][t & 31]));
       }
-      float mx = fmaxf(fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])), fmaxf(fmaxf(pm[4], pm[5]), fmaxf(pm[6], pm[7])));
+      float mx = fmax3(fmax3(pm[0], pm[1], pm[2]), fmax3(pm[3], pm[4], pm[5]), fmaxf(pm[6], pm[7]));
       mx *= p.scale_log2;
       if (__any_sync(0xffffffffu, mx > m_used + kRescaleThreshold)) {
         // the previous P.V must have finished before O is rescaled (its phase j - 1)
