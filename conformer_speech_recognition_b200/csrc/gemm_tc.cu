@@ -847,6 +847,213 @@ gemm_tc_pair_kernel(const __grid_constant__ CUtensorMap mA, const __grid_constan
 }
 
 // ---------------------------------------------------------------------------
+// Split-K for GEMMs with few tiles (batch-1 sizes, at most 256 rows): a cluster
+// of KS CTAs (2 .. 4) computes one 128 x BN tile, CTA r over the k-blocks
+// [r KB/KS, (r+1) KB/KS), so KS times as many SMs stream the weights.  The
+// CTAs other than the leader (rank 0) push their fp32 partial accumulators into
+// the leader's shared memory (st.shared::cluster) and arrive on its barrier; the
+// leader adds them to its own accumulator in rank order -- a fixed summation
+// order, so the result does not depend on timing -- and runs the usual epilogue.
+// One tile per cluster; no second kernel.
+// ---------------------------------------------------------------------------
+constexpr int kMaxSplit = 4;
+
+template <int BN, int EPI>
+struct SplitCfg {
+  static constexpr int B_TILE = BN * BK * 2;
+  static constexpr int STAGE = A_TILE + B_TILE;
+  static constexpr int SLOT = BM * BN * 4;                 // one partial accumulator, fp32 [BM][BN]
+  static constexpr int NSLOT = BN == 64 ? kMaxSplit - 1 : 1;  // KS <= 4 at 64 columns, <= 2 at 128
+  static constexpr int EPI_SMEM = EPI == EPI_RESID ? kEpiWarps * kStageTile : 0;  // one staging tile per warp
+  static constexpr int STAGES = min8((227 * 1024 - 1280 - EPI_SMEM - NSLOT * SLOT) / STAGE);
+  static constexpr int TMEM_COLS = BN == 64 ? 64 : 128;
+  static constexpr size_t SMEM = (size_t)STAGES * STAGE + (size_t)NSLOT * SLOT + EPI_SMEM + 1024 + 256;
+};
+
+__device__ __forceinline__ uint32_t cluster_size() {
+  uint32_t n;
+  asm volatile("mov.u32 %0, %%cluster_nctarank;" : "=r"(n));
+  return n;
+}
+__device__ __forceinline__ void st_cluster_v4(uint32_t addr, float4 v) {
+  asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "f"(v.x), "f"(v.y), "f"(v.z),
+               "f"(v.w)
+               : "memory");
+}
+__device__ __forceinline__ void acc_st32(uint32_t taddr, const uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+      "%15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]),
+      "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]),
+      "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]),
+      "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31]));
+}
+
+template <int BN, int EPI>
+__global__ void __launch_bounds__(threads_of<false>(), 1)
+gemm_tc_splitk_kernel(const __grid_constant__ CUtensorMap mA, const __grid_constant__ CUtensorMap mA2,
+                      const __grid_constant__ CUtensorMap mB, const __grid_constant__ CUtensorMap mX, const TcArgs p) {
+  using C = SplitCfg<BN, EPI>;
+  constexpr int STAGES = C::STAGES;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+  uint8_t* sA = base;
+  uint8_t* sB = base + STAGES * A_TILE;
+  float* slots = reinterpret_cast<float*>(base + STAGES * C::STAGE);  // [NSLOT][BM][BN], filled by ranks 1..KS-1
+  uint8_t* sEpi = reinterpret_cast<uint8_t*>(slots) + C::NSLOT * C::SLOT;
+  uint64_t* full = reinterpret_cast<uint64_t*>(sEpi + C::EPI_SMEM);
+  uint64_t* empty = full + STAGES;
+  uint64_t* tfull = empty + STAGES;
+  uint64_t* parts = tfull + 1;  // leader: every partial has arrived
+  uint64_t* drain = parts + 1;
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tslot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int ks = (int)cluster_size(), rank = (int)cluster_rank();
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    mbar_init(tfull, 1);
+    mbar_init(parts, (ks - 1) * kEpiWarps > 0 ? (ks - 1) * kEpiWarps : 1);
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&mA);
+    prefetch_tmap(&mA2);
+    prefetch_tmap(&mB);
+  }
+  if (warp == 1) tmem_alloc(tslot, C::TMEM_COLS);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  cluster_sync_all();  // the leader's barriers are initialised before any remote arrive
+  const uint32_t tmem = *tslot;
+  pdl_launch_dependents();
+  pdl_wait();
+
+  const int tile = blockIdx.x / ks;
+  const int nb = tile % p.n_blocks, mb = tile / p.n_blocks;
+  const int m0 = mb * BM, n0 = nb * BN;
+  const int KB = p.K / BK, kb0 = rank * KB / ks, kb1 = (rank + 1) * KB / ks;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      const CUtensorMap* ma = (n0 >= p.n_split) ? &mA2 : &mA;
+      int it = 0;
+      for (int kb = kb0; kb < kb1; ++kb, ++it) {
+        const int s = it % STAGES;
+        if (!mbar_wait(&empty[s], ((it / STAGES) & 1) ^ 1, abort_flag, p.wait_ns)) break;
+        mbar_arrive_expect_tx(&full[s], A_TILE + C::B_TILE);
+        tma_load_2d(sA + s * A_TILE, ma, &full[s], kb * BK, m0);
+        tma_load_2d(sB + s * C::B_TILE, &mB, &full[s], kb * BK, n0);
+      }
+      const int first = it > STAGES ? it - STAGES : 0;
+      for (int j = first; j < it; ++j) mbar_settle(&full[j % STAGES], (j / STAGES) & 1, abort_flag, p.wait_ns);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_f16_f32(BM, BN);
+      bool ok = true;
+      int it = 0;
+      for (int kb = kb0; kb < kb1; ++kb, ++it) {
+        const int s = it % STAGES;
+        if (!mbar_wait(&full[s], (it / STAGES) & 1, abort_flag, p.wait_ns)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint64_t da = sdesc_k_sw128(smem_u32(sA + s * A_TILE));
+        const uint64_t db = sdesc_k_sw128(smem_u32(sB + s * C::B_TILE));
+#pragma unroll
+        for (int k = 0; k < BK / 16; ++k) umma_f16(tmem, da + 2 * k, db + 2 * k, idesc, (it | k) != 0 ? 1u : 0u);
+        umma_commit(&empty[s]);
+      }
+      if (ok) umma_commit(tfull);
+      umma_commit(drain);
+      mbar_settle(drain, 0, abort_flag, p.wait_ns);
+    }
+  } else {
+    const int q = warp & 3, half = (warp - 2) / 4;
+    const int row = q * 32 + lane, r = m0 + row;
+    const uint32_t tbase = tmem + ((uint32_t)(q * 32) << 16);
+    const int c_lo = half * (BN / 2), c_hi = c_lo + BN / 2;
+    bool ok = __all_sync(0xffffffffu, mbar_wait(tfull, 0, abort_flag, p.wait_ns));
+    tc_fence_after();
+    if (rank != 0) {
+      // push this CTA's partial accumulator into slot rank - 1 of the leader
+      if (ok) {
+        float* slot = slots + (size_t)(rank - 1) * BM * BN + (size_t)row * BN;
+        for (int c = c_lo; c < c_hi; c += 32) {
+          uint32_t u[32];
+          tmem_ld32(tbase + c, u);
+          tmem_ld_wait();
+          const uint32_t dst = map_to_cta(slot + c, 0);
+#pragma unroll
+          for (int j = 0; j < 8; ++j)
+            st_cluster_v4(dst + 16 * j, make_float4(__uint_as_float(u[4 * j]), __uint_as_float(u[4 * j + 1]),
+                                                    __uint_as_float(u[4 * j + 2]), __uint_as_float(u[4 * j + 3])));
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive_remote(map_to_cta(parts, 0));  // release: the stores above come first
+    } else {
+      if (ks > 1 && ok) {
+        ok = __all_sync(0xffffffffu, mbar_wait(parts, 0, abort_flag, p.wait_ns));
+        asm volatile("fence.acq_rel.cluster;" ::: "memory");
+      }
+      // own accumulator + partials of ranks 1 .. KS-1, in that order, back into TMEM
+      if (ok) {
+        if (ks > 1) {
+          for (int c = c_lo; c < c_hi; c += 32) {
+            uint32_t u[32];
+            tmem_ld32(tbase + c, u);
+            tmem_ld_wait();
+            for (int sidx = 0; sidx < ks - 1; ++sidx) {
+              const float4* src = reinterpret_cast<const float4*>(slots + (size_t)sidx * BM * BN + (size_t)row * BN + c);
+#pragma unroll
+              for (int j = 0; j < 8; ++j) {
+                const float4 v = src[j];
+                u[4 * j] = __float_as_uint(__uint_as_float(u[4 * j]) + v.x);
+                u[4 * j + 1] = __float_as_uint(__uint_as_float(u[4 * j + 1]) + v.y);
+                u[4 * j + 2] = __float_as_uint(__uint_as_float(u[4 * j + 2]) + v.z);
+                u[4 * j + 3] = __float_as_uint(__uint_as_float(u[4 * j + 3]) + v.w);
+              }
+            }
+            acc_st32(tbase + c, u);
+          }
+          asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+        }
+      }
+      // every epilogue warp's sums are in TMEM before any epilogue reads them (the GLU
+      // epilogue of one column half reads the other half's gate columns); reached by
+      // all 8 epilogue warps of the leader whatever `ok` is
+      tc_fence_before();
+      asm volatile("bar.sync 1, %0;" ::"r"(32 * kEpiWarps) : "memory");
+      tc_fence_after();
+      if (ok) {
+        uint32_t stage_seq = 0;
+        epilogue_tile<BN, EPI, false, 1>(p, r, n0, tbase, half, &mX, sEpi + (warp - 2) * kStageTile, p.ep.bias + n0,
+                                         stage_seq);
+      }
+      if (EPI == EPI_RESID && lane == 0) bulk_wait0();  // reductions complete before the CTA exits
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (threadIdx.x == 0 && *abort_flag) atomicExch(p.status, 1);
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
+// ---------------------------------------------------------------------------
 // host side
 // ---------------------------------------------------------------------------
 
@@ -1008,6 +1215,62 @@ cudaError_t launch_width(int BN, int mt, TcGemmCache* cache, const CUtensorMap& 
   return launch_bn<128, QBITS>(cache, mA, mA2, mB, mX, args, s);
 }
 
+template <int BN, int EPI>
+cudaError_t launch_split_epi(const CUtensorMap& mA, const CUtensorMap& mA2, const CUtensorMap& mB,
+                             const CUtensorMap& mX, const TcArgs& args, int ks, cudaStream_t s) {
+  using C = SplitCfg<BN, EPI>;
+  auto kern = gemm_tc_splitk_kernel<BN, EPI>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::SMEM);
+  if (e != cudaSuccess) return e;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = ks;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(args.tiles * ks);
+  cfg.blockDim = dim3(threads_of<false>());
+  cfg.dynamicSmemBytes = C::SMEM;
+  cfg.stream = s;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl_enabled() ? 2 : 1;
+  e = cudaLaunchKernelEx(&cfg, kern, mA, mA2, mB, mX, args);
+  if (e != cudaSuccess) return e;
+  return cudaGetLastError();
+}
+
+cudaError_t launch_split(int BN, const CUtensorMap& mA, const CUtensorMap& mA2, const CUtensorMap& mB,
+                         const CUtensorMap& mX, const TcArgs& args, int ks, cudaStream_t s) {
+  if (BN == 128) {
+    if (args.epi == EPI_GLU) return launch_split_epi<128, EPI_GLU>(mA, mA2, mB, mX, args, ks, s);
+    return cudaErrorInvalidValue;
+  }
+  switch (args.epi) {
+    case EPI_SWISH: return launch_split_epi<64, EPI_SWISH>(mA, mA2, mB, mX, args, ks, s);
+    case EPI_RESID: return launch_split_epi<64, EPI_RESID>(mA, mA2, mB, mX, args, ks, s);
+    case EPI_QKV: return launch_split_epi<64, EPI_QKV>(mA, mA2, mB, mX, args, ks, s);
+    case EPI_F32: return launch_split_epi<64, EPI_F32>(mA, mA2, mB, mX, args, ks, s);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+// Split count for a GEMM of few rows: the largest KS in 2 .. 4 (2 for the GLU's
+// 128-column tiles) that divides the k-blocks and leaves each CTA at least two
+// of them (forced), or -- chosen by the library -- at least eight, with tiles x KS
+// within the SMs.  Measured at batch 1 (d768): the cluster's fixed cost (launch,
+// partial-sum exchange) pays off only for deep K (FFN down, K = 3072: 0.73 ->
+// 0.67 ms per step); at K = 768 a split made FFN up, QKV and the output
+// projection slower.  0 when none applies.
+int split_count(const TcGemmCache* cache, int M, int N, int K, int bn, bool forced) {
+  const int tiles = ((M + BM - 1) / BM) * (N / bn);
+  const int KB = K / BK;
+  for (int c = bn == 64 ? kMaxSplit : 2; c >= 2; --c)
+    if (KB % c == 0 && (forced ? KB / c >= 2 : (KB / c >= 8 && tiles * c <= cache->sm_count))) return c;
+  return 0;
+}
+
 }  // namespace
 
 bool tc_supported(int a_dtype, int b_dtype, int N, int K, int epi) {
@@ -1027,6 +1290,8 @@ cudaError_t tc_init(TcGemmCache* cache, int device) {
     else if (!std::strcmp(v, "pair")) cache->pair_mode = 2;
     else cache->pair_mode = 1;
   }
+  // GAM_SPLITK=0: no split-K for GEMMs of few rows
+  if (const char* v = std::getenv("GAM_SPLITK")) cache->splitk = std::strcmp(v, "0") != 0;
   // GAM_QB_TILES=m1|m2 (default m2): M tiles per CTA tile of the quantised-weight GEMMs
   if (const char* v = std::getenv("GAM_QB_TILES")) cache->qb_mt = std::strcmp(v, "m1") ? 2 : 1;
   e = cudaMalloc(&cache->status, sizeof(int));
@@ -1102,6 +1367,42 @@ cudaError_t launch_gemm_tc(TcGemmCache* cache, const void* A, const void* A2, in
   const bool qb = B.dtype >= 2;  // INT8 / INT6 / INT4 g64 weights: dequantised in the mainloop
   const int qbits = B.dtype == 2 ? 8 : B.dtype == 3 ? 6 : 4;
   if (qb && !B.scale_t) return cudaErrorInvalidValue;
+  // Few rows (batch-1 sizes): split K over a cluster when that multiplies the SMs
+  // streaming the weights (variant 2 forces it).  fp16 weights, plain A operand.
+  if (variant == 2 || (variant < 0 && width == 0 && cache->splitk && M <= 256)) {
+    const int bn = epi == EPI_GLU ? 128 : 64;
+    const bool fits = B.dtype == 1 && lda >= K && M <= 256 && N % bn == 0 && (!A2 || n_split % bn == 0) &&
+                      (epi == EPI_SWISH || epi == EPI_GLU || epi == EPI_RESID || epi == EPI_QKV || epi == EPI_F32);
+    const int ks = fits ? split_count(cache, M, N, K, bn, variant == 2) : 0;
+    if (ks >= 2) {
+      CUtensorMap mA, mA2, mB, mX;
+      cudaError_t e = make_map_f16(&mA, A, K, M, (uint64_t)lda * 2, BK, BM);
+      if (e == cudaSuccess) e = make_map_f16(&mA2, A2 ? A2 : A, K, M, (uint64_t)lda * 2, BK, BM);
+      if (e == cudaSuccess) e = make_map_f16(&mB, B.w, K, N, (uint64_t)K * 2, BK, bn);
+      mX = mB;
+      if (e == cudaSuccess && epi == EPI_RESID) e = make_map_f32(&mX, ep.x, N, M, (uint64_t)ep.ldo * 4, 32, 32);
+      if (e != cudaSuccess) return e;
+      TcArgs args;
+      args.M = M;
+      args.N = N;
+      args.K = K;
+      args.m_blocks = (M + BM - 1) / BM;
+      args.n_blocks = N / bn;
+      args.tiles = args.m_blocks * args.n_blocks;
+      args.n_split = A2 ? n_split : INT_MAX;
+      args.conv_c = 0;
+      args.epi = epi;
+      args.ep = ep;
+      args.scale_t = nullptr;
+      args.status = cache->status;
+      args.wait_ns = cache->debug_limit_ns ? cache->debug_limit_ns : kWaitLimitNs;
+      args.debug_skip = -1;
+      cache->debug_limit_ns = 0;
+      cache->debug_skip = -1;
+      return launch_split(bn, mA, mA2, mB, mX, args, ks, s);
+    }
+    if (variant == 2) return cudaErrorInvalidValue;  // forced, but no split applies
+  }
   const TileShape t = choose_tile(cache, M, N, epi, qb, variant, width, A2 ? n_split : 0);
   if (!t.width) return cudaErrorInvalidValue;
   const bool pair = t.pair;

@@ -22,6 +22,9 @@ struct TcGemmCache {
   // quantised-weight GEMMs: 128-row A tiles per CTA tile (2: one converted B stage
   // feeds two accumulators; 1: one), GAM_QB_TILES=m1|m2
   int qb_mt = 2;
+  // fp16 GEMMs of at most 256 rows: split K over a cluster of 2 .. 4 CTAs when that
+  // puts more SMs on the weight stream (GAM_SPLITK=0 turns it off)
+  bool splitk = true;
 };
 
 // Resolves the driver's tensor-map encoder and allocates the status word.
@@ -43,6 +46,10 @@ struct TileShape {
 TileShape choose_tile(const TcGemmCache* cache, int M, int N, int epi, bool int8_weights, int variant, int width,
                       int n_split = 0);
 
+// One tensor-core GEMM with a fused epilogue.  variant as for choose_tile, plus
+// 2: split K over a cluster (fp16 weights, at most 256 rows; fails where no split
+// applies).  With variant -1, width 0 and at most 256 rows the library splits K
+// by itself when that helps (TcGemmCache::splitk).
 cudaError_t launch_gemm_tc(TcGemmCache* cache, const void* A, const void* A2, int n_split, int lda, WeightOp B,
                            int M, int N, int K, int epi, const EpiParams& ep, cudaStream_t s, int variant = -1,
                            int width = 0);

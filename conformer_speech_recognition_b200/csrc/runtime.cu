@@ -1566,13 +1566,15 @@ gam_status gam_debug_gemm(gam_ctx* c, int impl, const void* a, int lda, const vo
   ep.ldo = ldo;
   WeightOp W{w, nullptr, 1, nullptr};
   const int kind = impl & 0xff, width = impl >> 8;
-  if (impl < 0 || kind > 3 || (kind == 1 && width) ||
+  if (impl < 0 || kind > 4 || ((kind == 1 || kind == 4) && width) ||
       (width && width != 64 && width != 128 && width != 192 && width != 256) || (width == 64 && kind == 3))
-    return fail(c, GAM_ERR_INVALID_ARG, "impl: kind 0 .. 3 plus (tile width 64 (single-CTA), 128, 192 or 256) << 8");
+    return fail(c, GAM_ERR_INVALID_ARG, "impl: kind 0 .. 4 plus (tile width 64 (single-CTA), 128, 192 or 256) << 8");
   if (kind != 1) {
     if (!tc_supported(1, 1, n, k, EPI_RESID)) return fail(c, GAM_ERR_SHAPE, "tensor-core GEMM needs N % 256 == 0, K % 64 == 0");
-    const int variant = kind == 0 ? -1 : kind == 2 ? 0 : 1;
-    if (!choose_tile(&c->tc, m, n, EPI_RESID, false, variant, width).width)
+    const int variant = kind == 0 ? -1 : kind == 2 ? 0 : kind == 3 ? 1 : 2;
+    if (kind == 4 && (m > 256 || lda < k))
+      return fail(c, GAM_ERR_SHAPE, "split-K GEMM: at most 256 rows, plain A operand");
+    if (kind != 4 && !choose_tile(&c->tc, m, n, EPI_RESID, false, variant, width).width)
       return fail(c, GAM_ERR_SHAPE, "no tile of that width divides N");
     return run_kernel(c, PK_MISC, s, [&] {
       return launch_gemm_tc(&c->tc, a, nullptr, 0, lda, W, m, n, k, EPI_RESID, ep, s, variant, width);

@@ -388,7 +388,11 @@ gam_status gam_graphs_enable(gam_ctx* ctx, int on);
  * rows on two SMs, cta_group::2); width 0 lets the library choose the tile
  * width, else 128, 192 or 256 output columns, or 64 with single-CTA tiles of at
  * most 256 rows (tensor-core kinds only; the library picks 64 for such few rows
- * so that more SMs share the weight stream).
+ * so that more SMs share the weight stream); 4 = tensor cores with K split over
+ * a cluster of 2 to 4 CTAs whose partial sums the first CTA adds in a fixed
+ * order (at most 256 rows, lda >= k, width 0; the library also picks this for
+ * such few rows when K is deep enough to leave each CTA at least 8 k-blocks of
+ * 64; GAM_ERR_SHAPE, or GAM_ERR_CUDA when no split count applies to the shape).
  * N % 256 == 0 and K % 64 == 0 for the tensor-core kinds, N % 128 == 0 and
  * K % 16 == 0 for CUDA cores; a width that does not divide N fails with
  * GAM_ERR_SHAPE, an impl outside these values with GAM_ERR_INVALID_ARG.

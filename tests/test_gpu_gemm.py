@@ -1,9 +1,9 @@
 """Unit parity of the encoder's GEMM kernels through the C ABI (gam_debug_gemm):
 out += A . W^T + bias with fp16 operands and fp32 accumulation, for the
 tensor-core (tcgen05) and CUDA-core implementations, against NumPy in fp64.
-impl 0 lets the library choose the tile shape, 2 forces single-CTA tiles and
-3 paired-CTA (cta_group::2) tiles; a tile width (128, 192, 256) shifted left by
-8 bits forces the width too."""
+impl 0 lets the library choose the tile shape, 2 forces single-CTA tiles,
+3 paired-CTA (cta_group::2) tiles and 4 K split over a cluster; a tile width
+(128, 192, 256) shifted left by 8 bits forces the width too."""
 import numpy as np
 import pytest
 
@@ -90,3 +90,14 @@ def test_gemm_width_must_divide_n(ctx):
         gam.gam_debug_gemm(ctx, 3 | (192 << 8), a, w, b, o)
     with pytest.raises(gam.GamError):
         gam.gam_debug_gemm(ctx, 3 | (100 << 8), a, w, b, o)
+
+
+@pytest.mark.parametrize("M,N,K", [(24, 768, 3072), (25, 768, 768), (200, 3072, 768), (129, 2304, 768),
+                                   (256, 768, 1536), (1, 256, 512)],
+                         ids=["batch1_ffn_down", "batch1_out_proj", "ffn_up_two_m_blocks", "qkv_ragged",
+                              "two_full_m_blocks", "one_row"])
+def test_gemm_split_k(ctx, M, N, K):
+    """K split over a cluster of 2 to 4 CTAs, the leader adding the partial sums
+    in rank order: forced (kind 4) and as the library chooses for few rows."""
+    test_gemm_parity(ctx, 4, M, N, K, K)
+    test_gemm_parity(ctx, 0, M, N, K, K)
