@@ -101,3 +101,35 @@ def test_transcribe_repeats_match(model):
         for i in range(2):
             assert np.array_equal(t[i, :c[i]], results[0][0][i, :c[i]])
     ctx.close()
+
+
+def test_more_keys_than_graph_slots(model):
+    """20 call keys against 16 table slots, called round-robin four times with
+    fresh audio each round: eager, captured (the last four evict the first four),
+    replayed or eager again, then the first four recaptured into slots whose last
+    replay may still be queued.  Every call must equal an eager run bit for bit."""
+    cfg, W = model
+    cfg = dict(cfg, n_layers=1)
+    W = {k: v for k, v in W.items() if not k.startswith("layers.") or k.startswith("layers.0.")}
+    n_keys = 20
+    lens_of = [[16000 + 1280 * k] for k in range(n_keys)]
+    ctx = gam.gam_create(cfg, W, 1, 48000)
+    eager = gam.gam_create(cfg, W, 1, 48000)
+    gam.gam_graphs_enable(eager, False)
+    outs = []
+    for lens in lens_of:
+        _, el, _, tmax = gam.gam_plan_lengths(cfg, lens)
+        outs.append(torch.empty((1, tmax, cfg["d_model"]), dtype=torch.float32, device="cuda"))
+    audio = torch.empty((1, 48000), dtype=torch.float32, device="cuda")
+    for rnd in range(4):
+        for k, lens in enumerate(lens_of):
+            a_np, _ = synth.random_audio([48000], seed=1000 * rnd + k)
+            audio.copy_(to_torch(a_np))
+            outs[k].fill_(float("nan"))
+            gam.gam_encode(ctx, audio, lens, out=outs[k])
+            ref, el = gam.gam_encode(eager, audio, lens)
+            torch.cuda.synchronize()
+            assert np.array_equal(outs[k].cpu().numpy()[0, :el[0]], ref.cpu().numpy()[0, :el[0]]), (rnd, k)
+    gam.gam_device_status(ctx)
+    ctx.close()
+    eager.close()
