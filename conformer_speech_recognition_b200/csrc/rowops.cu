@@ -344,133 +344,15 @@ __device__ __forceinline__ unsigned long long fma2(unsigned long long a, unsigne
   return d;
 }
 
-// fp16 activations: the same tile and clip handling as dwconv_kernel, but each
-// thread owns a pair of adjacent channels (one 64-bit shared-memory load and one
-// packed FMA per tap for both) and 16 rows in 2 groups of 8.  Every multiply-add
-// is still one fp32 fma per channel, in the same tap order.
-template <int K>
-__global__ void __launch_bounds__(256)
-dwconv_pair_kernel(const __half* __restrict__ g, const float* __restrict__ w, const float* __restrict__ bias,
-                   Clips clips, __half* __restrict__ out, int rows, int d) {
-  pdl_launch_dependents();
-  pdl_wait();
-  constexpr int PAD = (K - 1) / 2, R = 64, HALO = R + 2 * PAD;
-  __shared__ __align__(16) float tile[HALO][128];
-  __shared__ int s_lo[R], s_hi[R];
-  const int r0 = blockIdx.x * R, c0 = blockIdx.y * 128;
-  constexpr int ITEMS = (HALO * 32 + 255) / 256;
-  float4 v[ITEMS];
-#pragma unroll
-  for (int it = 0; it < ITEMS; ++it) {
-    const int idx = threadIdx.x + it * 256;
-    const int rr = idx >> 5, c4 = (idx & 31) * 4;
-    const int src = r0 - PAD + rr;
-    v[it] = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (idx < HALO * 32 && src >= 0 && src < rows) {
-      const uint2 raw = __ldg(reinterpret_cast<const uint2*>(g + (size_t)src * d + c0 + c4));
-      const float2 a = __half22float2(*reinterpret_cast<const __half2*>(&raw.x));
-      const float2 b = __half22float2(*reinterpret_cast<const __half2*>(&raw.y));
-      v[it] = make_float4(a.x, a.y, b.x, b.y);
-    }
-  }
-#pragma unroll
-  for (int it = 0; it < ITEMS; ++it) {
-    const int idx = threadIdx.x + it * 256;
-    if (idx < HALO * 32) *reinterpret_cast<float4*>(&tile[idx >> 5][(idx & 31) * 4]) = v[it];
-  }
-  if (threadIdx.x < R) {
-    const int r = r0 + threadIdx.x;
-    int lo = 0, hi = 0;
-    if (r < rows) {
-      const int ci = clips.find(r, 1, 0);
-      lo = clips.e(ci);
-      hi = lo + clips.L2(ci);
-    }
-    s_lo[threadIdx.x] = lo;
-    s_hi[threadIdx.x] = hi;
-  }
-  __syncthreads();
-  const int cc = 2 * (threadIdx.x & 63), c = c0 + cc;
-  unsigned long long wk[K];
-#pragma unroll
-  for (int k = 0; k < K; ++k) wk[k] = __ldg(reinterpret_cast<const unsigned long long*>(w + (size_t)k * d + c));
-  const unsigned long long bv = __ldg(reinterpret_cast<const unsigned long long*>(bias + c));
-  const int rbase = (threadIdx.x >> 6) * 16;
-#pragma unroll 1
-  for (int grp = 0; grp < 2; ++grp) {
-    const int j0 = rbase + grp * 8;
-    const int lo = s_lo[j0], hi = s_hi[j0];
-    const bool same = s_lo[j0 + 7] == lo;
-    const int r = r0 + j0;
-    float2 res[8];
-    if (same && r - PAD >= lo && r + 7 + PAD < hi) {
-      unsigned long long acc[8];
-#pragma unroll
-      for (int i = 0; i < 8; ++i) acc[i] = bv;
-#pragma unroll
-      for (int t = 0; t < K + 7; ++t) {
-        const unsigned long long x = *reinterpret_cast<const unsigned long long*>(&tile[j0 + t][cc]);
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const int k = t - i;
-          if (k >= 0 && k < K) acc[i] = fma2(wk[k], x, acc[i]);
-        }
-      }
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const float2 a = upk2(acc[i]);
-        res[i] = make_float2(swish_t<__half>(a.x), swish_t<__half>(a.y));
-      }
-    } else {
-#pragma unroll
-      for (int i = 0; i < 8; ++i) res[i] = make_float2(0.f, 0.f);
-      int i0 = 0;
-#pragma unroll 1
-      while (i0 < 8) {
-        const int li = s_lo[j0 + i0], hiI = s_hi[j0 + i0];
-        int i1 = i0 + 1;
-        while (i1 < 8 && s_lo[j0 + i1] == li) ++i1;
-        const unsigned span = (unsigned)(hiI - li);
-        unsigned long long a[8];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) a[i] = bv;
-#pragma unroll
-        for (int t = 0; t < K + 7; ++t) {
-          const unsigned long long x = ((unsigned)(r - PAD + t - li) < span)
-                                           ? *reinterpret_cast<const unsigned long long*>(&tile[j0 + t][cc])
-                                           : 0ull;
-#pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            const int k = t - i;
-            if (k >= 0 && k < K) a[i] = fma2(wk[k], x, a[i]);
-          }
-        }
-#pragma unroll
-        for (int i = 0; i < 8; ++i)
-          if (i >= i0 && i < i1 && (unsigned)(r + i - li) < span) {
-            const float2 q = upk2(a[i]);
-            res[i] = make_float2(swish_t<__half>(q.x), swish_t<__half>(q.y));
-          }
-        i0 = i1;
-      }
-    }
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      if (r + i >= rows) break;
-      *reinterpret_cast<__half2*>(out + (size_t)(r + i) * d + c) = __floats2half2_rn(res[i].x, res[i].y);
-    }
-  }
-}
-
 // fp16 activations, persistent and TMA-fed.  Work items are (64 rows, 128
 // channels) tiles; each CTA walks its items with a ring of kDwStages tiles in
 // shared memory that one thread fills by TMA (halo rows included: a negative or
 // past-the-end row coordinate reads zeros), so the load of the next tiles needs
-// no registers and overlaps this tile's arithmetic.  The arithmetic is that of
-// dwconv_pair_kernel, read straight from the fp16 tile: each thread owns two
-// adjacent channels and 16 rows in 2 groups of 8, one packed fma.rn.f32x2 per tap
-// for both channels (one fp32 fma per channel, in tap order), BN folded, clip
-// edges zeroed per row.  Waits are bounded; a wait that gives up sets `status`.
+// no registers and overlaps this tile's arithmetic, which reads the fp16 tile
+// directly: each thread owns two adjacent channels and 16 rows in 2 groups of 8,
+// one packed fma.rn.f32x2 per tap for both channels (one fp32 fma per channel, in
+// tap order), BN folded; a group of 8 rows that meets a clip edge runs once per
+// clip among its rows with the inputs outside that clip zeroed.  Waits are bounded; a wait that gives up sets `status`.
 constexpr int kDwStages = 2;
 
 template <int K>
@@ -898,14 +780,10 @@ cudaError_t dwconv_t(const void* g, const float* w, const float* bias, Clips cli
   const T* gi = (const T*)g;
   T* o = (T*)out;
   if constexpr (sizeof(T) == 2) {  // fp16 activations: TMA-fed persistent form
-    if (status && !(reinterpret_cast<uintptr_t>(g) & 15)) {
-      if (K == 31) return dwconv_tma<31>(gi, w, bias, clips, o, rows, d, sm_count, status, s);
-      if (K == 5) return dwconv_tma<5>(gi, w, bias, clips, o, rows, d, sm_count, status, s);
-      if (K == 15) return dwconv_tma<15>(gi, w, bias, clips, o, rows, d, sm_count, status, s);
-    }
-    if (K == 31) return launch_pdl(dwconv_pair_kernel<31>, grid, 256, 0, s, gi, w, bias, clips, o, rows, d);
-    if (K == 5) return launch_pdl(dwconv_pair_kernel<5>, grid, 256, 0, s, gi, w, bias, clips, o, rows, d);
-    if (K == 15) return launch_pdl(dwconv_pair_kernel<15>, grid, 256, 0, s, gi, w, bias, clips, o, rows, d);
+    if (!status || (reinterpret_cast<uintptr_t>(g) & 15)) return cudaErrorInvalidValue;
+    if (K == 31) return dwconv_tma<31>(gi, w, bias, clips, o, rows, d, sm_count, status, s);
+    if (K == 5) return dwconv_tma<5>(gi, w, bias, clips, o, rows, d, sm_count, status, s);
+    if (K == 15) return dwconv_tma<15>(gi, w, bias, clips, o, rows, d, sm_count, status, s);
   }
   if (K == 31) return launch_pdl(dwconv_kernel<T, 31>, grid, 256, 0, s, gi, w, bias, clips, o, rows, d);
   if (K == 5) return launch_pdl(dwconv_kernel<T, 5>, grid, 256, 0, s, gi, w, bias, clips, o, rows, d);
