@@ -293,7 +293,13 @@ gam_status gam_rnnt_attach(gam_ctx* ctx, const gam_rnnt_config* cfg, const gam_t
  * max_tokens]): the encoder frame of each symbol, -1 after the last;
  * counts_dev device i32 [batch]: symbols stored (at most max_tokens; symbols
  * past max_tokens are decoded but not stored, and t_max * max_symbols never
- * loses any). */
+ * loses any).  The encoder half of the joint is one tensor-core GEMM over all
+ * valid frames; the loop is one kernel, by default a cluster of 8 CTAs per clip
+ * holding the head's weights in shared memory; heads whose weight slices do not
+ * fit (e.g. 4096 classes or a 1024-wide predictor) stream the weights through
+ * one CTA per clip instead, and GAM_RNNT=ring in the environment forces that
+ * form.  Clips with more decisions take longer; the call's time is that of the
+ * slowest clip. */
 gam_status gam_rnnt_greedy(gam_ctx* ctx, const float* enc_dev, const int32_t* enc_len_host, int batch, int t_max,
                            int max_tokens, int32_t* tokens_dev, int32_t* frames_dev, int32_t* counts_dev,
                            void* stream);
