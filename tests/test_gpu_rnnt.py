@@ -45,7 +45,7 @@ def _compare(enc, lens, Wr, C, tok, fr, cnt, max_symbols=10, act="relu", min_che
 
 
 @pytest.mark.parametrize("precision,C,act", [("fp16", 34, "relu"), ("fp16", 1025, "relu"), ("int8_g64", 257, "relu"),
-                                             ("fp32", 34, "relu"), ("fp16", 34, "tanh")])
+                                             ("int4_g64", 34, "relu"), ("fp32", 34, "relu"), ("fp16", 34, "tanh")])
 def test_rnnt_greedy_matches_oracle(precision, C, act):
     cfg, W = config_and_weights(small_model(layers=1), 34, precision)
     d = cfg["d_model"]
