@@ -1456,10 +1456,9 @@ cudaError_t launch_gemm_tc(TcGemmCache* cache, const void* A, const void* A2, in
 
 cudaError_t launch_attention(TcGemmCache* cache, const void* qk, const void* vt, Clips clips, void* o, int t_half,
                              int rows_pad, int n_heads, int d_head, int t_max, cudaStream_t s) {
-  static const bool first_form = [] {
-    const char* v = std::getenv("GAM_ATTN");
-    return v && std::strcmp(v, "1") == 0;
-  }();
+  // GAM_ATTN=1 selects the earlier 128-key kernel (read at each launch)
+  const char* form = std::getenv("GAM_ATTN");
+  const bool first_form = form && std::strcmp(form, "1") == 0;
   if (t_half && !first_form) return launch_attention_tc2(cache, qk, vt, clips, o, rows_pad, n_heads, d_head, t_max, s);
   if (t_half) return launch_attention_tc(cache, qk, vt, clips, o, rows_pad, n_heads, d_head, t_max, s);
   return launch_attention_simt(qk, vt, clips, o, t_half, rows_pad, n_heads, d_head, t_max, s);

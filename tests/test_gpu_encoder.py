@@ -153,6 +153,27 @@ def test_c5_quantized_full_batch_sampled(name):
     ctx.close()
 
 
+@pytest.mark.parametrize("form", ["1", "2"], ids=["attn_128_key_blocks", "attn_64_key_blocks"])
+@pytest.mark.parametrize("K", [31, 5])
+def test_attention_forms_small_model(form, K, monkeypatch):
+    """Both tensor-core attention kernels (GAM_ATTN=1: 128-key blocks; the default:
+    64-key blocks with scores double-buffered in TMEM) on ragged clips, d_h 64,
+    against the oracle."""
+    monkeypatch.setenv("GAM_ATTN", form)
+    model = small_model(d=256, heads=4, ffn=512, layers=2, K=K)
+    cfg, W = config_and_weights(model, 34, "fp16")
+    audio, lens = synth.random_audio([48000, 17000, 30001], seed=11)
+    ctx = gam.gam_create(cfg, W, 3, 48000)
+    enc, el = gam.gam_encode(ctx, to_torch(audio), lens)
+    enc = enc.cpu().numpy()
+    for i in range(3):
+        ref = oracle.encode_clip(audio[i, :lens[i]].astype(np.float64), W, cfg)
+        assert rel_fro(enc[i, :el[i]], ref) <= TOL_REL_FRO, (form, i)
+        assert max_abs(enc[i, :el[i]], ref) <= TOL_MAX_ABS, (form, i)
+    gam.gam_device_status(ctx)
+    ctx.close()
+
+
 @pytest.mark.parametrize("tiles", ["m1", "m2"])
 @pytest.mark.parametrize("precision", ["int8_g64", "int6_g64", "int4_g64"])
 def test_quantized_small_model(precision, tiles, monkeypatch):
